@@ -1,0 +1,269 @@
+"""ctypes binding of the fp64 CPU oracle (``moe_oracle.c``).
+
+TEST INFRASTRUCTURE: only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. It shares no code with
+the CUDA library. Tensors are numpy arrays; bf16 tensors are ``uint16`` arrays
+holding the raw bf16 bits, binary32 tensors are ``float32`` arrays.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+
+def build(force: bool = False) -> str:
+    """Compile ``moe_oracle.c`` with gcc into ``oracle/liboracle.so``."""
+    src = os.path.join(_HERE, "moe_oracle.c")
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < max(
+        os.path.getmtime(src), os.path.getmtime(os.path.join(_HERE, "moe_oracle.h"))
+    ):
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-o", _LIB_PATH, src, "-lm"]
+        )
+    return _LIB_PATH
+
+
+class OracleCfg(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int32),
+        ("n_routed", ctypes.c_int32),
+        ("n_shared", ctypes.c_int32),
+        ("top_k", ctypes.c_int32),
+        ("n_group", ctypes.c_int32),
+        ("topk_group", ctypes.c_int32),
+        ("inter", ctypes.c_int32),
+        ("score_fn", ctypes.c_int32),
+        ("renormalize", ctypes.c_int32),
+        ("routed_scaling_factor", ctypes.c_double),
+        ("cap_policy", ctypes.c_int32),
+        ("capacity_factor", ctypes.c_double),
+        ("capacity", ctypes.c_int32),
+    ]
+
+
+class OracleStats(ctypes.Structure):
+    _fields_ = [
+        ("overflowed", ctypes.c_int64),
+        ("dropped", ctypes.c_int64),
+        ("exempt_tokens", ctypes.c_int64),
+        ("capacity", ctypes.c_int64),
+    ]
+
+
+class DsArch(ctypes.Structure):
+    _fields_ = [
+        (name, ctypes.c_int64)
+        for name in (
+            "n_layers d_model q_lora_rank kv_lora_rank n_heads qk_nope_dim qk_rope_dim v_head_dim "
+            "vocab first_k_dense dense_inter n_routed n_shared top_k moe_inter"
+        ).split()
+    ]
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        _lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i64, i32 = ctypes.c_int64, ctypes.c_int32
+        _lib.oracle_router_logits.argtypes = [i64, i32, i32, P, i32, P, i32, P]
+        _lib.oracle_route.argtypes = [P, i64, P, P, P, P, P, P, P]
+        _lib.oracle_route_capacity.argtypes = [P, i64, P, P, P, P, P, P]
+        _lib.oracle_capacity_value.argtypes = [P, i64]
+        _lib.oracle_capacity_value.restype = i64
+        _lib.oracle_dispatch.argtypes = [i64, i32, i32, P, P, P, P, P]
+        _lib.oracle_dispatch.restype = i64
+        _lib.oracle_swiglu.argtypes = [i32, i32, i64, P, P, P, P, i32, P]
+        _lib.oracle_combine.argtypes = [i64, i32, i32, P, P, P, P, P]
+        _lib.oracle_layer.argtypes = [P, i64] + [P] * 9 + [i32] + [P] * 6
+        _lib.oracle_ds_params.argtypes = [P, P, P]
+    return _lib
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dt(a: np.ndarray) -> int:
+    if a.dtype == np.float32:
+        return 0
+    if a.dtype == np.uint16:
+        return 1
+    raise TypeError(f"oracle tensors are float32 or uint16 (bf16 bits), got {a.dtype}")
+
+
+def _c(a, dtype=None):
+    if a is None:
+        return None
+    return np.ascontiguousarray(a if dtype is None else a.astype(dtype, copy=False))
+
+
+@dataclass
+class Cfg:
+    """Layer configuration in the pages' field names."""
+
+    d_model: int
+    n_routed: int
+    top_k: int
+    moe_intermediate_size: int
+    n_shared: int = 0
+    n_group: int = 1
+    topk_group: int = 1
+    score_fn: str = "softmax"  # or "sigmoid"
+    renormalize: bool = False
+    routed_scaling_factor: float = 1.0
+    cap_policy: str = "none"  # "none" | "overflow_next" | "drop"
+    capacity_factor: float = 0.0
+    capacity: int = 0
+
+    def c(self) -> OracleCfg:
+        return OracleCfg(
+            self.d_model,
+            self.n_routed,
+            self.n_shared,
+            self.top_k,
+            self.n_group,
+            self.topk_group,
+            self.moe_intermediate_size,
+            {"softmax": 0, "sigmoid": 1}[self.score_fn],
+            int(bool(self.renormalize)),
+            float(self.routed_scaling_factor),
+            {"none": 0, "overflow_next": 1, "drop": 2}[self.cap_policy],
+            float(self.capacity_factor),
+            int(self.capacity),
+        )
+
+
+def router_logits(x: np.ndarray, w_r: np.ndarray) -> np.ndarray:
+    x, w_r = _c(x), _c(w_r)
+    n, d = x.shape
+    E = w_r.shape[0]
+    out = np.empty((n, E), np.float64)
+    lib().oracle_router_logits(n, d, E, _ptr(x), _dt(x), _ptr(w_r), _dt(w_r), _ptr(out))
+    return out
+
+
+def route(cfg: Cfg, logits: np.ndarray, bias=None, want_ranking=False):
+    """Routing without capacity. Returns (topk_idx, topk_w, exempt, ranking|None, stats)."""
+    logits = _c(logits, np.float64)
+    bias = _c(bias, np.float32)
+    n = logits.shape[0]
+    k, E = cfg.top_k, cfg.n_routed
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    ex = np.empty(n, np.uint8)
+    rk = np.empty((n, E), np.int32) if want_ranking else None
+    st = OracleStats()
+    c = cfg.c()
+    lib().oracle_route(
+        ctypes.byref(c), n, _ptr(logits), _ptr(bias), _ptr(idx), _ptr(w), _ptr(ex), _ptr(rk),
+        ctypes.byref(st),
+    )
+    return idx, w, ex.astype(bool), rk, st
+
+
+def route_capacity(cfg: Cfg, logits: np.ndarray, bias=None):
+    """Routing with the configured capacity policy. Returns (topk_idx, topk_w, exempt, stats)."""
+    logits = _c(logits, np.float64)
+    bias = _c(bias, np.float32)
+    n = logits.shape[0]
+    k = cfg.top_k
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    ex = np.empty(n, np.uint8)
+    st = OracleStats()
+    c = cfg.c()
+    lib().oracle_route_capacity(
+        ctypes.byref(c), n, _ptr(logits), _ptr(bias), _ptr(idx), _ptr(w), _ptr(ex), ctypes.byref(st)
+    )
+    return idx, w, ex.astype(bool), st
+
+
+def capacity_value(cfg: Cfg, n: int) -> int:
+    c = cfg.c()
+    return int(lib().oracle_capacity_value(ctypes.byref(c), n))
+
+
+def dispatch(topk_idx: np.ndarray, E: int):
+    """Returns (counts[E], offsets[E+1], perm_token[kept], slot_dest[n,k])."""
+    topk_idx = _c(topk_idx, np.int32)
+    n, k = topk_idx.shape
+    counts = np.empty(E, np.int32)
+    offsets = np.empty(E + 1, np.int32)
+    perm = np.empty(max(n * k, 1), np.int32)
+    dest = np.empty((n, k), np.int32)
+    kept = lib().oracle_dispatch(n, k, E, _ptr(topk_idx), _ptr(counts), _ptr(offsets), _ptr(perm), _ptr(dest))
+    return counts, offsets, perm[:kept].copy(), dest
+
+
+def swiglu(x: np.ndarray, w_gate: np.ndarray, w_up: np.ndarray, w_down: np.ndarray) -> np.ndarray:
+    """x[m, d] (float64) through one SwiGLU expert with W_g, W_u [I, d], W_d [d, I]."""
+    x = _c(x, np.float64)
+    w_gate, w_up, w_down = _c(w_gate), _c(w_up), _c(w_down)
+    assert w_gate.dtype == w_up.dtype == w_down.dtype
+    m, d = x.shape
+    I = w_gate.shape[0]
+    out = np.empty((m, d), np.float64)
+    lib().oracle_swiglu(d, I, m, _ptr(x), _ptr(w_gate), _ptr(w_up), _ptr(w_down), _dt(w_gate), _ptr(out))
+    return out
+
+
+def combine(eo: np.ndarray, slot_dest: np.ndarray, topk_w: np.ndarray, sh=None) -> np.ndarray:
+    eo = _c(eo, np.float64)
+    slot_dest = _c(slot_dest, np.int32)
+    topk_w = _c(topk_w, np.float64)
+    sh = _c(sh, np.float64)
+    n, k = slot_dest.shape
+    d = eo.shape[1]
+    y = np.empty((n, d), np.float64)
+    lib().oracle_combine(n, k, d, _ptr(eo), _ptr(slot_dest), _ptr(topk_w), _ptr(sh), _ptr(y))
+    return y
+
+
+def layer(cfg: Cfg, x, w_r, w_gate, w_up, w_down, bias=None, ws_gate=None, ws_up=None, ws_down=None):
+    """Whole layer. Returns dict(y, topk_idx, topk_w, counts, exempt, stats)."""
+    x, w_r, w_gate, w_up, w_down = (_c(a) for a in (x, w_r, w_gate, w_up, w_down))
+    ws_gate, ws_up, ws_down = (_c(a) for a in (ws_gate, ws_up, ws_down))
+    bias = _c(bias, np.float32)
+    dt = _dt(x)
+    for a in (w_r, w_gate, w_up, w_down, ws_gate, ws_up, ws_down):
+        assert a is None or _dt(a) == dt
+    n = x.shape[0]
+    k, E, d = cfg.top_k, cfg.n_routed, cfg.d_model
+    y = np.empty((n, d), np.float64)
+    idx = np.empty((n, k), np.int32)
+    w = np.empty((n, k), np.float64)
+    counts = np.empty(E, np.int32)
+    ex = np.empty(n, np.uint8)
+    st = OracleStats()
+    c = cfg.c()
+    lib().oracle_layer(
+        ctypes.byref(c), n, _ptr(x), _ptr(w_r), _ptr(bias), _ptr(w_gate), _ptr(w_up), _ptr(w_down),
+        _ptr(ws_gate), _ptr(ws_up), _ptr(ws_down), dt, _ptr(y), _ptr(idx), _ptr(w), _ptr(counts),
+        _ptr(ex), ctypes.byref(st),
+    )
+    return dict(y=y, topk_idx=idx, topk_w=w, counts=counts, exempt=ex.astype(bool), stats=st)
+
+
+def ds_params(**fields) -> tuple[int, int]:
+    a = DsArch(**fields)
+    total, active = ctypes.c_int64(), ctypes.c_int64()
+    lib().oracle_ds_params(ctypes.byref(a), ctypes.byref(total), ctypes.byref(active))
+    return total.value, active.value
+
+
+def bf16_to_f64(a: np.ndarray) -> np.ndarray:
+    """Exact widening of raw bf16 bits (uint16) or float32 to float64 (input decoding only)."""
+    if a.dtype == np.uint16:
+        return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return a.astype(np.float64)

@@ -1,0 +1,453 @@
+"""Pins of the fp64 CPU oracle to facts outside itself.
+
+Each test ties one oracle function to something the oracle does not compute
+itself: integers printed on the pages, hand-worked examples, a library routine
+(numpy/torch/scipy) that solves a special case, brute-force enumeration, or a
+closed form. A dropped term, a wrong sign or index, or a transposed operand in
+the oracle fails at least one of these.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import scipy.special
+import torch
+
+from oracle import oracle as O
+from synth import workloads as W
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def _cfg(E, k, **kw):
+    base = dict(d_model=1, n_routed=E, top_k=k, moe_intermediate_size=1)
+    base.update(kw)
+    return O.Cfg(**base)
+
+
+# ---------------------------------------------------------------- parameter ledger (printed integers)
+
+
+def test_deepseek_v3_ledger_matches_printed_totals():
+    g = _gold("deepseek_param_ledger.json")["deepseek_v3"]
+    total, active = O.ds_params(**g["arch"])
+    assert total == g["total"] == 671026404352
+    assert active == g["active"] == 37552282624
+    a = g["arch"]
+    # per-module integers printed beside the totals
+    assert 3 * a["d_model"] * a["moe_inter"] == g["per_expert"]
+    assert 3 * a["d_model"] * a["dense_inter"] == g["dense_ffn"]
+    assert a["n_routed"] * a["d_model"] == g["router"]
+    assert a["vocab"] * a["d_model"] == g["embedding"]
+
+
+def test_deepseek_v2_ledger_matches_printed_total():
+    g = _gold("deepseek_param_ledger.json")["deepseek_v2"]
+    total, active = O.ds_params(**g["arch"])
+    assert total == g["total"] == 235741434880
+    assert round(active / 1e9) == 21  # the page's "21B activated"
+
+
+def test_ledger_mla_term():
+    # With every non-MLA term zeroed except norms, total = layers * MLA + norms.
+    g = _gold("deepseek_param_ledger.json")["deepseek_v3"]
+    a = dict(g["arch"], first_k_dense=0, dense_inter=0, n_routed=0, n_shared=0, top_k=0, vocab=0)
+    a["n_layers"] = 1
+    total, _ = O.ds_params(**a)
+    assert total - (2 * 7168 + 7168) == g["per_layer_mla"]
+
+
+# ---------------------------------------------------------------- router logits
+
+
+def test_router_logits_match_numpy_matmul():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((37, 53)).astype(np.float32)
+    w = rng.standard_normal((11, 53)).astype(np.float32)
+    ref = x.astype(np.float64) @ w.astype(np.float64).T
+    np.testing.assert_allclose(O.router_logits(x, w), ref, rtol=1e-12, atol=1e-12)
+
+
+def test_router_logits_bf16_inputs_widened_exactly():
+    w = W.get("mixtral_small")
+    inp = W.host_inputs(w, names=["x", "w_r"])
+    ref = O.bf16_to_f64(inp["x"]) @ O.bf16_to_f64(inp["w_r"]).T
+    np.testing.assert_allclose(O.router_logits(inp["x"], inp["w_r"]), ref, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- selection: worked examples
+
+
+@pytest.mark.parametrize("case", ["softmax_ties", "softmax_tie_at_cut"])
+def test_softmax_worked_examples(case):
+    g = _gold("routing_worked_examples.json")[case]
+    lg = np.array(g["logits"])
+    idx, w, ex, _, _ = O.route(_cfg(lg.shape[1], g["top_k"]), lg)
+    assert idx.tolist() == g["expect_idx"]
+
+
+def test_sigmoid_group_worked_example():
+    g = _gold("routing_worked_examples.json")["sigmoid_groups"]
+    lg = np.array(g["logits"])
+    cfg = _cfg(8, g["top_k"], score_fn="sigmoid", n_group=g["n_group"], topk_group=g["topk_group"],
+               renormalize=True, routed_scaling_factor=g["routed_scaling_factor"])
+    idx, w, ex, _, _ = O.route(cfg, lg, bias=np.zeros(8, np.float32))
+    assert idx.tolist() == g["expect_idx"]
+    np.testing.assert_allclose(w, g["expect_w"], rtol=1e-15)
+
+
+def test_sigmoid_bias_worked_example():
+    g = _gold("routing_worked_examples.json")["sigmoid_bias_selection_only"]
+    lg = np.array(g["logits"])
+    b = np.array(g["bias"], np.float32)
+    for renorm, key in ((True, "expect_w_renorm"), (False, "expect_w_raw")):
+        cfg = _cfg(4, 1, score_fn="sigmoid", renormalize=renorm)
+        idx, w, _, _, _ = O.route(cfg, lg, bias=b)
+        assert idx.tolist() == g["expect_idx"]
+        np.testing.assert_allclose(w, g[key], rtol=1e-15)
+
+
+# ---------------------------------------------------------------- selection: library and brute force
+
+
+def _lexsort_topk(vals, k):
+    """Plain top-k by a library sort: descending value, ties to lower index."""
+    E = vals.shape[1]
+    out = []
+    for row in vals:
+        order = np.lexsort((np.arange(E), -row))
+        out.append(order[:k])
+    return np.array(out, np.int32)
+
+
+def test_plain_topk_reduces_to_library_sort():
+    rng = np.random.default_rng(2)
+    lg = rng.standard_normal((200, 19))
+    lg[:20] = np.round(lg[:20])  # exact ties
+    idx, w, _, _, _ = O.route(_cfg(19, 5), lg)
+    np.testing.assert_array_equal(idx, _lexsort_topk(lg, 5))
+    p = scipy.special.softmax(lg, axis=1)
+    np.testing.assert_allclose(w, np.take_along_axis(p, idx, 1), rtol=1e-13)
+
+
+def test_renormalised_softmax_gates_equal_softmax_of_selected_logits():
+    rng = np.random.default_rng(3)
+    lg = rng.standard_normal((50, 8)) * 3
+    idx, w, _, _, _ = O.route(_cfg(8, 2, renormalize=True), lg)
+    sel = np.take_along_axis(lg, idx, 1)
+    np.testing.assert_allclose(w, scipy.special.softmax(sel, axis=1), rtol=1e-13)
+    np.testing.assert_allclose(w.sum(1), 1.0, rtol=1e-14)
+
+
+def _brute_group_topk(c, G, keep, k):
+    """Enumerate group subsets, then expert subsets (lexicographically first among the best)."""
+    E = len(c)
+    per = E // G
+    gscore = [max(c[g * per + a] + c[g * per + b] for a in range(per) for b in range(per) if a != b)
+              for g in range(G)]
+    best_groups = None
+    for gs in itertools.combinations(range(G), keep):
+        s = math.fsum(gscore[g] for g in gs)  # correctly rounded: order-independent
+        if best_groups is None or s > best_groups[0]:
+            best_groups = (s, gs)
+    elig = [e for e in range(E) if e // per in best_groups[1]]
+    best = None
+    for es in itertools.combinations(elig, k):
+        s = math.fsum(c[e] for e in es)
+        if best is None or s > best[0]:
+            best = (s, es)
+    return sorted(best[1], key=lambda e: (-c[e], e))
+
+
+@pytest.mark.parametrize("integer_logits", [False, True])
+def test_group_limited_topk_matches_brute_force(integer_logits):
+    rng = np.random.default_rng(4 + integer_logits)
+    E, G, keep, k = 12, 4, 2, 3
+    lg = rng.integers(-2, 3, (300, E)).astype(np.float64) if integer_logits else rng.standard_normal((300, E))
+    bias = np.zeros(E, np.float32) if integer_logits else rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    cfg = _cfg(E, k, score_fn="sigmoid", n_group=G, topk_group=keep, renormalize=True,
+               routed_scaling_factor=2.5)
+    idx, w, ex, _, _ = O.route(cfg, lg, bias=bias)
+    s = scipy.special.expit(lg)
+    c = s + bias.astype(np.float64)
+    for t in range(lg.shape[0]):
+        assert idx[t].tolist() == _brute_group_topk(c[t], G, keep, k), t
+    sel = np.take_along_axis(s, idx, 1)
+    np.testing.assert_allclose(w, sel / sel.sum(1, keepdims=True) * 2.5, rtol=1e-13)
+    if integer_logits:
+        assert ex.any()  # exact ties are flagged
+
+
+def test_group_invariants_on_v3_shapes():
+    rng = np.random.default_rng(6)
+    E, G, keep, k = 256, 8, 4, 8
+    lg = rng.standard_normal((400, E))
+    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    cfg = _cfg(E, k, score_fn="sigmoid", n_group=G, topk_group=keep, renormalize=True,
+               routed_scaling_factor=2.5)
+    idx, w, _, _, _ = O.route(cfg, lg, bias=bias)
+    c = scipy.special.expit(lg) + bias
+    gs = np.sort(c.reshape(-1, G, E // G), axis=2)[:, :, -2:].sum(2)
+    for t in range(lg.shape[0]):
+        assert len(set(idx[t].tolist())) == k
+        kept = set(np.lexsort((np.arange(G), -gs[t]))[:keep].tolist())
+        assert all(e // (E // G) in kept for e in idx[t])
+    np.testing.assert_allclose(w.sum(1), 2.5, rtol=1e-13)
+    # a huge bias on one expert forces it (and its group) in
+    b2 = bias.copy()
+    b2[77] = 100.0
+    idx2, _, _, _, _ = O.route(cfg, lg, bias=b2)
+    assert (idx2[:, 0] == 77).all()
+
+
+def test_bias_changes_selection_never_gate_values():
+    rng = np.random.default_rng(7)
+    E, k = 64, 6
+    lg = rng.standard_normal((500, E))
+    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    cfg = _cfg(E, k, score_fn="sigmoid", n_group=8, topk_group=4, renormalize=True, routed_scaling_factor=2.5)
+    i0, w0, _, _, _ = O.route(cfg, lg, bias=np.zeros(E, np.float32))
+    i1, w1, _, _, _ = O.route(cfg, lg, bias=bias)
+    same = (np.sort(i0, 1) == np.sort(i1, 1)).all(1)
+    assert same.any() and (~same).any()
+    for t in np.nonzero(same)[0]:
+        a = dict(zip(i0[t], w0[t]))
+        b = dict(zip(i1[t], w1[t]))
+        assert a.keys() == b.keys()
+        # same values up to the order of the normalising sum (slots may be reordered)
+        np.testing.assert_allclose([a[e] for e in a], [b[e] for e in a], rtol=1e-15)
+    # gates always use raw scores: w = s_sel / sum s_sel * rsf
+    s = scipy.special.expit(lg)
+    sel = np.take_along_axis(s, i1, 1)
+    np.testing.assert_allclose(w1, sel / sel.sum(1, keepdims=True) * 2.5, rtol=1e-13)
+
+
+def test_exemption_flags_near_ties_only():
+    lg = np.array([[3.0, 1.0, 1.0 + 1e-9, -2.0], [3.0, 1.0, 0.5, -2.0], [2.0, 2.0, 0.0, -1.0]])
+    _, _, ex, _, st = O.route(_cfg(4, 2), lg)
+    # row 0: 2nd and 3rd differ by 1e-9 relative; row 2: the two selected tie (order boundary)
+    assert ex.tolist() == [True, False, True]
+    assert st.exempt_tokens == 2
+
+
+# ---------------------------------------------------------------- capacity
+
+
+@pytest.mark.parametrize("case", ["capacity_k1", "capacity_k2", "capacity_drop_when_exhausted", "drop_policy"])
+def test_capacity_worked_examples(case):
+    g = _gold("routing_worked_examples.json")[case]
+    lg = np.array(g["logits"])
+    cfg = _cfg(lg.shape[1], g["top_k"], cap_policy=g.get("cap_policy", "overflow_next"),
+               capacity=g["capacity"], renormalize=True)
+    idx, w, _, st = O.route_capacity(cfg, lg)
+    assert idx.tolist() == g["expect_idx"]
+    assert st.overflowed == g["expect_overflowed"] and st.dropped == g["expect_dropped"]
+    assert (w[idx < 0] == 0).all()
+
+
+def _fill_event_routing(rankings, k, C):
+    """Event-driven reformulation of the greedy: between two fill events every token simply takes
+    its first k non-full experts, so commit up to the first token that fills an expert."""
+    n, E = rankings.shape
+    full = np.zeros(E, bool)
+    count = np.zeros(E, np.int64)
+    out = -np.ones((n, k), np.int64)
+    t0 = 0
+    while t0 < n:
+        choice = -np.ones((n - t0, k), np.int64)
+        for i, t in enumerate(range(t0, n)):
+            r = [e for e in rankings[t] if e >= 0 and not full[e]][:k]
+            choice[i, : len(r)] = r
+        # first token at which some expert reaches C
+        run = count.copy()
+        stop = n - t0 - 1
+        for i in range(n - t0):
+            hit = False
+            for e in choice[i]:
+                if e >= 0:
+                    run[e] += 1
+                    hit |= run[e] == C
+            if hit:
+                stop = i
+                break
+        out[t0 : t0 + stop + 1] = choice[: stop + 1]
+        for e in choice[: stop + 1].ravel():
+            if e >= 0:
+                count[e] += 1
+        full |= count >= C
+        t0 += stop + 1
+    return out
+
+
+@pytest.mark.parametrize("seed,n,E,k,C", [(8, 16, 4, 2, 5), (9, 300, 8, 2, 60), (10, 400, 16, 3, 50)])
+def test_capacity_greedy_matches_fill_event_reformulation(seed, n, E, k, C):
+    rng = np.random.default_rng(seed)
+    lg = rng.standard_normal((n, E)) - 1.2 * np.log(np.arange(E) + 1)  # skewed demand
+    cfg = _cfg(E, k, cap_policy="overflow_next", capacity=C)
+    idx, w, _, st = O.route_capacity(cfg, lg)
+    rankings = np.array([np.lexsort((np.arange(E), -row)) for row in lg])
+    np.testing.assert_array_equal(idx, _fill_event_routing(rankings, k, C))
+    counts = np.bincount(idx[idx >= 0], minlength=E)
+    assert counts.max() <= C
+    assert st.overflowed > 0
+
+
+def test_capacity_at_least_n_times_k_is_no_capacity():
+    rng = np.random.default_rng(11)
+    lg = rng.standard_normal((500, 16)) - 1.2 * np.log(np.arange(16) + 1)
+    i0, w0, _, _, _ = O.route(_cfg(16, 2), lg)
+    i1, w1, _, st = O.route_capacity(_cfg(16, 2, cap_policy="overflow_next", capacity=1000), lg)
+    np.testing.assert_array_equal(i0, i1)
+    np.testing.assert_array_equal(w0, w1)
+    assert st.overflowed == 0 and st.dropped == 0
+
+
+def test_capacity_value_formula():
+    cfg = _cfg(64, 2, cap_policy="overflow_next", capacity_factor=1.25)
+    assert O.capacity_value(cfg, 32768) == 1280  # 1.25 * 32768 * 2 / 64
+    assert O.capacity_value(cfg, 1000) == math.ceil(1.25 * 1000 * 2 / 64)
+
+
+def test_drop_policy_invariants():
+    rng = np.random.default_rng(12)
+    E, k, C = 16, 2, 40
+    lg = rng.standard_normal((600, E)) - 1.2 * np.log(np.arange(E) + 1)
+    i0, _, _, _, _ = O.route(_cfg(E, k), lg)
+    i1, w1, _, st = O.route_capacity(_cfg(E, k, cap_policy="drop", capacity=C), lg)
+    kept = i1 >= 0
+    assert (i1[kept] == i0[kept]).all()  # kept slots are the original choices, in place
+    counts = np.bincount(i1[kept], minlength=E)
+    assert counts.max() <= C and st.dropped == (~kept).sum() > 0
+    # a slot is dropped exactly when its expert already had C earlier slots
+    seen = np.zeros(E, int)
+    for t in range(i0.shape[0]):
+        for j in range(k):
+            e = i0[t, j]
+            assert kept[t, j] == (seen[e] < C)
+            seen[e] += kept[t, j]
+
+
+# ---------------------------------------------------------------- dispatch
+
+
+def test_dispatch_is_a_stable_argsort():
+    rng = np.random.default_rng(13)
+    n, k, E = 257, 3, 10
+    idx = np.stack([rng.permutation(E)[:k] for _ in range(n)]).astype(np.int32)
+    idx[5, 1] = -1  # a dropped slot
+    counts, offsets, perm, dest = O.dispatch(idx, E)
+    flat = idx.ravel()
+    keep = np.nonzero(flat >= 0)[0]
+    order = keep[np.argsort(flat[keep], kind="stable")]
+    np.testing.assert_array_equal(perm, order // k)
+    np.testing.assert_array_equal(counts, np.bincount(flat[keep], minlength=E))
+    np.testing.assert_array_equal(offsets, np.concatenate([[0], np.cumsum(counts)]))
+    d = dest.ravel()
+    assert d[5 * k + 1] == -1
+    np.testing.assert_array_equal(d[order], np.arange(len(order)))  # bijection, inverse of perm
+
+
+def test_identity_experts_reproduce_input_times_gate_sum():
+    w = W.get("deepseek_v3_small")
+    inp = W.host_inputs(w, names=["x", "w_r", "bias"])
+    cfg = O.Cfg(**w.cfg_fields())
+    lg = O.router_logits(inp["x"], inp["w_r"])
+    idx, tw, _, _, _ = O.route(cfg, lg, inp["bias"])
+    counts, offsets, perm, dest = O.dispatch(idx, w.n_routed)
+    x = O.bf16_to_f64(inp["x"])
+    y = O.combine(x[perm], dest, tw)  # expert = identity
+    np.testing.assert_allclose(y, x * tw.sum(1, keepdims=True), rtol=1e-14, atol=1e-14)
+
+
+# ---------------------------------------------------------------- SwiGLU, shared experts, combine
+
+
+def _torch_swiglu(x, wg, wu, wd):
+    x, wg, wu, wd = (torch.from_numpy(O.bf16_to_f64(a) if a.dtype == np.uint16 else a.astype(np.float64))
+                     for a in (x, wg, wu, wd))
+    return (torch.nn.functional.silu(x @ wg.T) * (x @ wu.T) @ wd.T).numpy()
+
+
+def test_silu_closed_form():
+    one = np.ones((1, 1), np.float32)
+    out = O.swiglu(np.array([[1.0]]), one, one, one)
+    assert out[0, 0] == pytest.approx(1.0 / (1.0 + math.exp(-1.0)), rel=1e-15)  # silu(1) * 1
+    out = O.swiglu(np.array([[-2.0]]), one, one, one)
+    assert out[0, 0] == pytest.approx(-2.0 / (1.0 + math.exp(2.0)) * -2.0, rel=1e-15)
+
+
+def test_swiglu_matches_torch_float64():
+    rng = np.random.default_rng(14)
+    d, I, m = 48, 80, 9
+    x = rng.standard_normal((m, d))
+    wg, wu = (rng.standard_normal((I, d)).astype(np.float32) for _ in range(2))
+    wd = rng.standard_normal((d, I)).astype(np.float32)
+    np.testing.assert_allclose(O.swiglu(x, wg, wu, wd), _torch_swiglu(x, wg, wu, wd), rtol=1e-11, atol=1e-11)
+
+
+def test_single_expert_layer_is_a_dense_ffn():
+    rng = np.random.default_rng(15)
+    d, I, n = 32, 48, 20
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    wr = rng.standard_normal((1, d)).astype(np.float32)
+    wg, wu = (rng.standard_normal((1, I, d)).astype(np.float32) for _ in range(2))
+    wd = rng.standard_normal((1, d, I)).astype(np.float32)
+    cfg = O.Cfg(d_model=d, n_routed=1, top_k=1, moe_intermediate_size=I)
+    r = O.layer(cfg, x, wr, wg, wu, wd)
+    np.testing.assert_allclose(r["y"], _torch_swiglu(x, wg[0], wu[0], wd[0]), rtol=1e-11, atol=1e-11)
+
+
+def test_k_equals_E_is_the_dense_softmax_mixture():
+    rng = np.random.default_rng(16)
+    d, I, n, E = 24, 40, 15, 5
+    x = rng.standard_normal((n, d)).astype(np.float32)
+    wr = rng.standard_normal((E, d)).astype(np.float32)
+    wg, wu = (rng.standard_normal((E, I, d)).astype(np.float32) for _ in range(2))
+    wd = rng.standard_normal((E, d, I)).astype(np.float32)
+    cfg = O.Cfg(d_model=d, n_routed=E, top_k=E, moe_intermediate_size=I)
+    r = O.layer(cfg, x, wr, wg, wu, wd)
+    p = scipy.special.softmax(x.astype(np.float64) @ wr.astype(np.float64).T, axis=1)
+    ref = sum(p[:, e : e + 1] * _torch_swiglu(x, wg[e], wu[e], wd[e]) for e in range(E))
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-10, atol=1e-11)
+
+
+def test_shared_experts_are_added_unweighted_and_concatenate():
+    w = W.get("deepseek_v2_small", n=30)
+    inp = W.host_inputs(w)
+    cfg = O.Cfg(**w.cfg_fields())
+    r = O.layer(cfg, inp["x"], inp["w_r"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                ws_gate=inp["ws_gate"], ws_up=inp["ws_up"], ws_down=inp["ws_down"])
+    r0 = O.layer(cfg.__class__(**{**cfg.__dict__, "n_shared": 0}), inp["x"], inp["w_r"], inp["w_gate"],
+                 inp["w_up"], inp["w_down"])
+    I = w.moe_intermediate_size
+    sh = sum(_torch_swiglu(inp["x"], inp["ws_gate"][s * I:(s + 1) * I], inp["ws_up"][s * I:(s + 1) * I],
+                           inp["ws_down"][:, s * I:(s + 1) * I]) for s in range(w.n_shared))
+    np.testing.assert_allclose(r["y"] - r0["y"], sh, rtol=1e-9, atol=1e-10)
+
+
+def test_layer_composes_route_dispatch_swiglu_combine():
+    w = W.get("mixtral_small", n=64)
+    inp = W.host_inputs(w)
+    cfg = O.Cfg(**w.cfg_fields())
+    r = O.layer(cfg, inp["x"], inp["w_r"], inp["w_gate"], inp["w_up"], inp["w_down"])
+    lg = O.bf16_to_f64(inp["x"]) @ O.bf16_to_f64(inp["w_r"]).T
+    idx = _lexsort_topk(lg, 2)
+    np.testing.assert_array_equal(r["topk_idx"], idx)
+    sel = np.take_along_axis(lg, idx, 1)
+    gw = scipy.special.softmax(sel, axis=1)
+    ref = np.zeros((w.n, w.d_model))
+    for t in range(w.n):
+        for j in range(2):
+            e = idx[t, j]
+            ref[t] += gw[t, j] * _torch_swiglu(inp["x"][t : t + 1], inp["w_gate"][e], inp["w_up"][e],
+                                               inp["w_down"][e])[0]
+    np.testing.assert_allclose(r["y"], ref, rtol=1e-9, atol=1e-10)
+    np.testing.assert_array_equal(r["counts"], np.bincount(idx.ravel(), minlength=8))
