@@ -1,0 +1,377 @@
+"""Benchmark of the sparse-MoE FFN layer forward on B200 (one process per GPU).
+
+python bench.py --gpus N --steps K --warmup W [--impl ours|reference] [--workload NAME]
+
+A step is one moe_layer_forward (route + permute + SwiGLU experts + shared
+experts + combine) over one batch of synthetic tokens whose inputs are already
+resident in HBM. The default workload is the Mixtral-8x7B-shaped layer
+(n = 4096 tokens, d = 4096, 8 experts, top-2, I = 14336, bf16). Ranks are
+independent replicas (weak scaling, no collective on the data path); the time
+is the maximum over ranks of the CUDA-event time of K steps.
+
+The reference arm (--impl reference) times the fp64 CPU oracle on the host
+cores on a bounded token sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer tokens/s (route+permute+SwiGLU+combine) and % of roofline, 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return p["hbm_gbs"], p["bf16_tflops"], p.get("bf16_tflops_sustained"), "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def layer_work(w, kept_slots, active_experts):
+    """Algorithmic FLOPs and bytes of one layer forward."""
+    b = 2 if w.dtype == "bf16" else 4
+    d, I, E, n = w.d_model, w.moe_intermediate_size, w.n_routed, w.n
+    flops = 2 * n * E * d + 6 * kept_slots * d * I + 6 * n * d * w.I_s
+    bytes_ = E * d * b + active_experts * 3 * d * I * b + 3 * d * w.I_s * b + 2 * n * d * b
+    return flops, bytes_
+
+
+def launches_per_step(w):
+    """Kernels of this library launched by one moe_layer_forward."""
+    n = 2  # router GEMM + route
+    if w.cap_policy != "none":
+        n += 2  # capacity + gates
+    n += 2  # counts: histogram + scan
+    n += 4  # permute: histogram + scan + scatter + gather
+    n += 2  # GEMM1 (SwiGLU) + GEMM2
+    if w.n_shared:
+        n += 2
+    n += 1  # combine
+    return n
+
+
+def _sources_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "top_routing_expert_router_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_key, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it matches the current sources."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        e = t[kernel_key][workload]
+        if e.get("sources_sha") == _sources_sha():
+            return e["bytes_per_launch"]
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.out,
+                                         stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            self.proc.wait(timeout=10)
+
+    def summary(self):
+        self.out.flush()
+        self.out.seek(0)
+        rows = [r.split(",") for r in self.out.read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import top_routing_expert_router_b200 as moe
+    from synth import workloads as W
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    w = W.get(args.workload)
+    dev = W.device_inputs(w, seed=rank, device=f"cuda:{local}")
+    cfg = moe.make_config(dtype=w.dtype, **w.cfg_fields())
+    n = w.n
+    ws = torch.empty(moe.moe_workspace_size(cfg, n), dtype=torch.uint8, device="cuda")
+    y = torch.empty((n, w.d_model), dtype=dev["x"].dtype, device="cuda")
+    counts = torch.empty(w.n_routed, dtype=torch.int32, device="cuda")
+    diag = torch.zeros(8, dtype=torch.int32, device="cuda")
+    weights = moe.make_weights(dev["w_r"], dev["w_gate"], dev["w_up"], dev["w_down"], dev.get("ws_gate"),
+                               dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+
+    def step():
+        moe.moe_layer_forward(cfg, n, dev["x"], weights, y, ws, counts=counts, diag=diag, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    st = moe.moe_sync_status(ws, s)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    gpu_index = phys[local] if len(phys) > local and phys[local] != "" else str(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_index) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    value = world * n * args.steps / (ms_total / 1e3)
+    clocks = clk.summary()
+
+    # Stage times through the staged entry points (same kernels), events on the launching stream.
+    nk = n * w.top_k
+    idx = torch.empty((n, w.top_k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((n, w.top_k), dtype=torch.float32, device="cuda")
+    offs = torch.empty(w.n_routed + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(nk, dtype=torch.int32, device="cuda")
+    dest = torch.empty((n, w.top_k), dtype=torch.int32, device="cuda")
+    xp = torch.empty((nk, w.d_model), dtype=dev["x"].dtype, device="cuda")
+    eo = torch.empty((nk, w.d_model), dtype=dev["x"].dtype, device="cuda")
+    stages = {
+        "route": lambda: moe.moe_route(cfg, n, dev["x"], weights, idx, tw, counts, diag, ws, s),
+        "permute": lambda: moe.moe_permute(cfg, n, dev["x"], idx, offs, perm, dest, xp, ws, s),
+        "expert_ffn": lambda: moe.moe_expert_ffn(cfg, n, xp, offs, weights, eo, ws, s),
+        "combine": lambda: moe.moe_combine(cfg, n, eo, dest, tw, dev["x"], weights, y, ws, s),
+    }
+    reps = max(3, min(args.steps, 20))
+    stage_ms = {}
+    for name, fn in stages.items():
+        fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        stage_ms[name] = a.elapsed_time(b) / reps
+    st = moe.moe_sync_status(ws, s)
+    if st != moe.MOE_OK:
+        raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
+    dg = dict(zip(moe.DIAG_FIELDS, diag.cpu().tolist()[:5]))
+    cnt = counts.cpu()
+    kept = int(cnt.sum())
+    active = int((cnt > 0).sum())
+    flops, bytes_ = layer_work(w, kept, active)
+
+    # End to end through the public API with host buffers: pinned x in, y out, every step.
+    x_host = dev["x"].cpu().pin_memory()
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(e2e_steps):
+        dev["x"].copy_(x_host, non_blocking=True)
+        step()
+        y_host.copy_(y, non_blocking=True)
+    b.record(stream)
+    barrier()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    bpe = dev["x"].element_size()
+
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    ffn_flops = 6.0 * kept * w.d_model * w.moe_intermediate_size
+    achieved = ffn_flops / (stage_ms["expert_ffn"] / 1e3) / 1e12
+    t_roof = max(flops / (tf_burst * 1e12), bytes_ / (hbm * 1e9))
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded counter-based generator; Irwin-Hall normals)",
+        "config": {"workload": w.name, "n_tokens": n, "d_model": w.d_model, "n_routed": w.n_routed,
+                   "top_k": w.top_k, "moe_intermediate_size": w.moe_intermediate_size, "n_shared": w.n_shared,
+                   "score_fn": w.score_fn, "cap_policy": w.cap_policy, "parallelism": f"replicas x{world}",
+                   "l2": f"inputs larger than L2: {active} experts x {3 * w.d_model * w.moe_intermediate_size * bpe / 1e6:.0f} MB of weights streamed per step"},
+        "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (grouped SwiGLU GEMM1 + down GEMM2)",
+                     "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst,
+                     "peak_kind": f"{peak_kind} bf16 burst", "frac_of_sustained": achieved / tf_sust if tf_sust else None,
+                     "flops_per_launch": ffn_flops, "traffic": _traffic("expert_ffn", w.name)},
+        "layer_roofline": {"flops": flops, "bytes": bytes_, "t_roof_ms": t_roof * 1e3,
+                           "frac": t_roof * 1e3 / ms_step, "active_experts": active, "kept_slots": kept},
+        "stages_ms": stage_ms,
+        "diag": dg,
+        "e2e": {"value": world * n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": n * w.d_model * bpe,
+                "d2h_bytes_per_step": n * w.d_model * bpe, "ms_per_step": e2e_ms},
+        "gpu_launches": launches_per_step(w) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def _oracle_inputs(w, tokens):
+    """Host inputs of the oracle's sample: the first `tokens` rows of x and all weights."""
+    from synth import workloads as W
+
+    names = ["w_r", "w_gate", "w_up", "w_down"] + (["bias"] if w.bias_range else []) + \
+        (["ws_gate", "ws_up", "ws_down"] if w.n_shared else [])
+    inp = W.host_inputs(w, names=names)
+    inp["x"] = W.host_rows(w, "x", range(tokens))
+    return inp
+
+
+def _oracle_time(w, inp, tokens):
+    """Seconds the oracle layer takes on the first `tokens` rows of the sample."""
+    from oracle import oracle as O
+
+    cfg = O.Cfg(**w.cfg_fields())
+    t0 = time.perf_counter()
+    O.layer(cfg, inp["x"][:tokens], inp["w_r"], inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("bias"),
+            inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"))
+    return time.perf_counter() - t0
+
+
+def _cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, tokens):
+    sec = _oracle_time(w, _oracle_inputs(w, tokens), tokens)
+    return {"value": tokens / sec, "unit": "tokens/s", "cores": int(os.environ.get("OMP_NUM_THREADS", _cores())),
+            "kind": "oracle",
+            "sample": f"fp64 oracle layer (routing of the sample as its own batch, experts, combine) on the first "
+                      f"{tokens} tokens of {w.name}: {sec:.1f} s"}
+
+
+def run_reference(args):
+    from synth import workloads as W
+
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    w = W.get(args.workload)
+    tokens = args.ref_sample
+    inp = _oracle_inputs(w, tokens)
+    for _ in range(args.warmup):
+        _oracle_time(w, inp, 1)
+    secs = [_oracle_time(w, inp, tokens) for _ in range(args.steps)]
+    total = sum(secs)
+    value = tokens * args.steps / total
+    cores = int(os.environ.get("OMP_NUM_THREADS", _cores()))
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / args.steps * 1e3,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic", "config": {"workload": w.name, "n_tokens_sampled_per_step": tokens},
+           "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                            "sample": f"fp64 oracle layer on {tokens} tokens of {w.name} per step (inputs generated before timing)"},
+           "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mixtral_8x7b")
+    ap.add_argument("--cpu-sample", type=int, default=16, help="tokens in the oracle's timed sample")
+    ap.add_argument("--ref-sample", type=int, default=1, help="tokens per step of the reference (oracle) arm")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("at least 3 warm-up steps")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,198 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts FFN layer,
+ * forward pass: router -> dispatch -> per-expert SwiGLU -> shared experts ->
+ * gate-weighted combine.
+ *
+ * Where each operation is defined (page title, then section):
+ *   [DS]   "15. DeepSeek: MLA, MoE and MTP" -- section "V3 MoE: how 8 of 256
+ *          experts are chosen": x @ W^T with W [E, d]; sigmoid scores; bias
+ *          (e_score_correction_bias) added for selection only; E experts viewed
+ *          as n_group groups, a group scored by the sum of its two best biased
+ *          scores, topk_group groups kept, the rest masked; top-k; gates taken
+ *          from the raw scores, divided by their sum and multiplied by
+ *          routed_scaling_factor; y = sum_k w_k expert_k(x) + shared_expert(x).
+ *          Section "V2": softmax scoring, 160 routed + 2 shared experts, top-6.
+ *          Section "671B and 37B": an expert is three matrices gate, up, down.
+ *   [MoE]  "MoE architecture revealed", section 3.1: a linear router maps x to
+ *          E logits, softmax turns them into probabilities, the top-k experts
+ *          are chosen; section 4.1: top-k of the probabilities as gates.
+ *   [1.8T] "1.8T parameters / 2% per token", section 2.2: each expert has a
+ *          capacity per batch and tokens beyond it are forced to the
+ *          next-best expert; section 4.1: gates as the softmax of the top-k
+ *          logits (renormalised); section 4.2: capacity_factor and
+ *          drop_tokens.
+ *   [KL]   "MoE" tag feed, section on activation functions: SwiGLU FFN.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named x, w_*, y, topk_*, offsets, perm_token, slot_dest,
+ *     x_perm, expert_out, expert_counts, diag and ws are DEVICE pointers
+ *     (one GPU); cfg, the moe_weights struct itself and bytes are HOST
+ *     pointers. The caller owns all memory; the library allocates nothing
+ *     and keeps no state between calls. Scratch space comes only from the
+ *     workspace ws of at least moe_workspace_size() bytes.
+ *   - Arrays are dense row-major. Weights use the out x in (nn.Linear)
+ *     convention: W_r [E, d]; w_gate, w_up [E, I, d]; w_down [E, d, I];
+ *     shared experts concatenated along I: ws_gate, ws_up [n_shared*I, d],
+ *     ws_down [d, n_shared*I]. Activations and weights share cfg->dtype
+ *     (MOE_F32 or MOE_BF16); gates are binary32; indices are int32.
+ *   - Every device pointer must be 16-byte aligned; ws must be 256-byte
+ *     aligned.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream). Results are deterministic run to run (fixed reduction
+ *     orders, no floating-point atomics).
+ *   - Argument and shape errors are returned synchronously before anything
+ *     is enqueued. A failed launch returns MOE_ERR_CUDA. Errors that only the
+ *     device can see (a bounded wait that ran out, an internal check) are
+ *     written to the status word in the workspace and are returned by
+ *     moe_sync_status(). n = 0 is a valid no-op.
+ *   - Expert order and tie rule: output slots are ordered by descending
+ *     selection score (logit for softmax, score + bias for sigmoid); equal
+ *     scores go to the lower expert index, equal group scores to the lower
+ *     group index. Dropped slots carry index -1, weight 0 and slot_dest -1.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st* moe_stream_t; /* same object as cudaStream_t */
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or field     */
+  MOE_ERR_UNSUPPORTED = 2, /* valid but outside what the kernels handle      */
+  MOE_ERR_WORKSPACE = 3,   /* ws_bytes below moe_workspace_size()            */
+  MOE_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed           */
+  MOE_ERR_TIMEOUT = 5,     /* a bounded device wait gave up                  */
+  MOE_ERR_INTERNAL = 6     /* a device-side consistency check failed         */
+} moe_status;
+
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_CAP_NONE = 0, MOE_CAP_OVERFLOW_NEXT = 1, MOE_CAP_DROP = 2 } moe_cap_policy;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+
+/* Layer configuration, in the field names of [DS] and [1.8T] 4.2. */
+typedef struct {
+  int32_t d_model;               /* d                                              */
+  int32_t n_routed;              /* E, 1..256                                      */
+  int32_t n_shared;              /* shared experts (0 = none)                      */
+  int32_t top_k;                 /* k, 1..min(E, 32)                               */
+  int32_t n_group;               /* expert groups; 1 = no group limit              */
+  int32_t topk_group;            /* groups kept per token                          */
+  int32_t moe_intermediate_size; /* I                                              */
+  int32_t score_fn;              /* moe_score_fn                                   */
+  int32_t renormalize;           /* 1: gates normalised over the kept slots        */
+  float routed_scaling_factor;   /* multiplies every gate ([DS]: 2.5 for V3)       */
+  int32_t cap_policy;            /* moe_cap_policy                                 */
+  float capacity_factor;         /* C = ceil(capacity_factor * n * k / E)          */
+  int32_t capacity;              /* > 0 overrides capacity_factor                  */
+  int32_t dtype;                 /* moe_dtype of activations and weights           */
+} moe_config;
+
+/* Caller-owned device weights. bias may be NULL (= 0); ws_* NULL when n_shared = 0. */
+typedef struct {
+  const void* w_router; /* [E, d]                */
+  const void* w_gate;   /* [E, I, d]             */
+  const void* w_up;     /* [E, I, d]             */
+  const void* w_down;   /* [E, d, I]             */
+  const void* ws_gate;  /* [n_shared*I, d]       */
+  const void* ws_up;    /* [n_shared*I, d]       */
+  const void* ws_down;  /* [d, n_shared*I]       */
+  const float* bias;    /* [E] selection bias    */
+} moe_weights;
+
+/* Device-resident diagnostics written by moe_route / moe_layer_forward. */
+typedef struct {
+  int32_t overflowed;     /* slots sent to an expert ranked below the k-th       */
+  int32_t dropped;        /* slots left empty                                     */
+  int32_t refined_tokens; /* tokens whose decision was re-taken in binary64       */
+  int32_t max_load;       /* largest per-expert slot count                        */
+  int32_t status;         /* moe_status seen on the device                        */
+  int32_t reserved[3];
+} moe_diag;
+
+/*
+ * Workspace bytes needed by any entry point for this cfg and token count n.
+ * Returns MOE_ERR_INVALID_ARG / MOE_ERR_UNSUPPORTED for a bad cfg.
+ */
+moe_status moe_workspace_size(const moe_config* cfg, int64_t n, size_t* bytes);
+
+/*
+ * Router ([DS] router; [MoE] 3.1; capacity: [1.8T] 2.2, 4.2).
+ *   in : x [n, d]; weights->w_router, weights->bias.
+ *   out: topk_idx [n, k] int32, topk_w [n, k] float, expert_counts [E] int32
+ *        (slots per expert after capacity; may be NULL), diag (may be NULL).
+ * Logits are accumulated in binary32 on tensor cores; a token whose decision
+ * (group cut, k-th/(k+1)-th expert, order of the kept experts, and under a
+ * capacity every rank cut) is closer than the binary32 error bound is
+ * re-decided from binary64 logits, so indices equal the binary64 definition.
+ */
+moe_status moe_route(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
+                     int32_t* topk_idx, float* topk_w, int32_t* expert_counts, moe_diag* diag,
+                     void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Dispatch: per-expert histogram, exclusive scan and stable permutation
+ * (token order within an expert), plus the row gather.
+ *   in : x [n, d], topk_idx [n, k] (-1 = dropped).
+ *   out: offsets [E + 1] (offsets[E] = kept slots), perm_token [n * k]
+ *        (first offsets[E] entries valid: source token of each permuted row),
+ *        slot_dest [n, k] (permuted row of each slot, -1 if dropped),
+ *        x_perm [n * k, d] (first offsets[E] rows valid).
+ */
+moe_status moe_permute(const moe_config* cfg, int64_t n, const void* x, const int32_t* topk_idx,
+                       int32_t* offsets, int32_t* perm_token, int32_t* slot_dest, void* x_perm,
+                       void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Routed experts ([DS] three matrices; [KL] SwiGLU): for every expert e and
+ * every permuted row r in [offsets[e], offsets[e+1]):
+ *   expert_out[r] = (silu(x_perm[r] W_gate[e]^T) * (x_perm[r] W_up[e]^T)) W_down[e]^T
+ * with silu(z) = z * sigmoid(z), binary32 accumulation, the intermediate
+ * rounded to cfg->dtype. n bounds the rows: offsets[E] <= n * k.
+ */
+moe_status moe_expert_ffn(const moe_config* cfg, int64_t n, const void* x_perm, const int32_t* offsets,
+                          const moe_weights* weights, void* expert_out, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * Combine ([DS] last line of the router listing):
+ *   y[t] = sum_{j<k, slot kept} topk_w[t, j] * expert_out[slot_dest[t, j]] + shared(x[t])
+ * summed in binary32 in slot order, the shared experts' SwiGLU (computed here
+ * from x and weights->ws_*) added last with weight 1. y [n, d].
+ */
+moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out, const int32_t* slot_dest,
+                       const float* topk_w, const void* x, const moe_weights* weights, void* y, void* ws,
+                       size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Whole layer: moe_route -> moe_permute -> moe_expert_ffn -> moe_combine with
+ * all intermediates in the workspace. y [n, d]. topk_idx_opt, topk_w_opt,
+ * counts_opt and diag_opt may be NULL; when given they receive the routing.
+ */
+moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
+                             void* y, int32_t* topk_idx_opt, float* topk_w_opt, int32_t* counts_opt,
+                             moe_diag* diag_opt, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Synchronises `stream`, then returns the device status word kept in the
+ * workspace (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_INTERNAL) and clears it. Every
+ * entry point clears the word when it starts, so it reports the most recent
+ * call made on this workspace.
+ */
+moe_status moe_sync_status(void* ws, moe_stream_t stream);
+
+/* Static text for a status code. */
+const char* moe_status_string(moe_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_H_ */

@@ -1,0 +1,199 @@
+"""Parity of the CUDA path (called through the C ABI) with the fp64 CPU oracle.
+
+Indices, permutations and counts must be bit-exact, except for tokens the
+oracle marks exempt (a decision boundary closer than 1e-6 relative); the
+tie-stress workloads have exact integer logits and must match on every token.
+Layer outputs must satisfy max_i |y_i - r_i| / max(|r_i|, rms(r)) <= 2e-2 (bf16)
+or 1e-4 (fp32).
+"""
+import numpy as np
+import pytest
+import torch
+
+import top_routing_expert_router_b200 as moe
+from oracle import oracle as O
+from synth import synth, workloads as W
+from tests import moe_harness as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "deepseek_v3_decode_small",
+         "skewed_small", "drop_small", "tie_softmax", "tie_sigmoid"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def _oracle_route(w, host):
+    lg = O.router_logits(host["x"], host["w_r"])
+    return O.route_capacity(H.oracle_cfg(w), lg, host.get("bias"))
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v3_small", "tiny_f32", "skewed_small"])
+def test_device_inputs_equal_host_inputs(name):
+    w = W.get(name)
+    dev = W.device_inputs(w)
+    host = W.host_inputs(w)
+    for k in host:
+        assert (H.to_np(dev[k]) == host[k]).all(), k
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_route_parity(name):
+    w = W.get(name)
+    dev, host = W.device_inputs(w), W.host_inputs(w)
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, w.n)
+    idx = torch.empty((w.n, w.top_k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((w.n, w.top_k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(w.n_routed, dtype=torch.int32, device="cuda")
+    dg = torch.zeros(8, dtype=torch.int32, device="cuda")
+    moe.moe_route(cfg, w.n, dev["x"], H.weights_for(dev), idx, tw, counts, dg, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    oi, ow, ex, st = _oracle_route(w, host)
+    gi, gw = idx.cpu().numpy(), tw.cpu().numpy()
+    diag = H.diag_dict(dg)
+    if w.ternary:
+        ex = np.zeros_like(ex)  # exact integer logits: every token must match, ties included
+        assert diag["refined_tokens"] > 0
+    if w.cap_policy != "none":
+        # a near-tie can cascade through the capacity counts: compare up to the first exempt token
+        stop = int(np.argmax(ex)) if ex.any() else w.n
+        np.testing.assert_array_equal(gi[:stop], oi[:stop])
+        if stop == w.n:
+            assert diag["overflowed"] == st.overflowed and diag["dropped"] == st.dropped
+        keep = np.arange(w.n) < stop
+    else:
+        keep = ~ex
+        np.testing.assert_array_equal(gi[keep], oi[keep])
+    np.testing.assert_allclose(gw[keep], ow[keep], rtol=2e-4, atol=1e-6)
+    if keep.all():
+        np.testing.assert_array_equal(counts.cpu().numpy(), np.bincount(oi[oi >= 0], minlength=w.n_routed))
+        assert diag["max_load"] == np.bincount(oi[oi >= 0], minlength=w.n_routed).max()
+    assert ex.mean() < 0.05
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "skewed_small", "drop_small", "tiny_f32"])
+def test_permute_parity(name):
+    w = W.get(name)
+    host = W.host_inputs(w, names=["x", "w_r", "bias"] if w.bias_range else ["x", "w_r"])
+    oi, _, _, _ = _oracle_route(w, host)
+    counts, offsets, perm, dest = O.dispatch(oi, w.n_routed)
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, w.n)
+    x = W.device_inputs(w, names=["x"])["x"]
+    nk = w.n * w.top_k
+    g_off = torch.empty(w.n_routed + 1, dtype=torch.int32, device="cuda")
+    g_perm = torch.full((nk,), -7, dtype=torch.int32, device="cuda")
+    g_dest = torch.empty((w.n, w.top_k), dtype=torch.int32, device="cuda")
+    g_xp = torch.empty((nk, w.d_model), dtype=x.dtype, device="cuda")
+    moe.moe_permute(cfg, w.n, x, torch.from_numpy(oi).cuda(), g_off, g_perm, g_dest, g_xp, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    np.testing.assert_array_equal(g_off.cpu().numpy(), offsets)
+    kept = int(offsets[-1])
+    np.testing.assert_array_equal(g_perm.cpu().numpy()[:kept], perm)
+    np.testing.assert_array_equal(g_dest.cpu().numpy(), dest)
+    assert (H.to_np(g_xp[:kept]) == host["x"][perm]).all()
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small",
+                                  "deepseek_v3_decode_small", "skewed_small"])
+def test_expert_ffn_parity(name):
+    w = W.get(name)
+    host = W.host_inputs(w)
+    dev = W.device_inputs(w)
+    oi, _, _, _ = _oracle_route(w, host)
+    counts, offsets, perm, dest = O.dispatch(oi, w.n_routed)
+    xp_host = host["x"][perm]
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, w.n)
+    xp = torch.from_numpy(xp_host.view(np.int16) if xp_host.dtype == np.uint16 else xp_host).cuda()
+    if w.dtype == "bf16":
+        xp = xp.view(torch.bfloat16)
+    eo = torch.empty((w.n * w.top_k, w.d_model), dtype=xp.dtype, device="cuda")
+    moe.moe_expert_ffn(cfg, w.n, xp, torch.from_numpy(offsets).cuda(), H.weights_for(dev), eo, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    got = H.as_f64(eo[: offsets[-1]])
+    x64 = O.bf16_to_f64(xp_host)
+    ref = np.zeros_like(got)
+    for e in range(w.n_routed):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            ref[lo:hi] = O.swiglu(x64[lo:hi], host["w_gate"][e], host["w_up"][e], host["w_down"][e])
+    assert H.rel_err(got, ref) <= H.TOL[w.dtype]
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "deepseek_v2_small", "deepseek_v3_small"])
+def test_combine_parity(name):
+    w = W.get(name)
+    host = W.host_inputs(w)
+    dev = W.device_inputs(w)
+    oi, ow, _, _ = _oracle_route(w, host)
+    counts, offsets, perm, dest = O.dispatch(oi, w.n_routed)
+    rows = int(offsets[-1])
+    # synthetic expert outputs in the layer's dtype
+    eo_host = synth.host((rows, w.d_model), w.dtype, 0, 77, synth.NORMAL, 1.0)
+    eo = torch.from_numpy(eo_host.view(np.int16) if w.dtype == "bf16" else eo_host).cuda()
+    if w.dtype == "bf16":
+        eo = eo.view(torch.bfloat16)
+    tw32 = ow.astype(np.float32)
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, w.n)
+    y = torch.empty((w.n, w.d_model), dtype=eo.dtype, device="cuda")
+    moe.moe_combine(cfg, w.n, eo, torch.from_numpy(dest).cuda(), torch.from_numpy(tw32).cuda(), dev["x"],
+                    H.weights_for(dev), y, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    sh = None
+    if w.n_shared:
+        sh = O.swiglu(O.bf16_to_f64(host["x"]), host["ws_gate"], host["ws_up"], host["ws_down"])
+    ref = O.combine(O.bf16_to_f64(eo_host), dest, tw32.astype(np.float64), sh)
+    assert H.rel_err(H.as_f64(y), ref) <= H.TOL[w.dtype]
+
+
+@pytest.mark.parametrize("name", SMALL)
+def test_layer_parity(name):
+    w = W.get(name)
+    dev, host = W.device_inputs(w), W.host_inputs(w)
+    got = H.run_layer(w, dev)
+    r = O.layer(H.oracle_cfg(w), host["x"], host["w_r"], host["w_gate"], host["w_up"], host["w_down"],
+                host.get("bias"), host.get("ws_gate"), host.get("ws_up"), host.get("ws_down"))
+    gi = got["topk_idx"].cpu().numpy()
+    ex = r["exempt"] if not w.ternary else np.zeros(w.n, bool)
+    if w.cap_policy != "none" and ex.any():
+        keep = np.arange(w.n) < int(np.argmax(ex))
+    else:
+        keep = ~ex
+    np.testing.assert_array_equal(gi[keep], r["topk_idx"][keep])
+    y = H.as_f64(got["y"])
+    assert H.rel_err(y[keep], r["y"][keep]) <= H.TOL[w.dtype]
+
+
+def test_layer_is_deterministic():
+    w = W.get("deepseek_v3_small")
+    dev = W.device_inputs(w)
+    a = H.run_layer(w, dev)["y"].clone()
+    b = H.run_layer(w, dev)["y"]
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_zero_tokens_is_a_noop():
+    w = W.get("mixtral_small")
+    dev = W.device_inputs(w)
+    got = H.run_layer(w, dev, n=0)
+    assert got["counts"].sum().item() == 0
+
+
+def test_single_token_and_ragged_sizes():
+    w = W.get("deepseek_v3_small")
+    dev, host = W.device_inputs(w), W.host_inputs(w)
+    for n in (1, 3, 129):
+        got = H.run_layer(w, {k: (v[:n] if k == "x" else v) for k, v in dev.items()}, n=n)
+        r = O.layer(H.oracle_cfg(w), host["x"][:n], host["w_r"], host["w_gate"], host["w_up"], host["w_down"],
+                    host.get("bias"), host.get("ws_gate"), host.get("ws_up"), host.get("ws_down"))
+        keep = ~r["exempt"]
+        np.testing.assert_array_equal(got["topk_idx"].cpu().numpy()[keep], r["topk_idx"][keep])
+        assert H.rel_err(H.as_f64(got["y"])[keep], r["y"][keep]) <= H.TOL[w.dtype]

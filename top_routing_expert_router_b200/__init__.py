@@ -1,0 +1,157 @@
+"""Python binding of the B200 sparse-MoE FFN layer library (``libmoe_b200.so``).
+
+Argument marshalling only: every function forwards device pointers, sizes and
+the current CUDA stream to the C entry point of the same name declared in
+``include/moe.h``. All computation runs in the library's CUDA kernels. Importing
+this module fails loudly when the library has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m top_routing_expert_router_b200.build` "
+                      "(or __graft_entry__.build()); there is no fallback implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
+    MOE_ERR_INTERNAL = range(7)
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+MOE_CAP_NONE, MOE_CAP_OVERFLOW_NEXT, MOE_CAP_DROP = 0, 1, 2
+MOE_F32, MOE_BF16 = 0, 1
+
+# Every symbol declared in include/moe.h.
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
+           "moe_layer_forward", "moe_sync_status", "moe_status_string")
+
+
+class moe_config(ctypes.Structure):
+    _fields_ = [
+        ("d_model", ctypes.c_int32), ("n_routed", ctypes.c_int32), ("n_shared", ctypes.c_int32),
+        ("top_k", ctypes.c_int32), ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32),
+        ("moe_intermediate_size", ctypes.c_int32), ("score_fn", ctypes.c_int32),
+        ("renormalize", ctypes.c_int32), ("routed_scaling_factor", ctypes.c_float),
+        ("cap_policy", ctypes.c_int32), ("capacity_factor", ctypes.c_float), ("capacity", ctypes.c_int32),
+        ("dtype", ctypes.c_int32),
+    ]
+
+
+class moe_weights(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_void_p) for n in
+                ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "bias")]
+
+
+class moe_diag(ctypes.Structure):
+    _fields_ = [("overflowed", ctypes.c_int32), ("dropped", ctypes.c_int32), ("refined_tokens", ctypes.c_int32),
+                ("max_load", ctypes.c_int32), ("status", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
+DIAG_FIELDS = ("overflowed", "dropped", "refined_tokens", "max_load", "status")
+
+_P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+_lib.moe_workspace_size.argtypes = [_P, _I64, ctypes.POINTER(ctypes.c_size_t)]
+_lib.moe_route.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_permute.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_expert_ffn.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_combine.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_layer_forward.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_sync_status.argtypes = [_P, _P]
+_lib.moe_status_string.argtypes = [ctypes.c_int]
+_lib.moe_status_string.restype = ctypes.c_char_p
+for _name in EXPORTS[:-1]:
+    getattr(_lib, _name).restype = ctypes.c_int
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {moe_status_string(status)} (status {status})")
+        self.status = status
+
+
+def moe_status_string(status: int) -> str:
+    return _lib.moe_status_string(status).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != MOE_OK:
+        raise MoeError(status, where)
+
+
+def make_config(d_model, n_routed, top_k, moe_intermediate_size, n_shared=0, n_group=1, topk_group=1,
+                score_fn="softmax", renormalize=False, routed_scaling_factor=1.0, cap_policy="none",
+                capacity_factor=0.0, capacity=0, dtype="bf16") -> moe_config:
+    """A moe_config from the pages' field names (strings for the enums)."""
+    return moe_config(
+        d_model, n_routed, n_shared, top_k, n_group, topk_group, moe_intermediate_size,
+        {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score_fn], int(bool(renormalize)),
+        float(routed_scaling_factor),
+        {"none": MOE_CAP_NONE, "overflow_next": MOE_CAP_OVERFLOW_NEXT, "drop": MOE_CAP_DROP}[cap_policy],
+        float(capacity_factor), int(capacity), {"f32": MOE_F32, "bf16": MOE_BF16}[dtype])
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(stream):
+    if stream is not None:
+        return stream
+    import torch
+
+    return torch.cuda.current_stream().cuda_stream
+
+
+def make_weights(w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None, bias=None) -> moe_weights:
+    """moe_weights from device tensors (the tensors must outlive every call that uses the struct)."""
+    return moe_weights(*(_ptr(t) for t in (w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, bias)))
+
+
+def moe_workspace_size(cfg: moe_config, n: int) -> int:
+    out = ctypes.c_size_t()
+    _check(_lib.moe_workspace_size(ctypes.byref(cfg), n, ctypes.byref(out)), "moe_workspace_size")
+    return out.value
+
+
+def moe_route(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, ws, stream=None):
+    _check(_lib.moe_route(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(topk_idx), _ptr(topk_w),
+                          _ptr(expert_counts), _ptr(diag), _ptr(ws), ws.numel() * ws.element_size(),
+                          _stream(stream)), "moe_route")
+
+
+def moe_permute(cfg, n, x, topk_idx, offsets, perm_token, slot_dest, x_perm, ws, stream=None):
+    _check(_lib.moe_permute(ctypes.byref(cfg), n, _ptr(x), _ptr(topk_idx), _ptr(offsets), _ptr(perm_token),
+                            _ptr(slot_dest), _ptr(x_perm), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream)), "moe_permute")
+
+
+def moe_expert_ffn(cfg, n, x_perm, offsets, weights, expert_out, ws, stream=None):
+    _check(_lib.moe_expert_ffn(ctypes.byref(cfg), n, _ptr(x_perm), _ptr(offsets), ctypes.byref(weights),
+                               _ptr(expert_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "moe_expert_ffn")
+
+
+def moe_combine(cfg, n, expert_out, slot_dest, topk_w, x, weights, y, ws, stream=None):
+    _check(_lib.moe_combine(ctypes.byref(cfg), n, _ptr(expert_out), _ptr(slot_dest), _ptr(topk_w), _ptr(x),
+                            ctypes.byref(weights), _ptr(y), _ptr(ws), ws.numel() * ws.element_size(),
+                            _stream(stream)), "moe_combine")
+
+
+def moe_layer_forward(cfg, n, x, weights, y, ws, topk_idx=None, topk_w=None, counts=None, diag=None, stream=None):
+    _check(_lib.moe_layer_forward(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(y), _ptr(topk_idx),
+                                  _ptr(topk_w), _ptr(counts), _ptr(diag), _ptr(ws), ws.numel() * ws.element_size(),
+                                  _stream(stream)), "moe_layer_forward")
+
+
+def moe_sync_status(ws, stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word of the workspace."""
+    return _lib.moe_sync_status(_ptr(ws), _stream(stream))
+
+
+def lib_handle():
+    return _lib

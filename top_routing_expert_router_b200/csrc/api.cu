@@ -1,0 +1,334 @@
+// api.cu -- the C ABI entry points declared in moe.h: argument checks,
+// workspace carving and the launch sequence of each stage on the caller's
+// stream. No allocation, no host synchronisation (except moe_sync_status).
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Workspace layout; every region starts on a 256-byte boundary.
+struct Plan {
+  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, total;
+};
+
+Plan make_plan(const moe_config& c, int64_t n) {
+  const size_t b = c.dtype == MOE_BF16 ? 2 : 4;
+  const int64_t nk = n * c.top_k;
+  const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size;
+  Plan p{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += (size_t)align_up((int64_t)(bytes > 0 ? bytes : 1), 256);
+    return at;
+  };
+  p.diag = take(sizeof(moe_diag));
+  p.logits = take((size_t)n * c.n_routed * 4);
+  p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
+  p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
+  p.idx = take((size_t)nk * 4);
+  p.w = take((size_t)nk * 4);
+  p.counts = take((size_t)c.n_routed * 4);
+  p.offsets = take((size_t)(c.n_routed + 1) * 4);
+  p.perm = take((size_t)nk * 4);
+  p.dest = take((size_t)nk * 4);
+  p.xperm = take((size_t)nk * c.d_model * b);
+  p.h = take((size_t)nk * c.moe_intermediate_size * b);
+  p.eo = take((size_t)nk * c.d_model * b);
+  p.shh = take((size_t)(Is > 0 ? n * Is : 0) * b);
+  p.sh = take((size_t)(Is > 0 ? n * c.d_model : 0) * b);
+  p.shoff = take(2 * 4);
+  p.total = off;
+  return p;
+}
+
+moe_status check_cfg(const moe_config* c, int64_t n) {
+  if (!c || n < 0) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->cap_policy < MOE_CAP_NONE || c->cap_policy > MOE_CAP_DROP) return MOE_ERR_INVALID_ARG;
+  if (c->d_model <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->moe_intermediate_size <= 0 || c->n_shared < 0 ||
+      c->n_group <= 0 || c->topk_group <= 0)
+    return MOE_ERR_INVALID_ARG;
+  if (c->top_k > c->n_routed || c->topk_group > c->n_group || c->n_routed % c->n_group != 0)
+    return MOE_ERR_INVALID_ARG;
+  if ((int64_t)c->topk_group * (c->n_routed / c->n_group) < c->top_k) return MOE_ERR_INVALID_ARG;
+  if (c->cap_policy != MOE_CAP_NONE && c->capacity <= 0 && !(c->capacity_factor > 0.0f)) return MOE_ERR_INVALID_ARG;
+  if (!isfinite(c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
+  if (c->n_routed > kMaxExperts || c->top_k > kMaxTopK || c->n_group > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  if (c->n_group > 1 && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_UNSUPPORTED;
+  if (c->d_model % 8 != 0 || c->moe_intermediate_size % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (n * c->top_k >= (int64_t)1 << 31 || n * (int64_t)c->n_routed >= (int64_t)1 << 40) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+int64_t capacity_of(const moe_config& c, int64_t n) {
+  if (c.capacity > 0) return c.capacity;
+  return (int64_t)ceil((double)c.capacity_factor * (double)n * (double)c.top_k / (double)c.n_routed);
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                         \
+  do {                                        \
+    const moe_status st_ = (expr);            \
+    if (st_ != MOE_OK) return st_;            \
+  } while (0)
+#define MOE_CUDA(expr) MOE_TRY(cuda_status(expr))
+
+struct Ctx {
+  moe_config c;
+  int64_t n;
+  Plan p;
+  char* ws;
+  cudaStream_t s;
+  template <typename T>
+  T* at(size_t off) const {
+    return reinterpret_cast<T*>(ws + off);
+  }
+  moe_diag* status() const { return at<moe_diag>(p.diag); }
+};
+
+moe_status begin(const moe_config* cfg, int64_t n, void* ws, size_t ws_bytes, moe_stream_t stream, Ctx* ctx) {
+  MOE_TRY(check_cfg(cfg, n));
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  ctx->c = *cfg;
+  ctx->n = n;
+  ctx->p = make_plan(*cfg, n);
+  if (ws_bytes < ctx->p.total) return MOE_ERR_WORKSPACE;
+  ctx->ws = static_cast<char*>(ws);
+  ctx->s = reinterpret_cast<cudaStream_t>(stream);
+  return MOE_OK;
+}
+
+// First enqueued work of every entry point, after all argument checks: the
+// status word reports the most recent entry point on this workspace.
+moe_status clear_status(const Ctx& ctx) {
+  return cuda_status(cudaMemsetAsync(&ctx.status()->status, 0, sizeof(int32_t), ctx.s));
+}
+
+bool ptr_ok(const void* p) { return p && aligned(p, 16); }
+
+moe_status check_weights(const moe_config& c, const moe_weights* w, bool routed, bool shared) {
+  if (!w) return MOE_ERR_INVALID_ARG;
+  if (routed && (!ptr_ok(w->w_gate) || !ptr_ok(w->w_up) || !ptr_ok(w->w_down))) return MOE_ERR_INVALID_ARG;
+  if (shared && c.n_shared > 0 && (!ptr_ok(w->ws_gate) || !ptr_ok(w->ws_up) || !ptr_ok(w->ws_down)))
+    return MOE_ERR_INVALID_ARG;
+  if (w->bias && !aligned(w->bias, 4)) return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Grouped GEMM dispatch: tcgen05 tensor cores for bf16 where the shape allows,
+// the CUDA-core kernel otherwise (binary32 layers).
+moe_status gemm(const Ctx& x, const GemmArgs& a, bool swiglu, bool out_f32) {
+  if (x.c.dtype == MOE_BF16 && gemm_tc_supported(a, swiglu, out_f32))
+    return cuda_status(launch_gemm_tc(a, swiglu, out_f32, x.status(), x.s));
+  return cuda_status(launch_gemm_simt(a, x.c.dtype, out_f32, swiglu, x.s));
+}
+
+moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, int32_t* counts,
+                      moe_diag* diag) {
+  const moe_config& c = x.c;
+  float* logits = x.at<float>(x.p.logits);
+  moe_diag* d = diag ? diag : x.status();
+  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), x.s));  // counters, not the status word
+  if (x.n == 0) return MOE_OK;
+  GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model};
+  MOE_TRY(gemm(x, g, false, true));
+  RouteArgs r{};
+  r.logits = logits;
+  r.x = X;
+  r.w_r = w->w_router;
+  r.bias = c.score_fn == MOE_SCORE_SIGMOID ? w->bias : nullptr;
+  r.dtype = c.dtype;
+  r.d = c.d_model;
+  r.n = x.n;
+  r.E = c.n_routed;
+  r.k = c.top_k;
+  r.G = c.n_group;
+  r.topk_group = c.topk_group;
+  r.score_fn = c.score_fn;
+  r.renorm = c.renormalize;
+  r.rsf = c.routed_scaling_factor;
+  r.topk_idx = idx;
+  r.topk_w = tw;
+  r.diag = d;
+  if (c.cap_policy == MOE_CAP_NONE) {
+    r.ranking = nullptr;
+    MOE_CUDA(launch_route(r, x.s));
+  } else {
+    r.ranking = x.at<uint16_t>(x.p.ranking);
+    MOE_CUDA(launch_route(r, x.s));
+    MOE_CUDA(launch_capacity(r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, x.s));
+    MOE_CUDA(launch_gates(r, x.s));
+  }
+  // per-expert slot counts and the largest load (histogram + scan, no scatter)
+  MOE_CUDA(launch_dispatch(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), counts,
+                           x.at<int32_t>(x.p.offsets), nullptr, nullptr, false, d, x.s));
+  return MOE_OK;
+}
+
+moe_status permute_impl(const Ctx& x, const void* X, const int32_t* idx, int32_t* offsets, int32_t* perm,
+                        int32_t* dest, void* xperm) {
+  const moe_config& c = x.c;
+  if (x.n == 0) {
+    MOE_CUDA(launch_fill_i32(offsets, c.n_routed + 1, 0, x.s));
+    return MOE_OK;
+  }
+  MOE_CUDA(launch_dispatch(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), nullptr, offsets, perm, dest,
+                           true, nullptr, x.s));
+  const int64_t row_bytes = (int64_t)c.d_model * (c.dtype == MOE_BF16 ? 2 : 4);
+  MOE_CUDA(launch_gather(X, perm, offsets, c.n_routed, x.n * c.top_k, row_bytes, xperm, x.s));
+  return MOE_OK;
+}
+
+moe_status ffn_impl(const Ctx& x, const void* xperm, const int32_t* offsets, const moe_weights* w, void* eo) {
+  const moe_config& c = x.c;
+  if (x.n == 0) return MOE_OK;
+  const int64_t I = c.moe_intermediate_size, d = c.d_model, nk = x.n * c.top_k;
+  void* h = x.ws + x.p.h;
+  GemmArgs g1{xperm, d, w->w_gate, w->w_up, I * d, h, I, offsets, c.n_routed, nk, (int32_t)I, (int32_t)d};
+  MOE_TRY(gemm(x, g1, true, false));
+  GemmArgs g2{h, I, w->w_down, nullptr, d * I, eo, d, offsets, c.n_routed, nk, (int32_t)d, (int32_t)I};
+  MOE_TRY(gemm(x, g2, false, false));
+  return MOE_OK;
+}
+
+moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void** sh_out) {
+  const moe_config& c = x.c;
+  *sh_out = nullptr;
+  if (c.n_shared == 0 || x.n == 0) return MOE_OK;
+  const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size, d = c.d_model;
+  void* shh = x.ws + x.p.shh;
+  void* sh = x.ws + x.p.sh;
+  GemmArgs g1{X, d, w->ws_gate, w->ws_up, 0, shh, Is, nullptr, 1, x.n, (int32_t)Is, (int32_t)d};
+  MOE_TRY(gemm(x, g1, true, false));
+  GemmArgs g2{shh, Is, w->ws_down, nullptr, 0, sh, d, nullptr, 1, x.n, (int32_t)d, (int32_t)Is};
+  MOE_TRY(gemm(x, g2, false, false));
+  *sh_out = sh;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+moe_status moe_workspace_size(const moe_config* cfg, int64_t n, size_t* bytes) {
+  MOE_TRY(check_cfg(cfg, n));
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = make_plan(*cfg, n).total;
+  return MOE_OK;
+}
+
+moe_status moe_route(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
+                     int32_t* topk_idx, float* topk_w, int32_t* expert_counts, moe_diag* diag, void* ws,
+                     size_t ws_bytes, moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (!weights || !ptr_ok(weights->w_router) || !ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(topk_w))
+    return MOE_ERR_INVALID_ARG;
+  if ((expert_counts && !aligned(expert_counts, 4)) || (diag && !aligned(diag, 16))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, false, false));
+  MOE_TRY(clear_status(c));
+  return route_impl(c, x, weights, topk_idx, topk_w, expert_counts, diag);
+}
+
+moe_status moe_permute(const moe_config* cfg, int64_t n, const void* x, const int32_t* topk_idx, int32_t* offsets,
+                       int32_t* perm_token, int32_t* slot_dest, void* x_perm, void* ws, size_t ws_bytes,
+                       moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (!ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(offsets) || !ptr_ok(perm_token) || !ptr_ok(slot_dest) ||
+      !ptr_ok(x_perm))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(clear_status(c));
+  return permute_impl(c, x, topk_idx, offsets, perm_token, slot_dest, x_perm);
+}
+
+moe_status moe_expert_ffn(const moe_config* cfg, int64_t n, const void* x_perm, const int32_t* offsets,
+                          const moe_weights* weights, void* expert_out, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (!ptr_ok(x_perm) || !ptr_ok(offsets) || !ptr_ok(expert_out)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, true, false));
+  MOE_TRY(clear_status(c));
+  return ffn_impl(c, x_perm, offsets, weights, expert_out);
+}
+
+moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out, const int32_t* slot_dest,
+                       const float* topk_w, const void* x, const moe_weights* weights, void* y, void* ws,
+                       size_t ws_bytes, moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (!ptr_ok(expert_out) || !ptr_ok(slot_dest) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
+  if (c.c.n_shared > 0 && !ptr_ok(x)) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, false, true));
+  MOE_TRY(clear_status(c));
+  void* sh = nullptr;
+  MOE_TRY(shared_impl(c, x, weights, &sh));
+  return cuda_status(launch_combine(expert_out, slot_dest, topk_w, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
+}
+
+moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights, void* y,
+                             int32_t* topk_idx_opt, float* topk_w_opt, int32_t* counts_opt, moe_diag* diag_opt,
+                             void* ws, size_t ws_bytes, moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (!ptr_ok(x) || !ptr_ok(y) || !weights || !ptr_ok(weights->w_router)) return MOE_ERR_INVALID_ARG;
+  if ((topk_idx_opt && !ptr_ok(topk_idx_opt)) || (topk_w_opt && !ptr_ok(topk_w_opt)) ||
+      (counts_opt && !aligned(counts_opt, 4)) || (diag_opt && !aligned(diag_opt, 16)))
+    return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, true, true));
+  MOE_TRY(clear_status(c));
+  int32_t* idx = topk_idx_opt ? topk_idx_opt : c.at<int32_t>(c.p.idx);
+  float* tw = topk_w_opt ? topk_w_opt : c.at<float>(c.p.w);
+  int32_t* counts = counts_opt ? counts_opt : c.at<int32_t>(c.p.counts);
+  int32_t* offsets = c.at<int32_t>(c.p.offsets);
+  int32_t* perm = c.at<int32_t>(c.p.perm);
+  int32_t* dest = c.at<int32_t>(c.p.dest);
+  void* xperm = c.ws + c.p.xperm;
+  void* eo = c.ws + c.p.eo;
+  MOE_TRY(route_impl(c, x, weights, idx, tw, counts, diag_opt));
+  if (n == 0) return MOE_OK;
+  MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm));
+  MOE_TRY(ffn_impl(c, xperm, offsets, weights, eo));
+  void* sh = nullptr;
+  MOE_TRY(shared_impl(c, x, weights, &sh));
+  return cuda_status(launch_combine(eo, dest, tw, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
+}
+
+moe_status moe_sync_status(void* ws, moe_stream_t stream) {
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  moe_diag* d = reinterpret_cast<moe_diag*>(ws);  // the diag region is first in the workspace
+  int32_t code = 0;
+  if (cudaMemcpy(&code, &d->status, sizeof(code), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (code != 0 && cudaMemset(&d->status, 0, sizeof(code)) != cudaSuccess) return MOE_ERR_CUDA;
+  return (moe_status)code;
+}
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_INTERNAL: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// kernels.h -- internal launch interface between the host entry points and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Grouped GEMM problem. Rows of group g are [offsets[g], offsets[g+1]) of A and
+// C (offsets == nullptr: one group of M rows). B holds G consecutive [N, K]
+// matrices (out x in) b_group_stride elements apart; B2 likewise (SwiGLU up).
+struct GemmArgs {
+  const void* A;
+  int64_t lda;
+  const void* B;
+  const void* B2;
+  int64_t b_group_stride;
+  void* C;
+  int64_t ldc;
+  const int32_t* offsets;
+  int32_t G;
+  int64_t M;  // upper bound on the total rows (exact when offsets == nullptr)
+  int32_t N;
+  int32_t K;
+};
+
+cudaError_t launch_gemm_simt(const GemmArgs& a, int dtype, bool out_f32, bool swiglu, cudaStream_t s);
+
+// tcgen05 grouped GEMM (bf16 in, fp32 accumulate in TMEM). Returns
+// cudaErrorNotSupported when the shape is outside what it handles.
+cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_diag* status, cudaStream_t s);
+bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32);
+
+// Router: scoring, group limit, top-k, certification / binary64 refinement, gates.
+struct RouteArgs {
+  const float* logits;  // [n, E]
+  const void* x;        // [n, d] for the binary64 refinement
+  const void* w_r;      // [E, d]
+  const float* bias;    // [E] or nullptr
+  int dtype;
+  int32_t d;
+  int64_t n;
+  int32_t E, k, G, topk_group, score_fn, renorm;
+  float rsf;
+  uint16_t* ranking;    // [n, E] eligible experts in selection order (capacity), or nullptr
+  int32_t* topk_idx;    // [n, k] (written when ranking == nullptr)
+  float* topk_w;        // [n, k]
+  moe_diag* diag;       // refined_tokens counter
+};
+cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+
+// Capacity rule over the ranking; writes topk_idx and the overflow/drop counts.
+cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32_t k, int64_t C, int policy,
+                            int32_t* topk_idx, moe_diag* diag, cudaStream_t s);
+// Gates of a given selection from the logits.
+cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s);
+
+// Dispatch.
+int64_t dispatch_blocks(int64_t n, int32_t k);
+cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, int32_t* blk_counts,
+                            int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* slot_dest,
+                            bool scatter, moe_diag* diag, cudaStream_t s);
+cudaError_t launch_gather(const void* x, const int32_t* perm_token, const int32_t* offsets, int32_t E,
+                          int64_t max_rows, int64_t row_bytes, void* x_perm, cudaStream_t s);
+
+// Combine.
+cudaError_t launch_combine(const void* eo, const int32_t* slot_dest, const float* topk_w, const void* sh,
+                           int64_t n, int32_t k, int32_t d, int dtype, void* y, cudaStream_t s);
+
+// Small utilities.
+cudaError_t launch_fill_i32(int32_t* p, int64_t count, int32_t value, cudaStream_t s);
+cudaError_t launch_set_offsets2(int32_t* p, int64_t n, cudaStream_t s);
+
+}  // namespace moe
