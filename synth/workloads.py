@@ -115,6 +115,8 @@ WORKLOADS = {w.name: w for w in [
         cap_policy="overflow_next", capacity_factor=1.25, zipf_s=1.2),
     _wl("drop_small", n=1000, d_model=128, n_routed=16, top_k=2, moe_intermediate_size=64,
         cap_policy="drop", capacity_factor=1.0, zipf_s=1.2),
+    _wl("ragged_small", n=77, d_model=200, n_routed=5, top_k=2, moe_intermediate_size=72, renormalize=True,
+        n_shared=1),
     _wl("tie_softmax", n=256, d_model=64, n_routed=16, top_k=4, moe_intermediate_size=64,
         ternary=True, renormalize=True),
     _wl("tie_sigmoid", n=256, d_model=64, n_routed=32, top_k=4, moe_intermediate_size=64,

@@ -45,10 +45,19 @@ def as_f64(t) -> np.ndarray:
 
 
 def rel_err(y: np.ndarray, r: np.ndarray) -> float:
-    """max_i |y_i - r_i| / max(|r_i|, rms(r))."""
-    rms = float(np.sqrt(np.mean(r * r))) if r.size else 1.0
-    den = np.maximum(np.abs(r), rms if rms > 0 else 1.0)
-    return float(np.max(np.abs(y - r) / den)) if r.size else 0.0
+    """max over elements of |y - r| / max(|r|, rms of r over the same token's row).
+
+    "Max relative error" is undefined where r ~ 0; the floor is the token's own
+    output scale (the row rms), so that tokens with small gates (e.g. capacity
+    overflow onto low-probability experts) are judged against their own size.
+    """
+    if not r.size:
+        return 0.0
+    r2 = r.reshape(-1, r.shape[-1]) if r.ndim > 1 else r.reshape(1, -1)
+    y2 = y.reshape(r2.shape)
+    rms = np.sqrt(np.mean(r2 * r2, axis=1, keepdims=True))
+    rms[rms == 0] = 1.0
+    return float(np.max(np.abs(y2 - r2) / np.maximum(np.abs(r2), rms)))
 
 
 def run_layer(w: W.Workload, inp: dict, n=None, diag=True):

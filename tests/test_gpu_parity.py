@@ -18,7 +18,7 @@ from tests import moe_harness as H
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "deepseek_v3_decode_small",
-         "skewed_small", "drop_small", "tie_softmax", "tie_sigmoid"]
+         "skewed_small", "drop_small", "ragged_small", "tie_softmax", "tie_sigmoid"]
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -101,7 +101,7 @@ def test_permute_parity(name):
 
 
 @pytest.mark.parametrize("name", ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small",
-                                  "deepseek_v3_decode_small", "skewed_small"])
+                                  "deepseek_v3_decode_small", "skewed_small", "ragged_small"])
 def test_expert_ffn_parity(name):
     w = W.get(name)
     host = W.host_inputs(w)

@@ -114,6 +114,8 @@ moe_status clear_status(const Ctx& ctx) {
 }
 
 bool ptr_ok(const void* p) { return p && aligned(p, 16); }
+// Per-token buffers may be null (zero-size tensors) when there are no tokens.
+bool tok_ok(const void* p, int64_t n) { return n == 0 ? (!p || aligned(p, 16)) : ptr_ok(p); }
 
 moe_status check_weights(const moe_config& c, const moe_weights* w, bool routed, bool shared) {
   if (!w) return MOE_ERR_INVALID_ARG;
@@ -138,7 +140,10 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   float* logits = x.at<float>(x.p.logits);
   moe_diag* d = diag ? diag : x.status();
   MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), x.s));  // counters, not the status word
-  if (x.n == 0) return MOE_OK;
+  if (x.n == 0) {
+    if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
+    return MOE_OK;
+  }
   GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model};
   MOE_TRY(gemm(x, g, false, true));
   RouteArgs r{};
@@ -234,7 +239,7 @@ moe_status moe_route(const moe_config* cfg, int64_t n, const void* x, const moe_
                      size_t ws_bytes, moe_stream_t stream) {
   Ctx c;
   MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
-  if (!weights || !ptr_ok(weights->w_router) || !ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(topk_w))
+  if (!weights || !ptr_ok(weights->w_router) || !tok_ok(x, n) || !tok_ok(topk_idx, n) || !tok_ok(topk_w, n))
     return MOE_ERR_INVALID_ARG;
   if ((expert_counts && !aligned(expert_counts, 4)) || (diag && !aligned(diag, 16))) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_weights(c.c, weights, false, false));
@@ -247,8 +252,8 @@ moe_status moe_permute(const moe_config* cfg, int64_t n, const void* x, const in
                        moe_stream_t stream) {
   Ctx c;
   MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
-  if (!ptr_ok(x) || !ptr_ok(topk_idx) || !ptr_ok(offsets) || !ptr_ok(perm_token) || !ptr_ok(slot_dest) ||
-      !ptr_ok(x_perm))
+  if (!tok_ok(x, n) || !tok_ok(topk_idx, n) || !ptr_ok(offsets) || !tok_ok(perm_token, n) ||
+      !tok_ok(slot_dest, n) || !tok_ok(x_perm, n))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY(clear_status(c));
   return permute_impl(c, x, topk_idx, offsets, perm_token, slot_dest, x_perm);
@@ -259,7 +264,7 @@ moe_status moe_expert_ffn(const moe_config* cfg, int64_t n, const void* x_perm, 
                           moe_stream_t stream) {
   Ctx c;
   MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
-  if (!ptr_ok(x_perm) || !ptr_ok(offsets) || !ptr_ok(expert_out)) return MOE_ERR_INVALID_ARG;
+  if (!tok_ok(x_perm, n) || !ptr_ok(offsets) || !tok_ok(expert_out, n)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_weights(c.c, weights, true, false));
   MOE_TRY(clear_status(c));
   return ffn_impl(c, x_perm, offsets, weights, expert_out);
@@ -270,12 +275,14 @@ moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out,
                        size_t ws_bytes, moe_stream_t stream) {
   Ctx c;
   MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
-  if (!ptr_ok(expert_out) || !ptr_ok(slot_dest) || !ptr_ok(topk_w) || !ptr_ok(y)) return MOE_ERR_INVALID_ARG;
-  if (c.c.n_shared > 0 && !ptr_ok(x)) return MOE_ERR_INVALID_ARG;
+  if (!tok_ok(expert_out, n) || !tok_ok(slot_dest, n) || !tok_ok(topk_w, n) || !tok_ok(y, n))
+    return MOE_ERR_INVALID_ARG;
+  if (c.c.n_shared > 0 && !tok_ok(x, n)) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_weights(c.c, weights, false, true));
   MOE_TRY(clear_status(c));
   void* sh = nullptr;
   MOE_TRY(shared_impl(c, x, weights, &sh));
+  if (n == 0) return MOE_OK;
   return cuda_status(launch_combine(expert_out, slot_dest, topk_w, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
 }
 
@@ -284,14 +291,14 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
                              void* ws, size_t ws_bytes, moe_stream_t stream) {
   Ctx c;
   MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
-  if (!ptr_ok(x) || !ptr_ok(y) || !weights || !ptr_ok(weights->w_router)) return MOE_ERR_INVALID_ARG;
-  if ((topk_idx_opt && !ptr_ok(topk_idx_opt)) || (topk_w_opt && !ptr_ok(topk_w_opt)) ||
+  if (!tok_ok(x, n) || !tok_ok(y, n) || !weights || !ptr_ok(weights->w_router)) return MOE_ERR_INVALID_ARG;
+  if ((topk_idx_opt && !tok_ok(topk_idx_opt, n)) || (topk_w_opt && !tok_ok(topk_w_opt, n)) ||
       (counts_opt && !aligned(counts_opt, 4)) || (diag_opt && !aligned(diag_opt, 16)))
     return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_weights(c.c, weights, true, true));
   MOE_TRY(clear_status(c));
-  int32_t* idx = topk_idx_opt ? topk_idx_opt : c.at<int32_t>(c.p.idx);
-  float* tw = topk_w_opt ? topk_w_opt : c.at<float>(c.p.w);
+  int32_t* idx = topk_idx_opt && n > 0 ? topk_idx_opt : c.at<int32_t>(c.p.idx);
+  float* tw = topk_w_opt && n > 0 ? topk_w_opt : c.at<float>(c.p.w);
   int32_t* counts = counts_opt ? counts_opt : c.at<int32_t>(c.p.counts);
   int32_t* offsets = c.at<int32_t>(c.p.offsets);
   int32_t* perm = c.at<int32_t>(c.p.perm);

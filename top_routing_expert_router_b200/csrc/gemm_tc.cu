@@ -1,8 +1,530 @@
-// gemm_tc.cu -- placeholder until the tcgen05 grouped GEMM lands.
+// gemm_tc.cu -- grouped GEMM on the 5th-generation tensor cores (tcgen05).
+//
+// For every group g (an expert, or the single shared-expert / router problem)
+// and every row r of that group:
+//   plain : C[r, n]  = sum_k A[r, k] * B_g[n, k]
+//   SwiGLU: C[r, i]  = silu(sum_k A[r, k] Bg_g[i, k]) * (sum_k A[r, k] Bu_g[i, k])
+// (page "15. DeepSeek: MLA, MoE and MTP", section "671B and 37B": gate, up,
+// down matrices; page "MoE" tag feed, activation functions: SwiGLU).
+//
+// Design (one CTA per SM, persistent, warp-specialised, 192 threads):
+//   warp 0      TMA producer: 128x64 A tile + 256x64 B tile per stage into a
+//               4-stage ring of 128B-swizzled shared memory (48 KB per stage);
+//               for SwiGLU the B tile is 128 gate rows over 128 up rows of the
+//               same output columns, so one MMA produces both.
+//   warp 1      TMEM owner (512 columns = two 128x256 fp32 accumulators) and
+//               MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32),
+//               M=128, N=256, K=16, four per stage; tcgen05.commit frees the
+//               stage and, after the last stage, hands the accumulator over.
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 16 columns, SwiGLU in fp32,
+//               bf16 (or fp32) stores of the rows inside the group; it drains
+//               one accumulator while the MMA fills the other.
+// Tiles are ordered (group, n-tile, m-tile) so that the CTAs running at the
+// same time share B tiles through L2. Every mbarrier wait is bounded: past the
+// limit the kernel records MOE_ERR_TIMEOUT in the status word, stops issuing,
+// waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
+#include <cuda.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace moe {
-bool gemm_tc_supported(const GemmArgs&, bool, bool) { return false; }
-cudaError_t launch_gemm_tc(const GemmArgs&, bool, bool, moe_diag*, cudaStream_t) { return cudaErrorNotSupported; }
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int BN_MAX = 256;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN_MAX * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int kMaxGroupsTc = 256;
+constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s for any single wait
+constexpr uint64_t kDrainNs = 200000000ull;     // 0.2 s per drain wait after an abort
+
+struct TcParams {
+  int32_t G;
+  const int32_t* offsets;  // [G + 1] row offsets, or nullptr: one group of M rows
+  int32_t M;
+  int32_t N;       // valid output columns per group
+  int32_t K;
+  int32_t n_mma;   // MMA N (multiple of 16, <= 256)
+  int32_t n_out;   // output columns per tile (SwiGLU: n_mma / 2)
+  int32_t b_rows;  // rows per group in the B tensor maps
+  int32_t swiglu;
+  int32_t out_f32;
+  void* C;
+  int64_t ldc;
+  moe_diag* status;
+};
+
+struct __align__(8) SmemCtl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t total_tiles;
+  int32_t n_tiles;
+  int32_t row_off[kMaxGroupsTc + 1];
+  int32_t tile_off[kMaxGroupsTc + 1];
+};
+
+// ---- PTX wrappers ------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of `parity` to complete. False on timeout or abort.
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SmemCtl* ctl, moe_diag* st) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(b, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        atomicExch(&ctl->abort, 1);
+        set_status(st, MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait used only while draining after an abort.
+__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t b = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(b, parity))
+    if (globaltimer() - t0 > kDrainNs) return;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
+                                            int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
+          "r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand, 128-byte swizzle: 8-row x 128-byte atoms stacked 1024 B apart.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
+  d |= (uint64_t)1 << 16;                   // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                   // descriptor version (tcgen05)
+  d |= (uint64_t)2 << 61;                   // SWIZZLE_128B
+  return d;
+}
+
+// kind::f16 instruction descriptor: bf16 A and B, fp32 D, both K-major, M = 128.
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ---- tile mapping ----------------------------------------------------------------
+struct Tile {
+  int g, m, nt;
+};
+
+// Tiles of group g are tile_off[g] .. tile_off[g+1]-1, ordered n-tile major, m minor.
+__device__ __forceinline__ Tile decode(const SmemCtl* ctl, int G, int t, int& g_hint) {
+  int g = g_hint;
+  while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
+  g_hint = g;
+  const int local = t - ctl->tile_off[g];
+  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM - 1) / BM;
+  return Tile{g, local % mt, local / mt};
+}
+
+__device__ __forceinline__ void store16(void* C, int64_t ldc, int64_t row, int col, int N, const float (&v)[16],
+                                        bool f32) {
+  if (f32) {
+    float* p = static_cast<float*>(C) + row * ldc + col;
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (col + 4 * q + 4 <= N)
+        *reinterpret_cast<float4*>(p + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+  } else {
+    bf16* p = static_cast<bf16*>(C) + row * ldc + col;
+    uint4 lo, hi;
+    __nv_bfloat162* l2 = reinterpret_cast<__nv_bfloat162*>(&lo);
+    __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&hi);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      l2[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+      h2[q] = __floats2bfloat162_rn(v[8 + 2 * q], v[8 + 2 * q + 1]);
+    }
+    if (col + 8 <= N) *reinterpret_cast<uint4*>(p) = lo;
+    if (col + 16 <= N) *reinterpret_cast<uint4*>(p + 8) = hi;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                   const __grid_constant__ CUtensorMap map_b2, TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  SmemCtl* ctl = reinterpret_cast<SmemCtl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- set-up: group row offsets, tile offsets, barriers, TMEM ----
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    const int n_tiles = (p.N + p.n_out - 1) / p.n_out;
+    for (int g = 0; g < p.G; ++g) {
+      const int lo = p.offsets ? p.offsets[g] : 0;
+      const int hi = p.offsets ? p.offsets[g + 1] : p.M;
+      ctl->row_off[g] = lo;
+      ctl->row_off[g + 1] = hi;
+      ctl->tile_off[g] = acc;
+      acc += ((hi - lo + BM - 1) / BM) * n_tiles;
+    }
+    ctl->tile_off[p.G] = acc;
+    ctl->total_tiles = acc;
+    ctl->n_tiles = n_tiles;
+    ctl->abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tmem_full[b], 1);
+      mbar_init(&ctl->tmem_empty[b], 4);
+    }
+    mbar_init(&ctl->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+    if (p.swiglu) tma_prefetch_desc(&map_b2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int total = ctl->total_tiles;
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int g_hint = 0;
+      uint32_t armed[STAGES] = {0, 0, 0, 0};
+      const uint32_t tx = A_BYTES + (uint32_t)p.n_mma * BK * 2;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        const Tile tl = decode(ctl, p.G, t, g_hint);
+        const int row0 = ctl->row_off[tl.g] + tl.m * BM;
+        const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          uint8_t* sb = sa + A_BYTES;
+          mbar_expect_tx(&ctl->full[stage], tx);
+          ++armed[stage];
+          tma_load_2d(sa, &map_a, &ctl->full[stage], kb * BK, row0);
+          if (p.swiglu) {
+            tma_load_2d(sb, &map_b, &ctl->full[stage], kb * BK, brow);
+            tma_load_2d(sb + (p.n_mma / 2) * BK * 2, &map_b2, &ctl->full[stage], kb * BK, brow);
+          } else {
+            tma_load_2d(sb, &map_b, &ctl->full[stage], kb * BK, brow);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let the copies already issued land before the block exits.
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) mbar_drain(&ctl->full[s], (armed[s] - 1) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc = idesc_bf16(p.n_mma);
+      bool ok = true;
+      bool issued = false;
+      int i = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+        if (!mbar_wait(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN_MAX);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait(&ctl->full[stage], phase, ctl, p.status)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = sw128_kmajor_desc(sa);
+          const uint64_t bdesc = sw128_kmajor_desc(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // advance 16 elements = 32 bytes inside the swizzle atom
+            mma_bf16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+          issued = true;
+          mma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&ctl->tmem_full[buf]);
+      }
+      if (!ok && issued) {
+        // Wait for the MMAs already issued before TMEM is released.
+        mma_commit(&ctl->drain);
+        mbar_drain(&ctl->drain, 0);
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5) =================
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_in_tile = q * 32 + lane;
+    int g_hint = 0;
+    int i = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      const Tile tl = decode(ctl, p.G, t, g_hint);
+      if (!mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status)) break;
+      fence_after();
+      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM + row_in_tile;
+      const bool valid = row < ctl->row_off[tl.g + 1];
+      const int col0 = tl.nt * p.n_out;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN_MAX);
+      if (p.swiglu) {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + (uint32_t)c, gv);
+          tmem_ld16(taddr + (uint32_t)(p.n_out + c), uv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) gv[e] = silu(gv[e]) * uv[e];
+          if (valid && col0 + c < p.N) store16(p.C, p.ldc, row, col0 + c, p.N, gv, false);
+        }
+      } else {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)c, v);
+          if (valid && col0 + c < p.N) store16(p.C, p.ldc, row, col0 + c, p.N, v, p.out_f32 != 0);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---- host side -----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous), box [box_rows, 64], 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int num_sms() {
+  static int sms = 0;
+  if (!sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (sms <= 0) sms = 148;
+  }
+  return sms;
+}
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SmemCtl);
+
+}  // namespace
+
+bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32) {
+  if (a.K % 8 != 0 || a.N % 8 != 0 || a.N <= 0 || a.K <= 0) return false;
+  if (a.G > kMaxGroupsTc || a.M >= ((int64_t)1 << 31)) return false;
+  if (a.lda != a.K) return false;
+  if (swiglu && out_f32) return false;
+  if (out_f32 && a.ldc % 4 != 0) return false;
+  if (!out_f32 && a.ldc % 8 != 0) return false;
+  if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.B) % 16 ||
+      reinterpret_cast<uintptr_t>(a.C) % 16 || (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
+    return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_diag* status, cudaStream_t s) {
+  if (!gemm_tc_supported(a, swiglu, out_f32)) return cudaErrorNotSupported;
+  if (a.M <= 0) return cudaSuccess;
+  TcParams p{};
+  p.G = a.G;
+  p.offsets = a.offsets;
+  p.M = (int32_t)a.M;
+  p.N = a.N;
+  p.K = a.K;
+  if (swiglu) {
+    p.n_mma = BN_MAX;
+    p.n_out = BN_MAX / 2;
+  } else {
+    p.n_mma = a.N >= BN_MAX ? BN_MAX : (int32_t)align_up(a.N, 16);
+    p.n_out = p.n_mma;
+  }
+  p.b_rows = a.N;
+  p.swiglu = swiglu;
+  p.out_f32 = out_f32;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.status = status;
+  CUtensorMap ma, mb, mb2;
+  const int64_t b_total_rows = (int64_t)a.G * a.N;
+  const int b_box = swiglu ? p.n_mma / 2 : p.n_mma;
+  if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mb, a.B, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
+  if (swiglu) {
+    if (!make_map(&mb2, a.B2, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
+  } else {
+    mb2 = mb;
+  }
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  // Upper bound on the tiles: every group may add one partial m-tile.
+  const int64_t n_tiles = ceil_div(a.N, p.n_out);
+  const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles;
+  const int grid = (int)(max_tiles < num_sms() ? max_tiles : num_sms());
+  gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mb2, p);
+  return cudaGetLastError();
+}
+
 }  // namespace moe
