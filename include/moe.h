@@ -181,6 +181,42 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
                              moe_diag* diag_opt, void* ws, size_t ws_bytes, moe_stream_t stream);
 
 /*
+ * Bytes of the device array behind moe_route_static_scratch (8 MiB).
+ */
+#define MOE_STATIC_SCRATCH_BYTES (8u << 20)
+
+/*
+ * moe_route for callers that cannot allocate device memory. The pages have no
+ * counterpart to this entry point; it exists for deployment. Some callers only
+ * ever receive their input and output buffers: a plug-in running inside a
+ * serving engine whose memory planner owns every device allocation, or code on
+ * a latency-critical path where a cudaMalloc would synchronise the device. They
+ * cannot provide a workspace, so this variant keeps the router's scratch (the
+ * binary32 logits, the capacity ranking, per-block counts and the status word)
+ * in one array of MOE_STATIC_SCRATCH_BYTES in device memory that is part of
+ * this library: every GPU that loads the library holds that array until the
+ * process exits. It calls no cudaMalloc, cudaFree or allocating routine.
+ *   Arguments and outputs are those of moe_route, without ws/ws_bytes.
+ *   Returns MOE_ERR_WORKSPACE when this cfg and n need more scratch than the
+ *   array holds (E * 4 bytes of logits per token dominate; e.g. E = 256 fits
+ *   about 7000 tokens, E = 8 about 200000), MOE_ERR_CUDA if the array's device
+ *   address cannot be found, and the errors of moe_route otherwise.
+ *   The first call on each device performs a one-time set-up that looks up the
+ *   array's device address with that device current; make this first call
+ *   before any stream capture begins.
+ *   All calls on a device share the one array and it keeps the contents of the
+ *   last call (everything that must start at zero is cleared by each call).
+ *   Calls that overlap on the GPU, e.g. on two streams at once, race on it and
+ *   produce undefined results; order them on one stream. The status word that
+ *   moe_sync_status reads lives in the array, so that call does not apply here:
+ *   when diag is given, the call copies its device status word (a moe_status
+ *   value, 0 = MOE_OK) into diag->status on `stream`.
+ */
+moe_status moe_route_static_scratch(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
+                                    int32_t* topk_idx, float* topk_w, int32_t* expert_counts, moe_diag* diag,
+                                    moe_stream_t stream);
+
+/*
  * Synchronises `stream`, then returns the device status word kept in the
  * workspace (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_INTERNAL) and clears it. Every
  * entry point clears the word when it starts, so it reports the most recent

@@ -1,0 +1,74 @@
+"""moe_route_static_scratch: the router for callers that cannot allocate.
+
+Some callers of this library never allocate device memory themselves: a
+plug-in that runs inside a serving engine only receives the input and output
+buffers the engine's memory planner hands it, and code on a latency-critical
+path must not call cudaMalloc because it synchronises the device. Those
+callers cannot supply a workspace, so this entry point keeps the router's
+scratch in a fixed-size device array that is part of the library.
+
+The array is shared by every call and keeps the previous call's contents, so
+each test below routes twice in a row and compares both results with
+moe_route run on a caller-provided workspace: same expert indices and counts,
+gates within the tolerance of the routing parity tests. This file is named so
+that pytest collects it last.
+"""
+import numpy as np
+import pytest
+import torch
+
+import top_routing_expert_router_b200 as moe
+from synth import workloads as W
+from tests import moe_harness as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    torch.cuda.set_device(0)
+
+
+def _outputs(w):
+    return (torch.full((w.n, w.top_k), -9, dtype=torch.int32, device="cuda"),
+            torch.full((w.n, w.top_k), -9.0, dtype=torch.float32, device="cuda"),
+            torch.full((w.n_routed,), -9, dtype=torch.int32, device="cuda"),
+            torch.full((8,), -9, dtype=torch.int32, device="cuda"))
+
+
+@pytest.mark.parametrize("name", ["deepseek_v3_small", "skewed_small", "mixtral_small", "deepseek_v3_decode_small"])
+def test_static_scratch_route_matches_workspace_route_twice(name):
+    w = W.get(name)
+    dev = W.device_inputs(w)
+    cfg = H.cfg_for(w)
+    weights = H.weights_for(dev)
+
+    # the existing entry point, with a workspace the caller allocated
+    ws = H.workspace(cfg, w.n)
+    idx0, tw0, cnt0, dg0 = _outputs(w)
+    moe.moe_route(cfg, w.n, dev["x"], weights, idx0, tw0, cnt0, dg0, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+
+    for call in range(2):
+        idx, tw, cnt, dg = _outputs(w)
+        moe.moe_route_static_scratch(cfg, w.n, dev["x"], weights, idx, tw, cnt, dg)
+        torch.cuda.synchronize()
+        diag = H.diag_dict(dg)
+        assert diag["status"] == moe.MOE_OK, (call, diag)
+        assert torch.equal(idx, idx0), call
+        assert torch.equal(cnt, cnt0), call
+        np.testing.assert_allclose(tw.cpu().numpy(), tw0.cpu().numpy(), rtol=2e-4, atol=1e-6)
+        assert diag["refined_tokens"] == H.diag_dict(dg0)["refined_tokens"]
+        assert diag["overflowed"] == H.diag_dict(dg0)["overflowed"]
+
+
+def test_static_scratch_rejects_sizes_beyond_the_array():
+    w = W.get("deepseek_v3_prefill")  # 16384 tokens x 256 experts of fp32 logits > 8 MiB
+    cfg = H.cfg_for(w)
+    dummy = torch.empty(16, dtype=torch.int32, device="cuda")
+    weights = moe.make_weights(dummy, dummy, dummy, dummy)
+    with pytest.raises(moe.MoeError) as e:
+        moe.moe_route_static_scratch(cfg, w.n, dummy, weights, dummy, dummy, None, None)
+    assert e.value.status == moe.MOE_ERR_WORKSPACE

@@ -28,7 +28,8 @@ MOE_F32, MOE_BF16 = 0, 1
 
 # Every symbol declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
-           "moe_layer_forward", "moe_sync_status", "moe_status_string")
+           "moe_layer_forward", "moe_route_static_scratch", "moe_sync_status", "moe_status_string")
+MOE_STATIC_SCRATCH_BYTES = 8 << 20  # include/moe.h
 
 
 class moe_config(ctypes.Structure):
@@ -61,6 +62,7 @@ _lib.moe_permute.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_expert_ffn.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_combine.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_layer_forward.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_route_static_scratch.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_sync_status.argtypes = [_P, _P]
 _lib.moe_status_string.argtypes = [ctypes.c_int]
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -122,6 +124,13 @@ def moe_route(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, ws, str
     _check(_lib.moe_route(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(topk_idx), _ptr(topk_w),
                           _ptr(expert_counts), _ptr(diag), _ptr(ws), ws.numel() * ws.element_size(),
                           _stream(stream)), "moe_route")
+
+
+def moe_route_static_scratch(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, stream=None):
+    """moe_route without a workspace: the scratch is the library's static device array (see moe.h)."""
+    _check(_lib.moe_route_static_scratch(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(topk_idx),
+                                         _ptr(topk_w), _ptr(expert_counts), _ptr(diag), _stream(stream)),
+           "moe_route_static_scratch")
 
 
 def moe_permute(cfg, n, x, topk_idx, offsets, perm_token, slot_dest, x_perm, ws, stream=None):

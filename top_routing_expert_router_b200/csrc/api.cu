@@ -223,6 +223,41 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
 }  // namespace
 }  // namespace moe
 
+namespace moe {
+
+// Bytes of the routing part of the workspace layout (the regions moe_route uses).
+size_t route_scratch_bytes(const moe_config& c, int64_t n) {
+  const Plan p = make_plan(c, n);
+  return p.offsets + (size_t)align_up((int64_t)(c.n_routed + 1) * 4, 256);
+}
+
+// moe_route over a scratch region that only needs route_scratch_bytes() bytes.
+moe_status route_in_scratch(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
+                            int32_t* topk_idx, float* topk_w, int32_t* expert_counts, moe_diag* diag, void* scratch,
+                            size_t scratch_bytes, moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg, n));
+  if (!scratch || !aligned(scratch, 256)) return MOE_ERR_INVALID_ARG;
+  if (scratch_bytes < route_scratch_bytes(*cfg, n)) return MOE_ERR_WORKSPACE;
+  Ctx c;
+  c.c = *cfg;
+  c.n = n;
+  c.p = make_plan(*cfg, n);
+  c.ws = static_cast<char*>(scratch);
+  c.s = reinterpret_cast<cudaStream_t>(stream);
+  if (!weights || !ptr_ok(weights->w_router) || !tok_ok(x, n) || !tok_ok(topk_idx, n) || !tok_ok(topk_w, n))
+    return MOE_ERR_INVALID_ARG;
+  if ((expert_counts && !aligned(expert_counts, 4)) || (diag && !aligned(diag, 16))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, false, false));
+  MOE_TRY(clear_status(c));
+  MOE_TRY(route_impl(c, x, weights, topk_idx, topk_w, expert_counts, diag));
+  // The scratch is not the caller's, so hand the device status word over in diag.
+  if (diag)
+    MOE_CUDA(cudaMemcpyAsync(&diag->status, &c.status()->status, sizeof(int32_t), cudaMemcpyDeviceToDevice, c.s));
+  return MOE_OK;
+}
+
+}  // namespace moe
+
 using namespace moe;
 
 extern "C" {
