@@ -104,6 +104,9 @@ WORKLOADS = {w.name: w for w in [
     _wl("skewed_capacity", n=32768, d_model=4096, n_routed=64, top_k=2, moe_intermediate_size=2048,
         cap_policy="overflow_next", capacity_factor=1.25, zipf_s=1.2,
         description="skewed softmax top-2, capacity 1.25*n*k/E, overflow to next-best"),
+    # profiling case: Mixtral shapes with 4 experts (1.4 GB of weights, still far larger than L2)
+    _wl("mixtral_4e", n=2048, d_model=4096, n_routed=4, top_k=2, moe_intermediate_size=14336,
+        renormalize=True, description="Mixtral-shaped layer with 4 experts (profiling size)"),
     # parity-size variants
     _wl("mixtral_small", n=700, d_model=256, n_routed=8, top_k=2, moe_intermediate_size=384,
         renormalize=True),

@@ -197,3 +197,18 @@ def test_single_token_and_ragged_sizes():
         keep = ~r["exempt"]
         np.testing.assert_array_equal(got["topk_idx"].cpu().numpy()[keep], r["topk_idx"][keep])
         assert H.rel_err(H.as_f64(got["y"])[keep], r["y"][keep]) <= H.TOL[w.dtype]
+
+
+@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+@pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v3_small", "ragged_small", "deepseek_v2_small"])
+def test_expert_ffn_both_tile_modes(name, mode, monkeypatch):
+    """The 128-row single-SM tiles and the 256-row SM-pair tiles both match the oracle."""
+    monkeypatch.setenv("MOE_TC_MODE", mode)
+    test_expert_ffn_parity(name)
+    w = W.get(name)
+    dev, host = W.device_inputs(w), W.host_inputs(w)
+    got = H.run_layer(w, dev)
+    r = O.layer(H.oracle_cfg(w), host["x"], host["w_r"], host["w_gate"], host["w_up"], host["w_down"],
+                host.get("bias"), host.get("ws_gate"), host.get("ws_up"), host.get("ws_down"))
+    keep = ~r["exempt"]
+    assert H.rel_err(H.as_f64(got["y"])[keep], r["y"][keep]) <= H.TOL[w.dtype]

@@ -17,6 +17,23 @@ struct Plan {
   size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, total;
 };
 
+// Split-K factor of the router GEMM: small token counts leave most SMs idle
+// (one 128-row tile per 128 tokens), so the k range is split and the route
+// kernel sums the partial logits in a fixed order. Capped at 4 MiB of partials.
+int router_splits(const moe_config& c, int64_t n) {
+  if (c.dtype != MOE_BF16 || c.n_routed % 8 != 0 || n <= 0) return 1;
+  const int64_t tiles = ceil_div(n, 128) * ceil_div(c.n_routed, 256);
+  if (tiles >= 74) return 1;
+  const int64_t num_kb = ceil_div(c.d_model, 64);
+  int64_t s = 148 / tiles;
+  const int64_t cap = ((int64_t)4 << 20) / (n * c.n_routed * 4);
+  if (s > cap) s = cap;
+  if (s > num_kb) s = num_kb;
+  if (s < 1) s = 1;
+  const int64_t kb_per = ceil_div(num_kb, s);
+  return (int)ceil_div(num_kb, kb_per);
+}
+
 Plan make_plan(const moe_config& c, int64_t n) {
   const size_t b = c.dtype == MOE_BF16 ? 2 : 4;
   const int64_t nk = n * c.top_k;
@@ -29,7 +46,7 @@ Plan make_plan(const moe_config& c, int64_t n) {
     return at;
   };
   p.diag = take(sizeof(moe_diag));
-  p.logits = take((size_t)n * c.n_routed * 4);
+  p.logits = take((size_t)router_splits(c, n) * n * c.n_routed * 4);
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
   p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
   p.idx = take((size_t)nk * 4);
@@ -144,10 +161,14 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
     return MOE_OK;
   }
-  GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model};
+  const int splits = router_splits(c, x.n);
+  GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model,
+             splits, x.n * c.n_routed};
   MOE_TRY(gemm(x, g, false, true));
   RouteArgs r{};
   r.logits = logits;
+  r.splits = splits;
+  r.split_stride = x.n * c.n_routed;
   r.x = X;
   r.w_r = w->w_router;
   r.bias = c.score_fn == MOE_SCORE_SIGMOID ? w->bias : nullptr;

@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(GemmArgs a) {
 int64_t gemm_simt_max_tiles_y(int64_t rows_total, int G) { return ceil_div(rows_total, BM) + G; }
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, int dtype, bool out_f32, bool swiglu, cudaStream_t s) {
+  if (a.k_splits > 1) return cudaErrorInvalidValue;  // split-K is a tensor-core path feature
   const int64_t ty = gemm_simt_max_tiles_y(a.M, a.G);
   if (ty <= 0 || a.N <= 0) return cudaSuccess;
   dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ty);

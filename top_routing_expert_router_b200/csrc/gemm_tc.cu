@@ -24,6 +24,8 @@
 // limit the kernel records MOE_ERR_TIMEOUT in the status word, stops issuing,
 // waits (bounded) for its copies and MMAs in flight, frees TMEM and returns.
 #include <cuda.h>
+#include <stdlib.h>
+#include <string.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -55,8 +57,11 @@ struct TcParams {
   int32_t b_rows;  // rows per group in the B tensor maps
   int32_t swiglu;
   int32_t out_f32;
+  int32_t k_splits;   // split-K factor (partials to C + split * c_split_stride)
+  int32_t kb_per;     // k-blocks per split
   void* C;
   int64_t ldc;
+  int64_t c_split_stride;
   moe_diag* status;
 };
 
@@ -197,17 +202,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 
 // ---- tile mapping ----------------------------------------------------------------
 struct Tile {
-  int g, m, nt;
+  int g, m, nt, split;
 };
 
-// Tiles of group g are tile_off[g] .. tile_off[g+1]-1, ordered n-tile major, m minor.
+// Tiles of group g are tile_off[g] .. tile_off[g+1]-1, ordered split major,
+// then n-tile, then m-tile.
 __device__ __forceinline__ Tile decode(const SmemCtl* ctl, int G, int t, int& g_hint) {
   int g = g_hint;
   while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
   g_hint = g;
   const int local = t - ctl->tile_off[g];
   const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM - 1) / BM;
-  return Tile{g, local % mt, local / mt};
+  const int per_split = mt * ctl->n_tiles;
+  const int rem = local % per_split;
+  return Tile{g, rem % mt, rem / mt, local / per_split};
 }
 
 __device__ __forceinline__ void store16(void* C, int64_t ldc, int64_t row, int col, int N, const float (&v)[16],
@@ -251,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctl->row_off[g] = lo;
       ctl->row_off[g + 1] = hi;
       ctl->tile_off[g] = acc;
-      acc += ((hi - lo + BM - 1) / BM) * n_tiles;
+      acc += ((hi - lo + BM - 1) / BM) * n_tiles * p.k_splits;
     }
     ctl->tile_off[p.G] = acc;
     ctl->total_tiles = acc;
@@ -285,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   fence_after();
   const uint32_t tmem_base = ctl->tmem_base;
   const int total = ctl->total_tiles;
-  const int num_kb = (p.K + BK - 1) / BK;
+  const int num_kb_all = (p.K + BK - 1) / BK;
 
   if (warp == 0) {
     // ================= TMA producer =================
@@ -300,7 +308,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const Tile tl = decode(ctl, p.G, t, g_hint);
         const int row0 = ctl->row_off[tl.g] + tl.m * BM;
         const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        const int kb0 = tl.split * p.kb_per, kb1 = min(num_kb_all, kb0 + p.kb_per);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
             ok = false;
             break;
@@ -337,7 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       bool issued = false;
       int i = 0;
+      int g_hint = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+        const Tile tl = decode(ctl, p.G, t, g_hint);
+        const int nkb = min(num_kb_all, (tl.split + 1) * p.kb_per) - tl.split * p.kb_per;
         const int buf = i & 1;
         const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
         if (!mbar_wait(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
@@ -346,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN_MAX);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&ctl->full[stage], phase, ctl, p.status)) {
             ok = false;
             break;
@@ -384,9 +396,315 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int buf = i & 1;
       const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
       const Tile tl = decode(ctl, p.G, t, g_hint);
-      if (!mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status)) break;
+      const bool got = mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
+      __syncwarp();  // tcgen05.ld below is warp-aligned
+      if (!got) break;
       fence_after();
       const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM + row_in_tile;
+      const bool valid = row < ctl->row_off[tl.g + 1];
+      const int col0 = tl.nt * p.n_out;
+      void* C = p.out_f32 ? (void*)(static_cast<float*>(p.C) + (int64_t)tl.split * p.c_split_stride)
+                          : (void*)(static_cast<bf16*>(p.C) + (int64_t)tl.split * p.c_split_stride);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN_MAX);
+      if (p.swiglu) {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + (uint32_t)c, gv);
+          tmem_ld16(taddr + (uint32_t)(p.n_out + c), uv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) gv[e] = silu(gv[e]) * uv[e];
+          if (valid && col0 + c < p.N) store16(C, p.ldc, row, col0 + c, p.N, gv, false);
+        }
+      } else {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)c, v);
+          if (valid && col0 + c < p.N) store16(C, p.ldc, row, col0 + c, p.N, v, p.out_f32 != 0);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---- 2-SM variant (cta_group::2) -----------------------------------------------------
+// A CTA pair (cluster of 2) computes a 256 x 256 tile: CTA r holds A rows
+// [128r, 128r+128) of the tile and B rows [128r, 128r+128) (for SwiGLU: the
+// gate half in CTA 0, the up half in CTA 1). The leader CTA (rank 0) issues
+// tcgen05.mma.cta_group::2 with M = 256, which reads the peer's operand halves
+// through the pair's shared memory, so each SM stages 32 KB per 64-k step
+// instead of 48 KB. Both CTAs' copies signal the leader's `full` barrier; the
+// leader's commits are multicast to both CTAs; both epilogues report to the
+// leader's `tmem_empty` barrier. No TMA multicast is used.
+constexpr int BM2 = 256;        // rows per pair tile
+constexpr int STAGES2 = 6;
+constexpr int A2_BYTES = 128 * BK * 2;
+constexpr int B2_BYTES = 128 * BK * 2;
+constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
+
+struct __align__(8) SmemCtl2 {
+  uint64_t full[STAGES2];
+  uint64_t empty[STAGES2];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t total_tiles;
+  int32_t n_tiles;
+  int32_t row_off[kMaxGroupsTc + 1];
+  int32_t tile_off[kMaxGroupsTc + 1];
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Shared-cluster address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
+  return out;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// Pair copy: lands in this CTA's shared memory, completes bytes on the leader's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t leader_bar, int32_t c0,
+                                                 int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+      "[%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+// Arrive on the barrier at this offset in both CTAs of the pair once the MMAs complete.
+__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          smem_u32(bar)),
+      "h"(mask)
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM2 >> 4) << 24);
+}
+
+__device__ __forceinline__ Tile decode2(const SmemCtl2* ctl, int G, int t, int& g_hint) {
+  int g = g_hint;
+  while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
+  g_hint = g;
+  const int local = t - ctl->tile_off[g];
+  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM2 - 1) / BM2;
+  return Tile{g, local % mt, local / mt, 0};
+}
+
+__device__ __noinline__ bool mbar_wait2(uint64_t* bar, uint32_t parity, SmemCtl2* ctl, moe_diag* st) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(b, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        atomicExch(&ctl->abort, 1);
+        set_status(st, MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __noinline__ void spin_ns(uint64_t ns) {
+  const uint64_t t0 = globaltimer();
+  while (globaltimer() - t0 < ns) {
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const __grid_constant__ CUtensorMap map_b2, TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw2[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
+  SmemCtl2* ctl = reinterpret_cast<SmemCtl2*>(smem + STAGES2 * STAGE2_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    const int n_tiles = (p.N + p.n_out - 1) / p.n_out;
+    for (int g = 0; g < p.G; ++g) {
+      const int lo = p.offsets ? p.offsets[g] : 0;
+      const int hi = p.offsets ? p.offsets[g + 1] : p.M;
+      ctl->row_off[g] = lo;
+      ctl->row_off[g + 1] = hi;
+      ctl->tile_off[g] = acc;
+      acc += ((hi - lo + BM2 - 1) / BM2) * n_tiles;
+    }
+    ctl->tile_off[p.G] = acc;
+    ctl->total_tiles = acc;
+    ctl->n_tiles = n_tiles;
+    ctl->abort = 0;
+    for (int s = 0; s < STAGES2; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tmem_full[b], 1);
+      mbar_init(&ctl->tmem_empty[b], 8);
+    }
+    mbar_init(&ctl->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_b);
+    if (p.swiglu) tma_prefetch_desc(&map_b2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised before any remote arrive or copy
+  fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int total = ctl->total_tiles;
+  const int num_kb = (p.K + BK - 1) / BK;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ================= TMA producer (both CTAs) =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int g_hint = 0;
+      const uint32_t tx = 2u * STAGE2_BYTES;
+      for (int t = pair; t < total && !aborted; t += npairs) {
+        const Tile tl = decode2(ctl, p.G, t, g_hint);
+        const int row0 = ctl->row_off[tl.g] + tl.m * BM2 + (int)rank * 128;
+        const CUtensorMap* bmap = (p.swiglu && rank == 1) ? &map_b2 : &map_b;
+        const int brow = p.swiglu ? tl.g * p.b_rows + tl.nt * p.n_out
+                                  : tl.g * p.b_rows + tl.nt * p.n_out + (int)rank * 128;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait2(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE2_BYTES;
+          const uint32_t leader_full = map_to_rank(&ctl->full[stage], 0);
+          if (rank == 0) mbar_expect_tx(&ctl->full[stage], tx);
+          tma_load_2d_pair(sa, &map_a, leader_full, kb * BK, row0);
+          tma_load_2d_pair(sa + A2_BYTES, bmap, leader_full, kb * BK, brow);
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (leader CTA) =================
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc = idesc_bf16_m256(BN_MAX);
+      bool issued = false;
+      int i = 0;
+      for (int t = pair; t < total && !aborted; t += npairs, ++i) {
+        const int buf = i & 1;
+        const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+        if (!mbar_wait2(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
+          aborted = true;
+          break;
+        }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN_MAX);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait2(&ctl->full[stage], phase, ctl, p.status)) {
+            aborted = true;
+            break;
+          }
+          fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
+          const uint64_t adesc = sw128_kmajor_desc(sa);
+          const uint64_t bdesc = sw128_kmajor_desc(sa + A2_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)
+            mma_bf16_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, (kb | k) != 0);
+          issued = true;
+          mma_commit_pair(&ctl->empty[stage]);
+          if (++stage == STAGES2) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (aborted) break;
+        mma_commit_pair(&ctl->tmem_full[buf]);
+      }
+      if (aborted && issued) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&ctl->drain))
+                     : "memory");
+        mbar_drain(&ctl->drain, 0);
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5, both CTAs) =================
+    const int q = warp & 3;
+    const int row_in_tile = (int)rank * 128 + q * 32 + lane;
+    const uint32_t leader_tmem_empty[2] = {map_to_rank(&ctl->tmem_empty[0], 0), map_to_rank(&ctl->tmem_empty[1], 0)};
+    int g_hint = 0;
+    int i = 0;
+    for (int t = pair; t < total; t += npairs, ++i) {
+      const int buf = i & 1;
+      const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      const Tile tl = decode2(ctl, p.G, t, g_hint);
+      const bool got = mbar_wait2(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
+      __syncwarp();  // tcgen05.ld below is warp-aligned
+      if (!got) {
+        aborted = true;
+        break;
+      }
+      fence_after();
+      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM2 + row_in_tile;
       const bool valid = row < ctl->row_off[tl.g + 1];
       const int col0 = tl.nt * p.n_out;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN_MAX);
@@ -408,15 +726,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+      if (lane == 0) mbar_arrive_cluster(leader_tmem_empty[buf]);
     }
   }
 
+  if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) spin_ns(1000000);  // let copies in flight land
   fence_before();
   __syncthreads();
+  __syncwarp();
+  cluster_sync();
   fence_after();
   if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
                  : "memory");
   }
 }
@@ -465,6 +787,19 @@ int num_sms() {
 }
 
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SmemCtl);
+constexpr size_t kSmemBytes2 = 1024 + STAGES2 * STAGE2_BYTES + sizeof(SmemCtl2);
+
+// 2-SM pair tiles (256 rows) pay off when groups carry enough rows; ragged
+// groups with few rows waste less with 128-row tiles. MOE_TC_MODE=1sm|2sm
+// overrides the choice (tuning and tests).
+bool use_pair_tiles(const GemmArgs& a, bool swiglu, bool out_f32) {
+  if (a.k_splits > 1 || out_f32) return false;
+  if (!swiglu && a.N < BN_MAX) return false;
+  const char* mode = getenv("MOE_TC_MODE");
+  if (mode && strcmp(mode, "1sm") == 0) return false;
+  if (mode && strcmp(mode, "2sm") == 0) return true;
+  return a.M / (a.offsets ? a.G : 1) >= 768;
+}
 
 }  // namespace
 
@@ -473,6 +808,7 @@ bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32) {
   if (a.G > kMaxGroupsTc || a.M >= ((int64_t)1 << 31)) return false;
   if (a.lda != a.K) return false;
   if (swiglu && out_f32) return false;
+  if (a.k_splits > 1 && (swiglu || !out_f32)) return false;
   if (out_f32 && a.ldc % 4 != 0) return false;
   if (!out_f32 && a.ldc % 8 != 0) return false;
   if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.B) % 16 ||
@@ -500,18 +836,58 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   p.b_rows = a.N;
   p.swiglu = swiglu;
   p.out_f32 = out_f32;
+  {
+    // Split-K: every split owns at least one k-block.
+    const int num_kb = (int)ceil_div(a.K, BK);
+    const int want = a.k_splits < 1 ? 1 : (a.k_splits > num_kb ? num_kb : a.k_splits);
+    p.kb_per = (int)ceil_div(num_kb, want);
+    p.k_splits = (int)ceil_div(num_kb, p.kb_per);
+    if (p.k_splits != a.k_splits) return cudaErrorInvalidValue;  // caller sized its partials for a.k_splits
+  }
   p.C = a.C;
   p.ldc = a.ldc;
+  p.c_split_stride = a.c_split_stride;
   p.status = status;
   CUtensorMap ma, mb, mb2;
   const int64_t b_total_rows = (int64_t)a.G * a.N;
-  const int b_box = swiglu ? p.n_mma / 2 : p.n_mma;
+  const bool pair = use_pair_tiles(a, swiglu, out_f32);
+  // Rows of B one CTA stages per copy: SwiGLU gate/up halves are 128 rows; on an
+  // SM pair each CTA also holds only a 128-row half of a plain 256-row B tile.
+  const int b_box = (swiglu || pair) ? p.n_mma / 2 : p.n_mma;
+  // Every copy must fit the shared-memory slot it lands in.
+  const int b_slot_rows = pair ? B2_BYTES / (BK * 2) : (swiglu ? BN_MAX / 2 : BN_MAX);
+  if (b_box > b_slot_rows || (pair && (p.n_mma != BN_MAX || A2_BYTES != BM * BK * 2))) return cudaErrorInvalidValue;
   if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
   if (!make_map(&mb, a.B, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
   if (swiglu) {
     if (!make_map(&mb2, a.B2, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
   } else {
     mb2 = mb;
+  }
+  const int64_t n_tiles_all = ceil_div(a.N, p.n_out);
+  if (pair) {
+    static bool attr2 = false;
+    if (!attr2) {
+      cudaError_t e =
+          cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes2);
+      if (e != cudaSuccess) return e;
+      attr2 = true;
+    }
+    const int64_t max_pair_tiles = (ceil_div(a.M, BM2) + (a.offsets ? a.G : 0)) * n_tiles_all;
+    const int64_t pairs = max_pair_tiles < num_sms() / 2 ? max_pair_tiles : num_sms() / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytes2;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, mb, mb2, p);
   }
   static bool attr_set = false;
   if (!attr_set) {
@@ -521,7 +897,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   }
   // Upper bound on the tiles: every group may add one partial m-tile.
   const int64_t n_tiles = ceil_div(a.N, p.n_out);
-  const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles;
+  const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles * p.k_splits;
   const int grid = (int)(max_tiles < num_sms() ? max_tiles : num_sms());
   gemm_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mb2, p);
   return cudaGetLastError();

@@ -24,6 +24,8 @@ struct GemmArgs {
   int64_t M;  // upper bound on the total rows (exact when offsets == nullptr)
   int32_t N;
   int32_t K;
+  int32_t k_splits = 1;         // > 1: split-K, partial results written k_splits times
+  int64_t c_split_stride = 0;   // elements between the partial result matrices
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, int dtype, bool out_f32, bool swiglu, cudaStream_t s);
@@ -35,7 +37,9 @@ bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32);
 
 // Router: scoring, group limit, top-k, certification / binary64 refinement, gates.
 struct RouteArgs {
-  const float* logits;  // [n, E]
+  const float* logits;  // [splits][n, E] partial logits, summed in order
+  int32_t splits;
+  int64_t split_stride;
   const void* x;        // [n, d] for the binary64 refinement
   const void* w_r;      // [E, d]
   const float* bias;    // [E] or nullptr

@@ -74,118 +74,319 @@ __device__ __forceinline__ double pick(const double (&r)[EPL], int j) {
   return out;
 }
 
-// Selection of one token. Writes the ranked experts to rank[0..R) (R = k, or
-// every eligible expert when `full_ranking`). Returns false when `check` is set
-// and some gap the decision depends on is within the binary32 error bound.
+// Selection values: softmax ranks the logits; sigmoid ranks s + bias.
 template <int EPL>
-__device__ bool decide(const RouteArgs& a, const double (&l)[EPL], bool check, bool full_ranking,
-                       int16_t* rank, int* n_ranked) {
+__device__ __forceinline__ void selection_values(const RouteArgs& a, const double (&l)[EPL], double (&v)[EPL],
+                                                 bool (&valid)[EPL]) {
   const int lane = threadIdx.x & 31;
-  const int E = a.E;
-  double v[EPL];
-  bool valid[EPL];
-  double amax = 0.0;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = lane + 32 * j;
-    valid[j] = e < E;
-    if (valid[j]) {
-      if (a.score_fn == MOE_SCORE_SIGMOID)
-        v[j] = sigmoid_d(l[j]) + (a.bias ? (double)a.bias[e] : 0.0);
-      else
-        v[j] = l[j];
-      amax = fmax(amax, fabs(l[j]));
-    } else {
+    valid[j] = e < a.E;
+    if (valid[j])
+      v[j] = a.score_fn == MOE_SCORE_SIGMOID ? sigmoid_d(l[j]) + (a.bias ? (double)a.bias[e] : 0.0) : l[j];
+    else
       v[j] = -INFINITY;
-    }
   }
-  double delta_v = 0.0;
-  if (check) {
-    amax = warp_max(amax);
-    const double delta_l = ldexp(fmax(1.0, amax), -14);
-    delta_v = a.score_fn == MOE_SCORE_SIGMOID ? 0.25 * delta_l : delta_l;
-  }
-  bool ok = true;
+}
 
-  // Group limit: keep the topk_group groups with the largest sum of two best scores.
-  bool elig[EPL];
-#pragma unroll
-  for (int j = 0; j < EPL; ++j) elig[j] = valid[j];
-  if (a.G > 1) {
-    const int per = E / a.G;
-    double gs[kMaxGroups];
-    for (int g = 0; g < a.G; ++g) {
-      double t1 = -INFINITY, t2 = -INFINITY;
-#pragma unroll
-      for (int j = 0; j < EPL; ++j) {
-        const int e = lane + 32 * j;
-        if (valid[j] && e / per == g) {
-          if (v[j] > t1) {
-            t2 = t1;
-            t1 = v[j];
-          } else if (v[j] > t2) {
-            t2 = v[j];
-          }
-        }
-      }
-#pragma unroll
-      for (int off = 16; off; off >>= 1) {
-        const double o1 = __shfl_xor_sync(kFull, t1, off);
-        const double o2 = __shfl_xor_sync(kFull, t2, off);
-        const double hi = fmax(t1, o1);
-        const double lo = fmax(fmin(t1, o1), fmax(t2, o2));
-        t1 = hi;
-        t2 = lo;
-      }
-      gs[g] = t1 + t2;
-    }
-    uint32_t keep = 0;
-    double min_kept = INFINITY, max_drop = -INFINITY;
-    for (int g = 0; g < a.G; ++g) {
-      int better = 0;
-      for (int h = 0; h < a.G; ++h) better += (gs[h] > gs[g]) || (gs[h] == gs[g] && h < g);
-      if (better < a.topk_group) {
-        keep |= 1u << g;
-        min_kept = fmin(min_kept, gs[g]);
-      } else {
-        max_drop = fmax(max_drop, gs[g]);
-      }
-    }
-    if (check && a.topk_group < a.G && !(min_kept - max_drop > 4.0 * delta_v)) ok = false;
+// Group limit with per-expert uncertainty (bit j of `exact`: value is binary64;
+// otherwise it may be off by delta_v). Sets *elig (bits over j) to the experts
+// of the kept groups. Returns false when the group cut is not certain, with the
+// inexact experts that could decide it in *mark. An expert can be in its group's
+// true top two only if v >= (second largest v) - 2 delta_v; once all of those
+// are exact the group score is exact.
+template <int EPL>
+__device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
+                              double delta_v, uint32_t* elig, uint32_t* mark) {
+  const int lane = threadIdx.x & 31;
+  const int per = a.E / a.G;
+  double gs[kMaxGroups], gu[kMaxGroups], t2s[kMaxGroups];
+  for (int g = 0; g < a.G; ++g) {
+    double t1 = -INFINITY, t2 = -INFINITY;
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = lane + 32 * j;
-      elig[j] = valid[j] && ((keep >> (e / per)) & 1u);
+      if (valid[j] && e / per == g) {
+        if (v[j] > t1) {
+          t2 = t1;
+          t1 = v[j];
+        } else if (v[j] > t2) {
+          t2 = v[j];
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const double o1 = __shfl_xor_sync(kFull, t1, off);
+      const double o2 = __shfl_xor_sync(kFull, t2, off);
+      const double hi = fmax(t1, o1);
+      const double lo = fmax(fmin(t1, o1), fmax(t2, o2));
+      t1 = hi;
+      t2 = lo;
+    }
+    bool inexact_cand = false;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      if (valid[j] && e / per == g && !((exact >> j) & 1u) && v[j] >= t2 - 2.0 * delta_v) inexact_cand = true;
+    }
+    gs[g] = t1 + t2;
+    gu[g] = __any_sync(kFull, inexact_cand) ? 2.0 * delta_v : 0.0;
+    t2s[g] = t2;
+  }
+  uint32_t keep = 0;
+  double min_kept = INFINITY, max_drop = -INFINITY;
+  for (int g = 0; g < a.G; ++g) {
+    int better = 0;
+    for (int h = 0; h < a.G; ++h) better += (gs[h] > gs[g]) || (gs[h] == gs[g] && h < g);
+    if (better < a.topk_group) {
+      keep |= 1u << g;
+      min_kept = fmin(min_kept, gs[g] - gu[g]);
+    } else {
+      max_drop = fmax(max_drop, gs[g] + gu[g]);
     }
   }
-
-  // Ranked selection by repeated warp arg-max.
-  int n_elig = 0;
+  bool ok = true;
+  uint32_t m = 0;
+  if (a.topk_group < a.G && !(min_kept > max_drop)) {
+    uint32_t involved = 0;
+    for (int g = 0; g < a.G; ++g) {
+      const bool kept = (keep >> g) & 1u;
+      if (gu[g] > 0.0 && (kept ? gs[g] - gu[g] <= max_drop : gs[g] + gu[g] >= min_kept)) involved |= 1u << g;
+    }
+    if (involved) {
+      ok = false;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) n_elig += elig[j];
+      for (int j = 0; j < EPL; ++j) {
+        const int e = lane + 32 * j;
+        if (valid[j] && ((involved >> (e / per)) & 1u) && !((exact >> j) & 1u) && v[j] >= t2s[e / per] - 2.0 * delta_v)
+          m |= 1u << j;
+      }
+    }
+  }
+  uint32_t el = 0;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = lane + 32 * j;
+    if (valid[j] && ((keep >> (e / per)) & 1u)) el |= 1u << j;
+  }
+  *elig = el;
+  *mark = m;
+  return ok;
+}
+
+// Top-k selection of one token with per-expert uncertainty. l[j] is the logit
+// of expert lane + 32j; bit j of `exact` says it is the binary64 value,
+// otherwise it is the binary32 GEMM result whose selection value may be off by
+// up to delta_v. Writes the k kept experts to rank[0..k). Returns true when
+// every comparison the decision depends on is certain: strictly separated
+// intervals, or both sides exact (exact ties then follow the index rule).
+// Otherwise sets, in *refine, the inexact experts an uncertain comparison involves.
+template <int EPL>
+__device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exact, double delta_v, int16_t* rank,
+                       int* n_ranked, uint32_t* refine) {
+  const int lane = threadIdx.x & 31;
+  double v[EPL];
+  bool valid[EPL];
+  selection_values<EPL>(a, l, v, valid);
+  auto unc = [&](int j) { return ((exact >> j) & 1u) ? 0.0 : delta_v; };
+  bool ok = true;
+  uint32_t mark = 0;
+  uint32_t elig_mask = 0;
+  if (a.G > 1) {
+    if (!decide_groups<EPL>(a, v, valid, exact, delta_v, &elig_mask, &mark)) ok = false;
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (valid[j]) elig_mask |= 1u << j;
+  }
+  int n_elig = __popc(elig_mask);
 #pragma unroll
   for (int off = 16; off; off >>= 1) n_elig += __shfl_xor_sync(kFull, n_elig, off);
-  const int want = full_ranking ? n_elig : min(n_elig, check ? a.k + 1 : a.k);
+  const int want = min(n_elig, a.k);
   uint32_t taken = 0;
-  double prev = 0.0;
+  double prev_lo = 0.0;
+  int prev_e = -1;
+  bool prev_exact = true;
+  double top_lo = INFINITY;  // min over the kept experts of v - u
   for (int r = 0; r < want; ++r) {
     VE best{-INFINITY, 0x7FFFFFFF};
 #pragma unroll
     for (int j = 0; j < EPL; ++j) {
       const int e = lane + 32 * j;
-      if (elig[j] && !((taken >> j) & 1u) && (v[j] > best.v || (v[j] == best.v && e < best.e))) {
+      if (((elig_mask & ~taken) >> j) & 1u && (v[j] > best.v || (v[j] == best.v && e < best.e))) {
         best.v = v[j];
         best.e = e;
       }
     }
     best = warp_best(best);
-    if ((best.e & 31) == lane) taken |= 1u << (best.e >> 5);
-    if (check && r > 0 && (full_ranking || r <= a.k) && !(prev - best.v > 2.0 * delta_v)) ok = false;
-    prev = best.v;
-    if (lane == 0 && (full_ranking || r < a.k)) rank[r] = (int16_t)best.e;
+    const int owner = best.e & 31, jb = best.e >> 5;
+    const bool b_exact = __shfl_sync(kFull, (int)((exact >> jb) & 1u), owner) != 0;
+    const double bu = b_exact ? 0.0 : delta_v;
+    if (lane == owner) taken |= 1u << jb;
+    if (r > 0 && !(prev_exact && b_exact) && !(prev_lo > best.v + bu)) {
+      // adjacent order not certain: refine whichever of the two is inexact
+      ok = false;
+      if (!prev_exact && (prev_e & 31) == lane) mark |= 1u << (prev_e >> 5);
+      if (!b_exact && lane == owner) mark |= 1u << jb;
+    }
+    prev_lo = best.v - bu;
+    prev_e = best.e;
+    prev_exact = b_exact;
+    top_lo = fmin(top_lo, best.v - bu);
+    if (lane == 0) rank[r] = (int16_t)best.e;
   }
-  *n_ranked = full_ranking ? n_elig : min(n_elig, a.k);
+  if (want < n_elig) {
+    // The cut between the k kept experts and every eligible expert below them.
+    double below_hi = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (((elig_mask & ~taken) >> j) & 1u) below_hi = fmax(below_hi, v[j] + unc(j));
+    below_hi = warp_max(below_hi);
+    if (!(top_lo > below_hi)) {
+      bool any = false;
+#pragma unroll
+      for (int j = 0; j < EPL; ++j) {
+        if (!((elig_mask >> j) & 1u) || ((exact >> j) & 1u)) continue;
+        const bool mine = (taken >> j) & 1u;
+        if (mine ? v[j] - delta_v <= below_hi : v[j] + delta_v >= top_lo) {
+          mark |= 1u << j;
+          any = true;
+        }
+      }
+      if (__any_sync(kFull, any)) ok = false;
+    }
+  }
+  *n_ranked = want;
+  *refine = mark;
   __syncwarp();
+  return ok;
+}
+
+// Key order of the ranking: larger value first, then lower expert index.
+__device__ __forceinline__ bool better(double va, int ea, double vb, int eb) {
+  return va > vb || (va == vb && ea < eb);
+}
+
+// Full ranking of one token's eligible experts (the capacity rule needs it),
+// by a bitonic sort across the warp: position p = lane * EPL + j. Each element
+// carries its expert index and exactness. After the sort, adjacent pairs are
+// certified like the top-k pairs; uncertain inexact experts are flagged in
+// `flags` (per-warp shared, one byte per expert) and returned in *refine.
+template <int EPL>
+__device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t exact, double delta_v,
+                            int16_t* rank, uint8_t* flags, int* n_ranked, uint32_t* refine) {
+  const int lane = threadIdx.x & 31;
+  const int E = a.E;
+  double v0[EPL];
+  bool valid[EPL];
+  selection_values<EPL>(a, l, v0, valid);
+  uint32_t elig_mask = 0;
+  bool ok = true;
+  uint32_t mark = 0;
+  if (a.G > 1) {
+    if (!decide_groups<EPL>(a, v0, valid, exact, delta_v, &elig_mask, &mark)) ok = false;
+  } else {
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (valid[j]) elig_mask |= 1u << j;
+  }
+  // keys in sort layout: lane holds positions lane*EPL .. lane*EPL+EPL-1
+  double kv[EPL];
+  int ke[EPL];  // expert | exact << 16, or -1 for empty
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int e = lane + 32 * j;
+    const bool el = (elig_mask >> j) & 1u;
+    kv[j] = el ? v0[j] : -INFINITY;
+    ke[j] = el ? (e | (int)(((exact >> j) & 1u) << 16)) : (0x7FFF | (1 << 16));
+  }
+  constexpr int S = 32 * EPL;
+#pragma unroll
+  for (int k = 2; k <= S; k <<= 1) {
+#pragma unroll
+    for (int d = k >> 1; d > 0; d >>= 1) {
+      if (d < EPL) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          const int jp = j ^ d;
+          if (jp > j) {
+            const int p = lane * EPL + j;
+            const bool up = (p & k) == 0;  // block sorted best-first
+            const bool swap = up ? better(kv[jp], ke[jp] & 0xFFFF, kv[j], ke[j] & 0xFFFF)
+                                 : better(kv[j], ke[j] & 0xFFFF, kv[jp], ke[jp] & 0xFFFF);
+            if (swap) {
+              const double tv = kv[j];
+              kv[j] = kv[jp];
+              kv[jp] = tv;
+              const int te = ke[j];
+              ke[j] = ke[jp];
+              ke[jp] = te;
+            }
+          }
+        }
+      } else {
+        const int ld = d / EPL;
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) {
+          const double ov = __shfl_xor_sync(kFull, kv[j], ld);
+          const int oe = __shfl_xor_sync(kFull, ke[j], ld);
+          const int p = lane * EPL + j;
+          const bool up = (p & k) == 0;
+          const bool lower = (lane & ld) == 0;  // this element sits at the smaller position
+          const bool other_better = better(ov, oe & 0xFFFF, kv[j], ke[j] & 0xFFFF);
+          // the smaller position keeps the better key in an ascending block
+          const bool take = (lower == up) ? other_better : !other_better;
+          if (take) {
+            kv[j] = ov;
+            ke[j] = oe;
+          }
+        }
+      }
+    }
+  }
+  int n_elig = __popc(elig_mask);
+#pragma unroll
+  for (int off = 16; off; off >>= 1) n_elig += __shfl_xor_sync(kFull, n_elig, off);
+  // certify adjacent pairs (p, p+1) inside the eligible prefix
+  const double nxt_v = __shfl_down_sync(kFull, kv[0], 1);
+  const int nxt_e = __shfl_down_sync(kFull, ke[0], 1);
+  bool any_flag = false;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int p = lane * EPL + j;
+    if (p + 1 >= n_elig) continue;
+    const double vb = (j + 1 < EPL) ? kv[(j + 1) % EPL] : nxt_v;
+    const int eb = (j + 1 < EPL) ? ke[(j + 1) % EPL] : nxt_e;
+    const bool ea_exact = (ke[j] >> 16) & 1, eb_exact = (eb >> 16) & 1;
+    const double ua = ea_exact ? 0.0 : delta_v, ub = eb_exact ? 0.0 : delta_v;
+    if (!(ea_exact && eb_exact) && !(kv[j] - ua > vb + ub)) {
+      if (!ea_exact) flags[ke[j] & 0xFFFF] = 1;
+      if (!eb_exact) flags[eb & 0xFFFF] = 1;
+      any_flag = true;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const int p = lane * EPL + j;
+    if (p < n_elig) rank[p] = (int16_t)(ke[j] & 0xFFFF);
+  }
+  if (__any_sync(kFull, any_flag)) {
+    ok = false;
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < EPL; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E && flags[e]) {
+        mark |= 1u << j;
+        flags[e] = 0;
+      }
+    }
+  }
+  __syncwarp();
+  *n_ranked = n_elig;
+  *refine = mark;
   return ok;
 }
 
@@ -222,64 +423,115 @@ __device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* id
   return (float)(mine / denom * (double)a.rsf);
 }
 
+// Binary64 dot product x[t] . W_r[e], computed by the whole warp: lanes take
+// 16-byte chunks of the row in turn (coalesced), then a butterfly sum.
+__device__ double dot64(const RouteArgs& a, int64_t t, int e) {
+  const int lane = threadIdx.x & 31;
+  double acc0 = 0.0, acc1 = 0.0;
+  if (a.dtype == MOE_BF16) {
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.x) + t * a.d);
+    const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.w_r) + (int64_t)e * a.d);
+    for (int i = lane; i < a.d / 8; i += 32) {
+      const uint4 xv = __ldg(xr + i), wv = __ldg(wr + i);
+      const bf16* xs = reinterpret_cast<const bf16*>(&xv);
+      const bf16* ws = reinterpret_cast<const bf16*>(&wv);
+#pragma unroll
+      for (int q = 0; q < 8; q += 2) {
+        acc0 = fma(to_f64(xs[q]), to_f64(ws[q]), acc0);
+        acc1 = fma(to_f64(xs[q + 1]), to_f64(ws[q + 1]), acc1);
+      }
+    }
+  } else {
+    const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + t * a.d);
+    const float4* wr = reinterpret_cast<const float4*>(static_cast<const float*>(a.w_r) + (int64_t)e * a.d);
+    for (int i = lane; i < a.d / 4; i += 32) {
+      const float4 xv = __ldg(xr + i), wv = __ldg(wr + i);
+      acc0 = fma((double)xv.x, (double)wv.x, acc0);
+      acc1 = fma((double)xv.y, (double)wv.y, acc1);
+      acc0 = fma((double)xv.z, (double)wv.z, acc0);
+      acc1 = fma((double)xv.w, (double)wv.w, acc1);
+    }
+  }
+  return warp_sum(acc0 + acc1);
+}
+
+// Replace the logits of the experts in `which` (bits over j, per lane) by binary64 values.
 template <int EPL>
-__device__ void refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL]) {
+__device__ void refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], uint32_t which) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    uint32_t m = __ballot_sync(kFull, (which >> j) & 1u);
+    while (m) {
+      const int src = __ffs(m) - 1;
+      m &= m - 1;
+      const double s = dot64(a, t, src + 32 * j);
+      if (lane == src) l[j] = s;
+    }
+  }
+}
+
+// Load a token's logits, summing the split-K partial GEMM results in order.
+template <int EPL>
+__device__ __forceinline__ void load_logits(const RouteArgs& a, int64_t t, double (&l)[EPL]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = lane + 32 * j;
-    double acc = 0.0;
-    if (e < a.E) {
-      if (a.dtype == MOE_BF16) {
-        const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.x) + t * a.d);
-        const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.w_r) + (int64_t)e * a.d);
-        for (int i = 0; i < a.d / 8; ++i) {
-          const uint4 xv = xr[i], wv = __ldg(wr + i);
-          const bf16* xs = reinterpret_cast<const bf16*>(&xv);
-          const bf16* ws = reinterpret_cast<const bf16*>(&wv);
-#pragma unroll
-          for (int q = 0; q < 8; ++q) acc = fma(to_f64(xs[q]), to_f64(ws[q]), acc);
-        }
-      } else {
-        const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + t * a.d);
-        const float4* wr = reinterpret_cast<const float4*>(static_cast<const float*>(a.w_r) + (int64_t)e * a.d);
-        for (int i = 0; i < a.d / 4; ++i) {
-          const float4 xv = xr[i], wv = __ldg(wr + i);
-          acc = fma((double)xv.x, (double)wv.x, acc);
-          acc = fma((double)xv.y, (double)wv.y, acc);
-          acc = fma((double)xv.z, (double)wv.z, acc);
-          acc = fma((double)xv.w, (double)wv.w, acc);
-        }
-      }
-    }
-    l[j] = acc;
+    double s = 0.0;
+    if (e < a.E)
+      for (int p = 0; p < a.splits; ++p) s += (double)a.logits[(int64_t)p * a.split_stride + t * a.E + e];
+    l[j] = s;
   }
 }
 
-template <int EPL>
+template <int EPL, bool FULL>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a) {
   __shared__ int16_t s_rank[kWarpsPerBlock][kMaxExperts];
+  __shared__ uint8_t s_flag[kWarpsPerBlock][kMaxExperts];
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  const bool full_ranking = a.ranking != nullptr;
+  constexpr bool full_ranking = FULL;  // the capacity rule needs every eligible expert ranked
+  for (int i = lane; i < kMaxExperts; i += 32) s_flag[wib][i] = 0;
+  __syncwarp();
+  uint32_t valid_mask = 0;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j)
+    if (lane + 32 * j < a.E) valid_mask |= 1u << j;
   for (int64_t t = warp; t < a.n; t += nwarps) {
     double l[EPL];
+    load_logits<EPL>(a, t, l);
+    double amax = 0.0;
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      l[j] = e < a.E ? (double)a.logits[t * a.E + e] : 0.0;
-    }
+    for (int j = 0; j < EPL; ++j)
+      if ((valid_mask >> j) & 1u) amax = fmax(amax, fabs(l[j]));
+    amax = warp_max(amax);
+    // binary32 error bound of the logits, mapped to selection values (sigmoid' <= 1/4)
+    const double delta_l = ldexp(fmax(1.0, amax), -13);
+    const double delta_v = a.score_fn == MOE_SCORE_SIGMOID ? 0.25 * delta_l : delta_l;
+    uint32_t exact = 0;
     int nr = 0;
-    bool ok = decide<EPL>(a, l, true, full_ranking, s_rank[wib], &nr);
-    if (!ok) {
-      refine_logits<EPL>(a, t, l);
-      decide<EPL>(a, l, false, full_ranking, s_rank[wib], &nr);
-      if (lane == 0 && a.diag) atomicAdd(&a.diag->refined_tokens, 1);
+    bool refined = false;
+    for (int it = 0;; ++it) {
+      uint32_t refine = 0;
+      bool ok;
+      if constexpr (FULL)
+        ok = decide_full<EPL>(a, l, exact, delta_v, s_rank[wib], s_flag[wib], &nr, &refine);
+      else
+        ok = decide<EPL>(a, l, exact, delta_v, s_rank[wib], &nr, &refine);
+      if (ok) break;
+      refine &= ~exact;
+      if (it >= 3 || !__any_sync(kFull, refine != 0)) refine = valid_mask & ~exact;  // refine the rest
+      refine_logits<EPL>(a, t, l, refine);
+      exact |= refine;
+      refined = true;
     }
+    if (refined && lane == 0 && a.diag) atomicAdd(&a.diag->refined_tokens, 1);
     if (full_ranking) {
       for (int r = lane; r < a.E; r += 32) a.ranking[t * a.E + r] = r < nr ? (uint16_t)s_rank[wib][r] : (uint16_t)0xFFFF;
+      __syncwarp();
       continue;
     }
     if (lane < a.k) s_idx[wib][lane] = lane < nr ? (int)s_rank[wib][lane] : -1;
@@ -293,7 +545,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
   }
 }
 
-// Gates of an existing selection (after the capacity rule), from binary32 logits.
+// Gates of an existing selection (after the capacity rule), from the binary32 logits.
 template <int EPL>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a) {
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
@@ -302,11 +554,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a)
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t t = warp; t < a.n; t += nwarps) {
     double l[EPL];
-#pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      l[j] = e < a.E ? (double)a.logits[t * a.E + e] : 0.0;
-    }
+    load_logits<EPL>(a, t, l);
     if (lane < a.k) s_idx[wib][lane] = a.topk_idx[t * a.k + lane];
     __syncwarp();
     const float w = gates<EPL>(a, l, s_idx[wib]);
@@ -323,10 +571,12 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a)
 // commits the chunk up to that token, marks the filled experts and continues
 // after it. There are at most E fill events.
 constexpr int kCapThreads = 1024;
+constexpr int kCapPrefix = 64;  // ranking entries per token staged in shared memory
 
 __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k,
                                                             int64_t C, int policy, int32_t* topk_idx,
                                                             moe_diag* diag) {
+  extern __shared__ __align__(16) uint16_t st[];  // [kCapThreads][P] staged ranking prefixes
   __shared__ int cnt[kMaxExperts];
   __shared__ int ccnt[kMaxExperts];
   __shared__ uint32_t full[kMaxExperts / 32];
@@ -336,6 +586,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
   __shared__ int stop;
   __shared__ unsigned long long s_over, s_drop;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  const int P = E < kCapPrefix ? E : kCapPrefix;
   for (int e = tid; e < kMaxExperts; e += kCapThreads) cnt[e] = 0;
   if (tid < kMaxExperts / 32) full[tid] = 0;
   if (tid == 0) s_over = s_drop = 0;
@@ -343,17 +594,31 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
   unsigned long long my_over = 0, my_drop = 0;
   int64_t base = 0;
   while (base < n) {
+    // stage the window's ranking prefixes (coalesced 16-byte copies when rows allow it)
+    const int cnt_tok = (int)((n - base) < kCapThreads ? (n - base) : kCapThreads);
+    if (E % 8 == 0) {
+      const int vpr = P / 8;  // 16-byte vectors per staged row
+      for (int i = tid; i < cnt_tok * vpr; i += kCapThreads) {
+        const int row = i / vpr, v = i % vpr;
+        reinterpret_cast<uint4*>(st)[row * vpr + v] =
+            reinterpret_cast<const uint4*>(ranking + (base + row) * E)[v];
+      }
+    } else {
+      for (int i = tid; i < cnt_tok * P; i += kCapThreads) st[i] = ranking[(base + i / P) * E + i % P];
+    }
+    __syncthreads();
     const int64_t t = base + tid;
-    const bool valid = t < n;
+    const bool valid = tid < cnt_tok;
     int ch[kMaxTopK];
     int over = 0;
     for (int j = 0; j < k; ++j) ch[j] = -1;
     if (valid) {
-      const uint16_t* rk = ranking + t * E;
+      const uint16_t* srow = st + tid * P;
+      const uint16_t* grow = ranking + t * E;
       if (policy == MOE_CAP_OVERFLOW_NEXT) {
         int taken = 0;
         for (int r = 0; r < E && taken < k; ++r) {
-          const int e = rk[r];
+          const int e = r < P ? srow[r] : grow[r];
           if (e == 0xFFFF) break;
           if (!((full[e >> 5] >> (e & 31)) & 1u)) {
             ch[taken++] = e;
@@ -362,7 +627,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
         }
       } else {
         for (int j = 0; j < k; ++j) {
-          const int e = rk[j];
+          const int e = j < P ? srow[j] : grow[j];
           ch[j] = (e != 0xFFFF && !((full[e >> 5] >> (e & 31)) & 1u)) ? e : -1;
         }
       }
@@ -449,11 +714,12 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   if (a.n <= 0) return cudaSuccess;
   const unsigned grid = route_grid(a.n);
   const unsigned block = 32 * kWarpsPerBlock;
+  const bool full = a.ranking != nullptr;
   switch (epl_for(a.E)) {
-    case 1: route_kernel<1><<<grid, block, 0, s>>>(a); break;
-    case 2: route_kernel<2><<<grid, block, 0, s>>>(a); break;
-    case 4: route_kernel<4><<<grid, block, 0, s>>>(a); break;
-    default: route_kernel<8><<<grid, block, 0, s>>>(a); break;
+    case 1: full ? route_kernel<1, true><<<grid, block, 0, s>>>(a) : route_kernel<1, false><<<grid, block, 0, s>>>(a); break;
+    case 2: full ? route_kernel<2, true><<<grid, block, 0, s>>>(a) : route_kernel<2, false><<<grid, block, 0, s>>>(a); break;
+    case 4: full ? route_kernel<4, true><<<grid, block, 0, s>>>(a) : route_kernel<4, false><<<grid, block, 0, s>>>(a); break;
+    default: full ? route_kernel<8, true><<<grid, block, 0, s>>>(a) : route_kernel<8, false><<<grid, block, 0, s>>>(a); break;
   }
   return cudaGetLastError();
 }
@@ -474,7 +740,16 @@ cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s) {
 cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32_t k, int64_t C, int policy,
                             int32_t* topk_idx, moe_diag* diag, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
-  capacity_kernel<<<1, kCapThreads, 0, s>>>(ranking, n, E, k, C, policy, topk_idx, diag);
+  const int P = E < kCapPrefix ? E : kCapPrefix;
+  const size_t smem = (size_t)kCapThreads * P * sizeof(uint16_t);
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(capacity_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kCapThreads * kCapPrefix * 2));
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  capacity_kernel<<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag);
   return cudaGetLastError();
 }
 
