@@ -310,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
         const int kb0 = tl.split * p.kb_per, kb1 = min(num_kb_all, kb0 + p.kb_per);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+          if (!mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
+              !mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
             ok = false;
             break;
           }
@@ -359,11 +360,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN_MAX);
         for (int kb = 0; kb < nkb; ++kb) {
-          if (!mbar_wait(&ctl->full[stage], phase, ctl, p.status)) {
+          // The copies completed on this barrier; the MMAs read them through the
+          // async proxy as well, so no tcgen05 fence is needed here.
+          if (!mbar_try(smem_u32(&ctl->full[stage]), phase) && !mbar_wait(&ctl->full[stage], phase, ctl, p.status)) {
             ok = false;
             break;
           }
-          fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint64_t adesc = sw128_kmajor_desc(sa);
           const uint64_t bdesc = sw128_kmajor_desc(sa + A_BYTES);
@@ -624,7 +626,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int brow = p.swiglu ? tl.g * p.b_rows + tl.nt * p.n_out
                                   : tl.g * p.b_rows + tl.nt * p.n_out + (int)rank * 128;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait2(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+          if (!mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
+              !mbar_wait2(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
             aborted = true;
             break;
           }
@@ -658,11 +661,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN_MAX);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait2(&ctl->full[stage], phase, ctl, p.status)) {
+          if (!mbar_try(smem_u32(&ctl->full[stage]), phase) && !mbar_wait2(&ctl->full[stage], phase, ctl, p.status)) {
             aborted = true;
             break;
           }
-          fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
           const uint64_t adesc = sw128_kmajor_desc(sa);
           const uint64_t bdesc = sw128_kmajor_desc(sa + A2_BYTES);
