@@ -43,7 +43,8 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int kThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kMaxGroupsTc = 256;
-constexpr uint64_t kTimeoutNs = 2000000000ull;  // 2 s for any single wait
+constexpr uint64_t kTimeoutNs = 2000000000ull;      // 2 s for any single wait
+constexpr uint64_t kTestTimeoutNs = 50000000ull;    // 50 ms under injected stalls
 constexpr uint64_t kDrainNs = 200000000ull;     // 0.2 s per drain wait after an abort
 
 struct TcParams {
@@ -63,9 +64,12 @@ struct TcParams {
   int64_t ldc;
   int64_t c_split_stride;
   moe_diag* status;
+  uint64_t timeout_ns;  // limit of any single barrier wait
+  int32_t test_stall;   // fault injection: withhold the first copy of each CTA
 };
 
 struct __align__(8) SmemCtl {
+  uint64_t timeout_ns;
   uint64_t full[STAGES];
   uint64_t empty[STAGES];
   uint64_t tmem_full[2];
@@ -115,7 +119,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SmemCtl* 
     if (mbar_try(b, parity)) return true;
     if ((it & 255u) == 0) {
       if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (globaltimer() - t0 > ctl->timeout_ns) {
         atomicExch(&ctl->abort, 1);
         set_status(st, MOE_ERR_TIMEOUT);
         return false;
@@ -265,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->total_tiles = acc;
     ctl->n_tiles = n_tiles;
     ctl->abort = 0;
+    ctl->timeout_ns = p.timeout_ns;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
@@ -317,6 +322,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
           uint8_t* sb = sa + A_BYTES;
+          if (p.test_stall && t == (int)blockIdx.x && kb == kb0) {
+            // injected fault: this stage is never filled, so the MMA's wait on it runs out
+            if (++stage == STAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           mbar_expect_tx(&ctl->full[stage], tx);
           ++armed[stage];
           tma_load_2d(sa, &map_a, &ctl->full[stage], kb * BK, row0);
@@ -456,6 +469,7 @@ constexpr int B2_BYTES = 128 * BK * 2;
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
 
 struct __align__(8) SmemCtl2 {
+  uint64_t timeout_ns;
   uint64_t full[STAGES2];
   uint64_t empty[STAGES2];
   uint64_t tmem_full[2];
@@ -540,7 +554,7 @@ __device__ __noinline__ bool mbar_wait2(uint64_t* bar, uint32_t parity, SmemCtl2
     if (mbar_try(b, parity)) return true;
     if ((it & 255u) == 0) {
       if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
-      if (globaltimer() - t0 > kTimeoutNs) {
+      if (globaltimer() - t0 > ctl->timeout_ns) {
         atomicExch(&ctl->abort, 1);
         set_status(st, MOE_ERR_TIMEOUT);
         return false;
@@ -580,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ctl->total_tiles = acc;
     ctl->n_tiles = n_tiles;
     ctl->abort = 0;
+    ctl->timeout_ns = p.timeout_ns;
     for (int s = 0; s < STAGES2; ++s) {
       mbar_init(&ctl->full[s], 1);
       mbar_init(&ctl->empty[s], 1);
@@ -632,6 +647,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* sa = smem + stage * STAGE2_BYTES;
+          if (p.test_stall && t == pair && kb == 0) {
+            // injected fault: this stage is never filled, so the MMA's wait on it runs out
+            if (++stage == STAGES2) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           const uint32_t leader_full = map_to_rank(&ctl->full[stage], 0);
           if (rank == 0) mbar_expect_tx(&ctl->full[stage], tx);
           tma_load_2d_pair(sa, &map_a, leader_full, kb * BK, row0);
@@ -850,6 +873,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   p.ldc = a.ldc;
   p.c_split_stride = a.c_split_stride;
   p.status = status;
+  // MOE_TEST_STALL=1 injects a stalled pipeline stage to exercise the bounded
+  // waits and the MOE_ERR_TIMEOUT status path (fault injection for tests).
+  const char* stall = getenv("MOE_TEST_STALL");
+  p.test_stall = stall && stall[0] == '1';
+  p.timeout_ns = p.test_stall ? kTestTimeoutNs : kTimeoutNs;
   CUtensorMap ma, mb, mb2;
   const int64_t b_total_rows = (int64_t)a.G * a.N;
   const bool pair = use_pair_tiles(a, swiglu, out_f32);
