@@ -27,9 +27,12 @@
  *   - Pointers named x, w_*, y, topk_*, offsets, perm_token, slot_dest,
  *     x_perm, expert_out, expert_counts, diag and ws are DEVICE pointers
  *     (one GPU); cfg, the moe_weights struct itself and bytes are HOST
- *     pointers. The caller owns all memory; the library allocates nothing
- *     and keeps no state between calls. Scratch space comes only from the
- *     workspace ws of at least moe_workspace_size() bytes.
+ *     pointers. The caller owns all memory; the library allocates no device
+ *     memory and keeps no data between calls. Scratch space comes only from
+ *     the workspace ws of at least moe_workspace_size() bytes. The one
+ *     runtime resource it keeps is, per device, a non-blocking stream and two
+ *     events created on the first moe_layer_forward with shared experts: the
+ *     shared experts run there, joined back to `stream` before the combine.
  *   - Arrays are dense row-major. Weights use the out x in (nn.Linear)
  *     convention: W_r [E, d]; w_gate, w_up [E, I, d]; w_down [E, d, I];
  *     shared experts concatenated along I: ws_gate, ws_up [n_shared*I, d],

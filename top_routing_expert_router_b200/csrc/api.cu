@@ -4,6 +4,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -241,6 +243,33 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
   return MOE_OK;
 }
 
+// Per-device side stream with fork/join events: the shared experts depend only
+// on x, so their GEMMs run there while routing and dispatch (CUDA-core and HBM
+// bound) run on the caller's stream. Created on first use, kept until exit.
+struct SideStream {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+};
+
+SideStream* side_stream() {
+  constexpr int kMaxDevices = 64;
+  static SideStream table[kMaxDevices];
+  static std::mutex lock;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> g(lock);
+  SideStream& ss = table[dev];
+  if (!ss.s) {
+    if (cudaStreamCreateWithFlags(&ss.s, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+      ss.s = nullptr;
+      return nullptr;
+    }
+  }
+  return &ss;
+}
+
 }  // namespace
 }  // namespace moe
 
@@ -361,12 +390,25 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
   int32_t* dest = c.at<int32_t>(c.p.dest);
   void* xperm = c.ws + c.p.xperm;
   void* eo = c.ws + c.p.eo;
+  // Shared experts first, on the side stream, overlapping routing and dispatch.
+  void* sh = nullptr;
+  SideStream* side = (n > 0 && c.c.n_shared > 0) ? side_stream() : nullptr;
+  if (side) {
+    MOE_CUDA(cudaEventRecord(side->fork, c.s));
+    MOE_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    Ctx cs = c;
+    cs.s = side->s;
+    MOE_TRY(shared_impl(cs, x, weights, &sh));
+    MOE_CUDA(cudaEventRecord(side->join, side->s));
+  }
   MOE_TRY(route_impl(c, x, weights, idx, tw, counts, diag_opt));
   if (n == 0) return MOE_OK;
   MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm));
   MOE_TRY(ffn_impl(c, xperm, offsets, weights, eo));
-  void* sh = nullptr;
-  MOE_TRY(shared_impl(c, x, weights, &sh));
+  if (side)
+    MOE_CUDA(cudaStreamWaitEvent(c.s, side->join, 0));
+  else
+    MOE_TRY(shared_impl(c, x, weights, &sh));
   return cuda_status(launch_combine(eo, dest, tw, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
 }
 

@@ -431,6 +431,7 @@ __device__ double dot64(const RouteArgs& a, int64_t t, int e) {
   if (a.dtype == MOE_BF16) {
     const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.x) + t * a.d);
     const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.w_r) + (int64_t)e * a.d);
+#pragma unroll 4
     for (int i = lane; i < a.d / 8; i += 32) {
       const uint4 xv = __ldg(xr + i), wv = __ldg(wr + i);
       const bf16* xs = reinterpret_cast<const bf16*>(&xv);
@@ -444,6 +445,7 @@ __device__ double dot64(const RouteArgs& a, int64_t t, int e) {
   } else {
     const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + t * a.d);
     const float4* wr = reinterpret_cast<const float4*>(static_cast<const float*>(a.w_r) + (int64_t)e * a.d);
+#pragma unroll 4
     for (int i = lane; i < a.d / 4; i += 32) {
       const float4 xv = __ldg(xr + i), wv = __ldg(wr + i);
       acc0 = fma((double)xv.x, (double)wv.x, acc0);
@@ -573,6 +575,14 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a)
 constexpr int kCapThreads = 1024;
 constexpr int kCapPrefix = 64;  // ranking entries per token staged in shared memory
 
+// counts[e] += 1 for every lane whose slot holds e (e < 0: nothing), one
+// shared-memory atomic per distinct expert in the warp: popular experts would
+// otherwise serialise hundreds of atomics on one address.
+__device__ __forceinline__ void warp_count(int* counts, int e) {
+  const unsigned peers = __match_any_sync(kFull, e);
+  if (e >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&counts[e], __popc(peers));
+}
+
 __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k,
                                                             int64_t C, int policy, int32_t* topk_idx,
                                                             moe_diag* diag) {
@@ -638,9 +648,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
       stop = kCapThreads;
     }
     __syncthreads();
-    if (valid)
-      for (int j = 0; j < k; ++j)
-        if (ch[j] >= 0) atomicAdd(&ccnt[ch[j]], 1);
+    for (int j = 0; j < k; ++j) warp_count(ccnt, valid ? ch[j] : -1);
     __syncthreads();
     for (int e = tid; e < E; e += kCapThreads)
       if (cnt[e] < C && cnt[e] + ccnt[e] >= C) cand[atomicAdd(&n_cand, 1)] = e;
@@ -680,9 +688,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
     if (s < kCapThreads) {
       for (int e = tid; e < E; e += kCapThreads) ccnt[e] = 0;
       __syncthreads();
-      if (commit)
-        for (int j = 0; j < k; ++j)
-          if (ch[j] >= 0) atomicAdd(&ccnt[ch[j]], 1);
+      for (int j = 0; j < k; ++j) warp_count(ccnt, commit ? ch[j] : -1);
       __syncthreads();
     }
     for (int e = tid; e < E; e += kCapThreads) {
