@@ -41,6 +41,15 @@ static int near_tie(double a, double b) {
 
 static double sigmoid(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+/* sqrt(softplus(z)), softplus(z) = log(1 + e^z) written without overflow. */
+static double sqrtsoftplus(double z) {
+  double sp = (z > 0 ? z : 0.0) + log1p(exp(-fabs(z)));
+  return sqrt(sp);
+}
+
+/* Raw score of the biased-score routers: sigmoid ([DS] V3) or sqrtsoftplus ([DS] V4). */
+static double raw_score(int32_t score_fn, double z) { return score_fn == 2 ? sqrtsoftplus(z) : sigmoid(z); }
+
 /* ---- router logits ([DS] router listing; [MoE] 3.1 linear router) --------- */
 
 void oracle_router_logits(int64_t n, int32_t d, int32_t E, const void* x, int32_t x_dt,
@@ -84,8 +93,8 @@ static int32_t token_ranking(const oracle_cfg* cfg, const double* l, const float
                              int32_t* rank, int* exempt) {
   const int32_t E = cfg->n_routed;
   for (int32_t e = 0; e < E; ++e) {
-    if (cfg->score_fn == 1)
-      v[e] = sigmoid(l[e]) + (bias ? (double)bias[e] : 0.0);
+    if (cfg->score_fn != 0)
+      v[e] = raw_score(cfg->score_fn, l[e]) + (bias ? (double)bias[e] : 0.0);
     else
       v[e] = l[e];
   }
@@ -140,8 +149,8 @@ static void token_gates(const oracle_cfg* cfg, const double* l, const int32_t* i
   const int32_t E = cfg->n_routed, k = cfg->top_k;
   double denom = 1.0;
   double* p = (double*)malloc(sizeof(double) * (size_t)E);
-  if (cfg->score_fn == 1) {
-    for (int32_t e = 0; e < E; ++e) p[e] = sigmoid(l[e]);
+  if (cfg->score_fn != 0) {
+    for (int32_t e = 0; e < E; ++e) p[e] = raw_score(cfg->score_fn, l[e]);
   } else {
     double mx = -INFINITY, z = 0.0;
     for (int32_t e = 0; e < E; ++e) mx = l[e] > mx ? l[e] : mx;
@@ -284,6 +293,39 @@ void oracle_route_capacity(const oracle_cfg* cfg, int64_t n, const double* logit
   free(vals);
   free(group_exempt);
   free(ranking);
+}
+
+/*
+ * Hash routing ([DS] section V4: the first layers choose experts by a fixed
+ * table indexed by token id; the router only weights the chosen experts).
+ * topk_idx[t, j] = tid2eid[token_id[t], j]; gates as token_gates().
+ */
+void oracle_route_hash(const oracle_cfg* cfg, int64_t n, const double* logits, const int32_t* token_ids,
+                       const int32_t* tid2eid, int32_t* topk_idx, double* topk_w) {
+  const int32_t E = cfg->n_routed, k = cfg->top_k;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < n; ++t) {
+    for (int32_t j = 0; j < k; ++j) topk_idx[t * k + j] = tid2eid[(int64_t)token_ids[t] * k + j];
+    token_gates(cfg, logits + t * (int64_t)E, topk_idx + t * k, topk_w + t * k);
+  }
+}
+
+/*
+ * Auxiliary-loss-free balancing step ([DS] V3: after each step the bias of an
+ * over-loaded expert is decreased by gamma and that of an under-loaded one
+ * increased by gamma). Load is compared with the mean load sum(counts) / E;
+ * an expert exactly at the mean keeps its bias.
+ */
+void oracle_bias_update(int32_t E, const int32_t* counts, const float* bias, double gamma, double* out) {
+  double total = 0.0;
+  for (int32_t e = 0; e < E; ++e) total += counts[e];
+  const double mean = total / E;
+  for (int32_t e = 0; e < E; ++e) {
+    double b = (double)bias[e];
+    if (counts[e] > mean) b -= gamma;
+    else if (counts[e] < mean) b += gamma;
+    out[e] = b;
+  }
 }
 
 /* ---- dispatch: histogram, exclusive scan, stable permutation -------------- */

@@ -13,6 +13,8 @@
  *         gate weights, routed_scaling_factor, shared expert) and section
  *         "671B and 37B parameter ledger" (three matrices per expert).
  *         Section "V2" gives 160 routed + 2 shared experts, top-6, softmax.
+ *         Section "V4": sqrtsoftplus scores with the bias and no group limit;
+ *         hash routing of the first layers through a token-id table.
  *   [MoE] "MoE architecture revealed", section 3.1 (linear router, softmax,
  *         top-k) and section 4.1 (router logits -> softmax -> topk probs).
  *   [1.8T] "1.8T parameters / 2% per token", section 2.2 (expert capacity:
@@ -42,7 +44,7 @@ typedef struct {
   int32_t n_group;       /* expert groups (1 = no group limit)                   */
   int32_t topk_group;    /* groups kept per token                                */
   int32_t inter;         /* I = moe_intermediate_size                            */
-  int32_t score_fn;      /* 0 = softmax, 1 = sigmoid + selection bias            */
+  int32_t score_fn;      /* 0 = softmax, 1 = sigmoid, 2 = sqrtsoftplus (+ bias)  */
   int32_t renormalize;   /* gates normalised over the selected experts           */
   double routed_scaling_factor;
   int32_t cap_policy;    /* 0 = none, 1 = overflow to next-best, 2 = drop        */
@@ -82,6 +84,13 @@ void oracle_route(const oracle_cfg* cfg, int64_t n, const double* logits, const 
 void oracle_route_capacity(const oracle_cfg* cfg, int64_t n, const double* logits,
                            const float* bias, int32_t* topk_idx, double* topk_w, uint8_t* exempt,
                            oracle_stats* stats);
+
+/* Hash routing: topk_idx[t] = tid2eid[token_ids[t]] ([DS] V4), gates from the scores. */
+void oracle_route_hash(const oracle_cfg* cfg, int64_t n, const double* logits, const int32_t* token_ids,
+                       const int32_t* tid2eid, int32_t* topk_idx, double* topk_w);
+
+/* Bias update of the auxiliary-loss-free balancing ([DS] V3): out = bias -/+ gamma. */
+void oracle_bias_update(int32_t E, const int32_t* counts, const float* bias, double gamma, double* out);
 
 /* Capacity C = capacity if > 0, else ceil(capacity_factor * n * k / E). */
 int64_t oracle_capacity_value(const oracle_cfg* cfg, int64_t n);

@@ -87,6 +87,8 @@ def lib():
         _lib.oracle_combine.argtypes = [i64, i32, i32, P, P, P, P, P]
         _lib.oracle_layer.argtypes = [P, i64] + [P] * 9 + [i32] + [P] * 6
         _lib.oracle_ds_params.argtypes = [P, P, P]
+        _lib.oracle_route_hash.argtypes = [P, i64, P, P, P, P, P]
+        _lib.oracle_bias_update.argtypes = [i32, P, P, ctypes.c_double, P]
     return _lib
 
 
@@ -119,7 +121,7 @@ class Cfg:
     n_shared: int = 0
     n_group: int = 1
     topk_group: int = 1
-    score_fn: str = "softmax"  # or "sigmoid"
+    score_fn: str = "softmax"  # or "sigmoid", "sqrtsoftplus"
     renormalize: bool = False
     routed_scaling_factor: float = 1.0
     cap_policy: str = "none"  # "none" | "overflow_next" | "drop"
@@ -135,7 +137,7 @@ class Cfg:
             self.n_group,
             self.topk_group,
             self.moe_intermediate_size,
-            {"softmax": 0, "sigmoid": 1}[self.score_fn],
+            {"softmax": 0, "sigmoid": 1, "sqrtsoftplus": 2}[self.score_fn],
             int(bool(self.renormalize)),
             float(self.routed_scaling_factor),
             {"none": 0, "overflow_next": 1, "drop": 2}[self.cap_policy],
@@ -187,6 +189,27 @@ def route_capacity(cfg: Cfg, logits: np.ndarray, bias=None):
         ctypes.byref(c), n, _ptr(logits), _ptr(bias), _ptr(idx), _ptr(w), _ptr(ex), ctypes.byref(st)
     )
     return idx, w, ex.astype(bool), st
+
+
+def route_hash(cfg: Cfg, logits: np.ndarray, token_ids: np.ndarray, tid2eid: np.ndarray):
+    """Hash routing: (topk_idx, topk_w)."""
+    logits = _c(logits, np.float64)
+    token_ids = _c(token_ids, np.int32)
+    tid2eid = _c(tid2eid, np.int32)
+    n = logits.shape[0]
+    idx = np.empty((n, cfg.top_k), np.int32)
+    w = np.empty((n, cfg.top_k), np.float64)
+    c = cfg.c()
+    lib().oracle_route_hash(ctypes.byref(c), n, _ptr(logits), _ptr(token_ids), _ptr(tid2eid), _ptr(idx), _ptr(w))
+    return idx, w
+
+
+def bias_update(counts: np.ndarray, bias: np.ndarray, gamma: float) -> np.ndarray:
+    counts = _c(counts, np.int32)
+    bias = _c(bias, np.float32)
+    out = np.empty(len(counts), np.float64)
+    lib().oracle_bias_update(len(counts), _ptr(counts), _ptr(bias), gamma, _ptr(out))
+    return out
 
 
 def capacity_value(cfg: Cfg, n: int) -> int:

@@ -451,3 +451,51 @@ def test_layer_composes_route_dispatch_swiglu_combine():
                                                inp["w_down"][e])[0]
     np.testing.assert_allclose(r["y"], ref, rtol=1e-9, atol=1e-10)
     np.testing.assert_array_equal(r["counts"], np.bincount(idx.ravel(), minlength=8))
+
+
+# ---------------------------------------------------------------- V4 routing variants and the bias update
+
+
+def test_sqrtsoftplus_closed_forms():
+    one = lambda l: O.route(_cfg(1, 1, score_fn="sqrtsoftplus"), np.array([[l]]))[1][0, 0]
+    assert one(0.0) == pytest.approx(math.sqrt(math.log(2.0)), rel=1e-15)
+    assert one(30.0) == pytest.approx(math.sqrt(30.0 + math.log1p(math.exp(-30.0))), rel=1e-15)
+    assert one(-30.0) == pytest.approx(math.sqrt(math.log1p(math.exp(-30.0))), rel=1e-12)
+    assert one(2.5) == pytest.approx(math.sqrt(math.log(1.0 + math.exp(2.5))), rel=1e-14)
+
+
+def test_sqrtsoftplus_selection_with_bias_matches_library_sort_and_brute_force():
+    rng = np.random.default_rng(21)
+    E, k = 12, 3
+    lg = rng.standard_normal((300, E)) * 2
+    bias = rng.uniform(-0.1, 0.1, E).astype(np.float32)
+    s = np.sqrt(np.logaddexp(0.0, lg))  # numpy softplus, then sqrt
+    c = s + bias.astype(np.float64)
+    idx, w, _, _, _ = O.route(_cfg(E, k, score_fn="sqrtsoftplus", renormalize=True, routed_scaling_factor=1.5), lg, bias)
+    np.testing.assert_array_equal(idx, _lexsort_topk(c, k))
+    sel = np.take_along_axis(s, idx, 1)
+    np.testing.assert_allclose(w, sel / sel.sum(1, keepdims=True) * 1.5, rtol=1e-13)
+    # with a group limit the same brute force as for sigmoid applies
+    idx2, _, _, _, _ = O.route(_cfg(E, k, score_fn="sqrtsoftplus", n_group=4, topk_group=2), lg, bias)
+    for t in range(60):
+        assert idx2[t].tolist() == _brute_group_topk(c[t], 4, 2, k), t
+
+
+def test_hash_routing_uses_the_table_and_scores_only_weight():
+    rng = np.random.default_rng(22)
+    E, k, vocab, n = 16, 3, 50, 120
+    table = np.stack([rng.permutation(E)[:k] for _ in range(vocab)]).astype(np.int32)
+    tok = rng.integers(0, vocab, n).astype(np.int32)
+    lg = rng.standard_normal((n, E))
+    cfg = _cfg(E, k, score_fn="sqrtsoftplus", renormalize=True, routed_scaling_factor=2.0)
+    idx, w = O.route_hash(cfg, lg, tok, table)
+    np.testing.assert_array_equal(idx, table[tok])
+    s = np.sqrt(np.logaddexp(0.0, lg))
+    sel = np.take_along_axis(s, idx, 1)
+    np.testing.assert_allclose(w, sel / sel.sum(1, keepdims=True) * 2.0, rtol=1e-13)
+
+
+def test_bias_update_worked_example():
+    g = _gold("routing_worked_examples.json")["bias_update"]
+    out = O.bias_update(np.array(g["counts"]), np.array(g["bias"], np.float32), g["gamma"])
+    np.testing.assert_allclose(out, g["expect"], rtol=0, atol=1e-12)
