@@ -22,6 +22,10 @@
  *          logits (renormalised); section 4.2: capacity_factor and
  *          drop_tokens.
  *   [KL]   "MoE" tag feed, section on activation functions: SwiGLU FFN.
+ *   [DS4]  "15. DeepSeek: MLA, MoE and MTP", section "V4": scores are
+ *          sqrt(softplus(l)) with the selection bias and no group limit; the
+ *          first layers choose experts by a fixed token-id table (tid2eid) and
+ *          the router only weights them.
  *
  * Conventions for every entry point:
  *   - Pointers named x, w_*, y, topk_*, offsets, perm_token, slot_dest,
@@ -76,7 +80,7 @@ typedef enum {
   MOE_ERR_INTERNAL = 6     /* a device-side consistency check failed         */
 } moe_status;
 
-typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score_fn;
+typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1, MOE_SCORE_SQRTSOFTPLUS = 2 } moe_score_fn;
 typedef enum { MOE_CAP_NONE = 0, MOE_CAP_OVERFLOW_NEXT = 1, MOE_CAP_DROP = 2 } moe_cap_policy;
 typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
 
@@ -89,7 +93,7 @@ typedef struct {
   int32_t n_group;               /* expert groups; 1 = no group limit              */
   int32_t topk_group;            /* groups kept per token                          */
   int32_t moe_intermediate_size; /* I                                              */
-  int32_t score_fn;              /* moe_score_fn                                   */
+  int32_t score_fn;              /* moe_score_fn; SIGMOID and SQRTSOFTPLUS add bias */
   int32_t renormalize;           /* 1: gates normalised over the kept slots        */
   float routed_scaling_factor;   /* multiplies every gate ([DS]: 2.5 for V3)       */
   int32_t cap_policy;            /* moe_cap_policy                                 */
@@ -182,6 +186,33 @@ moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out,
 moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
                              void* y, int32_t* topk_idx_opt, float* topk_w_opt, int32_t* counts_opt,
                              moe_diag* diag_opt, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * Hash routing ([DS4]): the experts of token t are row token_ids[t] of the
+ * fixed table tid2eid (device int32 [vocab, k], row-major); the gates come
+ * from the router scores of those experts exactly as in moe_route (score_fn,
+ * renormalize, routed_scaling_factor; cap_policy must be MOE_CAP_NONE).
+ *   in : x [n, d], token_ids [n] (device int32), tid2eid, vocab, weights->w_router.
+ *   out: topk_idx [n, k] in table order, topk_w [n, k], expert_counts [E]
+ *        (may be NULL), diag (may be NULL).
+ * A token id outside [0, vocab) or a table entry outside [0, E) leaves that
+ * slot empty (-1, weight 0) and sets MOE_ERR_INVALID_ARG in the status word
+ * (moe_sync_status).
+ */
+moe_status moe_route_hash(const moe_config* cfg, int64_t n, const void* x, const int32_t* token_ids,
+                          const int32_t* tid2eid, int32_t vocab, const moe_weights* weights, int32_t* topk_idx,
+                          float* topk_w, int32_t* expert_counts, moe_diag* diag, void* ws, size_t ws_bytes,
+                          moe_stream_t stream);
+
+/*
+ * One step of the auxiliary-loss-free balancing ([DS] V3): with counts the
+ * per-expert slot counts of a batch (device int32 [E], e.g. expert_counts of
+ * moe_route) and mean = sum(counts) / E, bias[e] (device float [E], updated in
+ * place) is decreased by gamma where counts[e] > mean, increased by gamma where
+ * counts[e] < mean, and kept where equal. Computed in binary64, stored binary32.
+ */
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* bias, float gamma,
+                           moe_stream_t stream);
 
 /*
  * Bytes of the device array behind moe_route_static_scratch (8 MiB).

@@ -120,6 +120,9 @@ WORKLOADS = {w.name: w for w in [
         cap_policy="drop", capacity_factor=1.0, zipf_s=1.2),
     _wl("ragged_small", n=77, d_model=200, n_routed=5, top_k=2, moe_intermediate_size=72, renormalize=True,
         n_shared=1),
+    _wl("deepseek_v4_small", n=300, d_model=256, n_routed=64, n_shared=1, top_k=6, moe_intermediate_size=128,
+        score_fn="sqrtsoftplus", renormalize=True, bias_range=(-0.1, 0.1),
+        description="DeepSeek-V4-style routing: sqrtsoftplus scores + bias, no group limit"),
     _wl("tie_softmax", n=256, d_model=64, n_routed=16, top_k=4, moe_intermediate_size=64,
         ternary=True, renormalize=True),
     _wl("tie_sigmoid", n=256, d_model=64, n_routed=32, top_k=4, moe_intermediate_size=64,

@@ -18,7 +18,7 @@ from tests import moe_harness as H
 pytestmark = pytest.mark.gpu
 
 SMALL = ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "deepseek_v3_decode_small",
-         "skewed_small", "drop_small", "ragged_small", "tie_softmax", "tie_sigmoid"]
+         "skewed_small", "drop_small", "ragged_small", "deepseek_v4_small", "tie_softmax", "tie_sigmoid"]
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -22,13 +22,13 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT, \
     MOE_ERR_INTERNAL = range(7)
-MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID = 0, 1
+MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID, MOE_SCORE_SQRTSOFTPLUS = 0, 1, 2
 MOE_CAP_NONE, MOE_CAP_OVERFLOW_NEXT, MOE_CAP_DROP = 0, 1, 2
 MOE_F32, MOE_BF16 = 0, 1
 
 # Every symbol declared in include/moe.h.
-EXPORTS = ("moe_workspace_size", "moe_route", "moe_permute", "moe_expert_ffn", "moe_combine",
-           "moe_layer_forward", "moe_route_static_scratch", "moe_sync_status", "moe_status_string")
+EXPORTS = ("moe_workspace_size", "moe_route", "moe_route_hash", "moe_bias_update", "moe_permute", "moe_expert_ffn",
+           "moe_combine", "moe_layer_forward", "moe_route_static_scratch", "moe_sync_status", "moe_status_string")
 MOE_STATIC_SCRATCH_BYTES = 8 << 20  # include/moe.h
 
 
@@ -62,6 +62,8 @@ _lib.moe_permute.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_expert_ffn.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_combine.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_layer_forward.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_route_hash.argtypes = [_P, _I64, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+_lib.moe_bias_update.argtypes = [_P, _P, _P, ctypes.c_float, _P]
 _lib.moe_route_static_scratch.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_sync_status.argtypes = [_P, _P]
 _lib.moe_status_string.argtypes = [ctypes.c_int]
@@ -91,7 +93,8 @@ def make_config(d_model, n_routed, top_k, moe_intermediate_size, n_shared=0, n_g
     """A moe_config from the pages' field names (strings for the enums)."""
     return moe_config(
         d_model, n_routed, n_shared, top_k, n_group, topk_group, moe_intermediate_size,
-        {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID}[score_fn], int(bool(renormalize)),
+        {"softmax": MOE_SCORE_SOFTMAX, "sigmoid": MOE_SCORE_SIGMOID, "sqrtsoftplus": MOE_SCORE_SQRTSOFTPLUS}[score_fn],
+        int(bool(renormalize)),
         float(routed_scaling_factor),
         {"none": MOE_CAP_NONE, "overflow_next": MOE_CAP_OVERFLOW_NEXT, "drop": MOE_CAP_DROP}[cap_policy],
         float(capacity_factor), int(capacity), {"f32": MOE_F32, "bf16": MOE_BF16}[dtype])
@@ -124,6 +127,18 @@ def moe_route(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, ws, str
     _check(_lib.moe_route(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(topk_idx), _ptr(topk_w),
                           _ptr(expert_counts), _ptr(diag), _ptr(ws), ws.numel() * ws.element_size(),
                           _stream(stream)), "moe_route")
+
+
+def moe_route_hash(cfg, n, x, token_ids, tid2eid, vocab, weights, topk_idx, topk_w, expert_counts, diag, ws,
+                   stream=None):
+    _check(_lib.moe_route_hash(ctypes.byref(cfg), n, _ptr(x), _ptr(token_ids), _ptr(tid2eid), vocab,
+                               ctypes.byref(weights), _ptr(topk_idx), _ptr(topk_w), _ptr(expert_counts), _ptr(diag),
+                               _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "moe_route_hash")
+
+
+def moe_bias_update(cfg, counts, bias, gamma, stream=None):
+    _check(_lib.moe_bias_update(ctypes.byref(cfg), _ptr(counts), _ptr(bias), float(gamma), _stream(stream)),
+           "moe_bias_update")
 
 
 def moe_route_static_scratch(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, stream=None):

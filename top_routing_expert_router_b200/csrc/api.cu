@@ -70,7 +70,8 @@ Plan make_plan(const moe_config& c, int64_t n) {
 moe_status check_cfg(const moe_config* c, int64_t n) {
   if (!c || n < 0) return MOE_ERR_INVALID_ARG;
   if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
-  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID && c->score_fn != MOE_SCORE_SQRTSOFTPLUS)
+    return MOE_ERR_INVALID_ARG;
   if (c->cap_policy < MOE_CAP_NONE || c->cap_policy > MOE_CAP_DROP) return MOE_ERR_INVALID_ARG;
   if (c->d_model <= 0 || c->n_routed <= 0 || c->top_k <= 0 || c->moe_intermediate_size <= 0 || c->n_shared < 0 ||
       c->n_group <= 0 || c->topk_group <= 0)
@@ -81,7 +82,7 @@ moe_status check_cfg(const moe_config* c, int64_t n) {
   if (c->cap_policy != MOE_CAP_NONE && c->capacity <= 0 && !(c->capacity_factor > 0.0f)) return MOE_ERR_INVALID_ARG;
   if (!isfinite(c->routed_scaling_factor)) return MOE_ERR_INVALID_ARG;
   if (c->n_routed > kMaxExperts || c->top_k > kMaxTopK || c->n_group > kMaxGroups) return MOE_ERR_UNSUPPORTED;
-  if (c->n_group > 1 && c->score_fn != MOE_SCORE_SIGMOID) return MOE_ERR_UNSUPPORTED;
+  if (c->n_group > 1 && c->score_fn == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
   if (c->d_model % 8 != 0 || c->moe_intermediate_size % 8 != 0) return MOE_ERR_UNSUPPORTED;
   if (n * c->top_k >= (int64_t)1 << 31 || n * (int64_t)c->n_routed >= (int64_t)1 << 40) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -153,16 +154,11 @@ moe_status gemm(const Ctx& x, const GemmArgs& a, bool swiglu, bool out_f32) {
   return cuda_status(launch_gemm_simt(a, x.c.dtype, out_f32, swiglu, x.s));
 }
 
-moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, int32_t* counts,
-                      moe_diag* diag) {
+// Router logits (binary32, split-K partials for small batches) and the route arguments.
+moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, moe_diag* d,
+                         RouteArgs* out) {
   const moe_config& c = x.c;
   float* logits = x.at<float>(x.p.logits);
-  moe_diag* d = diag ? diag : x.status();
-  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), x.s));  // counters, not the status word
-  if (x.n == 0) {
-    if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
-    return MOE_OK;
-  }
   const int splits = router_splits(c, x.n);
   GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model,
              splits, x.n * c.n_routed};
@@ -173,7 +169,7 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   r.split_stride = x.n * c.n_routed;
   r.x = X;
   r.w_r = w->w_router;
-  r.bias = c.score_fn == MOE_SCORE_SIGMOID ? w->bias : nullptr;
+  r.bias = c.score_fn != MOE_SCORE_SOFTMAX ? w->bias : nullptr;
   r.dtype = c.dtype;
   r.d = c.d_model;
   r.n = x.n;
@@ -187,6 +183,22 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   r.topk_idx = idx;
   r.topk_w = tw;
   r.diag = d;
+  r.ranking = nullptr;
+  *out = r;
+  return MOE_OK;
+}
+
+moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, int32_t* counts,
+                      moe_diag* diag) {
+  const moe_config& c = x.c;
+  moe_diag* d = diag ? diag : x.status();
+  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), x.s));  // counters, not the status word
+  if (x.n == 0) {
+    if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
+    return MOE_OK;
+  }
+  RouteArgs r;
+  MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
   if (c.cap_policy == MOE_CAP_NONE) {
     r.ranking = nullptr;
     MOE_CUDA(launch_route(r, x.s));
@@ -330,6 +342,42 @@ moe_status moe_route(const moe_config* cfg, int64_t n, const void* x, const moe_
   MOE_TRY(check_weights(c.c, weights, false, false));
   MOE_TRY(clear_status(c));
   return route_impl(c, x, weights, topk_idx, topk_w, expert_counts, diag);
+}
+
+moe_status moe_route_hash(const moe_config* cfg, int64_t n, const void* x, const int32_t* token_ids,
+                          const int32_t* tid2eid, int32_t vocab, const moe_weights* weights, int32_t* topk_idx,
+                          float* topk_w, int32_t* expert_counts, moe_diag* diag, void* ws, size_t ws_bytes,
+                          moe_stream_t stream) {
+  Ctx c;
+  MOE_TRY(begin(cfg, n, ws, ws_bytes, stream, &c));
+  if (cfg->cap_policy != MOE_CAP_NONE || vocab <= 0) return MOE_ERR_INVALID_ARG;
+  if (!weights || !ptr_ok(weights->w_router) || !tok_ok(x, n) || !tok_ok(topk_idx, n) || !tok_ok(topk_w, n) ||
+      (n > 0 && (!token_ids || !aligned(token_ids, 4))) || !tid2eid || !aligned(tid2eid, 4))
+    return MOE_ERR_INVALID_ARG;
+  if ((expert_counts && !aligned(expert_counts, 4)) || (diag && !aligned(diag, 16))) return MOE_ERR_INVALID_ARG;
+  MOE_TRY(check_weights(c.c, weights, false, false));
+  MOE_TRY(clear_status(c));
+  moe_diag* d = diag ? diag : c.status();
+  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), c.s));
+  if (n == 0) {
+    if (expert_counts) MOE_CUDA(launch_fill_i32(expert_counts, c.c.n_routed, 0, c.s));
+    return MOE_OK;
+  }
+  RouteArgs r;
+  MOE_TRY(router_logits(c, x, weights, topk_idx, topk_w, d, &r));
+  MOE_CUDA(launch_hash_select(token_ids, tid2eid, vocab, n, c.c.top_k, c.c.n_routed, topk_idx, c.status(), c.s));
+  MOE_CUDA(launch_gates(r, c.s));
+  MOE_CUDA(launch_dispatch(topk_idx, n, c.c.top_k, c.c.n_routed, c.at<int32_t>(c.p.blk), expert_counts,
+                           c.at<int32_t>(c.p.offsets), nullptr, nullptr, false, d, c.s));
+  return MOE_OK;
+}
+
+moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* bias, float gamma,
+                           moe_stream_t stream) {
+  MOE_TRY(check_cfg(cfg, 0));
+  if (!counts || !bias || !aligned(counts, 4) || !aligned(bias, 4) || !isfinite(gamma)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_bias_update(counts, cfg->n_routed, gamma, bias, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 moe_status moe_permute(const moe_config* cfg, int64_t n, const void* x, const int32_t* topk_idx, int32_t* offsets,

@@ -58,6 +58,10 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 // Capacity rule over the ranking; writes topk_idx and the overflow/drop counts.
 cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32_t k, int64_t C, int policy,
                             int32_t* topk_idx, moe_diag* diag, cudaStream_t s);
+// Hash routing selection and the balancing-bias update.
+cudaError_t launch_hash_select(const int32_t* token_ids, const int32_t* tid2eid, int32_t vocab, int64_t n, int32_t k,
+                               int32_t E, int32_t* topk_idx, moe_diag* status, cudaStream_t s);
+cudaError_t launch_bias_update(const int32_t* counts, int32_t E, float gamma, float* bias, cudaStream_t s);
 // Gates of a given selection from the logits.
 cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s);
 

@@ -65,6 +65,14 @@ __device__ __forceinline__ double warp_sum(double v) {
 
 __device__ __forceinline__ double sigmoid_d(double z) { return 1.0 / (1.0 + exp(-z)); }
 
+// sqrt(softplus(z)) ("sqrtsoftplus", page "15. DeepSeek: MLA, MoE and MTP", section V4).
+__device__ __forceinline__ double sqrtsoftplus_d(double z) { return sqrt(fmax(z, 0.0) + log1p(exp(-fabs(z)))); }
+
+// Raw score of the routers that add a selection bias.
+__device__ __forceinline__ double raw_score(int score_fn, double z) {
+  return score_fn == MOE_SCORE_SQRTSOFTPLUS ? sqrtsoftplus_d(z) : sigmoid_d(z);
+}
+
 template <int EPL>
 __device__ __forceinline__ double pick(const double (&r)[EPL], int j) {
   double out = 0.0;
@@ -84,7 +92,7 @@ __device__ __forceinline__ void selection_values(const RouteArgs& a, const doubl
     const int e = lane + 32 * j;
     valid[j] = e < a.E;
     if (valid[j])
-      v[j] = a.score_fn == MOE_SCORE_SIGMOID ? sigmoid_d(l[j]) + (a.bias ? (double)a.bias[e] : 0.0) : l[j];
+      v[j] = a.score_fn != MOE_SCORE_SOFTMAX ? raw_score(a.score_fn, l[j]) + (a.bias ? (double)a.bias[e] : 0.0) : l[j];
     else
       v[j] = -INFINITY;
   }
@@ -415,7 +423,7 @@ __device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* id
     const int src = e >= 0 ? (e & 31) : 0;
     const double le = __shfl_sync(kFull, pick(l, e >= 0 ? (e >> 5) : 0), src);
     double p = 0.0;
-    if (e >= 0) p = a.score_fn == MOE_SCORE_SOFTMAX ? exp(le - m) / z : sigmoid_d(le);
+    if (e >= 0) p = a.score_fn == MOE_SCORE_SOFTMAX ? exp(le - m) / z : raw_score(a.score_fn, le);
     if (lane == r) mine = p;
   }
   double denom = 1.0;
@@ -510,9 +518,12 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     for (int j = 0; j < EPL; ++j)
       if ((valid_mask >> j) & 1u) amax = fmax(amax, fabs(l[j]));
     amax = warp_max(amax);
-    // binary32 error bound of the logits, mapped to selection values (sigmoid' <= 1/4)
+    // binary32 error bound of the logits, mapped to selection values
+    // (sigmoid' <= 1/4; sqrtsoftplus' = sigmoid / (2 sqrtsoftplus) < 1/2)
     const double delta_l = ldexp(fmax(1.0, amax), -13);
-    const double delta_v = a.score_fn == MOE_SCORE_SIGMOID ? 0.25 * delta_l : delta_l;
+    const double delta_v = a.score_fn == MOE_SCORE_SIGMOID ? 0.25 * delta_l
+                           : a.score_fn == MOE_SCORE_SQRTSOFTPLUS ? 0.5 * delta_l
+                                                                  : delta_l;
     uint32_t exact = 0;
     int nr = 0;
     bool refined = false;
@@ -562,6 +573,47 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a)
     const float w = gates<EPL>(a, l, s_idx[wib]);
     if (lane < a.k) a.topk_w[t * a.k + lane] = w;
     __syncwarp();
+  }
+}
+
+// ---- hash routing and the balancing-bias update ------------------------------------
+// Hash routing (page "15. DeepSeek: MLA, MoE and MTP", section V4): the experts
+// of token t are row token_ids[t] of the fixed table tid2eid [vocab, k]; the
+// router only weights them (gates_kernel). Out-of-range ids or table entries
+// leave the slot empty (-1) and report MOE_ERR_INVALID_ARG in the status word.
+__global__ void hash_select_kernel(const int32_t* token_ids, const int32_t* tid2eid, int32_t vocab, int64_t n,
+                                   int32_t k, int32_t E, int32_t* topk_idx, moe_diag* status) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n * k; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / k;
+    const int32_t tok = token_ids[t];
+    int32_t e = -1;
+    if (tok >= 0 && tok < vocab) e = tid2eid[(int64_t)tok * k + i % k];
+    if (e < 0 || e >= E) {
+      e = -1;
+      set_status(status, MOE_ERR_INVALID_ARG);
+    }
+    topk_idx[i] = e;
+  }
+}
+
+// Auxiliary-loss-free balancing (same page, section V3): an expert that received
+// more slots than the mean has its selection bias lowered by gamma, one below
+// the mean raised by gamma; the mean is sum(counts) / E.
+__global__ void bias_update_kernel(const int32_t* counts, int32_t E, float gamma, float* bias) {
+  __shared__ double total;
+  if (threadIdx.x == 0) {
+    double s = 0.0;
+    for (int e = 0; e < E; ++e) s += counts[e];
+    total = s;
+  }
+  __syncthreads();
+  const double mean = total / E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const double c = counts[e];
+    double b = (double)bias[e];
+    if (c > mean) b -= (double)gamma;
+    else if (c < mean) b += (double)gamma;
+    bias[e] = (float)b;
   }
 }
 
@@ -740,6 +792,20 @@ cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s) {
     case 4: gates_kernel<4><<<grid, block, 0, s>>>(a); break;
     default: gates_kernel<8><<<grid, block, 0, s>>>(a); break;
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hash_select(const int32_t* token_ids, const int32_t* tid2eid, int32_t vocab, int64_t n, int32_t k,
+                               int32_t E, int32_t* topk_idx, moe_diag* status, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  const int64_t blocks = ceil_div(n * k, 256);
+  hash_select_kernel<<<(unsigned)(blocks < 148 * 8 ? blocks : 148 * 8), 256, 0, s>>>(token_ids, tid2eid, vocab, n, k, E,
+                                                                                  topk_idx, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bias_update(const int32_t* counts, int32_t E, float gamma, float* bias, cudaStream_t s) {
+  bias_update_kernel<<<1, 256, 0, s>>>(counts, E, gamma, bias);
   return cudaGetLastError();
 }
 
