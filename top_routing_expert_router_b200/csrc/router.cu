@@ -428,7 +428,9 @@ __device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* id
   }
   double denom = 1.0;
   if (a.renorm) denom = warp_sum(lane < a.k ? mine : 0.0);
-  return (float)(mine / denom * (double)a.rsf);
+  // a dropped slot weighs 0, also when every slot of the token was dropped
+  const bool kept = lane < a.k && idx_of_slot[lane] >= 0;
+  return kept ? (float)(mine / denom * (double)a.rsf) : 0.0f;
 }
 
 // Binary64 dot product x[t] . W_r[e], computed by the whole warp: lanes take
@@ -635,6 +637,10 @@ __device__ __forceinline__ void warp_count(int* counts, int e) {
   if (e >= 0 && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&counts[e], __popc(peers));
 }
 
+// The block holds a window of 1024 tokens, one per thread. Each token keeps
+// its current choices and a cursor into its ranking; after a fill event only
+// the tokens that lost a choice walk on from their cursor, so every ranking
+// entry of a window is read at most once.
 __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k,
                                                             int64_t C, int policy, int32_t* topk_idx,
                                                             moe_diag* diag) {
@@ -653,102 +659,140 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
   if (tid < kMaxExperts / 32) full[tid] = 0;
   if (tid == 0) s_over = s_drop = 0;
   __syncthreads();
+  auto is_full = [&](int e) { return (full[e >> 5] >> (e & 31)) & 1u; };
   unsigned long long my_over = 0, my_drop = 0;
-  int64_t base = 0;
-  while (base < n) {
-    // stage the window's ranking prefixes (coalesced 16-byte copies when rows allow it)
-    const int cnt_tok = (int)((n - base) < kCapThreads ? (n - base) : kCapThreads);
+  for (int64_t w0 = 0; w0 < n; w0 += kCapThreads) {
+    const int cnt_tok = (int)((n - w0) < kCapThreads ? (n - w0) : kCapThreads);
     if (E % 8 == 0) {
       const int vpr = P / 8;  // 16-byte vectors per staged row
       for (int i = tid; i < cnt_tok * vpr; i += kCapThreads) {
         const int row = i / vpr, v = i % vpr;
-        reinterpret_cast<uint4*>(st)[row * vpr + v] =
-            reinterpret_cast<const uint4*>(ranking + (base + row) * E)[v];
+        reinterpret_cast<uint4*>(st)[row * vpr + v] = reinterpret_cast<const uint4*>(ranking + (w0 + row) * E)[v];
       }
     } else {
-      for (int i = tid; i < cnt_tok * P; i += kCapThreads) st[i] = ranking[(base + i / P) * E + i % P];
+      for (int i = tid; i < cnt_tok * P; i += kCapThreads) st[i] = ranking[(w0 + i / P) * E + i % P];
     }
     __syncthreads();
-    const int64_t t = base + tid;
+    const int64_t t = w0 + tid;
     const bool valid = tid < cnt_tok;
-    int ch[kMaxTopK];
-    int over = 0;
-    for (int j = 0; j < k; ++j) ch[j] = -1;
-    if (valid) {
-      const uint16_t* srow = st + tid * P;
-      const uint16_t* grow = ranking + t * E;
-      if (policy == MOE_CAP_OVERFLOW_NEXT) {
-        int taken = 0;
-        for (int r = 0; r < E && taken < k; ++r) {
-          const int e = r < P ? srow[r] : grow[r];
-          if (e == 0xFFFF) break;
-          if (!((full[e >> 5] >> (e & 31)) & 1u)) {
-            ch[taken++] = e;
-            over += r >= k;
-          }
+    const uint16_t* srow = st + tid * P;
+    const uint16_t* grow = ranking + t * E;
+    int ch[kMaxTopK];  // current choices (in ranking order); -1 = empty slot
+    int pos[kMaxTopK];  // their ranking positions
+    int taken = 0, cursor = 0;
+    // walk on from the cursor until k non-full experts are held (overflow policy)
+    auto refill = [&]() {
+      while (taken < k && cursor < E) {
+        const int e = cursor < P ? srow[cursor] : grow[cursor];
+        if (e == 0xFFFF) {
+          cursor = E;
+          break;
         }
+        if (!is_full(e)) {
+          ch[taken] = e;
+          pos[taken] = cursor;
+          ++taken;
+        }
+        ++cursor;
+      }
+    };
+    if (valid) {
+      if (policy == MOE_CAP_OVERFLOW_NEXT) {
+        refill();
       } else {
         for (int j = 0; j < k; ++j) {
-          const int e = j < P ? srow[j] : grow[j];
-          ch[j] = (e != 0xFFFF && !((full[e >> 5] >> (e & 31)) & 1u)) ? e : -1;
+          const int e = srow[j];
+          ch[j] = (e != 0xFFFF && !is_full(e)) ? e : -1;
         }
       }
     }
-    for (int e = tid; e < E; e += kCapThreads) ccnt[e] = 0;
-    if (tid == 0) {
-      n_cand = 0;
-      stop = kCapThreads;
-    }
-    __syncthreads();
-    for (int j = 0; j < k; ++j) warp_count(ccnt, valid ? ch[j] : -1);
-    __syncthreads();
-    for (int e = tid; e < E; e += kCapThreads)
-      if (cnt[e] < C && cnt[e] + ccnt[e] >= C) cand[atomicAdd(&n_cand, 1)] = e;
-    __syncthreads();
-    const int nc = n_cand;
-    for (int c = 0; c < nc; ++c) {
-      const int e = cand[c];
-      bool mine = false;
-      if (valid)
-        for (int j = 0; j < k; ++j) mine |= ch[j] == e;
-      const uint32_t b = __ballot_sync(kFull, mine);
-      if (lane == 0) ballots[wid] = b;
-      __syncthreads();
-      if (tid == 0) {
-        int need = (int)(C - cnt[e]);  // this expert's C-th slot is taken by the need-th chooser
-        for (int w = 0; w < kCapThreads / 32; ++w) {
-          const int pc = __popc(ballots[w]);
-          if (need <= pc) {
-            uint32_t bb = ballots[w];
-            for (int q = 1; q < need; ++q) bb &= bb - 1;
-            const int pos = w * 32 + __ffs(bb) - 1;
-            if (pos < stop) stop = pos;
-            break;
-          }
-          need -= pc;
-        }
-      }
-      __syncthreads();
-    }
-    const int s = stop;  // relative index of the last committed token
-    const bool commit = valid && tid <= s;
-    if (commit) {
-      for (int j = 0; j < k; ++j) topk_idx[t * k + j] = ch[j];
-      my_over += over;
-      for (int j = 0; j < k; ++j) my_drop += ch[j] < 0;
-    }
-    if (s < kCapThreads) {
+    int f = 0;  // first window position not committed yet (uniform across the block)
+    while (true) {
+      const bool active = valid && tid >= f;
+      auto slot = [&](int j) {
+        if (policy == MOE_CAP_OVERFLOW_NEXT) return j < taken ? ch[j] : -1;
+        return ch[j];
+      };
       for (int e = tid; e < E; e += kCapThreads) ccnt[e] = 0;
+      if (tid == 0) {
+        n_cand = 0;
+        stop = kCapThreads;
+      }
       __syncthreads();
-      for (int j = 0; j < k; ++j) warp_count(ccnt, commit ? ch[j] : -1);
+      for (int j = 0; j < k; ++j) warp_count(ccnt, active ? slot(j) : -1);
       __syncthreads();
-    }
-    for (int e = tid; e < E; e += kCapThreads) {
-      cnt[e] += ccnt[e];
-      if (cnt[e] >= C) atomicOr(&full[e >> 5], 1u << (e & 31));
+      for (int e = tid; e < E; e += kCapThreads)
+        if (cnt[e] < C && cnt[e] + ccnt[e] >= C) cand[atomicAdd(&n_cand, 1)] = e;
+      __syncthreads();
+      const int nc = n_cand;
+      for (int c = 0; c < nc; ++c) {
+        const int e = cand[c];
+        bool mine = false;
+        if (active)
+          for (int j = 0; j < k; ++j) mine |= slot(j) == e;
+        const uint32_t b = __ballot_sync(kFull, mine);
+        if (lane == 0) ballots[wid] = b;
+        __syncthreads();
+        if (tid == 0) {
+          int need = (int)(C - cnt[e]);  // this expert's C-th slot goes to its need-th chooser
+          for (int w = 0; w < kCapThreads / 32; ++w) {
+            const int pc = __popc(ballots[w]);
+            if (need <= pc) {
+              uint32_t bb = ballots[w];
+              for (int q = 1; q < need; ++q) bb &= bb - 1;
+              const int at = w * 32 + __ffs(bb) - 1;
+              if (at < stop) stop = at;
+              break;
+            }
+            need -= pc;
+          }
+        }
+        __syncthreads();
+      }
+      const int s = stop;  // last committed window position (kCapThreads: all of them)
+      const bool commit = active && tid <= s;
+      if (commit) {
+        for (int j = 0; j < k; ++j) {
+          const int e = slot(j);
+          topk_idx[t * k + j] = e;
+          my_drop += e < 0;
+          if (policy == MOE_CAP_OVERFLOW_NEXT && j < taken) my_over += pos[j] >= k;
+        }
+      }
+      if (s < kCapThreads) {
+        for (int e = tid; e < E; e += kCapThreads) ccnt[e] = 0;
+        __syncthreads();
+        for (int j = 0; j < k; ++j) warp_count(ccnt, commit ? slot(j) : -1);
+        __syncthreads();
+      }
+      for (int e = tid; e < E; e += kCapThreads) {
+        cnt[e] += ccnt[e];
+        if (cnt[e] >= C) atomicOr(&full[e >> 5], 1u << (e & 31));
+      }
+      __syncthreads();
+      if (s >= cnt_tok - 1) break;  // the whole window is committed
+      f = s + 1;
+      // tokens still to come drop the experts that just filled
+      if (valid && tid >= f) {
+        if (policy == MOE_CAP_OVERFLOW_NEXT) {
+          int kept = 0;
+          for (int j = 0; j < taken; ++j)
+            if (!is_full(ch[j])) {
+              ch[kept] = ch[j];
+              pos[kept] = pos[j];
+              ++kept;
+            }
+          if (kept < taken) {
+            taken = kept;
+            refill();
+          }
+        } else {
+          for (int j = 0; j < k; ++j)
+            if (ch[j] >= 0 && is_full(ch[j])) ch[j] = -1;
+        }
+      }
     }
     __syncthreads();
-    base += s < kCapThreads ? (int64_t)s + 1 : (int64_t)kCapThreads;
   }
   atomicAdd(&s_over, my_over);
   atomicAdd(&s_drop, my_drop);
