@@ -47,6 +47,23 @@ def _dist():
     return ws, rank, local
 
 
+def reduce_max(x: float, world: int, device="cpu") -> float:
+    """Maximum of a per-rank scalar over all ranks (every rank gets it)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, world: int, ms_total_max: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch (replicas), time = slowest rank."""
+    return world * tokens_per_rank * steps / (ms_total_max / 1e3)
+
+
 def layer_work(w, kept_slots, active_experts):
     """Algorithmic FLOPs and bytes of one layer forward."""
     b = 2 if w.dtype == "bf16" else 4
@@ -71,9 +88,10 @@ def launches_per_step(w):
 
 
 def _sources_sha():
+    """Hash of the sources of the dominant kernel (the tensor-core grouped GEMM)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "top_routing_expert_router_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
+    for fn in ("gemm_tc.cu", "common.cuh"):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
@@ -184,13 +202,9 @@ def run_ours(args):
             step()
         ev1.record(stream)
         barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    t = torch.tensor([ms_total], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_total = float(t.item())
+    ms_total = reduce_max(ev0.elapsed_time(ev1), world, "cuda")
     ms_step = ms_total / args.steps
-    value = world * n * args.steps / (ms_total / 1e3)
+    value = job_throughput(n, args.steps, world, ms_total)
     clocks = clk.summary()
 
     # Stage times through the staged entry points (same kernels), events on the launching stream.
@@ -242,11 +256,7 @@ def run_ours(args):
         y_host.copy_(y, non_blocking=True)
     b.record(stream)
     barrier()
-    e2e_ms = a.elapsed_time(b) / e2e_steps
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = reduce_max(a.elapsed_time(b) / e2e_steps, world, "cuda")
     bpe = dev["x"].element_size()
 
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
