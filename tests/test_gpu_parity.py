@@ -199,6 +199,38 @@ def test_single_token_and_ragged_sizes():
         assert H.rel_err(H.as_f64(got["y"])[keep], r["y"][keep]) <= H.TOL[w.dtype]
 
 
+# Group sizes around the 128-row and 256-row tile edges: empty groups, one row,
+# exact multiples, one past them, and groups whose last tile is half height.
+EDGE_COUNTS = [0, 1, 64, 127, 128, 129, 255, 256, 257, 300, 384, 385, 513, 640, 0]
+
+
+@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+def test_expert_ffn_tile_edges(mode, monkeypatch):
+    """Caller-given group offsets at every tile edge; d and I leave ragged n- and k-tiles."""
+    monkeypatch.setenv("MOE_TC_MODE", mode)
+    counts = np.array(EDGE_COUNTS, np.int32)
+    rows = int(counts.sum())
+    w = W.get("ragged_small", n=rows, d_model=320, n_routed=len(counts), top_k=1, moe_intermediate_size=200,
+              n_shared=0, renormalize=False)
+    host = W.host_inputs(w, names=["x", "w_gate", "w_up", "w_down"])
+    dev = W.device_inputs(w, names=["x", "w_gate", "w_up", "w_down"])
+    offsets = np.zeros(len(counts) + 1, np.int32)
+    offsets[1:] = np.cumsum(counts)
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, rows)
+    eo = torch.empty((rows, w.d_model), dtype=dev["x"].dtype, device="cuda")
+    wts = moe.make_weights(None, dev["w_gate"], dev["w_up"], dev["w_down"])
+    moe.moe_expert_ffn(cfg, rows, dev["x"], torch.from_numpy(offsets).cuda(), wts, eo, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    got = H.as_f64(eo)
+    x64 = O.bf16_to_f64(host["x"])
+    for e in range(len(counts)):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            ref = O.swiglu(x64[lo:hi], host["w_gate"][e], host["w_up"][e], host["w_down"][e])
+            assert H.rel_err(got[lo:hi], ref) <= H.TOL[w.dtype], (e, int(counts[e]))
+
+
 @pytest.mark.parametrize("mode", ["1sm", "2sm"])
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v3_small", "ragged_small", "deepseek_v2_small"])
 def test_expert_ffn_both_tile_modes(name, mode, monkeypatch):

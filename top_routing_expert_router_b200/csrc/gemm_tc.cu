@@ -207,6 +207,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // ---- tile mapping ----------------------------------------------------------------
 struct Tile {
   int g, m, nt, split;
+  int half;    // SM-pair kernel: half-height (M = 128) last tile of its group
+  int lo, hi;  // SM-pair kernel: the group's rows
 };
 
 // Tiles of group g are tile_off[g] .. tile_off[g+1]-1, ordered split major,
@@ -219,7 +221,7 @@ __device__ __forceinline__ Tile decode(const SmemCtl* ctl, int G, int t, int& g_
   const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM - 1) / BM;
   const int per_split = mt * ctl->n_tiles;
   const int rem = local % per_split;
-  return Tile{g, rem % mt, rem / mt, local / per_split};
+  return Tile{g, rem % mt, rem / mt, local / per_split, 0, 0, 0};
 }
 
 __device__ __forceinline__ void store16(void* C, int64_t ldc, int64_t row, int col, int N, const float (&v)[16],
@@ -455,16 +457,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ---- 2-SM variant (cta_group::2) -----------------------------------------------------
 // A CTA pair (cluster of 2) computes a 256 x 256 tile: CTA r holds A rows
-// [128r, 128r+128) of the tile and B rows [128r, 128r+128) (for SwiGLU: the
-// gate half in CTA 0, the up half in CTA 1). The leader CTA (rank 0) issues
-// tcgen05.mma.cta_group::2 with M = 256, which reads the peer's operand halves
-// through the pair's shared memory, so each SM stages 32 KB per 64-k step
-// instead of 48 KB. Both CTAs' copies signal the leader's `full` barrier; the
-// leader's commits are multicast to both CTAs; both epilogues report to the
-// leader's `tmem_empty` barrier. No TMA multicast is used.
+// [128r, 128r+128) of the tile and B rows [128r, 128r+128). The leader CTA
+// (rank 0) issues tcgen05.mma.cta_group::2 with M = 256, which reads the peer's
+// operand halves through the pair's shared memory, so each SM stages 32 KB per
+// 64-k step instead of 48 KB. The last m-tile of a group whose remainder is at
+// most 128 rows is a half-height tile: M = 128, 64 A rows per CTA, so groups
+// are padded to 128 rows, not 256. For SwiGLU, CTA r stages gate rows
+// [64r, 64r+64) of the tile's 128 output columns over the up rows of the same
+// columns, so each output column finds its gate and up accumulators in one TMEM
+// lane in both tile heights. Both CTAs' copies signal the leader's `full`
+// barrier; the leader's commits are multicast to both CTAs; both epilogues
+// report to the leader's `tmem_empty` barrier. No TMA multicast is used.
 constexpr int BM2 = 256;        // rows per pair tile
-constexpr int STAGES2 = 6;
+constexpr int STAGES2 = 7;      // 7 x 32 KB ring; the group row offsets stay in global memory to make room
 constexpr int A2_BYTES = 128 * BK * 2;
+constexpr int A2_HALF_BYTES = 64 * BK * 2;  // half-height tile: 64 A rows per CTA
 constexpr int B2_BYTES = 128 * BK * 2;
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
 
@@ -479,7 +486,6 @@ struct __align__(8) SmemCtl2 {
   int32_t abort;
   int32_t total_tiles;
   int32_t n_tiles;
-  int32_t row_off[kMaxGroupsTc + 1];
   int32_t tile_off[kMaxGroupsTc + 1];
 };
 
@@ -533,17 +539,26 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
       : "memory");
 }
 
-__device__ __forceinline__ uint32_t idesc_bf16_m256(int n) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM2 >> 4) << 24);
+__device__ __forceinline__ uint32_t idesc_bf16_pair(int m, int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ Tile decode2(const SmemCtl2* ctl, int G, int t, int& g_hint) {
+__device__ __forceinline__ int group_row(const TcParams& p, int g) {
+  return p.offsets ? __ldg(p.offsets + g) : (g == 0 ? 0 : p.M);
+}
+
+__device__ __forceinline__ Tile decode2(const SmemCtl2* ctl, const TcParams& p, int t, int& g_hint) {
   int g = g_hint;
-  while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
+  while (g + 1 <= p.G && ctl->tile_off[g + 1] <= t) ++g;
   g_hint = g;
   const int local = t - ctl->tile_off[g];
-  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM2 - 1) / BM2;
-  return Tile{g, local % mt, local / mt, 0};
+  const int lo = group_row(p, g);
+  const int rows = group_row(p, g + 1) - lo;
+  const int mt = (rows + BM2 - 1) / BM2;
+  const int m = local % mt;
+  // the last m-tile is half height when at most 128 rows remain
+  const int half = (m == mt - 1 && rows - m * BM2 <= BM2 / 2) ? 1 : 0;
+  return Tile{g, m, local / mt, 0, half, lo, lo + rows};
 }
 
 __device__ __noinline__ bool mbar_wait2(uint64_t* bar, uint32_t parity, SmemCtl2* ctl, moe_diag* st) {
@@ -570,8 +585,8 @@ __device__ __noinline__ void spin_ns(uint64_t ns) {
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
-                    const __grid_constant__ CUtensorMap map_b2, TcParams p) {
+    gemm_tc2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a_half,
+                    const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_b2, TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw2[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw2) + 1023) & ~uintptr_t(1023));
   SmemCtl2* ctl = reinterpret_cast<SmemCtl2*>(smem + STAGES2 * STAGE2_BYTES);
@@ -585,8 +600,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < p.G; ++g) {
       const int lo = p.offsets ? p.offsets[g] : 0;
       const int hi = p.offsets ? p.offsets[g + 1] : p.M;
-      ctl->row_off[g] = lo;
-      ctl->row_off[g + 1] = hi;
       ctl->tile_off[g] = acc;
       acc += ((hi - lo + BM2 - 1) / BM2) * n_tiles;
     }
@@ -609,6 +622,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_a_half);
     tma_prefetch_desc(&map_b);
     if (p.swiglu) tma_prefetch_desc(&map_b2);
   }
@@ -633,12 +647,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int g_hint = 0;
-      const uint32_t tx = 2u * STAGE2_BYTES;
       for (int t = pair; t < total && !aborted; t += npairs) {
-        const Tile tl = decode2(ctl, p.G, t, g_hint);
-        const int row0 = ctl->row_off[tl.g] + tl.m * BM2 + (int)rank * 128;
-        const CUtensorMap* bmap = (p.swiglu && rank == 1) ? &map_b2 : &map_b;
-        const int brow = p.swiglu ? tl.g * p.b_rows + tl.nt * p.n_out
+        const Tile tl = decode2(ctl, p, t, g_hint);
+        const bool half = tl.half != 0;
+        const uint32_t tx = 2u * ((half ? A2_HALF_BYTES : A2_BYTES) + B2_BYTES);
+        const CUtensorMap* amap = half ? &map_a_half : &map_a;
+        const int row0 = tl.lo + tl.m * BM2 + (int)rank * (half ? 64 : 128);
+        // SwiGLU: 64 gate rows over the 64 up rows of the same output columns; plain: 128 rows of B
+        const int brow = p.swiglu ? tl.g * p.b_rows + tl.nt * p.n_out + (int)rank * 64
                                   : tl.g * p.b_rows + tl.nt * p.n_out + (int)rank * 128;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
@@ -657,8 +673,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t leader_full = map_to_rank(&ctl->full[stage], 0);
           if (rank == 0) mbar_expect_tx(&ctl->full[stage], tx);
-          tma_load_2d_pair(sa, &map_a, leader_full, kb * BK, row0);
-          tma_load_2d_pair(sa + A2_BYTES, bmap, leader_full, kb * BK, brow);
+          tma_load_2d_pair(sa, amap, leader_full, kb * BK, row0);
+          if (p.swiglu) {
+            tma_load_2d_pair(sa + A2_BYTES, &map_b, leader_full, kb * BK, brow);
+            tma_load_2d_pair(sa + A2_BYTES + 64 * BK * 2, &map_b2, leader_full, kb * BK, brow);
+          } else {
+            tma_load_2d_pair(sa + A2_BYTES, &map_b, leader_full, kb * BK, brow);
+          }
           if (++stage == STAGES2) {
             stage = 0;
             phase ^= 1u;
@@ -671,10 +692,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && rank == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t idesc = idesc_bf16_m256(BN_MAX);
+      const uint32_t idesc_full = idesc_bf16_pair(BM2, BN_MAX);
+      const uint32_t idesc_half = idesc_bf16_pair(BM2 / 2, BN_MAX);
       bool issued = false;
       int i = 0;
+      int g_hint = 0;
       for (int t = pair; t < total && !aborted; t += npairs, ++i) {
+        const uint32_t idesc = decode2(ctl, p, t, g_hint).half ? idesc_half : idesc_full;
         const int buf = i & 1;
         const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
         if (!mbar_wait2(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
@@ -713,15 +737,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ================= epilogue (warps 2..5, both CTAs) =================
+    // TMEM lane quarter q of CTA r. Full tile: lane = row 128r + 32q + lane,
+    // column = MMA column n. Half tile (M = 128, 64 rows per CTA): MMA columns
+    // [0, 128) sit in lanes 0..63 and columns [128, 256) in lanes 64..127, both
+    // at TMEM columns [0, 128), so quarters 0-1 hold the first half of the
+    // columns and quarters 2-3 the second half, each for rows 64r + 32(q & 1) + lane.
     const int q = warp & 3;
-    const int row_in_tile = (int)rank * 128 + q * 32 + lane;
     const uint32_t leader_tmem_empty[2] = {map_to_rank(&ctl->tmem_empty[0], 0), map_to_rank(&ctl->tmem_empty[1], 0)};
     int g_hint = 0;
     int i = 0;
     for (int t = pair; t < total; t += npairs, ++i) {
       const int buf = i & 1;
       const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
-      const Tile tl = decode2(ctl, p.G, t, g_hint);
+      const Tile tl = decode2(ctl, p, t, g_hint);
+      const bool half = tl.half != 0;
       const bool got = mbar_wait2(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
       __syncwarp();  // tcgen05.ld below is warp-aligned
       if (!got) {
@@ -729,21 +758,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       fence_after();
-      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM2 + row_in_tile;
-      const bool valid = row < ctl->row_off[tl.g + 1];
-      const int col0 = tl.nt * p.n_out;
+      const int row_in_tile = half ? (int)rank * 64 + (q & 1) * 32 + lane : (int)rank * 128 + q * 32 + lane;
+      const int64_t row = (int64_t)tl.lo + tl.m * BM2 + row_in_tile;
+      const bool valid = row < tl.hi;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN_MAX);
       if (p.swiglu) {
-        for (int c = 0; c < p.n_out; c += 16) {
+        // Output column j of the tile: gate at MMA column 128(j/64) + j%64, up 64 further.
+        const int j0 = half ? (q >> 1) * 64 : 0;
+        const int nj = half ? 64 : 128;
+        const int col0 = tl.nt * p.n_out + j0;
+        for (int c = 0; c < nj; c += 16) {
+          const uint32_t gcol = half ? (uint32_t)c : (uint32_t)(128 * (c >> 6) + (c & 63));
           float gv[16], uv[16];
-          tmem_ld16(taddr + (uint32_t)c, gv);
-          tmem_ld16(taddr + (uint32_t)(p.n_out + c), uv);
+          tmem_ld16(taddr + gcol, gv);
+          tmem_ld16(taddr + gcol + 64u, uv);
 #pragma unroll
           for (int e = 0; e < 16; ++e) gv[e] = silu(gv[e]) * uv[e];
           if (valid && col0 + c < p.N) store16(p.C, p.ldc, row, col0 + c, p.N, gv, false);
         }
       } else {
-        for (int c = 0; c < p.n_out; c += 16) {
+        const int j0 = half ? (q >> 1) * 128 : 0;
+        const int nj = half ? 128 : p.n_out;
+        const int col0 = tl.nt * p.n_out + j0;
+        for (int c = 0; c < nj; c += 16) {
           float v[16];
           tmem_ld16(taddr + (uint32_t)c, v);
           if (valid && col0 + c < p.N) store16(p.C, p.ldc, row, col0 + c, p.N, v, p.out_f32 != 0);
@@ -811,19 +848,39 @@ int num_sms() {
   return sms;
 }
 
+// Clusters of two gemm_tc2_kernel CTAs that fit on the device at once, per device.
+int max_resident_pairs(const cudaLaunchConfig_t& cfg) {
+  static int cached[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 0;
+  if (!cached[dev]) {
+    cudaLaunchConfig_t q = cfg;
+    q.gridDim = dim3((unsigned)num_sms(), 1, 1);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, (void*)gemm_tc2_kernel, &q) != cudaSuccess || clusters <= 0)
+      return 0;
+    cached[dev] = clusters;
+  }
+  return cached[dev];
+}
+
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SmemCtl);
 constexpr size_t kSmemBytes2 = 1024 + STAGES2 * STAGE2_BYTES + sizeof(SmemCtl2);
+static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448, "dynamic shared memory above 227 KB");
 
-// 2-SM pair tiles (256 rows) pay off when groups carry enough rows; ragged
-// groups with few rows waste less with 128-row tiles. MOE_TC_MODE=1sm|2sm
-// overrides the choice (tuning and tests).
+// SM-pair tiles stage fewer bytes per FLOP and, with half-height last tiles,
+// pad groups to 128 rows like the single-SM tiles; they are used once groups
+// average at least 128 rows. Below that (decode) every tile is mostly padding
+// and the single-SM kernel keeps twice as many independent weight streams in
+// flight. MOE_TC_MODE=1sm|2sm overrides the choice (tuning and tests).
 bool use_pair_tiles(const GemmArgs& a, bool swiglu, bool out_f32) {
   if (a.k_splits > 1 || out_f32) return false;
   if (!swiglu && a.N < BN_MAX) return false;
   const char* mode = getenv("MOE_TC_MODE");
   if (mode && strcmp(mode, "1sm") == 0) return false;
   if (mode && strcmp(mode, "2sm") == 0) return true;
-  return a.M / (a.offsets ? a.G : 1) >= 768;
+  return a.M / (a.offsets ? a.G : 1) >= 128;
 }
 
 }  // namespace
@@ -881,13 +938,17 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   CUtensorMap ma, mb, mb2;
   const int64_t b_total_rows = (int64_t)a.G * a.N;
   const bool pair = use_pair_tiles(a, swiglu, out_f32);
-  // Rows of B one CTA stages per copy: SwiGLU gate/up halves are 128 rows; on an
-  // SM pair each CTA also holds only a 128-row half of a plain 256-row B tile.
-  const int b_box = (swiglu || pair) ? p.n_mma / 2 : p.n_mma;
+  // Rows of B one CTA stages per copy. One SM: SwiGLU gate and up halves of 128
+  // rows, or the whole plain tile. SM pair: each CTA holds 128 of the tile's 256
+  // B rows, as 64 gate over 64 up rows for SwiGLU.
+  const int b_box = pair ? (swiglu ? p.n_mma / 4 : p.n_mma / 2) : (swiglu ? p.n_mma / 2 : p.n_mma);
   // Every copy must fit the shared-memory slot it lands in.
-  const int b_slot_rows = pair ? B2_BYTES / (BK * 2) : (swiglu ? BN_MAX / 2 : BN_MAX);
-  if (b_box > b_slot_rows || (pair && (p.n_mma != BN_MAX || A2_BYTES != BM * BK * 2))) return cudaErrorInvalidValue;
+  const int b_slot_rows = pair ? (swiglu ? B2_BYTES / (BK * 2) / 2 : B2_BYTES / (BK * 2)) : (swiglu ? BN_MAX / 2 : BN_MAX);
+  if (b_box > b_slot_rows || (pair && (p.n_mma != BN_MAX || A2_BYTES != BM * BK * 2 || 2 * A2_HALF_BYTES != A2_BYTES)))
+    return cudaErrorInvalidValue;
   if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
+  CUtensorMap ma_half;
+  if (pair && !make_map(&ma_half, a.A, a.M, a.K, BM / 2)) return cudaErrorInvalidValue;
   if (!make_map(&mb, a.B, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
   if (swiglu) {
     if (!make_map(&mb2, a.B2, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
@@ -904,9 +965,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
       attr2 = true;
     }
     const int64_t max_pair_tiles = (ceil_div(a.M, BM2) + (a.offsets ? a.G : 0)) * n_tiles_all;
-    const int64_t pairs = max_pair_tiles < num_sms() / 2 ? max_pair_tiles : num_sms() / 2;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmemBytes2;
     cfg.stream = s;
@@ -917,7 +976,15 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, mb, mb2, p);
+    // Tiles are dealt round-robin to a persistent grid, so every pair must be
+    // resident at once: a pair that only starts when another one exits would
+    // run its whole share after the others. On parts whose GPCs hold odd SM
+    // counts fewer than SMs/2 pairs fit, hence the occupancy query.
+    const int pairs_resident = max_resident_pairs(cfg);
+    if (pairs_resident <= 0) return cudaErrorInvalidConfiguration;
+    const int64_t pairs = max_pair_tiles < pairs_resident ? max_pair_tiles : pairs_resident;
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, ma_half, mb, mb2, p);
   }
   static bool attr_set = false;
   if (!attr_set) {
