@@ -237,7 +237,7 @@ def run_ours(args):
     st = moe.moe_sync_status(ws, s)
     if st != moe.MOE_OK:
         raise RuntimeError(f"device status: {moe.moe_status_string(st)}")
-    dg = dict(zip(moe.DIAG_FIELDS, diag.cpu().tolist()[:5]))
+    dg = dict(zip(moe.DIAG_FIELDS, diag.cpu().tolist()))
     cnt = counts.cpu()
     kept = int(cnt.sum())
     active = int((cnt > 0).sum())

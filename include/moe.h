@@ -120,8 +120,9 @@ typedef struct {
   int32_t dropped;        /* slots left empty                                     */
   int32_t refined_tokens; /* tokens whose decision was re-taken in binary64       */
   int32_t max_load;       /* largest per-expert slot count                        */
+  int32_t refined_logits; /* router logits recomputed in binary64 (all tokens)    */
   int32_t status;         /* moe_status seen on the device                        */
-  int32_t reserved[3];
+  int32_t reserved[2];
 } moe_diag;
 
 /*

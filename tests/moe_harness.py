@@ -79,7 +79,7 @@ def run_layer(w: W.Workload, inp: dict, n=None, diag=True):
 
 def diag_dict(dg: torch.Tensor) -> dict:
     v = dg.cpu().tolist()
-    return dict(zip(moe.DIAG_FIELDS, v[:5]))
+    return dict(zip(moe.DIAG_FIELDS, v))
 
 
 def first_mismatch(a: np.ndarray, b: np.ndarray) -> int:

@@ -199,6 +199,42 @@ def test_single_token_and_ragged_sizes():
         assert H.rel_err(H.as_f64(got["y"])[keep], r["y"][keep]) <= H.TOL[w.dtype]
 
 
+def _staged_layer(w, dev):
+    """The layer through the staged entry points: route, permute (permuted copy), expert FFN, combine."""
+    n, k, d = w.n, w.top_k, w.d_model
+    cfg = H.cfg_for(w)
+    ws = H.workspace(cfg, n)
+    wts = H.weights_for(dev)
+    idx = torch.empty((n, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((n, k), dtype=torch.float32, device="cuda")
+    counts = torch.empty(w.n_routed, dtype=torch.int32, device="cuda")
+    dg = torch.zeros(8, dtype=torch.int32, device="cuda")
+    offs = torch.empty(w.n_routed + 1, dtype=torch.int32, device="cuda")
+    perm = torch.empty(n * k, dtype=torch.int32, device="cuda")
+    dest = torch.empty((n, k), dtype=torch.int32, device="cuda")
+    xp = torch.empty((n * k, d), dtype=dev["x"].dtype, device="cuda")
+    eo = torch.empty((n * k, d), dtype=dev["x"].dtype, device="cuda")
+    y = torch.empty((n, d), dtype=dev["x"].dtype, device="cuda")
+    moe.moe_route(cfg, n, dev["x"], wts, idx, tw, counts, dg, ws)
+    moe.moe_permute(cfg, n, dev["x"], idx, offs, perm, dest, xp, ws)
+    moe.moe_expert_ffn(cfg, n, xp, offs, wts, eo, ws)
+    moe.moe_combine(cfg, n, eo, dest, tw, dev["x"], wts, y, ws)
+    assert moe.moe_sync_status(ws) == moe.MOE_OK
+    return y
+
+
+@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+@pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "ragged_small"])
+def test_layer_equals_staged_path(name, mode, monkeypatch):
+    """moe_layer_forward (shared experts on the side stream) equals route -> permute ->
+    expert FFN -> combine through the staged entry points bit for bit."""
+    monkeypatch.setenv("MOE_TC_MODE", mode)
+    w = W.get(name)
+    dev = W.device_inputs(w)
+    fused = H.run_layer(w, dev)["y"]
+    assert torch.equal(fused, _staged_layer(w, dev))
+
+
 # Group sizes around the 128-row and 256-row tile edges: empty groups, one row,
 # exact multiples, one past them, and groups whose last tile is half height.
 EDGE_COUNTS = [0, 1, 64, 127, 128, 129, 255, 256, 257, 300, 384, 385, 513, 640, 0]

@@ -50,10 +50,11 @@ class moe_weights(ctypes.Structure):
 
 class moe_diag(ctypes.Structure):
     _fields_ = [("overflowed", ctypes.c_int32), ("dropped", ctypes.c_int32), ("refined_tokens", ctypes.c_int32),
-                ("max_load", ctypes.c_int32), ("status", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("max_load", ctypes.c_int32), ("refined_logits", ctypes.c_int32), ("status", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
-DIAG_FIELDS = ("overflowed", "dropped", "refined_tokens", "max_load", "status")
+DIAG_FIELDS = ("overflowed", "dropped", "refined_tokens", "max_load", "refined_logits", "status")
 
 _P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
 _lib.moe_workspace_size.argtypes = [_P, _I64, ctypes.POINTER(ctypes.c_size_t)]

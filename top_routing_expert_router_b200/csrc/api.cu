@@ -2,6 +2,7 @@
 // workspace carving and the launch sequence of each stage on the caller's
 // stream. No allocation, no host synchronisation (except moe_sync_status).
 #include <math.h>
+#include <stddef.h>
 #include <string.h>
 
 #include <mutex>
@@ -192,13 +193,17 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
                       moe_diag* diag) {
   const moe_config& c = x.c;
   moe_diag* d = diag ? diag : x.status();
-  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), x.s));  // counters, not the status word
+  static_assert(offsetof(moe_diag, status) == 5 * sizeof(int32_t), "the counters precede the status word");
+  MOE_CUDA(cudaMemsetAsync(d, 0, 5 * sizeof(int32_t), x.s));  // the counters, not the status word
   if (x.n == 0) {
     if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
     return MOE_OK;
   }
   RouteArgs r;
   MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
+  // token cursor of the router's warps, in the workspace's own diag block
+  r.cursor = &x.status()->reserved[0];
+  MOE_CUDA(cudaMemsetAsync(r.cursor, 0, sizeof(int32_t), x.s));
   if (c.cap_policy == MOE_CAP_NONE) {
     r.ranking = nullptr;
     MOE_CUDA(launch_route(r, x.s));
@@ -358,7 +363,7 @@ moe_status moe_route_hash(const moe_config* cfg, int64_t n, const void* x, const
   MOE_TRY(check_weights(c.c, weights, false, false));
   MOE_TRY(clear_status(c));
   moe_diag* d = diag ? diag : c.status();
-  MOE_CUDA(cudaMemsetAsync(d, 0, 4 * sizeof(int32_t), c.s));
+  MOE_CUDA(cudaMemsetAsync(d, 0, 5 * sizeof(int32_t), c.s));
   if (n == 0) {
     if (expert_counts) MOE_CUDA(launch_fill_i32(expert_counts, c.c.n_routed, 0, c.s));
     return MOE_OK;

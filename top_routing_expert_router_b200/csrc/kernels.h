@@ -51,7 +51,8 @@ struct RouteArgs {
   uint16_t* ranking;    // [n, E] eligible experts in selection order (capacity), or nullptr
   int32_t* topk_idx;    // [n, k] (written when ranking == nullptr)
   float* topk_w;        // [n, k]
-  moe_diag* diag;       // refined_tokens counter
+  moe_diag* diag;       // refined_tokens / refined_logits counters
+  int32_t* cursor;      // zeroed before the launch: next token to route (warps fetch tokens from it)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 

@@ -467,13 +467,16 @@ __device__ double dot64(const RouteArgs& a, int64_t t, int e) {
   return warp_sum(acc0 + acc1);
 }
 
-// Replace the logits of the experts in `which` (bits over j, per lane) by binary64 values.
+// Replace the logits of the experts in `which` (bits over j, per lane) by
+// binary64 values. Returns how many were recomputed.
 template <int EPL>
-__device__ void refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], uint32_t which) {
+__device__ int refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], uint32_t which) {
   const int lane = threadIdx.x & 31;
+  int total = 0;
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     uint32_t m = __ballot_sync(kFull, (which >> j) & 1u);
+    total += __popc(m);
     while (m) {
       const int src = __ffs(m) - 1;
       m &= m - 1;
@@ -481,6 +484,7 @@ __device__ void refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], u
       if (lane == src) l[j] = s;
     }
   }
+  return total;
 }
 
 // Load a token's logits, summing the split-K partial GEMM results in order.
@@ -503,8 +507,6 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
   __shared__ uint8_t s_flag[kWarpsPerBlock][kMaxExperts];
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   constexpr bool full_ranking = FULL;  // the capacity rule needs every eligible expert ranked
   for (int i = lane; i < kMaxExperts; i += 32) s_flag[wib][i] = 0;
   __syncwarp();
@@ -512,7 +514,13 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
 #pragma unroll
   for (int j = 0; j < EPL; ++j)
     if (lane + 32 * j < a.E) valid_mask |= 1u << j;
-  for (int64_t t = warp; t < a.n; t += nwarps) {
+  // Warps take the next token from a shared cursor: a token that needs binary64
+  // refinement holds up only its own warp, never a whole block of tokens.
+  for (;;) {
+    int tok = 0;
+    if (lane == 0) tok = atomicAdd(a.cursor, 1);
+    const int64_t t = __shfl_sync(kFull, tok, 0);
+    if (t >= a.n) break;
     double l[EPL];
     load_logits<EPL>(a, t, l);
     double amax = 0.0;
@@ -528,7 +536,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
                                                                   : delta_l;
     uint32_t exact = 0;
     int nr = 0;
-    bool refined = false;
+    int n_refined = 0;
     for (int it = 0;; ++it) {
       uint32_t refine = 0;
       bool ok;
@@ -539,11 +547,13 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
       if (ok) break;
       refine &= ~exact;
       if (it >= 3 || !__any_sync(kFull, refine != 0)) refine = valid_mask & ~exact;  // refine the rest
-      refine_logits<EPL>(a, t, l, refine);
+      n_refined += refine_logits<EPL>(a, t, l, refine);
       exact |= refine;
-      refined = true;
     }
-    if (refined && lane == 0 && a.diag) atomicAdd(&a.diag->refined_tokens, 1);
+    if (n_refined && lane == 0 && a.diag) {
+      atomicAdd(&a.diag->refined_tokens, 1);
+      atomicAdd(&a.diag->refined_logits, n_refined);
+    }
     if (full_ranking) {
       for (int r = lane; r < a.E; r += 32) a.ranking[t * a.E + r] = r < nr ? (uint16_t)s_rank[wib][r] : (uint16_t)0xFFFF;
       __syncwarp();
@@ -629,6 +639,10 @@ __global__ void bias_update_kernel(const int32_t* counts, int32_t E, float gamma
 constexpr int kCapThreads = 1024;
 constexpr int kCapPrefix = 64;  // ranking entries per token staged in shared memory
 
+// 32-bit words per staged row: enough for P entries and odd, so that the lanes
+// of a warp reading the same ranking position hit 32 different banks.
+__host__ __device__ constexpr int cap_row_words(int P) { return ((P + 1) / 2) | 1; }
+
 // counts[e] += 1 for every lane whose slot holds e (e < 0: nothing), one
 // shared-memory atomic per distinct expert in the warp: popular experts would
 // otherwise serialise hundreds of atomics on one address.
@@ -644,7 +658,7 @@ __device__ __forceinline__ void warp_count(int* counts, int e) {
 __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k,
                                                             int64_t C, int policy, int32_t* topk_idx,
                                                             moe_diag* diag) {
-  extern __shared__ __align__(16) uint16_t st[];  // [kCapThreads][P] staged ranking prefixes
+  extern __shared__ __align__(16) uint16_t st[];  // [kCapThreads][2 * row words] staged ranking prefixes
   __shared__ int cnt[kMaxExperts];
   __shared__ int ccnt[kMaxExperts];
   __shared__ uint32_t full[kMaxExperts / 32];
@@ -655,6 +669,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
   __shared__ unsigned long long s_over, s_drop;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   const int P = E < kCapPrefix ? E : kCapPrefix;
+  const int RW = cap_row_words(P);  // 32-bit words per staged row
   for (int e = tid; e < kMaxExperts; e += kCapThreads) cnt[e] = 0;
   if (tid < kMaxExperts / 32) full[tid] = 0;
   if (tid == 0) s_over = s_drop = 0;
@@ -664,18 +679,24 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
   for (int64_t w0 = 0; w0 < n; w0 += kCapThreads) {
     const int cnt_tok = (int)((n - w0) < kCapThreads ? (n - w0) : kCapThreads);
     if (E % 8 == 0) {
-      const int vpr = P / 8;  // 16-byte vectors per staged row
+      const int vpr = P / 8;  // 16-byte vectors per staged row, stored as four words each
+      uint32_t* st32 = reinterpret_cast<uint32_t*>(st);
       for (int i = tid; i < cnt_tok * vpr; i += kCapThreads) {
         const int row = i / vpr, v = i % vpr;
-        reinterpret_cast<uint4*>(st)[row * vpr + v] = reinterpret_cast<const uint4*>(ranking + (w0 + row) * E)[v];
+        const uint4 q = reinterpret_cast<const uint4*>(ranking + (w0 + row) * E)[v];
+        uint32_t* dst = st32 + row * RW + 4 * v;
+        dst[0] = q.x;
+        dst[1] = q.y;
+        dst[2] = q.z;
+        dst[3] = q.w;
       }
     } else {
-      for (int i = tid; i < cnt_tok * P; i += kCapThreads) st[i] = ranking[(w0 + i / P) * E + i % P];
+      for (int i = tid; i < cnt_tok * P; i += kCapThreads) st[(i / P) * 2 * RW + i % P] = ranking[(w0 + i / P) * E + i % P];
     }
     __syncthreads();
     const int64_t t = w0 + tid;
     const bool valid = tid < cnt_tok;
-    const uint16_t* srow = st + tid * P;
+    const uint16_t* srow = st + tid * 2 * RW;
     const uint16_t* grow = ranking + t * E;
     int ch[kMaxTopK];  // current choices (in ranking order); -1 = empty slot
     int pos[kMaxTopK];  // their ranking positions
@@ -812,18 +833,38 @@ unsigned route_grid(int64_t n) {
 
 }  // namespace
 
+// Persistent grid: as many blocks as fit on the device at once (tokens come
+// from the cursor), never more than the tokens need.
+template <int EPL, bool FULL>
+cudaError_t launch_route_t(const RouteArgs& a, cudaStream_t s) {
+  static int resident = 0;
+  if (!resident) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, route_kernel<EPL, FULL>, 32 * kWarpsPerBlock, 0) !=
+            cudaSuccess ||
+        per_sm <= 0)
+      per_sm = 1;
+    int dev = 0, sms = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    resident = per_sm * (sms > 0 ? sms : 148);
+  }
+  const int64_t need = ceil_div(a.n, kWarpsPerBlock);
+  const unsigned grid = (unsigned)(need < resident ? need : resident);
+  route_kernel<EPL, FULL><<<grid, 32 * kWarpsPerBlock, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
   if (a.n <= 0) return cudaSuccess;
-  const unsigned grid = route_grid(a.n);
-  const unsigned block = 32 * kWarpsPerBlock;
+  if (!a.cursor) return cudaErrorInvalidValue;
   const bool full = a.ranking != nullptr;
   switch (epl_for(a.E)) {
-    case 1: full ? route_kernel<1, true><<<grid, block, 0, s>>>(a) : route_kernel<1, false><<<grid, block, 0, s>>>(a); break;
-    case 2: full ? route_kernel<2, true><<<grid, block, 0, s>>>(a) : route_kernel<2, false><<<grid, block, 0, s>>>(a); break;
-    case 4: full ? route_kernel<4, true><<<grid, block, 0, s>>>(a) : route_kernel<4, false><<<grid, block, 0, s>>>(a); break;
-    default: full ? route_kernel<8, true><<<grid, block, 0, s>>>(a) : route_kernel<8, false><<<grid, block, 0, s>>>(a); break;
+    case 1: return full ? launch_route_t<1, true>(a, s) : launch_route_t<1, false>(a, s);
+    case 2: return full ? launch_route_t<2, true>(a, s) : launch_route_t<2, false>(a, s);
+    case 4: return full ? launch_route_t<4, true>(a, s) : launch_route_t<4, false>(a, s);
+    default: return full ? launch_route_t<8, true>(a, s) : launch_route_t<8, false>(a, s);
   }
-  return cudaGetLastError();
 }
 
 cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s) {
@@ -857,11 +898,11 @@ cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32
                             int32_t* topk_idx, moe_diag* diag, cudaStream_t s) {
   if (n <= 0) return cudaSuccess;
   const int P = E < kCapPrefix ? E : kCapPrefix;
-  const size_t smem = (size_t)kCapThreads * P * sizeof(uint16_t);
+  const size_t smem = (size_t)kCapThreads * cap_row_words(P) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(capacity_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(kCapThreads * kCapPrefix * 2));
+    const cudaError_t e = cudaFuncSetAttribute(capacity_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)(kCapThreads * cap_row_words(kCapPrefix) * sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
     attr = true;
   }
