@@ -17,7 +17,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace layout; every region starts on a 256-byte boundary.
 struct Plan {
-  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, total;
+  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched, total;
 };
 
 // Split-K factor of the router GEMM: small token counts leave most SMs idle
@@ -64,6 +64,7 @@ Plan make_plan(const moe_config& c, int64_t n) {
   p.shh = take((size_t)(Is > 0 ? n * Is : 0) * b);
   p.sh = take((size_t)(Is > 0 ? n * c.d_model : 0) * b);
   p.shoff = take(2 * 4);
+  p.sched = take(4 * 4);  // tile counters of the SM-pair GEMM launches (routed GEMM1/2, shared GEMM1/2)
   p.total = off;
   return p;
 }
@@ -238,9 +239,12 @@ moe_status ffn_impl(const Ctx& x, const void* xperm, const int32_t* offsets, con
   if (x.n == 0) return MOE_OK;
   const int64_t I = c.moe_intermediate_size, d = c.d_model, nk = x.n * c.top_k;
   void* h = x.ws + x.p.h;
+  int32_t* sched = x.at<int32_t>(x.p.sched);
   GemmArgs g1{xperm, d, w->w_gate, w->w_up, I * d, h, I, offsets, c.n_routed, nk, (int32_t)I, (int32_t)d};
+  g1.tile_counter = sched;
   MOE_TRY(gemm(x, g1, true, false));
   GemmArgs g2{h, I, w->w_down, nullptr, d * I, eo, d, offsets, c.n_routed, nk, (int32_t)d, (int32_t)I};
+  g2.tile_counter = sched + 1;
   MOE_TRY(gemm(x, g2, false, false));
   return MOE_OK;
 }
@@ -252,9 +256,12 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
   const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size, d = c.d_model;
   void* shh = x.ws + x.p.shh;
   void* sh = x.ws + x.p.sh;
+  int32_t* sched = x.at<int32_t>(x.p.sched);
   GemmArgs g1{X, d, w->ws_gate, w->ws_up, 0, shh, Is, nullptr, 1, x.n, (int32_t)Is, (int32_t)d};
+  g1.tile_counter = sched + 2;
   MOE_TRY(gemm(x, g1, true, false));
   GemmArgs g2{shh, Is, w->ws_down, nullptr, 0, sh, d, nullptr, 1, x.n, (int32_t)d, (int32_t)Is};
+  g2.tile_counter = sched + 3;
   MOE_TRY(gemm(x, g2, false, false));
   *sh_out = sh;
   return MOE_OK;

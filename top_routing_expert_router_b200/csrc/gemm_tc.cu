@@ -66,6 +66,7 @@ struct TcParams {
   moe_diag* status;
   uint64_t timeout_ns;  // limit of any single barrier wait
   int32_t test_stall;   // fault injection: withhold the first copy of each CTA
+  int32_t* tile_counter;  // SM-pair kernel: next tile to hand out (zeroed before the launch)
 };
 
 struct __align__(8) SmemCtl {
@@ -475,12 +476,18 @@ constexpr int A2_HALF_BYTES = 64 * BK * 2;  // half-height tile: 64 A rows per C
 constexpr int B2_BYTES = 128 * BK * 2;
 constexpr int STAGE2_BYTES = A2_BYTES + B2_BYTES;
 
+constexpr int kTileSlots = 4;    // tile indices published ahead of the slowest reader
+constexpr int kTileReaders = 10;  // leader MMA + 4 leader epilogue warps + peer producer + 4 peer epilogue warps
+
 struct __align__(8) SmemCtl2 {
   uint64_t timeout_ns;
   uint64_t full[STAGES2];
   uint64_t empty[STAGES2];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
+  uint64_t tile_full[kTileSlots];   // both CTAs: tile_ring[slot] holds the next tile
+  uint64_t tile_empty[kTileSlots];  // leader CTA: every reader of both CTAs took the slot's tile
+  int32_t tile_ring[kTileSlots];
   uint64_t drain;
   uint32_t tmem_base;
   int32_t abort;
@@ -578,6 +585,66 @@ __device__ __noinline__ bool mbar_wait2(uint64_t* bar, uint32_t parity, SmemCtl2
   }
 }
 
+// Cluster-scope acquire: the tile barriers order data written by the other CTA of the pair.
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, SmemCtl2* ctl, moe_diag* st) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try_cluster(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_cluster(b, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > ctl->timeout_ns) {
+        atomicExch(&ctl->abort, 1);
+        set_status(st, MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// Dynamic tile schedule of a CTA pair. The leader's producer takes the next
+// tile index from the global counter and publishes it in slot i % kTileSlots of
+// both CTAs; every other role reads it from there, so all roles of the pair
+// walk the same tile sequence and the pairs stay within about one tile of each
+// other in the global tile order (tiles that share B run at the same time).
+__device__ int publish_tile(SmemCtl2* ctl, int i, const TcParams& p) {
+  const int slot = i % kTileSlots;
+  const uint32_t par = (uint32_t)(i / kTileSlots) & 1u;
+  if (!mbar_wait_cluster(&ctl->tile_empty[slot], par ^ 1u, ctl, p.status)) return -1;
+  const int t = atomicAdd(p.tile_counter, 1);
+  ctl->tile_ring[slot] = t;
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(map_to_rank(&ctl->tile_ring[slot], 1)), "r"(t) : "memory");
+  mbar_arrive(&ctl->tile_full[slot]);
+  mbar_arrive_cluster(map_to_rank(&ctl->tile_full[slot], 1));
+  return t;
+}
+
+// A reader's next tile (one thread per role); -1 after a timeout or an abort.
+__device__ int take_tile(SmemCtl2* ctl, int i, uint32_t rank, const TcParams& p) {
+  const int slot = i % kTileSlots;
+  const uint32_t par = (uint32_t)(i / kTileSlots) & 1u;
+  if (!mbar_wait_cluster(&ctl->tile_full[slot], par, ctl, p.status)) return -1;
+  const int t = *reinterpret_cast<volatile int32_t*>(&ctl->tile_ring[slot]);
+  if (rank == 0)
+    mbar_arrive(&ctl->tile_empty[slot]);
+  else
+    mbar_arrive_cluster(map_to_rank(&ctl->tile_empty[slot], 0));
+  return t;
+}
+
 __device__ __noinline__ void spin_ns(uint64_t ns) {
   const uint64_t t0 = globaltimer();
   while (globaltimer() - t0 < ns) {
@@ -592,7 +659,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   SmemCtl2* ctl = reinterpret_cast<SmemCtl2*>(smem + STAGES2 * STAGE2_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_rank();
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     int acc = 0;
@@ -615,6 +681,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tmem_full[b], 1);
       mbar_init(&ctl->tmem_empty[b], 8);
+    }
+    for (int q = 0; q < kTileSlots; ++q) {
+      mbar_init(&ctl->tile_full[q], 1);
+      mbar_init(&ctl->tile_empty[q], kTileReaders);
     }
     mbar_init(&ctl->drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -647,7 +717,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0;
       uint32_t phase = 0;
       int g_hint = 0;
-      for (int t = pair; t < total && !aborted; t += npairs) {
+      for (int i = 0; !aborted; ++i) {
+        const int t = rank == 0 ? publish_tile(ctl, i, p) : take_tile(ctl, i, rank, p);
+        if (t < 0) {
+          aborted = true;
+          break;
+        }
+        if (t >= total) break;
         const Tile tl = decode2(ctl, p, t, g_hint);
         const bool half = tl.half != 0;
         const uint32_t tx = 2u * ((half ? A2_HALF_BYTES : A2_BYTES) + B2_BYTES);
@@ -663,7 +739,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           uint8_t* sa = smem + stage * STAGE2_BYTES;
-          if (p.test_stall && t == pair && kb == 0) {
+          if (p.test_stall && i == 0 && kb == 0) {
             // injected fault: this stage is never filled, so the MMA's wait on it runs out
             if (++stage == STAGES2) {
               stage = 0;
@@ -695,9 +771,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t idesc_full = idesc_bf16_pair(BM2, BN_MAX);
       const uint32_t idesc_half = idesc_bf16_pair(BM2 / 2, BN_MAX);
       bool issued = false;
-      int i = 0;
       int g_hint = 0;
-      for (int t = pair; t < total && !aborted; t += npairs, ++i) {
+      for (int i = 0; !aborted; ++i) {
+        const int t = take_tile(ctl, i, 0, p);
+        if (t < 0) {
+          aborted = true;
+          break;
+        }
+        if (t >= total) break;
         const uint32_t idesc = decode2(ctl, p, t, g_hint).half ? idesc_half : idesc_full;
         const int buf = i & 1;
         const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
@@ -745,8 +826,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const uint32_t leader_tmem_empty[2] = {map_to_rank(&ctl->tmem_empty[0], 0), map_to_rank(&ctl->tmem_empty[1], 0)};
     int g_hint = 0;
-    int i = 0;
-    for (int t = pair; t < total; t += npairs, ++i) {
+    for (int i = 0;; ++i) {
+      int t = 0;
+      if (lane == 0) t = take_tile(ctl, i, rank, p);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t < 0) {
+        aborted = true;
+        break;
+      }
+      if (t >= total) break;
       const int buf = i & 1;
       const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
       const Tile tl = decode2(ctl, p, t, g_hint);
@@ -935,6 +1023,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   const char* stall = getenv("MOE_TEST_STALL");
   p.test_stall = stall && stall[0] == '1';
   p.timeout_ns = p.test_stall ? kTestTimeoutNs : kTimeoutNs;
+  p.tile_counter = a.tile_counter;
   CUtensorMap ma, mb, mb2;
   const int64_t b_total_rows = (int64_t)a.G * a.N;
   const bool pair = use_pair_tiles(a, swiglu, out_f32);
@@ -980,6 +1069,11 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
     // resident at once: a pair that only starts when another one exits would
     // run its whole share after the others. On parts whose GPCs hold odd SM
     // counts fewer than SMs/2 pairs fit, hence the occupancy query.
+    if (!a.tile_counter) return cudaErrorInvalidValue;
+    {
+      const cudaError_t e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s);
+      if (e != cudaSuccess) return e;
+    }
     const int pairs_resident = max_resident_pairs(cfg);
     if (pairs_resident <= 0) return cudaErrorInvalidConfiguration;
     const int64_t pairs = max_pair_tiles < pairs_resident ? max_pair_tiles : pairs_resident;

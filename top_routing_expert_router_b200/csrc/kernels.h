@@ -26,6 +26,7 @@ struct GemmArgs {
   int32_t K;
   int32_t k_splits = 1;         // > 1: split-K, partial results written k_splits times
   int64_t c_split_stride = 0;   // elements between the partial result matrices
+  int32_t* tile_counter = nullptr;  // device int32 the SM-pair kernel hands out tiles from (zeroed per launch)
 };
 
 cudaError_t launch_gemm_simt(const GemmArgs& a, int dtype, bool out_f32, bool swiglu, cudaStream_t s);
