@@ -43,8 +43,8 @@ def test_device_inputs_equal_host_inputs(name):
 
 
 @pytest.mark.parametrize("name", SMALL)
-def test_route_parity(name):
-    w = W.get(name)
+def test_route_parity(name, w=None):
+    w = w or W.get(name)
     dev, host = W.device_inputs(w), W.host_inputs(w)
     cfg = H.cfg_for(w)
     ws = H.workspace(cfg, w.n)
@@ -75,6 +75,15 @@ def test_route_parity(name):
         np.testing.assert_array_equal(counts.cpu().numpy(), np.bincount(oi[oi >= 0], minlength=w.n_routed))
         assert diag["max_load"] == np.bincount(oi[oi >= 0], minlength=w.n_routed).max()
     assert ex.mean() < 0.05
+
+
+@pytest.mark.parametrize("policy", ["overflow_next", "drop"])
+@pytest.mark.parametrize("k", [1, 3, 4, 6, 8])
+def test_capacity_route_parity_across_top_k(k, policy):
+    """The capacity kernel keeps a token's choices in registers for top_k 1, 2, 4, 8 and in a
+    local array otherwise; both match the oracle's greedy."""
+    w = W.get("skewed_small", top_k=k, cap_policy=policy, n=1500)
+    test_route_parity(w.name, w)
 
 
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "skewed_small", "drop_small", "tiny_f32"])

@@ -655,9 +655,40 @@ __device__ __forceinline__ void warp_count(int* counts, int e) {
 // its current choices and a cursor into its ranking; after a fill event only
 // the tokens that lost a choice walk on from their cursor, so every ranking
 // entry of a window is read at most once.
-__global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k,
+// A token's current choices and their ranking positions. For k known at
+// compile time (REG) the slots live in registers (indexed through unrolled
+// selects); otherwise in a local array of kMaxTopK.
+template <int KA, bool REG>
+struct Slots {
+  int v[KA];
+  __device__ __forceinline__ int get(int i) const {
+    if constexpr (REG) {
+      int r = -1;
+#pragma unroll
+      for (int q = 0; q < KA; ++q)
+        if (q == i) r = v[q];
+      return r;
+    } else {
+      return v[i];
+    }
+  }
+  __device__ __forceinline__ void set(int i, int x) {
+    if constexpr (REG) {
+#pragma unroll
+      for (int q = 0; q < KA; ++q)
+        if (q == i) v[q] = x;
+    } else {
+      v[i] = x;
+    }
+  }
+};
+
+template <int KT>  // KT = top_k when it is 1, 2, 4 or 8; 0 = any top_k up to kMaxTopK
+__global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* ranking, int64_t n, int E, int k_arg,
                                                             int64_t C, int policy, int32_t* topk_idx,
                                                             moe_diag* diag) {
+  constexpr int KA = KT > 0 ? KT : kMaxTopK;
+  const int k = KT > 0 ? KT : k_arg;
   extern __shared__ __align__(16) uint16_t st[];  // [kCapThreads][2 * row words] staged ranking prefixes
   __shared__ int cnt[kMaxExperts];
   __shared__ int ccnt[kMaxExperts];
@@ -698,8 +729,8 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
     const bool valid = tid < cnt_tok;
     const uint16_t* srow = st + tid * 2 * RW;
     const uint16_t* grow = ranking + t * E;
-    int ch[kMaxTopK];  // current choices (in ranking order); -1 = empty slot
-    int pos[kMaxTopK];  // their ranking positions
+    Slots<KA, (KT > 0)> ch;   // current choices (in ranking order); -1 = empty slot
+    Slots<KA, (KT > 0)> pos;  // their ranking positions
     int taken = 0, cursor = 0;
     // walk on from the cursor until k non-full experts are held (overflow policy)
     auto refill = [&]() {
@@ -710,8 +741,8 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
           break;
         }
         if (!is_full(e)) {
-          ch[taken] = e;
-          pos[taken] = cursor;
+          ch.set(taken, e);
+          pos.set(taken, cursor);
           ++taken;
         }
         ++cursor;
@@ -723,7 +754,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
       } else {
         for (int j = 0; j < k; ++j) {
           const int e = srow[j];
-          ch[j] = (e != 0xFFFF && !is_full(e)) ? e : -1;
+          ch.set(j, (e != 0xFFFF && !is_full(e)) ? e : -1);
         }
       }
     }
@@ -731,8 +762,8 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
     while (true) {
       const bool active = valid && tid >= f;
       auto slot = [&](int j) {
-        if (policy == MOE_CAP_OVERFLOW_NEXT) return j < taken ? ch[j] : -1;
-        return ch[j];
+        if (policy == MOE_CAP_OVERFLOW_NEXT) return j < taken ? ch.get(j) : -1;
+        return ch.get(j);
       };
       for (int e = tid; e < E; e += kCapThreads) ccnt[e] = 0;
       if (tid == 0) {
@@ -777,7 +808,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
           const int e = slot(j);
           topk_idx[t * k + j] = e;
           my_drop += e < 0;
-          if (policy == MOE_CAP_OVERFLOW_NEXT && j < taken) my_over += pos[j] >= k;
+          if (policy == MOE_CAP_OVERFLOW_NEXT && j < taken) my_over += pos.get(j) >= k;
         }
       }
       if (s < kCapThreads) {
@@ -797,11 +828,15 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
       if (valid && tid >= f) {
         if (policy == MOE_CAP_OVERFLOW_NEXT) {
           int kept = 0;
-          for (int j = 0; j < taken; ++j)
-            if (!is_full(ch[j])) {
-              ch[kept] = ch[j];
-              pos[kept] = pos[j];
-              ++kept;
+          for (int j = 0; j < k; ++j)
+            if (j < taken) {
+              const int cj = ch.get(j);
+              if (!is_full(cj)) {
+                const int pj = pos.get(j);
+                ch.set(kept, cj);
+                pos.set(kept, pj);
+                ++kept;
+              }
             }
           if (kept < taken) {
             taken = kept;
@@ -809,7 +844,7 @@ __global__ void __launch_bounds__(kCapThreads) capacity_kernel(const uint16_t* r
           }
         } else {
           for (int j = 0; j < k; ++j)
-            if (ch[j] >= 0 && is_full(ch[j])) ch[j] = -1;
+            if (ch.get(j) >= 0 && is_full(ch.get(j))) ch.set(j, -1);
         }
       }
     }
@@ -901,12 +936,21 @@ cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32
   const size_t smem = (size_t)kCapThreads * cap_row_words(P) * sizeof(uint32_t);
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(capacity_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)(kCapThreads * cap_row_words(kCapPrefix) * sizeof(uint32_t)));
-    if (e != cudaSuccess) return e;
+    const int bytes = (int)(kCapThreads * cap_row_words(kCapPrefix) * sizeof(uint32_t));
+    for (const void* f : {(const void*)capacity_kernel<1>, (const void*)capacity_kernel<2>, (const void*)capacity_kernel<4>,
+                          (const void*)capacity_kernel<8>, (const void*)capacity_kernel<0>}) {
+      const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+      if (e != cudaSuccess) return e;
+    }
     attr = true;
   }
-  capacity_kernel<<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag);
+  switch (k) {
+    case 1: capacity_kernel<1><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
+    case 2: capacity_kernel<2><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
+    case 4: capacity_kernel<4><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
+    case 8: capacity_kernel<8><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
+    default: capacity_kernel<0><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
+  }
   return cudaGetLastError();
 }
 
