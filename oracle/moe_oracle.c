@@ -475,3 +475,74 @@ void oracle_ds_params(const oracle_ds_arch* a, int64_t* total, int64_t* active) 
   *active = a->n_layers * mla + a->first_k_dense * dense +
             moe_layers * (router + (a->top_k + a->n_shared) * expert) + 2 * embed + norms;
 }
+
+/* ---- FP8 E4M3 codes and UE8M0 block scales ([DS] FP8 section) -------------- */
+
+double oracle_e4m3_value(uint8_t code) {
+  const int sign = code >> 7, ex = (code >> 3) & 15, man = code & 7;
+  double mag;
+  if (ex == 15 && man == 7) return NAN;
+  if (ex == 0)
+    mag = ldexp((double)man, -9);                  /* subnormal: man/8 * 2^-6   */
+  else
+    mag = ldexp(1.0 + man / 8.0, ex - 7);          /* normal: 1.man * 2^(ex-7) */
+  return sign ? -mag : mag;
+}
+
+uint8_t oracle_e4m3_encode(double v) {
+  if (isnan(v)) return 0x7F;
+  const uint8_t sign = signbit(v) ? 0x80 : 0x00;
+  const double a = fabs(v);
+  if (a >= 448.0) return sign | 0x7E;
+  if (a < ldexp(1.0, -6)) {
+    /* subnormal range: multiples of 2^-9; 8 * 2^-9 is the smallest normal, code 0x08 */
+    const double q = nearbyint(ldexp(a, 9));       /* round half to even */
+    return sign | (uint8_t)q;
+  }
+  int x;
+  const double f = frexp(a, &x);                   /* a = f * 2^x, f in [0.5, 1) */
+  int ex = x - 1;                                  /* a = (2f) * 2^ex, 2f in [1, 2) */
+  double m = nearbyint((2.0 * f - 1.0) * 8.0);     /* three mantissa bits, half to even */
+  if (m == 8.0) {
+    m = 0.0;
+    ++ex;
+  }
+  const int field = ex + 7;
+  if (field > 15 || (field == 15 && m > 6.0)) return sign | 0x7E;
+  return sign | (uint8_t)((field << 3) | (int)m);
+}
+
+int32_t oracle_ue8m0_exponent(double amax) {
+  if (!(amax > 0.0)) return 0;
+  int x;
+  const double f = frexp(amax, &x);                /* amax = f * 2^x, f in [0.5, 1) */
+  /* amax <= 448 * 2^e  <=>  f * 2^(x - 8 - e) <= 1.75 (448 = 1.75 * 2^8):
+   * e = x - 8 always holds; e = x - 9 holds iff f <= 0.875; e = x - 10 never. */
+  int32_t e = f <= 0.875 ? x - 9 : x - 8;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+void oracle_quantize_rows(int64_t rows, int32_t cols, const void* src, int32_t src_dt, uint8_t* codes,
+                          uint8_t* scale_byte) {
+  const int32_t tiles = cols / 128;
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int32_t t = 0; t < tiles; ++t) {
+      double amax = 0.0;
+      for (int32_t c = 0; c < 128; ++c) {
+        const int64_t i = r * cols + t * 128 + c;
+        const double v = src_dt == 2 ? ((const double*)src)[i] : elem(src, src_dt, i);
+        if (fabs(v) > amax) amax = fabs(v);
+      }
+      const int32_t e = oracle_ue8m0_exponent(amax);
+      scale_byte[r * tiles + t] = (uint8_t)(e + 127);
+      for (int32_t c = 0; c < 128; ++c) {
+        const int64_t i = r * cols + t * 128 + c;
+        const double v = src_dt == 2 ? ((const double*)src)[i] : elem(src, src_dt, i);
+        codes[i] = oracle_e4m3_encode(ldexp(v, -e));
+      }
+    }
+  }
+}

@@ -125,6 +125,27 @@ void oracle_layer(const oracle_cfg* cfg, int64_t n, const void* x, const void* w
                   double* y, int32_t* topk_idx, double* topk_w, int32_t* counts,
                   uint8_t* exempt, oracle_stats* stats);
 
+/*
+ * FP8 experts ([DS] section "FP8 training is a recipe, not the architecture"):
+ * matrix inputs in E4M3, one scale per 1 x 128 tile of activations and per
+ * 128 x 128 block of weights; V3.1 stores the scales as UE8M0 (an 8-bit
+ * exponent: scale = 2^(byte - 127)).
+ *
+ * E4M3: 1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits, no infinities,
+ * S.1111.111 is NaN, largest finite magnitude 448, subnormals m/8 * 2^-6.
+ */
+double oracle_e4m3_value(uint8_t code);
+/* Nearest E4M3 value, ties to the even mantissa; |v| > 448 saturates to +-448. */
+uint8_t oracle_e4m3_encode(double v);
+/* UE8M0 scale of a block whose largest magnitude is amax: the smallest power of
+ * two 2^e with amax <= 448 * 2^e (e = 0 when amax = 0). Returns e. */
+int32_t oracle_ue8m0_exponent(double amax);
+/* Rows of `cols` values (cols a multiple of 128) quantised in 1 x 128 tiles:
+ * scale_byte[r, t] = e + 127 for tile t, codes[r, c] = encode(v * 2^-e).
+ * src dtype: 0 = binary32, 1 = bf16 bits, 2 = binary64. */
+void oracle_quantize_rows(int64_t rows, int32_t cols, const void* src, int32_t src_dt, uint8_t* codes,
+                          uint8_t* scale_byte);
+
 /* DeepSeek-style architecture fields for the parameter ledger of [DS]. */
 typedef struct {
   int64_t n_layers, d_model, q_lora_rank, kv_lora_rank, n_heads, qk_nope_dim, qk_rope_dim,

@@ -89,6 +89,13 @@ def lib():
         _lib.oracle_ds_params.argtypes = [P, P, P]
         _lib.oracle_route_hash.argtypes = [P, i64, P, P, P, P, P]
         _lib.oracle_bias_update.argtypes = [i32, P, P, ctypes.c_double, P]
+        _lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+        _lib.oracle_e4m3_value.restype = ctypes.c_double
+        _lib.oracle_e4m3_encode.argtypes = [ctypes.c_double]
+        _lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        _lib.oracle_ue8m0_exponent.argtypes = [ctypes.c_double]
+        _lib.oracle_ue8m0_exponent.restype = i32
+        _lib.oracle_quantize_rows.argtypes = [i64, i32, P, i32, P, P]
     return _lib
 
 
@@ -290,3 +297,90 @@ def bf16_to_f64(a: np.ndarray) -> np.ndarray:
     if a.dtype == np.uint16:
         return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return a.astype(np.float64)
+
+
+# ---- FP8 experts (page "15. DeepSeek: MLA, MoE and MTP", FP8 section) -------------------------
+# E4M3 matrix inputs with one UE8M0 scale (2^(byte - 127)) per 1 x 128 activation tile and per
+# 128 x 128 weight block. The layer below quantises activations (x, and h between the two expert
+# matrices) exactly as defined by oracle_quantize_rows and multiplies the dequantised values in
+# binary64 (each dequantised value is exact: a 4-bit significand times a power of two).
+
+def e4m3_value(code: int) -> float:
+    return lib().oracle_e4m3_value(code)
+
+
+def e4m3_encode(v: float) -> int:
+    return lib().oracle_e4m3_encode(float(v))
+
+
+def ue8m0_exponent(amax: float) -> int:
+    return lib().oracle_ue8m0_exponent(float(amax))
+
+
+def e4m3_table() -> np.ndarray:
+    """binary64 value of every code 0..255 (NaN for the two NaN codes)."""
+    return np.array([lib().oracle_e4m3_value(c) for c in range(256)], np.float64)
+
+
+def quantize_rows(a: np.ndarray):
+    """Rows of a [rows, cols] (binary64, binary32 or bf16 bits) in 1 x 128 tiles -> (codes uint8, scale bytes uint8)."""
+    a = _c(a)
+    if a.dtype == np.float64:
+        dt = 2
+    else:
+        dt = _dt(a)
+    rows, cols = a.shape
+    assert cols % 128 == 0
+    codes = np.empty((rows, cols), np.uint8)
+    sb = np.empty((rows, cols // 128), np.uint8)
+    lib().oracle_quantize_rows(rows, cols, _ptr(a), dt, _ptr(codes), _ptr(sb))
+    return codes, sb
+
+
+def dequant_rows(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
+    """codes [rows, cols] with one scale byte per 1 x 128 tile -> binary64."""
+    v = e4m3_table()[codes]
+    s = np.ldexp(1.0, scale_bytes.astype(np.int32) - 127)
+    return v * np.repeat(s, 128, axis=1)
+
+
+def dequant_blocks(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
+    """Weight codes [N, K] with one scale byte per 128 x 128 block [ceil(N/128), K/128] -> binary64."""
+    N, K = codes.shape
+    v = e4m3_table()[codes]
+    s = np.ldexp(1.0, scale_bytes.astype(np.int32) - 127)
+    s = np.repeat(np.repeat(s, 128, axis=0)[:N], 128, axis=1)[:, :K]
+    return v * s
+
+
+def swiglu_fp8(x64: np.ndarray, wg, wu, wd) -> np.ndarray:
+    """One FP8 expert on rows x64 [m, d]: quantise x, gate/up with dequantised weights, SwiGLU,
+    quantise h, down. wg/wu/wd are (codes, scale bytes) pairs."""
+    xq, xs = quantize_rows(x64)
+    xd = dequant_rows(xq, xs)
+    g = xd @ dequant_blocks(*wg).T
+    u = xd @ dequant_blocks(*wu).T
+    h = g / (1.0 + np.exp(-g)) * u
+    hq, hs = quantize_rows(h)
+    return dequant_rows(hq, hs) @ dequant_blocks(*wd).T
+
+
+def layer_fp8(cfg: Cfg, x, w_r, bias, w8: dict, ws8: dict = None):
+    """Whole layer with FP8 experts. x, w_r are bf16 bits (routing as in layer()); w8 holds
+    gate/up/down as (codes [E, N, K], scale bytes [E, N/128, K/128]); ws8 the shared experts'
+    (codes [N, K], scale bytes). Returns dict(y, topk_idx, topk_w, counts, exempt, stats)."""
+    lg = router_logits(x, w_r)
+    idx, w, ex, st = route_capacity(cfg, lg, bias)
+    counts, offsets, perm, dest = dispatch(idx, cfg.n_routed)
+    x64 = bf16_to_f64(x)
+    eo = np.zeros((max(len(perm), 1), cfg.d_model), np.float64)
+    for e in range(cfg.n_routed):
+        lo, hi = offsets[e], offsets[e + 1]
+        if hi > lo:
+            eo[lo:hi] = swiglu_fp8(x64[perm[lo:hi]], (w8["gate"][0][e], w8["gate"][1][e]),
+                                   (w8["up"][0][e], w8["up"][1][e]), (w8["down"][0][e], w8["down"][1][e]))
+    sh = None
+    if ws8 is not None:
+        sh = swiglu_fp8(x64, ws8["gate"], ws8["up"], ws8["down"])
+    y = combine(eo, dest, w, sh)
+    return dict(y=y, topk_idx=idx, topk_w=w, counts=counts, exempt=ex, stats=st)

@@ -54,14 +54,21 @@ enum {
   SYNTH_STREAM_WDOWN = 6,   /* W_down[E, d, I]                           */
   SYNTH_STREAM_WSGATE = 7,  /* shared gate [I_s, d]                      */
   SYNTH_STREAM_WSUP = 8,    /* shared up   [I_s, d]                      */
-  SYNTH_STREAM_WSDOWN = 9   /* shared down [d, I_s]                      */
+  SYNTH_STREAM_WSDOWN = 9,  /* shared down [d, I_s]                      */
+  /* FP8 experts: E4M3 codes and UE8M0 block-scale bytes of each weight */
+  SYNTH_STREAM_WGATE_Q = 10, SYNTH_STREAM_WUP_Q = 11, SYNTH_STREAM_WDOWN_Q = 12,
+  SYNTH_STREAM_WSGATE_Q = 13, SYNTH_STREAM_WSUP_Q = 14, SYNTH_STREAM_WSDOWN_Q = 15,
+  SYNTH_STREAM_WGATE_S = 16, SYNTH_STREAM_WUP_S = 17, SYNTH_STREAM_WDOWN_S = 18,
+  SYNTH_STREAM_WSGATE_S = 19, SYNTH_STREAM_WSUP_S = 20, SYNTH_STREAM_WSDOWN_S = 21
 };
 
 /* Value kinds. */
 enum {
   SYNTH_NORMAL = 0,   /* Irwin-Hall(12) - 6, times sigma                */
   SYNTH_UNIFORM = 1,  /* lo + (hi - lo) * u, u in [0, 1)                */
-  SYNTH_TERNARY = 2   /* one of {-1, 0, +1}, each with probability 1/3  */
+  SYNTH_TERNARY = 2,  /* one of {-1, 0, +1}, each with probability 1/3  */
+  SYNTH_BYTE = 3,     /* integer uniform on [a, b] (0 <= a <= b <= 255)  */
+  SYNTH_SIGNED_CODE = 4 /* byte (sign << 7) | m, m uniform on [a, b] <= 127, sign a fair bit */
 };
 
 SYNTH_FN uint64_t synth_mix64(uint64_t z) {
@@ -100,6 +107,15 @@ SYNTH_FN double synth_value(uint64_t key, uint64_t i, int kind, double a, double
   if (kind == SYNTH_NORMAL) return SYNTH_DMUL(synth_irwin_hall(key, i), a);
   if (kind == SYNTH_UNIFORM) return SYNTH_DADD(a, SYNTH_DMUL(SYNTH_DADD(b, -a), synth_unit(key, i)));
   return (double)((int)(synth_word(key, i) % 3u) - 1);
+}
+
+/* Element i of an integer (byte) stream: integer operations only. */
+SYNTH_FN uint8_t synth_byte(uint64_t key, uint64_t i, int kind, int lo, int hi) {
+  const uint64_t w = synth_word(key, i);
+  const uint32_t span = (uint32_t)(hi - lo + 1);
+  const uint32_t v = (uint32_t)lo + (uint32_t)((w >> 8) % span);
+  if (kind == SYNTH_SIGNED_CODE) return (uint8_t)(((uint32_t)(w & 1u) << 7) | v);
+  return (uint8_t)v;
 }
 
 /* binary32 -> bf16 bits, round to nearest even (inputs here are finite). */

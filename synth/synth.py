@@ -12,8 +12,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 HOST_LIB = os.path.join(_HERE, "libsynth.so")
 CUDA_LIB = os.path.join(_HERE, "libsynth_cuda.so")
 
-NORMAL, UNIFORM, TERNARY = 0, 1, 2
-STREAM = dict(x=1, w_r=2, bias=3, w_gate=4, w_up=5, w_down=6, ws_gate=7, ws_up=8, ws_down=9)
+NORMAL, UNIFORM, TERNARY, BYTE, SIGNED_CODE = 0, 1, 2, 3, 4
+STREAM = dict(x=1, w_r=2, bias=3, w_gate=4, w_up=5, w_down=6, ws_gate=7, ws_up=8, ws_down=9,
+              w_gate_q=10, w_up_q=11, w_down_q=12, ws_gate_q=13, ws_up_q=14, ws_down_q=15,
+              w_gate_s=16, w_up_s=17, w_down_s=18, ws_gate_s=19, ws_up_s=20, ws_down_s=21)
 
 
 def _stale(out, *srcs):
@@ -48,6 +50,7 @@ def _host_lib():
                 ctypes.c_int, ctypes.c_double, ctypes.c_double]
         _host.synth_fill_f32.argtypes = args
         _host.synth_fill_bf16.argtypes = args
+        _host.synth_fill_u8.argtypes = args
     return _host
 
 
@@ -66,7 +69,7 @@ def _cuda_lib():
 
 def host(shape, dtype: str, seed: int, stream: int, kind: int, a: float, b: float = 0.0,
          start: int = 0) -> np.ndarray:
-    """Elements [start, start + prod(shape)) of a stream, as float32 or raw bf16 bits (uint16)."""
+    """Elements [start, start + prod(shape)) of a stream, as float32, raw bf16 bits (uint16) or bytes ("u8")."""
     count = int(np.prod(shape))
     if dtype == "f32":
         out = np.empty(count, np.float32)
@@ -74,17 +77,20 @@ def host(shape, dtype: str, seed: int, stream: int, kind: int, a: float, b: floa
     elif dtype == "bf16":
         out = np.empty(count, np.uint16)
         _host_lib().synth_fill_bf16(out.ctypes.data, count, seed, stream, start, kind, a, b)
+    elif dtype == "u8":
+        out = np.empty(count, np.uint8)
+        _host_lib().synth_fill_u8(out.ctypes.data, count, seed, stream, start, kind, a, b)
     else:
         raise ValueError(dtype)
     return out.reshape(shape)
 
 
 def device(t, seed: int, stream: int, kind: int, a: float, b: float = 0.0, start: int = 0):
-    """Fill a contiguous CUDA tensor (torch.float32 or torch.bfloat16) in place on its current stream."""
+    """Fill a contiguous CUDA tensor (torch.float32, torch.bfloat16 or torch.uint8) in place on its current stream."""
     import torch
 
     assert t.is_cuda and t.is_contiguous()
-    dt = {torch.float32: 0, torch.bfloat16: 1}[t.dtype]
+    dt = {torch.float32: 0, torch.bfloat16: 1, torch.uint8: 2}[t.dtype]
     s = torch.cuda.current_stream(t.device).cuda_stream
     rc = _cuda_lib().synth_cuda_fill(t.data_ptr(), dt, t.numel(), seed, stream, start, kind, a, b, s)
     if rc != 0:

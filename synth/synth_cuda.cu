@@ -15,6 +15,10 @@ __global__ void synth_fill_kernel(void* out, int dtype, int64_t count, uint64_t 
                                   int kind, double a, double b) {
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < count; i += stride) {
+    if (dtype == 2) {
+      static_cast<uint8_t*>(out)[i] = synth_byte(key, (uint64_t)(start + i), kind, (int)a, (int)b);
+      continue;
+    }
     const float v = (float)synth_value(key, (uint64_t)(start + i), kind, a, b);
     if (dtype == 0)
       static_cast<float*>(out)[i] = v;
@@ -25,7 +29,7 @@ __global__ void synth_fill_kernel(void* out, int dtype, int64_t count, uint64_t 
 
 }  // namespace
 
-/* dtype: 0 = binary32, 1 = bf16. Returns a cudaError_t value (0 on success). */
+/* dtype: 0 = binary32, 1 = bf16, 2 = bytes (integer kinds). Returns a cudaError_t value (0 on success). */
 extern "C" int synth_cuda_fill(void* out, int dtype, int64_t count, uint64_t seed, uint64_t stream,
                                int64_t start, int kind, double a, double b, void* cuda_stream) {
   if (count <= 0) return 0;

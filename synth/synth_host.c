@@ -23,3 +23,10 @@ void synth_fill_bf16(uint16_t* out, int64_t count, uint64_t seed, uint64_t strea
   for (int64_t i = 0; i < count; ++i)
     out[i] = synth_f32_to_bf16_bits((float)synth_value(key, (uint64_t)(start + i), kind, a, b));
 }
+
+void synth_fill_u8(uint8_t* out, int64_t count, uint64_t seed, uint64_t stream, int64_t start, int kind, double a,
+                   double b) {
+  const uint64_t key = synth_key(seed, stream);
+#pragma omp parallel for schedule(static)
+  for (int64_t i = 0; i < count; ++i) out[i] = synth_byte(key, (uint64_t)(start + i), kind, (int)a, (int)b);
+}

@@ -81,7 +81,33 @@ class Workload:
             specs["ws_gate"] = ((Is, d), synth.STREAM["ws_gate"], synth.NORMAL, 1.0 / math.sqrt(d), 0.0, dt)
             specs["ws_up"] = ((Is, d), synth.STREAM["ws_up"], synth.NORMAL, 1.0 / math.sqrt(d), 0.0, dt)
             specs["ws_down"] = ((d, Is), synth.STREAM["ws_down"], synth.NORMAL, 1.0 / math.sqrt(I), 0.0, dt)
+        if dt == "fp8":
+            # FP8 experts: activations and router stay bf16; every expert matrix is E4M3 codes plus one
+            # UE8M0 scale byte per 128 x 128 block, drawn directly as bytes (no conversion arithmetic).
+            for nm in ("x", "w_r"):
+                specs[nm] = specs[nm][:5] + ("bf16",)
+            for nm in ("w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down"):
+                if nm not in specs:
+                    continue
+                shape = specs.pop(nm)[0]
+                fan_in = shape[-1]
+                lo, hi = _fp8_scale_bytes(fan_in)
+                sshape = shape[:-2] + (-(-shape[-2] // 128), shape[-1] // 128)
+                specs[nm + "_q"] = (shape, synth.STREAM[nm + "_q"], synth.SIGNED_CODE, FP8_CODE_LO, FP8_CODE_HI, "u8")
+                specs[nm + "_s"] = (sshape, synth.STREAM[nm + "_s"], synth.BYTE, lo, hi, "u8")
         return specs
+
+
+# FP8 weight codes: sign plus a magnitude code uniform on [0x28, 0x47], i.e. E4M3 values of magnitude
+# 0.25 .. 3.75 (exponent fields 5..8, all mantissas); their root mean square is about 1.69.
+FP8_CODE_LO, FP8_CODE_HI, FP8_CODE_RMS = 0x28, 0x47, 1.69
+
+
+def _fp8_scale_bytes(fan_in: int) -> tuple:
+    """UE8M0 scale bytes (e + 127) of the two powers of two around 1 / (1.69 sqrt(fan_in)), so that the
+    weights' root mean square is close to 1/sqrt(fan_in) like the bf16 recipe."""
+    e = math.floor(math.log2(1.0 / (FP8_CODE_RMS * math.sqrt(fan_in))))
+    return e + 127, e + 128
 
 
 def _wl(name, **kw) -> Workload:
@@ -123,6 +149,12 @@ WORKLOADS = {w.name: w for w in [
     _wl("deepseek_v4_small", n=300, d_model=256, n_routed=64, n_shared=1, top_k=6, moe_intermediate_size=128,
         score_fn="sqrtsoftplus", renormalize=True, bias_range=(-0.1, 0.1),
         description="DeepSeek-V4-style routing: sqrtsoftplus scores + bias, no group limit"),
+    # FP8 experts (DeepSeek-V3 checkpoint format: E4M3 with UE8M0 128 x 128 block scales)
+    _wl("deepseek_v3_prefill_fp8", n=16384, dtype="fp8", description="DeepSeek-V3-shaped prefill, FP8 experts", **_V3),
+    _wl("deepseek_v3_decode_fp8", n=64, dtype="fp8", description="DeepSeek-V3-shaped decode, FP8 experts", **_V3),
+    _wl("deepseek_v3_small_fp8", n=333, dtype="fp8", **{**_V3, "d_model": 256, "moe_intermediate_size": 128}),
+    _wl("fp8_ragged_small", n=300, d_model=384, n_routed=12, top_k=3, moe_intermediate_size=256, n_shared=1,
+        dtype="fp8", renormalize=True),
     _wl("tie_softmax", n=256, d_model=64, n_routed=16, top_k=4, moe_intermediate_size=64,
         ternary=True, renormalize=True),
     _wl("tie_sigmoid", n=256, d_model=64, n_routed=32, top_k=4, moe_intermediate_size=64,
@@ -193,7 +225,8 @@ def device_inputs(w: Workload, seed: int = 0, device="cuda", names=None) -> dict
     out = {}
     for nm in names:
         shape, stream, kind, a, b, dt = specs[nm]
-        t = torch.empty(shape, dtype=torch.float32 if dt == "f32" else torch.bfloat16, device=device)
+        t = torch.empty(shape, dtype={"f32": torch.float32, "bf16": torch.bfloat16, "u8": torch.uint8}[dt],
+                        device=device)
         synth.device(t, seed, stream, kind, a, b)
         if w.zipf_s and nm in ("x", "w_r"):
             if nm == "x":
