@@ -353,14 +353,25 @@ def dequant_blocks(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
     return v * s
 
 
+def round_to_bf16(a64: np.ndarray) -> np.ndarray:
+    """binary64 -> binary32 -> bf16 (each round to nearest even), widened back to binary64: the
+    precision in which the kernel holds h when it quantises it."""
+    u = a64.astype(np.float32).view(np.uint32).astype(np.uint64)
+    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
 def swiglu_fp8(x64: np.ndarray, wg, wu, wd) -> np.ndarray:
     """One FP8 expert on rows x64 [m, d]: quantise x, gate/up with dequantised weights, SwiGLU,
-    quantise h, down. wg/wu/wd are (codes, scale bytes) pairs."""
+    quantise h, down. wg/wu/wd are (codes, scale bytes) pairs. The E4M3 codes of h are decided on
+    h held in bf16, the precision the kernel stores it in between the two expert matrices (an E4M3
+    step is 2^4 bf16 steps, so deciding the codes from binary64 h instead moves about 1 in 64
+    codes by one E4M3 step)."""
     xq, xs = quantize_rows(x64)
     xd = dequant_rows(xq, xs)
     g = xd @ dequant_blocks(*wg).T
     u = xd @ dequant_blocks(*wu).T
-    h = g / (1.0 + np.exp(-g)) * u
+    h = round_to_bf16(g / (1.0 + np.exp(-g)) * u)
     hq, hs = quantize_rows(h)
     return dequant_rows(hq, hs) @ dequant_blocks(*wd).T
 

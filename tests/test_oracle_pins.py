@@ -605,3 +605,10 @@ def test_fp8_layer_close_to_unquantised_layer():
     np.testing.assert_array_equal(r8["topk_idx"], ref["topk_idx"])
     err = np.sqrt(((r8["y"] - ref["y"]) ** 2).mean() / (ref["y"] ** 2).mean())
     assert 1e-4 < err < 0.05, err
+
+
+def test_round_to_bf16_matches_torch():
+    rng = np.random.default_rng(5)
+    a = np.concatenate([rng.normal(0, 1, 5000) * rng.lognormal(0, 4, 5000), [0.0, -0.0, 1.0, 3.0 / 7.0]])
+    ref = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(O.round_to_bf16(a), ref)
