@@ -42,6 +42,16 @@
  *     shared experts concatenated along I: ws_gate, ws_up [n_shared*I, d],
  *     ws_down [d, n_shared*I]. Activations and weights share cfg->dtype
  *     (MOE_F32 or MOE_BF16); gates are binary32; indices are int32.
+ *   - MOE_FP8 ([DS] FP8 section: E4M3 matrix inputs, one scale per 1 x 128
+ *     activation tile and per 128 x 128 weight block, scales stored as UE8M0):
+ *     x, y, x_perm, expert_out and w_router are bf16; every expert matrix
+ *     (w_gate, w_up, w_down, ws_*) holds E4M3 codes (one byte per element) with
+ *     its UE8M0 scale bytes (scale = 2^(byte - 127)) in the matching *_scale
+ *     array, [E, ceil(rows/128), cols/128] (shared: [ceil(rows/128), cols/128]).
+ *     Activations entering an expert matrix (x, and h between gate/up and
+ *     down) are quantised to E4M3 in 1 x 128 tiles by the library:
+ *     e = the smallest integer with max|tile| <= 448 * 2^e, code = E4M3 of
+ *     v * 2^-e, round to nearest even. d and I must be multiples of 128.
  *   - Every device pointer must be 16-byte aligned; ws must be 256-byte
  *     aligned.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
@@ -82,7 +92,7 @@ typedef enum {
 
 typedef enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1, MOE_SCORE_SQRTSOFTPLUS = 2 } moe_score_fn;
 typedef enum { MOE_CAP_NONE = 0, MOE_CAP_OVERFLOW_NEXT = 1, MOE_CAP_DROP = 2 } moe_cap_policy;
-typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8 = 2 } moe_dtype;
 
 /* Layer configuration, in the field names of [DS] and [1.8T] 4.2. */
 typedef struct {
@@ -112,6 +122,13 @@ typedef struct {
   const void* ws_up;    /* [n_shared*I, d]       */
   const void* ws_down;  /* [d, n_shared*I]       */
   const float* bias;    /* [E] selection bias    */
+  /* MOE_FP8 only: UE8M0 block-scale bytes of the expert matrices (NULL otherwise). */
+  const uint8_t* w_gate_scale;   /* [E, ceil(I/128), d/128]  */
+  const uint8_t* w_up_scale;     /* [E, ceil(I/128), d/128]  */
+  const uint8_t* w_down_scale;   /* [E, d/128, I/128]        */
+  const uint8_t* ws_gate_scale;  /* [ceil(I_s/128), d/128]   */
+  const uint8_t* ws_up_scale;    /* [ceil(I_s/128), d/128]   */
+  const uint8_t* ws_down_scale;  /* [d/128, I_s/128]         */
 } moe_weights;
 
 /* Device-resident diagnostics written by moe_route / moe_layer_forward. */
@@ -187,6 +204,19 @@ moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out,
 moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
                              void* y, int32_t* topk_idx_opt, float* topk_w_opt, int32_t* counts_opt,
                              moe_diag* diag_opt, void* ws, size_t ws_bytes, moe_stream_t stream);
+
+/*
+ * E4M3 quantisation of bf16 rows in 1 x 128 tiles, the activation format of
+ * the MOE_FP8 experts ([DS] FP8 section): for row r and tile t,
+ * e = the smallest integer with max|x[r, 128t .. 128t+127]| <= 448 * 2^e
+ * (0 for an all-zero tile), scale_bytes[r, t] = e + 127 (UE8M0) and
+ * codes[r, c] = E4M3 of x[r, c] * 2^-e, round to nearest even.
+ *   in : x [rows, cols] bf16 (device), cols a multiple of 128.
+ *   out: codes [rows, cols] and scale_bytes [rows, cols / 128] (device bytes).
+ * No workspace; MOE_ERR_INVALID_ARG for bad pointers or shapes.
+ */
+moe_status moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, uint8_t* codes, uint8_t* scale_bytes,
+                            moe_stream_t stream);
 
 /*
  * Hash routing ([DS4]): the experts of token t are row token_ids[t] of the

@@ -24,11 +24,12 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUD
     MOE_ERR_INTERNAL = range(7)
 MOE_SCORE_SOFTMAX, MOE_SCORE_SIGMOID, MOE_SCORE_SQRTSOFTPLUS = 0, 1, 2
 MOE_CAP_NONE, MOE_CAP_OVERFLOW_NEXT, MOE_CAP_DROP = 0, 1, 2
-MOE_F32, MOE_BF16 = 0, 1
+MOE_F32, MOE_BF16, MOE_FP8 = 0, 1, 2
 
 # Every symbol declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_route_hash", "moe_bias_update", "moe_permute", "moe_expert_ffn",
-           "moe_combine", "moe_layer_forward", "moe_route_static_scratch", "moe_sync_status", "moe_status_string")
+           "moe_combine", "moe_layer_forward", "moe_route_static_scratch", "moe_quantize_fp8", "moe_sync_status",
+           "moe_status_string")
 MOE_STATIC_SCRATCH_BYTES = 8 << 20  # include/moe.h
 
 
@@ -45,7 +46,8 @@ class moe_config(ctypes.Structure):
 
 class moe_weights(ctypes.Structure):
     _fields_ = [(n, ctypes.c_void_p) for n in
-                ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "bias")]
+                ("w_router", "w_gate", "w_up", "w_down", "ws_gate", "ws_up", "ws_down", "bias",
+                 "w_gate_scale", "w_up_scale", "w_down_scale", "ws_gate_scale", "ws_up_scale", "ws_down_scale")]
 
 
 class moe_diag(ctypes.Structure):
@@ -66,6 +68,7 @@ _lib.moe_layer_forward.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P, _P, _SZ
 _lib.moe_route_hash.argtypes = [_P, _I64, _P, _P, _P, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _SZ, _P]
 _lib.moe_bias_update.argtypes = [_P, _P, _P, ctypes.c_float, _P]
 _lib.moe_route_static_scratch.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P]
+_lib.moe_quantize_fp8.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
 _lib.moe_sync_status.argtypes = [_P, _P]
 _lib.moe_status_string.argtypes = [ctypes.c_int]
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -98,7 +101,7 @@ def make_config(d_model, n_routed, top_k, moe_intermediate_size, n_shared=0, n_g
         int(bool(renormalize)),
         float(routed_scaling_factor),
         {"none": MOE_CAP_NONE, "overflow_next": MOE_CAP_OVERFLOW_NEXT, "drop": MOE_CAP_DROP}[cap_policy],
-        float(capacity_factor), int(capacity), {"f32": MOE_F32, "bf16": MOE_BF16}[dtype])
+        float(capacity_factor), int(capacity), {"f32": MOE_F32, "bf16": MOE_BF16, "fp8": MOE_FP8}[dtype])
 
 
 def _ptr(t):
@@ -113,9 +116,14 @@ def _stream(stream):
     return torch.cuda.current_stream().cuda_stream
 
 
-def make_weights(w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None, bias=None) -> moe_weights:
-    """moe_weights from device tensors (the tensors must outlive every call that uses the struct)."""
-    return moe_weights(*(_ptr(t) for t in (w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, bias)))
+def make_weights(w_router, w_gate, w_up, w_down, ws_gate=None, ws_up=None, ws_down=None, bias=None,
+                 scales=None) -> moe_weights:
+    """moe_weights from device tensors (the tensors must outlive every call that uses the struct).
+    For MOE_FP8 the expert matrices are E4M3 codes (torch.uint8) and `scales` maps
+    gate/up/down/ws_gate/ws_up/ws_down to their UE8M0 block-scale bytes."""
+    sc = scales or {}
+    return moe_weights(*(_ptr(t) for t in (w_router, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, bias)),
+                       *(_ptr(sc.get(k)) for k in ("gate", "up", "down", "ws_gate", "ws_up", "ws_down")))
 
 
 def moe_workspace_size(cfg: moe_config, n: int) -> int:
@@ -171,6 +179,13 @@ def moe_layer_forward(cfg, n, x, weights, y, ws, topk_idx=None, topk_w=None, cou
     _check(_lib.moe_layer_forward(ctypes.byref(cfg), n, _ptr(x), ctypes.byref(weights), _ptr(y), _ptr(topk_idx),
                                   _ptr(topk_w), _ptr(counts), _ptr(diag), _ptr(ws), ws.numel() * ws.element_size(),
                                   _stream(stream)), "moe_layer_forward")
+
+
+def moe_quantize_fp8(x, codes, scale_bytes, stream=None):
+    """E4M3 codes and UE8M0 scale bytes of bf16 rows x [rows, cols] in 1 x 128 tiles."""
+    rows, cols = x.shape
+    _check(_lib.moe_quantize_fp8(_ptr(x), rows, cols, _ptr(codes), _ptr(scale_bytes), _stream(stream)),
+           "moe_quantize_fp8")
 
 
 def moe_sync_status(ws, stream=None) -> int:

@@ -17,14 +17,20 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace layout; every region starts on a 256-byte boundary.
 struct Plan {
-  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched, total;
+  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
+  size_t xq, sfx, hq, sfh, xsq, sfxs, hsq, sfhs;  // FP8 experts: E4M3 activations and their scale blocks
+  size_t total;
 };
+
+// Element type of the activations (x, y, x_perm, expert_out) and of the router
+// weight: bf16 for the FP8 experts, whose matrices alone are E4M3.
+int act_dtype(const moe_config& c) { return c.dtype == MOE_FP8 ? MOE_BF16 : c.dtype; }
 
 // Split-K factor of the router GEMM: small token counts leave most SMs idle
 // (one 128-row tile per 128 tokens), so the k range is split and the route
 // kernel sums the partial logits in a fixed order. Capped at 4 MiB of partials.
 int router_splits(const moe_config& c, int64_t n) {
-  if (c.dtype != MOE_BF16 || c.n_routed % 8 != 0 || n <= 0) return 1;
+  if (act_dtype(c) != MOE_BF16 || c.n_routed % 8 != 0 || n <= 0) return 1;
   const int64_t tiles = ceil_div(n, 128) * ceil_div(c.n_routed, 256);
   if (tiles >= 74) return 1;
   const int64_t num_kb = ceil_div(c.d_model, 64);
@@ -38,7 +44,7 @@ int router_splits(const moe_config& c, int64_t n) {
 }
 
 Plan make_plan(const moe_config& c, int64_t n) {
-  const size_t b = c.dtype == MOE_BF16 ? 2 : 4;
+  const size_t b = act_dtype(c) == MOE_BF16 ? 2 : 4;
   const int64_t nk = n * c.top_k;
   const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size;
   Plan p{};
@@ -65,13 +71,23 @@ Plan make_plan(const moe_config& c, int64_t n) {
   p.sh = take((size_t)(Is > 0 ? n * c.d_model : 0) * b);
   p.shoff = take(2 * 4);
   p.sched = take(4 * 4);  // tile counters of the SM-pair GEMM launches (routed GEMM1/2, shared GEMM1/2)
+  const bool fp8 = c.dtype == MOE_FP8;
+  const int64_t I = c.moe_intermediate_size, d = c.d_model;
+  p.xq = take(fp8 ? (size_t)nk * d : 0);
+  p.sfx = take(fp8 ? (size_t)fp8_sf_tiles_bound(nk, c.n_routed) * (d / 128) * 512 : 0);
+  p.hq = take(fp8 ? (size_t)nk * I : 0);
+  p.sfh = take(fp8 ? (size_t)fp8_sf_tiles_bound(nk, c.n_routed) * (I / 128) * 512 : 0);
+  p.xsq = take(fp8 && Is > 0 ? (size_t)n * d : 0);
+  p.sfxs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (d / 128) * 512 : 0);
+  p.hsq = take(fp8 && Is > 0 ? (size_t)n * Is : 0);
+  p.sfhs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (Is / 128) * 512 : 0);
   p.total = off;
   return p;
 }
 
 moe_status check_cfg(const moe_config* c, int64_t n) {
   if (!c || n < 0) return MOE_ERR_INVALID_ARG;
-  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (c->dtype != MOE_F32 && c->dtype != MOE_BF16 && c->dtype != MOE_FP8) return MOE_ERR_INVALID_ARG;
   if (c->score_fn != MOE_SCORE_SOFTMAX && c->score_fn != MOE_SCORE_SIGMOID && c->score_fn != MOE_SCORE_SQRTSOFTPLUS)
     return MOE_ERR_INVALID_ARG;
   if (c->cap_policy < MOE_CAP_NONE || c->cap_policy > MOE_CAP_DROP) return MOE_ERR_INVALID_ARG;
@@ -86,6 +102,11 @@ moe_status check_cfg(const moe_config* c, int64_t n) {
   if (c->n_routed > kMaxExperts || c->top_k > kMaxTopK || c->n_group > kMaxGroups) return MOE_ERR_UNSUPPORTED;
   if (c->n_group > 1 && c->score_fn == MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
   if (c->d_model % 8 != 0 || c->moe_intermediate_size % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  // FP8 experts: 128-wide scale tiles along every matrix dimension, at most 128 of them along k
+  if (c->dtype == MOE_FP8 && (c->d_model % 128 != 0 || c->moe_intermediate_size % 128 != 0 ||
+                              c->d_model > 128 * 128 || (int64_t)c->n_shared * c->moe_intermediate_size > 128 * 128 ||
+                              c->moe_intermediate_size > 128 * 128))
+    return MOE_ERR_UNSUPPORTED;
   if (n * c->top_k >= (int64_t)1 << 31 || n * (int64_t)c->n_routed >= (int64_t)1 << 40) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -145,15 +166,20 @@ moe_status check_weights(const moe_config& c, const moe_weights* w, bool routed,
   if (shared && c.n_shared > 0 && (!ptr_ok(w->ws_gate) || !ptr_ok(w->ws_up) || !ptr_ok(w->ws_down)))
     return MOE_ERR_INVALID_ARG;
   if (w->bias && !aligned(w->bias, 4)) return MOE_ERR_INVALID_ARG;
+  if (c.dtype == MOE_FP8) {
+    if (routed && (!w->w_gate_scale || !w->w_up_scale || !w->w_down_scale)) return MOE_ERR_INVALID_ARG;
+    if (shared && c.n_shared > 0 && (!w->ws_gate_scale || !w->ws_up_scale || !w->ws_down_scale))
+      return MOE_ERR_INVALID_ARG;
+  }
   return MOE_OK;
 }
 
 // Grouped GEMM dispatch: tcgen05 tensor cores for bf16 where the shape allows,
 // the CUDA-core kernel otherwise (binary32 layers).
 moe_status gemm(const Ctx& x, const GemmArgs& a, bool swiglu, bool out_f32) {
-  if (x.c.dtype == MOE_BF16 && gemm_tc_supported(a, swiglu, out_f32))
+  if (act_dtype(x.c) == MOE_BF16 && gemm_tc_supported(a, swiglu, out_f32))
     return cuda_status(launch_gemm_tc(a, swiglu, out_f32, x.status(), x.s));
-  return cuda_status(launch_gemm_simt(a, x.c.dtype, out_f32, swiglu, x.s));
+  return cuda_status(launch_gemm_simt(a, act_dtype(x.c), out_f32, swiglu, x.s));
 }
 
 // Router logits (binary32, split-K partials for small batches) and the route arguments.
@@ -172,7 +198,7 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
   r.x = X;
   r.w_r = w->w_router;
   r.bias = c.score_fn != MOE_SCORE_SOFTMAX ? w->bias : nullptr;
-  r.dtype = c.dtype;
+  r.dtype = act_dtype(c);
   r.d = c.d_model;
   r.n = x.n;
   r.E = c.n_routed;
@@ -229,14 +255,38 @@ moe_status permute_impl(const Ctx& x, const void* X, const int32_t* idx, int32_t
   }
   MOE_CUDA(launch_dispatch(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), nullptr, offsets, perm, dest,
                            true, nullptr, x.s));
-  const int64_t row_bytes = (int64_t)c.d_model * (c.dtype == MOE_BF16 ? 2 : 4);
+  if (!xperm) return MOE_OK;  // the FP8 quantiser gathers the rows itself
+  const int64_t row_bytes = (int64_t)c.d_model * (act_dtype(c) == MOE_BF16 ? 2 : 4);
   MOE_CUDA(launch_gather(X, perm, offsets, c.n_routed, x.n * c.top_k, row_bytes, xperm, x.s));
+  return MOE_OK;
+}
+
+// FP8 experts: quantise the rows (gathered through a_rows when given), gate/up GEMM with the
+// SwiGLU epilogue, quantise h, down GEMM; the scale blocks follow the same row groups.
+moe_status ffn_fp8(const Ctx& x, const void* A, const int32_t* a_rows, const int32_t* offsets, const moe_weights* w,
+                   void* eo) {
+  const moe_config& c = x.c;
+  const int64_t I = c.moe_intermediate_size, d = c.d_model, nk = x.n * c.top_k;
+  uint8_t* xq = x.at<uint8_t>(x.p.xq);
+  uint32_t* sfx = x.at<uint32_t>(x.p.sfx);
+  uint8_t* hq = x.at<uint8_t>(x.p.hq);
+  uint32_t* sfh = x.at<uint32_t>(x.p.sfh);
+  void* h = x.ws + x.p.h;
+  MOE_CUDA(launch_quantize_rows(A, a_rows, offsets, c.n_routed, nk, (int32_t)d, xq, sfx, x.s));
+  GemmFp8Args g1{xq, w->w_gate, w->w_up, sfx, w->w_gate_scale, w->w_up_scale, h, I, offsets, c.n_routed, nk,
+                 (int32_t)I, (int32_t)d};
+  MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
+  MOE_CUDA(launch_quantize_rows(h, nullptr, offsets, c.n_routed, nk, (int32_t)I, hq, sfh, x.s));
+  GemmFp8Args g2{hq, w->w_down, nullptr, sfh, w->w_down_scale, nullptr, eo, d, offsets, c.n_routed, nk,
+                 (int32_t)d, (int32_t)I};
+  MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
   return MOE_OK;
 }
 
 moe_status ffn_impl(const Ctx& x, const void* xperm, const int32_t* offsets, const moe_weights* w, void* eo) {
   const moe_config& c = x.c;
   if (x.n == 0) return MOE_OK;
+  if (c.dtype == MOE_FP8) return ffn_fp8(x, xperm, nullptr, offsets, w, eo);
   const int64_t I = c.moe_intermediate_size, d = c.d_model, nk = x.n * c.top_k;
   void* h = x.ws + x.p.h;
   int32_t* sched = x.at<int32_t>(x.p.sched);
@@ -256,6 +306,22 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
   const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size, d = c.d_model;
   void* shh = x.ws + x.p.shh;
   void* sh = x.ws + x.p.sh;
+  if (c.dtype == MOE_FP8) {
+    uint8_t* xq = x.at<uint8_t>(x.p.xsq);
+    uint32_t* sfx = x.at<uint32_t>(x.p.sfxs);
+    uint8_t* hq = x.at<uint8_t>(x.p.hsq);
+    uint32_t* sfh = x.at<uint32_t>(x.p.sfhs);
+    MOE_CUDA(launch_quantize_rows(X, nullptr, nullptr, 1, x.n, (int32_t)d, xq, sfx, x.s));
+    GemmFp8Args g1{xq, w->ws_gate, w->ws_up, sfx, w->ws_gate_scale, w->ws_up_scale, shh, Is, nullptr, 1, x.n,
+                   (int32_t)Is, (int32_t)d};
+    MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
+    MOE_CUDA(launch_quantize_rows(shh, nullptr, nullptr, 1, x.n, (int32_t)Is, hq, sfh, x.s));
+    GemmFp8Args g2{hq, w->ws_down, nullptr, sfh, w->ws_down_scale, nullptr, sh, d, nullptr, 1, x.n, (int32_t)d,
+                   (int32_t)Is};
+    MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
+    *sh_out = sh;
+    return MOE_OK;
+  }
   int32_t* sched = x.at<int32_t>(x.p.sched);
   GemmArgs g1{X, d, w->ws_gate, w->ws_up, 0, shh, Is, nullptr, 1, x.n, (int32_t)Is, (int32_t)d};
   g1.tile_counter = sched + 2;
@@ -428,7 +494,7 @@ moe_status moe_combine(const moe_config* cfg, int64_t n, const void* expert_out,
   void* sh = nullptr;
   MOE_TRY(shared_impl(c, x, weights, &sh));
   if (n == 0) return MOE_OK;
-  return cuda_status(launch_combine(expert_out, slot_dest, topk_w, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
+  return cuda_status(launch_combine(expert_out, slot_dest, topk_w, sh, n, c.c.top_k, c.c.d_model, act_dtype(c.c), y, c.s));
 }
 
 moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights, void* y,
@@ -463,13 +529,28 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
   }
   MOE_TRY(route_impl(c, x, weights, idx, tw, counts, diag_opt));
   if (n == 0) return MOE_OK;
-  MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm));
-  MOE_TRY(ffn_impl(c, xperm, offsets, weights, eo));
+  if (c.c.dtype == MOE_FP8) {
+    // the quantiser gathers the token rows itself: no bf16 permuted copy
+    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, nullptr));
+    MOE_TRY(ffn_fp8(c, x, perm, offsets, weights, eo));
+  } else {
+    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm));
+    MOE_TRY(ffn_impl(c, xperm, offsets, weights, eo));
+  }
   if (side)
     MOE_CUDA(cudaStreamWaitEvent(c.s, side->join, 0));
   else
     MOE_TRY(shared_impl(c, x, weights, &sh));
-  return cuda_status(launch_combine(eo, dest, tw, sh, n, c.c.top_k, c.c.d_model, c.c.dtype, y, c.s));
+  return cuda_status(launch_combine(eo, dest, tw, sh, n, c.c.top_k, c.c.d_model, act_dtype(c.c), y, c.s));
+}
+
+moe_status moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, uint8_t* codes, uint8_t* scale_bytes,
+                            moe_stream_t stream) {
+  if (rows < 0 || cols <= 0 || cols % 128 != 0 || rows * (int64_t)cols >= (int64_t)1 << 40) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  if (!ptr_ok(x) || !ptr_ok(codes) || !scale_bytes) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_rows(x, nullptr, nullptr, 1, rows, cols, codes, nullptr,
+                                          reinterpret_cast<cudaStream_t>(stream), scale_bytes));
 }
 
 moe_status moe_sync_status(void* ws, moe_stream_t stream) {

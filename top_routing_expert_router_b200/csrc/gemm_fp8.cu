@@ -1,0 +1,545 @@
+// gemm_fp8.cu -- grouped GEMM of the FP8 experts on the tcgen05 tensor cores.
+//
+// Page "15. DeepSeek: MLA, MoE and MTP", FP8 section: matrix inputs in E4M3,
+// one UE8M0 scale per 1 x 128 tile of the activations A and per 128 x 128
+// block of the weights B. For every group g and row r of that group:
+//   plain : C[r, n] = sum_k (A[r, k] sa[r, k/128]) (B_g[n, k] sb_g[n/128, k/128])
+//   SwiGLU: C[r, i] = silu(gate) * up, gate and up the plain sums with Bg_g, Bu_g
+// computed by tcgen05.mma kind::mxf8f6f4.block_scale (E4M3 x E4M3 -> fp32 in
+// TMEM, the scales applied by the tensor core per 32-wide k sub-block). C is bf16.
+//
+// Design (one CTA per SM, persistent, warp-specialised, 192 threads):
+//   warp 0      producer: per 128-k stage TMA copies of the 128 x 128 A tile,
+//               the 128 x 128 B tile (SwiGLU: 64 gate over 64 up rows) and a
+//               512-byte bulk copy of A's scale-factor block (laid out by the
+//               quantiser); the warp writes B's scale words from the block
+//               scale bytes (prefetched per tile) into the stage.
+//   warp 1      TMEM owner and MMA issuer: tcgen05.cp of both scale-factor
+//               blocks into TMEM (32x128b.warpx4: rows p and p+32k of the tile
+//               in lane p, column k), then four MMAs of K = 32 that select the
+//               scale byte of their sub-block; tcgen05.commit frees the stage.
+//   warps 2..5  epilogue: tcgen05.ld, SwiGLU in fp32, bf16 stores.
+// Every mbarrier wait is bounded like the bf16 kernels'.
+#include <cuda.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128, BN = 128, BK = 128;  // BK in E4M3 elements (128 bytes per row)
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, SF_BYTES = 512;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;  // 33 KB, keeps 1024-byte alignment
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = 2 * BN;  // scale factors after the two accumulators
+constexpr int kMaxGroupsFp8 = 256;
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr uint64_t kDrainNs = 200000000ull;
+static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+static_assert(SF_COL0 + 8 * STAGES <= TMEM_COLS, "TMEM budget");
+
+struct Fp8Params {
+  int32_t G;
+  const int32_t* offsets;
+  int32_t M;
+  int32_t N;      // valid output columns per group
+  int32_t K;
+  int32_t n_out;  // output columns per tile
+  int32_t b_rows; // rows per group in B
+  int32_t swiglu;
+  const uint32_t* sfa;        // A scale-factor blocks from the quantiser
+  const uint8_t* sb;          // B scale bytes [G][ceil(b_rows/128)][K/128]
+  const uint8_t* sb2;         // up-matrix scale bytes (SwiGLU)
+  void* C;
+  int64_t ldc;
+  moe_diag* status;
+};
+
+struct __align__(8) Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+  int32_t total_tiles;
+  int32_t n_tiles;
+  int32_t row_off[kMaxGroupsFp8 + 1];
+  int32_t tile_off[kMaxGroupsFp8 + 1];
+  int32_t sf_off[kMaxGroupsFp8 + 1];  // first 128-row scale tile of each group
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
+
+__device__ __forceinline__ uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, moe_diag* st) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(b, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        atomicExch(&ctl->abort, 1);
+        set_status(st, MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t b = smem_u32(bar);
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try(b, parity))
+    if (globaltimer() - t0 > kDrainNs) return;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0, int32_t c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
+      : "memory");
+}
+
+// Untiled bulk copy (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// K-major operand, 128-byte swizzle (8-row x 128-byte atoms, 1024 B apart).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Scale-factor block (32 rows x 16 bytes, rows contiguous), no swizzle: core
+// matrices of 8 rows x 16 bytes, 128 bytes apart.
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// kind::mxf8f6f4 instruction descriptor: E4M3 A and B (format 0), K-major,
+// UE8M0 scales, M = 128, N = BN; scale-factor byte `id` of A and of B.
+__device__ __forceinline__ uint32_t idesc_fp8(int id) {
+  return ((uint32_t)id << 4) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
+         ((uint32_t)id << 29);
+}
+
+__device__ __forceinline__ void mma_fp8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t sfa,
+                                        uint32_t sfb, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+__device__ __forceinline__ void sf_copy(uint32_t taddr, uint64_t desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(desc) : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+struct Tile {
+  int g, m, nt;
+};
+
+__device__ __forceinline__ Tile decode(const Ctl* ctl, int G, int t, int& g_hint) {
+  int g = g_hint;
+  while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
+  g_hint = g;
+  const int local = t - ctl->tile_off[g];
+  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM - 1) / BM;
+  return Tile{g, local % mt, local / mt};
+}
+
+__device__ __forceinline__ void store16(bf16* C, int64_t ldc, int64_t row, int col, int N, const float (&v)[16]) {
+  bf16* p = C + row * ldc + col;
+  uint4 lo, hi;
+  __nv_bfloat162* l2 = reinterpret_cast<__nv_bfloat162*>(&lo);
+  __nv_bfloat162* h2 = reinterpret_cast<__nv_bfloat162*>(&hi);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    l2[q] = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    h2[q] = __floats2bfloat162_rn(v[8 + 2 * q], v[8 + 2 * q + 1]);
+  }
+  if (col + 8 <= N) *reinterpret_cast<uint4*>(p) = lo;
+  if (col + 16 <= N) *reinterpret_cast<uint4*>(p + 8) = hi;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_fp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                    const __grid_constant__ CUtensorMap map_b2, Fp8Params p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    int acc = 0, sacc = 0;
+    const int n_tiles = (p.N + p.n_out - 1) / p.n_out;
+    for (int g = 0; g < p.G; ++g) {
+      const int lo = p.offsets ? p.offsets[g] : 0;
+      const int hi = p.offsets ? p.offsets[g + 1] : p.M;
+      const int mt = (hi - lo + BM - 1) / BM;
+      ctl->row_off[g] = lo;
+      ctl->row_off[g + 1] = hi;
+      ctl->tile_off[g] = acc;
+      ctl->sf_off[g] = sacc;
+      acc += mt * n_tiles;
+      sacc += mt;
+    }
+    ctl->tile_off[p.G] = acc;
+    ctl->sf_off[p.G] = sacc;
+    ctl->total_tiles = acc;
+    ctl->n_tiles = n_tiles;
+    ctl->abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 2);  // the producer's expect_tx arrival + its scale-word arrival
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tmem_full[b], 1);
+      mbar_init(&ctl->tmem_empty[b], 4);
+    }
+    mbar_init(&ctl->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int total = ctl->total_tiles;
+  const int nkb = p.K / BK;
+  const int nbr = (p.b_rows + 127) / 128;  // scale rows of B per group
+
+  if (warp == 0) {
+    // ================= producer (whole warp) =================
+    int stage = 0;
+    uint32_t phase = 0;
+    int g_hint = 0;
+    bool ok = true;
+    uint32_t armed[STAGES] = {};
+    const uint32_t tx = A_BYTES + B_BYTES + SF_BYTES;
+    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      const Tile tl = decode(ctl, p.G, t, g_hint);
+      const int row0 = ctl->row_off[tl.g] + tl.m * BM;
+      const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
+      const uint32_t* sfa_tile = p.sfa + (int64_t)(ctl->sf_off[tl.g] + tl.m) * nkb * 128;
+      // B scale bytes of this tile: lane l keeps k-blocks l, l + 32, l + 64, l + 96
+      const int brow_local = tl.nt * p.n_out;
+      const uint8_t* sb_g = p.sb + ((int64_t)tl.g * nbr + brow_local / 128) * nkb;
+      const uint8_t* sb2_g = p.swiglu ? p.sb2 + ((int64_t)tl.g * nbr + brow_local / 128) * nkb : sb_g;
+      uint32_t sbg[4], sbu[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kb = lane + 32 * j;
+        sbg[j] = kb < nkb ? sb_g[kb] : 127u;
+        sbu[j] = kb < nkb ? sb2_g[kb] : 127u;
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        int go = 1;
+        if (lane == 0 && !mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
+            !mbar_wait(&ctl->empty[stage], phase ^ 1u, ctl, p.status))
+          go = 0;
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        uint8_t* sbm = sa + A_BYTES;
+        uint8_t* sfa_s = sbm + B_BYTES;
+        uint8_t* sfb_s = sfa_s + SF_BYTES;
+        if (lane == 0) {
+          mbar_expect_tx(&ctl->full[stage], tx);
+          ++armed[stage];
+          tma_load_2d(sa, &map_a, &ctl->full[stage], kb * BK, row0);
+          if (p.swiglu) {
+            tma_load_2d(sbm, &map_b, &ctl->full[stage], kb * BK, brow);
+            tma_load_2d(sbm + (BN / 2) * BK, &map_b2, &ctl->full[stage], kb * BK, brow);
+          } else {
+            tma_load_2d(sbm, &map_b, &ctl->full[stage], kb * BK, brow);
+          }
+          bulk_load(sfa_s, sfa_tile + (int64_t)kb * 128, SF_BYTES, &ctl->full[stage]);
+        }
+        // B scale words: tile row p of B sits at word 4 (p % 32) + p / 32; rows 0..63 are the
+        // gate half and 64..127 the up half for SwiGLU, all one 128-row block otherwise.
+        const uint32_t bg = __shfl_sync(0xffffffffu, sbg[kb >> 5], kb & 31) * 0x01010101u;
+        const uint32_t bu = __shfl_sync(0xffffffffu, sbu[kb >> 5], kb & 31) * 0x01010101u;
+        const uint32_t w2 = p.swiglu ? bu : bg;
+        *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, w2, w2);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->full[stage]);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0)
+      for (int s = 0; s < STAGES; ++s)
+        if (armed[s]) mbar_drain(&ctl->full[s], (armed[s] - 1) & 1u);
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      int i = 0;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+        if (!mbar_wait(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_try(smem_u32(&ctl->full[stage]), phase) && !mbar_wait(&ctl->full[stage], phase, ctl, p.status)) {
+            ok = false;
+            break;
+          }
+          fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint32_t sfa_t = tmem_base + SF_COL0 + 8u * (uint32_t)stage;
+          const uint32_t sfb_t = sfa_t + 4u;
+          sf_copy(sfa_t, sf_desc(sa + A_BYTES + B_BYTES));
+          sf_copy(sfb_t, sf_desc(sa + A_BYTES + B_BYTES + SF_BYTES));
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 elements = 32 bytes per MMA
+            mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(k), sfa_t, sfb_t,
+                    (kb | k) != 0);
+          issued = true;
+          mma_commit(&ctl->empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(&ctl->tmem_full[buf]);
+      }
+      if (!ok && issued) {
+        mma_commit(&ctl->drain);
+        mbar_drain(&ctl->drain, 0);
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..5) =================
+    const int q = warp & 3;
+    const int row_in_tile = q * 32 + lane;
+    int g_hint = 0;
+    int i = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      const Tile tl = decode(ctl, p.G, t, g_hint);
+      const bool got = mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
+      __syncwarp();
+      if (!got) break;
+      fence_after();
+      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM + row_in_tile;
+      const bool valid = row < ctl->row_off[tl.g + 1];
+      const int col0 = tl.nt * p.n_out;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
+      bf16* C = static_cast<bf16*>(p.C);
+      if (p.swiglu) {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + (uint32_t)c, gv);
+          tmem_ld16(taddr + (uint32_t)(p.n_out + c), uv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) gv[e] = silu(gv[e]) * uv[e];
+          if (valid && col0 + c < p.N) store16(C, p.ldc, row, col0 + c, p.N, gv);
+        }
+      } else {
+        for (int c = 0; c < p.n_out; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + (uint32_t)c, v);
+          if (valid && col0 + c < p.N) store16(C, p.ldc, row, col0 + c, p.N, v);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// ---- host side -----------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  if (!tried) {
+    tried = true;
+    void* q = nullptr;
+    cudaDriverEntryPointQueryResult r;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
+        r == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(q);
+  }
+  return fn;
+}
+
+// 2-D byte tensor [rows, cols] (cols contiguous), box [box_rows, 128], 128-byte swizzle.
+bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
+
+}  // namespace
+
+cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
+  if (a.M <= 0) return cudaSuccess;
+  if (a.K % BK != 0 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8) return cudaErrorInvalidValue;
+  if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.B) % 16 ||
+      reinterpret_cast<uintptr_t>(a.sfa) % 16 || reinterpret_cast<uintptr_t>(a.C) % 16 || a.ldc % 8 != 0 ||
+      (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
+    return cudaErrorInvalidValue;
+  Fp8Params p{};
+  p.G = a.G;
+  p.offsets = a.offsets;
+  p.M = (int32_t)a.M;
+  p.N = a.N;
+  p.K = a.K;
+  p.n_out = swiglu ? BN / 2 : BN;
+  p.b_rows = a.N;
+  p.swiglu = swiglu;
+  p.sfa = a.sfa;
+  p.sb = a.sb;
+  p.sb2 = swiglu ? a.sb2 : a.sb;
+  p.C = a.C;
+  p.ldc = a.ldc;
+  p.status = status;
+  CUtensorMap ma, mb, mb2;
+  const int b_box = swiglu ? BN / 2 : BN;
+  if (!make_map_u8(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
+  if (!make_map_u8(&mb, a.B, (int64_t)a.G * a.N, a.K, b_box)) return cudaErrorInvalidValue;
+  if (swiglu) {
+    if (!make_map_u8(&mb2, a.B2, (int64_t)a.G * a.N, a.K, b_box)) return cudaErrorInvalidValue;
+  } else {
+    mb2 = mb;
+  }
+  static bool attr = false;
+  if (!attr) {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  int sms = 0, dev = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  const int64_t n_tiles = ceil_div(a.N, p.n_out);
+  const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles;
+  const int grid = (int)(max_tiles < sms ? max_tiles : sms);
+  gemm_fp8_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mb2, p);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -36,6 +36,33 @@ cudaError_t launch_gemm_simt(const GemmArgs& a, int dtype, bool out_f32, bool sw
 cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_diag* status, cudaStream_t s);
 bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32);
 
+// FP8 experts: E4M3 A (quantised rows, scale-factor blocks from launch_quantize_rows)
+// times E4M3 B with UE8M0 128 x 128 block-scale bytes, bf16 C; grouped like GemmArgs.
+struct GemmFp8Args {
+  const void* A;          // [rows, K] E4M3 codes
+  const void* B;          // [G * N, K] E4M3 codes
+  const void* B2;         // SwiGLU up matrix, like B
+  const uint32_t* sfa;    // A scale-factor blocks (512 bytes per 128-row tile and 128-wide k block)
+  const uint8_t* sb;      // [G, ceil(N/128), K/128] UE8M0 bytes of B
+  const uint8_t* sb2;     // same for B2
+  void* C;
+  int64_t ldc;
+  const int32_t* offsets; // [G + 1] or nullptr (one group of M rows)
+  int32_t G;
+  int64_t M;
+  int32_t N;
+  int32_t K;
+};
+cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s);
+
+// E4M3 quantisation of bf16 rows in 1 x 128 tiles (row r reads src[src_row[r]] when
+// src_row is given); scale words go to the GEMM's scale-factor blocks of the groups.
+int64_t fp8_sf_tiles_bound(int64_t rows, int32_t G);
+// sf_plain given: scale bytes [rows, cols/128] instead of the GEMM's blocks.
+cudaError_t launch_quantize_rows(const void* src, const int32_t* src_row, const int32_t* offsets, int32_t G,
+                                 int64_t rows_bound, int32_t cols, uint8_t* q, uint32_t* sf, cudaStream_t s,
+                                 uint8_t* sf_plain = nullptr);
+
 // Router: scoring, group limit, top-k, certification / binary64 refinement, gates.
 struct RouteArgs {
   const float* logits;  // [splits][n, E] partial logits, summed in order
