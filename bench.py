@@ -66,10 +66,11 @@ def job_throughput(tokens_per_rank: int, steps: int, world: int, ms_total_max: f
 
 def layer_work(w, kept_slots, active_experts):
     """Algorithmic FLOPs and bytes of one layer forward."""
-    b = 2 if w.dtype == "bf16" else 4
+    b = 4 if w.dtype == "f32" else 2       # activations and router weight (bf16 for the FP8 experts)
+    bw = 1 + 1 / 16384 if w.dtype == "fp8" else b  # expert weights: E4M3 codes plus one scale byte per 128 x 128
     d, I, E, n = w.d_model, w.moe_intermediate_size, w.n_routed, w.n
     flops = 2 * n * E * d + 6 * kept_slots * d * I + 6 * n * d * w.I_s
-    bytes_ = E * d * b + active_experts * 3 * d * I * b + 3 * d * w.I_s * b + 2 * n * d * b
+    bytes_ = E * d * b + active_experts * 3 * d * I * bw + 3 * d * w.I_s * bw + 2 * n * d * b
     return flops, bytes_
 
 
@@ -79,10 +80,14 @@ def launches_per_step(w):
     if w.cap_policy != "none":
         n += 2  # capacity + gates
     n += 2  # counts: histogram + scan
-    n += 4  # permute: histogram + scan + scatter + gather
-    n += 2  # GEMM1 (SwiGLU) + GEMM2
-    if w.n_shared:
-        n += 2
+    if w.dtype == "fp8":
+        n += 3  # permute: histogram + scan + scatter (the quantiser gathers the rows)
+        n += 4  # quantise x, GEMM1 (SwiGLU), quantise h, GEMM2
+        n += 4 if w.n_shared else 0
+    else:
+        n += 4  # permute: histogram + scan + scatter + gather
+        n += 2  # GEMM1 (SwiGLU) + GEMM2
+        n += 2 if w.n_shared else 0
     n += 1  # combine
     return n
 
@@ -173,8 +178,15 @@ def run_ours(args):
     y = torch.empty((n, w.d_model), dtype=dev["x"].dtype, device="cuda")
     counts = torch.empty(w.n_routed, dtype=torch.int32, device="cuda")
     diag = torch.zeros(8, dtype=torch.int32, device="cuda")
-    weights = moe.make_weights(dev["w_r"], dev["w_gate"], dev["w_up"], dev["w_down"], dev.get("ws_gate"),
-                               dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
+    if w.dtype == "fp8":
+        mats = ("gate", "up", "down")
+        scales = {k: dev["w_%s_s" % k] for k in mats}
+        scales.update({"ws_" + k: dev["ws_%s_s" % k] for k in mats if "ws_%s_s" % k in dev})
+        weights = moe.make_weights(dev["w_r"], dev["w_gate_q"], dev["w_up_q"], dev["w_down_q"], dev.get("ws_gate_q"),
+                                   dev.get("ws_up_q"), dev.get("ws_down_q"), dev.get("bias"), scales=scales)
+    else:
+        weights = moe.make_weights(dev["w_r"], dev["w_gate"], dev["w_up"], dev["w_down"], dev.get("ws_gate"),
+                                   dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
     stream = torch.cuda.current_stream()
     s = stream.cuda_stream
 
@@ -286,6 +298,9 @@ def run_ours(args):
     bpe = dev["x"].element_size()
 
     hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    peak_dtype = "bf16"
+    if w.dtype == "fp8":  # E4M3 contraction: the measured bf16 peak times the nominal FP8/bf16 ratio (4.5 / 2.25)
+        tf_burst, tf_sust, peak_dtype = 2 * tf_burst, 2 * tf_sust if tf_sust else None, "bf16 x 2 (nominal fp8/bf16) for fp8"
     ffn_flops = 6.0 * kept * w.d_model * w.moe_intermediate_size
     achieved = ffn_flops / (stage_ms["expert_ffn"] / 1e3) / 1e12
     t_roof = max(flops / (tf_burst * 1e12), bytes_ / (hbm * 1e9))
@@ -300,15 +315,15 @@ def run_ours(args):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": w.dtype,
+        "dtype": "e4m3 x e4m3 -> f32 (bf16 activations)" if w.dtype == "fp8" else w.dtype,
         "data": "synthetic (seeded counter-based generator; Irwin-Hall normals)",
         "config": {"workload": w.name, "n_tokens": n, "d_model": w.d_model, "n_routed": w.n_routed,
                    "top_k": w.top_k, "moe_intermediate_size": w.moe_intermediate_size, "n_shared": w.n_shared,
                    "score_fn": w.score_fn, "cap_policy": w.cap_policy, "parallelism": f"replicas x{world}",
-                   "l2": f"inputs larger than L2: {active} experts x {3 * w.d_model * w.moe_intermediate_size * bpe / 1e6:.0f} MB of weights streamed per step"},
+                   "l2": f"inputs larger than L2: {active} experts x {3 * w.d_model * w.moe_intermediate_size * (1 if w.dtype == 'fp8' else bpe) / 1e6:.0f} MB of weights streamed per step"},
         "roofline": {"bound": "tensor", "kernel": "moe_expert_ffn (grouped SwiGLU GEMM1 + down GEMM2)",
                      "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst,
-                     "peak_kind": f"{peak_kind} bf16 burst", "frac_of_sustained": achieved / tf_sust if tf_sust else None,
+                     "peak_kind": f"{peak_kind} {peak_dtype} burst", "frac_of_sustained": achieved / tf_sust if tf_sust else None,
                      "flops_per_launch": ffn_flops, "traffic": _traffic("expert_ffn", w.name)},
         "layer_roofline": {"flops": flops, "bytes": bytes_, "t_roof_ms": t_roof * 1e3,
                            "frac": t_roof * 1e3 / ms_step, "active_experts": active, "kept_slots": kept},
@@ -332,8 +347,10 @@ def _oracle_inputs(w, tokens):
     """Host inputs of the oracle's sample: the first `tokens` rows of x and all weights."""
     from synth import workloads as W
 
-    names = ["w_r", "w_gate", "w_up", "w_down"] + (["bias"] if w.bias_range else []) + \
-        (["ws_gate", "ws_up", "ws_down"] if w.n_shared else [])
+    mats = ["w_gate", "w_up", "w_down"] + (["ws_gate", "ws_up", "ws_down"] if w.n_shared else [])
+    if w.dtype == "fp8":
+        mats = [m + suffix for m in mats for suffix in ("_q", "_s")]
+    names = ["w_r"] + mats + (["bias"] if w.bias_range else [])
     inp = W.host_inputs(w, names=names)
     inp["x"] = W.host_rows(w, "x", range(tokens))
     return inp
@@ -345,8 +362,13 @@ def _oracle_time(w, inp, tokens):
 
     cfg = O.Cfg(**w.cfg_fields())
     t0 = time.perf_counter()
-    O.layer(cfg, inp["x"][:tokens], inp["w_r"], inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("bias"),
-            inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"))
+    if w.dtype == "fp8":
+        w8 = {k: (inp["w_%s_q" % k], inp["w_%s_s" % k]) for k in ("gate", "up", "down")}
+        ws8 = {k: (inp["ws_%s_q" % k], inp["ws_%s_s" % k]) for k in ("gate", "up", "down")} if w.n_shared else None
+        O.layer_fp8(cfg, inp["x"][:tokens], inp["w_r"], inp.get("bias"), w8, ws8)
+    else:
+        O.layer(cfg, inp["x"][:tokens], inp["w_r"], inp["w_gate"], inp["w_up"], inp["w_down"], inp.get("bias"),
+                inp.get("ws_gate"), inp.get("ws_up"), inp.get("ws_down"))
     return time.perf_counter() - t0
 
 

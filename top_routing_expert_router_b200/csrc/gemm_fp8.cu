@@ -30,18 +30,28 @@
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 128;  // BK in E4M3 elements (128 bytes per row)
-constexpr int STAGES = 6;
-constexpr int A_BYTES = BM * BK, B_BYTES = BN * BK, SF_BYTES = 512;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + 2 * SF_BYTES;  // 33 KB, keeps 1024-byte alignment
+constexpr int BM = 128, BK = 128;  // BK in E4M3 elements (128 bytes per row)
+constexpr int A_BYTES = BM * BK, SF_BYTES = 512;  // SF_BYTES: one 128-row scale-factor block
 constexpr int kThreads = 192;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = 2 * BN;  // scale factors after the two accumulators
 constexpr int kMaxGroupsFp8 = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr uint64_t kDrainNs = 200000000ull;
-static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-static_assert(SF_COL0 + 8 * STAGES <= TMEM_COLS, "TMEM budget");
+
+// Tile shapes: BN = 128 keeps two TMEM accumulators (the epilogue of one tile
+// overlaps the next); BN = 256 halves the copies of A per MMA but leaves TMEM
+// room for one accumulator next to the scale factors.
+template <int BN>
+struct Shape {
+  static constexpr int ACC_BUFS = BN == 256 ? 1 : 2;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int SFB_BYTES = (BN / 128) * SF_BYTES;
+  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr uint32_t SF_COL0 = ACC_BUFS * BN;   // scale factors after the accumulators
+  static constexpr uint32_t SF_COLS = 4 + BN / 32;     // per stage: A (128 rows) and B (BN rows)
+  static_assert(SF_COL0 + SF_COLS * STAGES <= TMEM_COLS, "TMEM budget");
+};
 
 struct Fp8Params {
   int32_t G;
@@ -60,9 +70,11 @@ struct Fp8Params {
   moe_diag* status;
 };
 
+constexpr int kMaxStages = 6;
+
 struct __align__(8) Ctl {
-  uint64_t full[STAGES];
-  uint64_t empty[STAGES];
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
   uint64_t drain;
@@ -174,8 +186,8 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
 
 // kind::mxf8f6f4 instruction descriptor: E4M3 A and B (format 0), K-major,
 // UE8M0 scales, M = 128, N = BN; scale-factor byte `id` of A and of B.
-__device__ __forceinline__ uint32_t idesc_fp8(int id) {
-  return ((uint32_t)id << 4) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
+__device__ __forceinline__ uint32_t idesc_fp8(int bn, int id) {
+  return ((uint32_t)id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
          ((uint32_t)id << 29);
 }
 
@@ -238,9 +250,12 @@ __device__ __forceinline__ void store16(bf16* C, int64_t ldc, int64_t row, int c
   if (col + 16 <= N) *reinterpret_cast<uint4*>(p + 8) = hi;
 }
 
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_b2, Fp8Params p) {
+  using S = Shape<BN>;
+  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES, B_BYTES = S::B_BYTES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
@@ -269,7 +284,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ctl->full[s], 2);  // the producer's expect_tx arrival + its scale-word arrival
       mbar_init(&ctl->empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < S::ACC_BUFS; ++b) {
       mbar_init(&ctl->tmem_full[b], 1);
       mbar_init(&ctl->tmem_empty[b], 4);
     }
@@ -298,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g_hint = 0;
     bool ok = true;
     uint32_t armed[STAGES] = {};
-    const uint32_t tx = A_BYTES + B_BYTES + SF_BYTES;
+    const uint32_t tx = A_BYTES + B_BYTES + SF_BYTES;  // TMA tiles and A's scale block
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile tl = decode(ctl, p.G, t, g_hint);
       const int row0 = ctl->row_off[tl.g] + tl.m * BM;
@@ -308,12 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int brow_local = tl.nt * p.n_out;
       const uint8_t* sb_g = p.sb + ((int64_t)tl.g * nbr + brow_local / 128) * nkb;
       const uint8_t* sb2_g = p.swiglu ? p.sb2 + ((int64_t)tl.g * nbr + brow_local / 128) * nkb : sb_g;
-      uint32_t sbg[4], sbu[4];
+      const uint8_t* sbn_g = sb_g + ((brow_local / 128 + 1 < nbr) ? nkb : 0);  // next 128-row block (plain, BN = 256)
+      uint32_t sbg[4], sbu[4], sbn[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int kb = lane + 32 * j;
         sbg[j] = kb < nkb ? sb_g[kb] : 127u;
         sbu[j] = kb < nkb ? sb2_g[kb] : 127u;
+        sbn[j] = kb < nkb ? sbn_g[kb] : 127u;
       }
       for (int kb = 0; kb < nkb; ++kb) {
         int go = 1;
@@ -341,12 +358,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           bulk_load(sfa_s, sfa_tile + (int64_t)kb * 128, SF_BYTES, &ctl->full[stage]);
         }
-        // B scale words: tile row p of B sits at word 4 (p % 32) + p / 32; rows 0..63 are the
-        // gate half and 64..127 the up half for SwiGLU, all one 128-row block otherwise.
+        // B scale words, one 128-row block per 512 bytes: block row p at word 4 (p % 32) + p / 32.
+        // SwiGLU: the first BN/2 tile rows are gate rows, the rest up rows (one scale block each,
+        // as BN/2 <= 128 rows never straddle a 128-row block); plain: one block per 128 rows.
         const uint32_t bg = __shfl_sync(0xffffffffu, sbg[kb >> 5], kb & 31) * 0x01010101u;
         const uint32_t bu = __shfl_sync(0xffffffffu, sbu[kb >> 5], kb & 31) * 0x01010101u;
-        const uint32_t w2 = p.swiglu ? bu : bg;
-        *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, w2, w2);
+        if (BN == 128) {
+          const uint32_t w2 = p.swiglu ? bu : bg;
+          *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, w2, w2);
+        } else {  // BN = 256: block 0 holds tile rows 0..127, block 1 rows 128..255
+          const uint32_t w2 = p.swiglu ? bu : __shfl_sync(0xffffffffu, sbn[kb >> 5], kb & 31) * 0x01010101u;
+          *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, bg, bg);
+          *reinterpret_cast<uint4*>(sfb_s + SF_BYTES + 16 * lane) = make_uint4(w2, w2, w2, w2);
+        }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->full[stage]);
@@ -367,8 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true, issued = false;
       int i = 0;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++i) {
-        const int buf = i & 1;
-        const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+        const int buf = S::ACC_BUFS == 2 ? (i & 1) : 0;
+        const uint32_t acc_phase = (uint32_t)(S::ACC_BUFS == 2 ? (i >> 1) : i) & 1u;
         if (!mbar_wait(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
           ok = false;
           break;
@@ -382,15 +406,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sfa_t = tmem_base + SF_COL0 + 8u * (uint32_t)stage;
+          const uint32_t sfa_t = tmem_base + S::SF_COL0 + S::SF_COLS * (uint32_t)stage;
           const uint32_t sfb_t = sfa_t + 4u;
           sf_copy(sfa_t, sf_desc(sa + A_BYTES + B_BYTES));
-          sf_copy(sfb_t, sf_desc(sa + A_BYTES + B_BYTES + SF_BYTES));
+#pragma unroll
+          for (int blk = 0; blk < BN / 128; ++blk)  // B rows 128 blk .. : TMEM columns 4 blk ..
+            sf_copy(sfb_t + 4u * blk, sf_desc(sa + A_BYTES + B_BYTES + SF_BYTES + SF_BYTES * blk));
           const uint64_t adesc = sw128_desc(sa);
           const uint64_t bdesc = sw128_desc(sa + A_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 elements = 32 bytes per MMA
-            mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(k), sfa_t, sfb_t,
+            mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(BN, k), sfa_t, sfb_t,
                     (kb | k) != 0);
           issued = true;
           mma_commit(&ctl->empty[stage]);
@@ -414,8 +440,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g_hint = 0;
     int i = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
-      const int buf = i & 1;
-      const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      const int buf = S::ACC_BUFS == 2 ? (i & 1) : 0;
+      const uint32_t acc_phase = (uint32_t)(S::ACC_BUFS == 2 ? (i >> 1) : i) & 1u;
       const Tile tl = decode(ctl, p.G, t, g_hint);
       const bool got = mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
       __syncwarp();
@@ -489,18 +515,15 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
-static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
+template <int BN>
+constexpr size_t smem_bytes() {
+  return 1024 + Shape<BN>::STAGES * Shape<BN>::STAGE_BYTES + sizeof(Ctl);
+}
+static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448, "dynamic shared memory above 227 KB");
+static_assert(Shape<128>::STAGES <= kMaxStages && Shape<256>::STAGES <= kMaxStages, "barrier arrays");
 
-}  // namespace
-
-cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
-  if (a.M <= 0) return cudaSuccess;
-  if (a.K % BK != 0 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8) return cudaErrorInvalidValue;
-  if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.B) % 16 ||
-      reinterpret_cast<uintptr_t>(a.sfa) % 16 || reinterpret_cast<uintptr_t>(a.C) % 16 || a.ldc % 8 != 0 ||
-      (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
-    return cudaErrorInvalidValue;
+template <int BN>
+cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
   Fp8Params p{};
   p.G = a.G;
   p.offsets = a.offsets;
@@ -527,7 +550,8 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
   }
   static bool attr = false;
   if (!attr) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_fp8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    const cudaError_t e =
+        cudaFuncSetAttribute(gemm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<BN>());
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -538,8 +562,26 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
   const int64_t n_tiles = ceil_div(a.N, p.n_out);
   const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles;
   const int grid = (int)(max_tiles < sms ? max_tiles : sms);
-  gemm_fp8_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mb, mb2, p);
+  gemm_fp8_kernel<BN><<<grid, kThreads, smem_bytes<BN>(), s>>>(ma, mb, mb2, p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+// SwiGLU GEMMs (gate/up, the larger contraction) run 128 x 256 tiles; the down
+// GEMM keeps 128 x 128 tiles with two accumulators. MOE_FP8_BN=128|256 overrides
+// the SwiGLU choice (tuning and tests).
+cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
+  if (a.M <= 0) return cudaSuccess;
+  if (a.K % BK != 0 || a.K / BK > 128 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8)
+    return cudaErrorInvalidValue;
+  if (reinterpret_cast<uintptr_t>(a.A) % 16 || reinterpret_cast<uintptr_t>(a.B) % 16 ||
+      reinterpret_cast<uintptr_t>(a.sfa) % 16 || reinterpret_cast<uintptr_t>(a.C) % 16 || a.ldc % 8 != 0 ||
+      (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
+    return cudaErrorInvalidValue;
+  const char* bn = getenv("MOE_FP8_BN");
+  const bool wide = bn ? strcmp(bn, "256") == 0 : swiglu;
+  return wide ? launch_bn<256>(a, swiglu, status, s) : launch_bn<128>(a, swiglu, status, s);
 }
 
 }  // namespace moe

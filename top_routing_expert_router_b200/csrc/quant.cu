@@ -69,27 +69,37 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
     const int64_t srow = src_row ? (int64_t)src_row[r] : r;
     const uint2* in = reinterpret_cast<const uint2*>(src + srow * cols);
     uint32_t* out = reinterpret_cast<uint32_t*>(q + r * cols);
-    for (int t = 0; t < tiles; ++t) {
-      const uint2 raw = __ldg(in + t * 32 + lane);
-      const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-      const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-      const float v0 = __low2float(a), v1 = __high2float(a), v2 = __low2float(b), v3 = __high2float(b);
-      float m = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+    // eight tiles' loads in flight at a time, then their reductions and stores
+    for (int t0 = 0; t0 < tiles; t0 += 8) {
+      uint2 raws[8];
 #pragma unroll
-      for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-      const int e = ue8m0_exponent(m);
-      // multiplying by 2^-e is exact for these magnitudes
-      const __nv_fp8x2_storage_t c01 =
-          __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v0, -e), ldexpf(v1, -e)), __NV_SATFINITE, __NV_E4M3);
-      const __nv_fp8x2_storage_t c23 =
-          __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v2, -e), ldexpf(v3, -e)), __NV_SATFINITE, __NV_E4M3);
-      out[t * 32 + lane] = (uint32_t)c01 | ((uint32_t)c23 << 16);
-      if (lane == 0) {
-        const uint32_t byte = (uint32_t)(e + 127);
-        if (sf_plain)
-          sf_plain[r * tiles + t] = (uint8_t)byte;
-        else
-          sf[(tile * tiles + t) * 128 + 4 * (p % 32) + p / 32] = byte * 0x01010101u;
+      for (int u = 0; u < 8; ++u)
+        if (t0 + u < tiles) raws[u] = __ldg(in + (t0 + u) * 32 + lane);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = t0 + u;
+        if (t >= tiles) break;
+        const uint2 raw = raws[u];
+        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+        const float v0 = __low2float(a), v1 = __high2float(a), v2 = __low2float(b), v3 = __high2float(b);
+        float m = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+#pragma unroll
+        for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        const int e = ue8m0_exponent(m);
+        // multiplying by 2^-e is exact for these magnitudes
+        const __nv_fp8x2_storage_t c01 =
+            __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v0, -e), ldexpf(v1, -e)), __NV_SATFINITE, __NV_E4M3);
+        const __nv_fp8x2_storage_t c23 =
+            __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v2, -e), ldexpf(v3, -e)), __NV_SATFINITE, __NV_E4M3);
+        out[t * 32 + lane] = (uint32_t)c01 | ((uint32_t)c23 << 16);
+        if (lane == 0) {
+          const uint32_t byte = (uint32_t)(e + 127);
+          if (sf_plain)
+            sf_plain[r * tiles + t] = (uint8_t)byte;
+          else
+            sf[(tile * tiles + t) * 128 + 4 * (p % 32) + p / 32] = byte * 0x01010101u;
+        }
       }
     }
   }
