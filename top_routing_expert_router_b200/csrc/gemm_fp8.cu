@@ -314,24 +314,40 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     uint32_t armed[STAGES] = {};
     const uint32_t tx = A_BYTES + B_BYTES + SF_BYTES;  // TMA tiles and A's scale block
+    // B scale bytes of a tile: lane l keeps k-blocks l, l + 32, l + 64, l + 96 of the gate (or
+    // plain) block, the up block and, for plain 256-wide tiles, the next 128-row block. They are
+    // loaded one tile ahead, so a tile's first stage does not wait for them.
+    int pf_hint = 0;
+    auto load_scales = [&](int tt, uint32_t (&g)[4], uint32_t (&u)[4], uint32_t (&nx)[4]) {
+      if (tt >= total) return;
+      const Tile tl = decode(ctl, p.G, tt, pf_hint);
+      const int brow_local = tl.nt * p.n_out;
+      const uint8_t* sb_g = p.sb + ((int64_t)tl.g * nbr + brow_local / 128) * nkb;
+      const uint8_t* sb2_g = p.swiglu ? p.sb2 + ((int64_t)tl.g * nbr + brow_local / 128) * nkb : sb_g;
+      const uint8_t* sbn_g = sb_g + ((brow_local / 128 + 1 < nbr) ? nkb : 0);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int kb = lane + 32 * j;
+        g[j] = kb < nkb ? sb_g[kb] : 127u;
+        u[j] = kb < nkb ? sb2_g[kb] : 127u;
+        nx[j] = kb < nkb ? sbn_g[kb] : 127u;
+      }
+    };
+    uint32_t nsbg[4], nsbu[4], nsbn[4];
+    load_scales(blockIdx.x, nsbg, nsbu, nsbn);
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
       const Tile tl = decode(ctl, p.G, t, g_hint);
       const int row0 = ctl->row_off[tl.g] + tl.m * BM;
       const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
       const uint32_t* sfa_tile = p.sfa + (int64_t)(ctl->sf_off[tl.g] + tl.m) * nkb * 128;
-      // B scale bytes of this tile: lane l keeps k-blocks l, l + 32, l + 64, l + 96
-      const int brow_local = tl.nt * p.n_out;
-      const uint8_t* sb_g = p.sb + ((int64_t)tl.g * nbr + brow_local / 128) * nkb;
-      const uint8_t* sb2_g = p.swiglu ? p.sb2 + ((int64_t)tl.g * nbr + brow_local / 128) * nkb : sb_g;
-      const uint8_t* sbn_g = sb_g + ((brow_local / 128 + 1 < nbr) ? nkb : 0);  // next 128-row block (plain, BN = 256)
       uint32_t sbg[4], sbu[4], sbn[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const int kb = lane + 32 * j;
-        sbg[j] = kb < nkb ? sb_g[kb] : 127u;
-        sbu[j] = kb < nkb ? sb2_g[kb] : 127u;
-        sbn[j] = kb < nkb ? sbn_g[kb] : 127u;
+        sbg[j] = nsbg[j];
+        sbu[j] = nsbu[j];
+        sbn[j] = nsbn[j];
       }
+      load_scales(t + (int)gridDim.x, nsbg, nsbu, nsbn);
       for (int kb = 0; kb < nkb; ++kb) {
         int go = 1;
         if (lane == 0 && !mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
@@ -568,9 +584,10 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
 
 }  // namespace
 
-// SwiGLU GEMMs (gate/up, the larger contraction) run 128 x 256 tiles; the down
-// GEMM keeps 128 x 128 tiles with two accumulators. MOE_FP8_BN=128|256 overrides
-// the SwiGLU choice (tuning and tests).
+// Both expert GEMMs run 128 x 256 tiles: at the FP8 MMA rate the L2 -> SM copies
+// bound the kernel, and 256-wide tiles copy 25 % fewer bytes per MAC than 128-wide
+// ones, which outweighs the epilogue no longer overlapping the next tile (measured
+// on the DeepSeek-V3 shapes). MOE_FP8_BN=128|256 overrides (tuning and tests).
 cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   if (a.K % BK != 0 || a.K / BK > 128 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8)
@@ -580,7 +597,7 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
       (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
     return cudaErrorInvalidValue;
   const char* bn = getenv("MOE_FP8_BN");
-  const bool wide = bn ? strcmp(bn, "256") == 0 : swiglu;
+  const bool wide = bn ? strcmp(bn, "256") == 0 : true;
   return wide ? launch_bn<256>(a, swiglu, status, s) : launch_bn<128>(a, swiglu, status, s);
 }
 
