@@ -584,10 +584,12 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
 
 }  // namespace
 
-// Both expert GEMMs run 128 x 256 tiles: at the FP8 MMA rate the L2 -> SM copies
-// bound the kernel, and 256-wide tiles copy 25 % fewer bytes per MAC than 128-wide
-// ones, which outweighs the epilogue no longer overlapping the next tile (measured
-// on the DeepSeek-V3 shapes). MOE_FP8_BN=128|256 overrides (tuning and tests).
+// Groups averaging at least 128 rows (prefill) run 128 x 256 tiles: at the FP8 MMA
+// rate the L2 -> SM copies bound the kernel, and 256-wide tiles copy 25 % fewer
+// bytes per MAC, which outweighs the epilogue no longer overlapping the next tile.
+// Smaller groups (decode) stream weights: 128-wide tiles with two accumulators keep
+// twice as many independent tiles in flight. MOE_FP8_BN=128|256 overrides (tuning
+// and tests).
 cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   if (a.K % BK != 0 || a.K / BK > 128 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8)
@@ -597,7 +599,7 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
       (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
     return cudaErrorInvalidValue;
   const char* bn = getenv("MOE_FP8_BN");
-  const bool wide = bn ? strcmp(bn, "256") == 0 : true;
+  const bool wide = bn ? strcmp(bn, "256") == 0 : a.M / (a.offsets ? a.G : 1) >= 128;
   return wide ? launch_bn<256>(a, swiglu, status, s) : launch_bn<128>(a, swiglu, status, s);
 }
 

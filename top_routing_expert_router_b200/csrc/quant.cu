@@ -19,19 +19,31 @@
 namespace moe {
 namespace {
 
-// UE8M0 exponent of a tile whose largest magnitude is amax (finite binary32).
+// UE8M0 exponent of a tile whose largest magnitude is amax (finite binary32):
+// with amax = f * 2^x, f in [0.5, 1), amax <= 448 * 2^e  <=>  f * 2^(x - 8 - e) <= 1.75,
+// so e = x - 9 when f <= 0.875 and x - 8 otherwise. For a normal amax = 1.m * 2^(E - 127)
+// that is x = E - 126 and f <= 0.875 <=> m <= 0.75, read straight off the bits.
 __device__ __forceinline__ int ue8m0_exponent(float amax) {
   if (!(amax > 0.0f)) return 0;
-  int x;
-  const float f = frexpf(amax, &x);  // amax = f * 2^x, f in [0.5, 1)
-  // amax <= 448 * 2^e  <=>  f * 2^(x - 8 - e) <= 1.75: e = x - 9 iff f <= 0.875, else x - 8
-  int e = f <= 0.875f ? x - 9 : x - 8;
+  const uint32_t u = __float_as_uint(amax);
+  const int E = (int)(u >> 23);
+  int e;
+  if (E > 0) {
+    e = (u & 0x7FFFFFu) <= 0x600000u ? E - 135 : E - 134;
+  } else {  // binary32 subnormal
+    int x;
+    const float f = frexpf(amax, &x);
+    e = f <= 0.875f ? x - 9 : x - 8;
+  }
   return e < -127 ? -127 : (e > 127 ? 127 : e);
 }
 
+// 2^-e as a binary32 (normal for the exponents bf16 inputs produce, -127 <= e <= 119).
+__device__ __forceinline__ float pow2_neg(int e) { return __uint_as_float((uint32_t)(127 - e) << 23); }
+
 constexpr int kQuantWarps = 8;
 
-// One warp per row; lane l holds columns 4l .. 4l+3 of each 128-column tile.
+// One warp per row, two 128-column tiles at a time (one per half-warp).
 __global__ void __launch_bounds__(32 * kQuantWarps)
     quantize_rows_kernel(const bf16* src, const int32_t* src_row, const int32_t* offsets, int G, int64_t rows_single,
                          int cols, uint8_t* q, uint32_t* sf, uint8_t* sf_plain) {
@@ -67,33 +79,50 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
     const int64_t tile = tile_off[g] + local / 128;
     const int p = (int)(local % 128);
     const int64_t srow = src_row ? (int64_t)src_row[r] : r;
-    const uint2* in = reinterpret_cast<const uint2*>(src + srow * cols);
-    uint32_t* out = reinterpret_cast<uint32_t*>(q + r * cols);
-    // eight tiles' loads in flight at a time, then their reductions and stores
-    for (int t0 = 0; t0 < tiles; t0 += 8) {
-      uint2 raws[8];
+    // Half-warp h of the warp owns tile 2c + h of chunk c (256 columns); lane l of a
+    // half-warp holds columns 8 (l % 16) .. +7 of its tile: one 16-byte load and one
+    // 8-byte store per lane, four chunks of loads in flight.
+    const uint4* in = reinterpret_cast<const uint4*>(src + srow * cols);
+    uint2* out = reinterpret_cast<uint2*>(q + r * cols);
+    const int half = lane >> 4, hl = lane & 15;
+    const unsigned hmask = half ? 0xffff0000u : 0x0000ffffu;
+    const int chunks = (tiles + 1) / 2;
+    for (int c0 = 0; c0 < chunks; c0 += 4) {
+      uint4 raws[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (t0 + u < tiles) raws[u] = __ldg(in + (t0 + u) * 32 + lane);
+      for (int u = 0; u < 4; ++u) {
+        const int t = 2 * (c0 + u) + half;
+        if (c0 + u < chunks && t < tiles) raws[u] = __ldg(in + t * 16 + hl);
+      }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int t = t0 + u;
-        if (t >= tiles) break;
-        const uint2 raw = raws[u];
-        const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-        const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-        const float v0 = __low2float(a), v1 = __high2float(a), v2 = __low2float(b), v3 = __high2float(b);
-        float m = fmaxf(fmaxf(fabsf(v0), fabsf(v1)), fmaxf(fabsf(v2), fabsf(v3)));
+      for (int u = 0; u < 4; ++u) {
+        const int t = 2 * (c0 + u) + half;
+        if (c0 + u >= chunks || t >= tiles) continue;  // uniform within each half-warp
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raws[u]);
+        float v[8];
 #pragma unroll
-        for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+        for (int j = 0; j < 4; ++j) {
+          v[2 * j] = __low2float(h2[j]);
+          v[2 * j + 1] = __high2float(h2[j]);
+        }
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[j]));
+#pragma unroll
+        for (int off = 8; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(hmask, m, off));
         const int e = ue8m0_exponent(m);
-        // multiplying by 2^-e is exact for these magnitudes
-        const __nv_fp8x2_storage_t c01 =
-            __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v0, -e), ldexpf(v1, -e)), __NV_SATFINITE, __NV_E4M3);
-        const __nv_fp8x2_storage_t c23 =
-            __nv_cvt_float2_to_fp8x2(make_float2(ldexpf(v2, -e), ldexpf(v3, -e)), __NV_SATFINITE, __NV_E4M3);
-        out[t * 32 + lane] = (uint32_t)c01 | ((uint32_t)c23 << 16);
-        if (lane == 0) {
+        const float sc = pow2_neg(e);  // multiplying by 2^-e is exact for these magnitudes
+        uint32_t w[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const __nv_fp8x2_storage_t c01 = __nv_cvt_float2_to_fp8x2(
+              make_float2(v[4 * j] * sc, v[4 * j + 1] * sc), __NV_SATFINITE, __NV_E4M3);
+          const __nv_fp8x2_storage_t c23 = __nv_cvt_float2_to_fp8x2(
+              make_float2(v[4 * j + 2] * sc, v[4 * j + 3] * sc), __NV_SATFINITE, __NV_E4M3);
+          w[j] = (uint32_t)c01 | ((uint32_t)c23 << 16);
+        }
+        out[t * 16 + hl] = make_uint2(w[0], w[1]);
+        if (hl == 0) {
           const uint32_t byte = (uint32_t)(e + 127);
           if (sf_plain)
             sf_plain[r * tiles + t] = (uint8_t)byte;
