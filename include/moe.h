@@ -282,6 +282,108 @@ moe_status moe_route_static_scratch(const moe_config* cfg, int64_t n, const void
                                     moe_stream_t stream);
 
 /*
+ * ---- Expert parallelism -----------------------------------------------------
+ * [DS] section "V3 MoE: how 8 of 256 experts are chosen" places one expert
+ * group per node and limits each token to topk_group of them; [MoE] 4.2
+ * spreads the experts evenly over the GPUs with the routing decision known to
+ * every GPU. Here R ranks (one GPU each) share a layer: rank q owns the routed
+ * experts [q E/R, (q+1) E/R) and holds only their matrices; every rank holds
+ * the router, the bias and the shared experts, and routes its own tokens.
+ * One layer step per rank:
+ *   1. route its n tokens; write its per-expert slot counts into row `rank` of
+ *      every rank's count table;
+ *   2. push every kept slot's token row into the owner's receive buffer;
+ *   3. run the owned experts over the rows it received;
+ *   4. y[t] = sum_j topk_w[t, j] * (owner's output row of slot j) + shared(x[t]),
+ *      pulling the rows from the owners' output buffers, binary32 in slot order
+ *      then the shared experts, as in moe_combine.
+ * A flag barrier separates the steps (and ends the call), so the buffers may
+ * be reused by the next call. Receive layout at owner q: its experts in order,
+ * inside an expert the source ranks in order, inside a source its tokens in
+ * order. With the ranks' batches concatenated in rank order this is the
+ * stable permutation of moe_permute restricted to q's experts, so a layer
+ * split over R ranks computes what moe_layer_forward computes on the
+ * concatenated batch. cfg->cap_policy must be MOE_CAP_NONE (a capacity is a
+ * property of one batch in one token order) and E must be a multiple of R.
+ */
+#define MOE_EP_MAX_RANKS 8
+
+/*
+ * The exchange buffers of a group of `world` ranks as seen from the calling
+ * device: entry q is rank q's buffer (device memory of the calling GPU for
+ * q = the caller's rank, a peer mapping -- moe_ep_open_handle -- otherwise).
+ * Every rank allocates the same buffers:
+ *   recv_x[q], recv_out[q]: [recv_rows, d] activations (cfg->dtype; bf16 for
+ *     MOE_FP8), the rows owner q receives and its experts' outputs;
+ *   counts[q]: [world, E] int32 count table;
+ *   flags[q]:  [world + 1] uint32 barrier words, zeroed once before the first
+ *     call and then left to the library.
+ * recv_rows bounds the rows an owner receives: the sum over ranks of
+ * n_r * min(k, E / world) can never be exceeded. More rows than that set
+ * MOE_ERR_WORKSPACE in the status word and the excess slots are skipped.
+ */
+typedef struct {
+  int32_t world;
+  int32_t reserved;
+  int64_t recv_rows;
+  void* recv_x[MOE_EP_MAX_RANKS];
+  void* recv_out[MOE_EP_MAX_RANKS];
+  int32_t* counts[MOE_EP_MAX_RANKS];
+  uint32_t* flags[MOE_EP_MAX_RANKS];
+} moe_ep_group;
+
+/*
+ * One rank's inputs and outputs. x [n, d], y [n, d] device; weights (host
+ * struct): w_router [E, d] and bias [E] of the whole layer, w_gate/w_up/w_down
+ * (and their FP8 scales) holding only this rank's E / world experts in order,
+ * ws_* the shared experts. topk_idx_opt [n, k] and topk_w_opt [n, k] may be
+ * NULL. ws: at least moe_ep_workspace_size() bytes, 256-byte aligned; its
+ * status word (moe_sync_status) reports this rank's device errors.
+ */
+typedef struct {
+  int64_t n;
+  const void* x;
+  const moe_weights* weights;
+  void* y;
+  int32_t* topk_idx_opt;
+  float* topk_w_opt;
+  void* ws;
+  size_t ws_bytes;
+} moe_ep_rank;
+
+/* Workspace bytes of one rank with n tokens in a group of `world` ranks. */
+moe_status moe_ep_workspace_size(const moe_config* cfg, int32_t world, int64_t n, int64_t recv_rows, size_t* bytes);
+
+/*
+ * One MoE layer step of ranks [first_rank, first_rank + num_ranks) of the
+ * group, ranks[i] describing rank first_rank + i, all on `stream`.
+ *   num_ranks == 1: the call of one process driving one rank; the steps are
+ *     separated by the flag barrier, whose wait is bounded (MOE_EP_TIMEOUT_MS
+ *     in the environment, default 5000 ms): past it the rank records
+ *     MOE_ERR_TIMEOUT in its status word and does not wait at later barriers
+ *     of the call. Every rank of the group must make the call.
+ *   num_ranks == world: one process drives every rank on one device (all
+ *     buffers local); the steps of all ranks run in stream order, no barrier.
+ * Returns MOE_ERR_INVALID_ARG for a bad group, rank range or buffer,
+ * MOE_ERR_UNSUPPORTED for a capacity policy or world > MOE_EP_MAX_RANKS.
+ */
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* group, int32_t first_rank,
+                                int32_t num_ranks, const moe_ep_rank* ranks, moe_stream_t stream);
+
+/*
+ * Peer mappings for moe_ep_group: an opaque 72-byte record of a device
+ * allocation (a CUDA IPC handle of the allocation holding ptr, and ptr's
+ * offset inside it), made by the process owning it and opened by the others
+ * (one per GPU of the same node, peer access between the GPUs). open returns
+ * the address of the same byte in the calling process; close releases a
+ * mapping made by open (pass the address open returned).
+ */
+#define MOE_EP_HANDLE_BYTES 72
+moe_status moe_ep_export_handle(const void* ptr, void* handle);
+moe_status moe_ep_open_handle(const void* handle, void** ptr);
+moe_status moe_ep_close_handle(void* ptr);
+
+/*
  * Synchronises `stream`, then returns the device status word kept in the
  * workspace (MOE_OK, MOE_ERR_TIMEOUT or MOE_ERR_INTERNAL) and clears it. Every
  * entry point clears the word when it starts, so it reports the most recent

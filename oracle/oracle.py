@@ -395,3 +395,23 @@ def layer_fp8(cfg: Cfg, x, w_r, bias, w8: dict, ws8: dict = None):
         sh = swiglu_fp8(x64, ws8["gate"], ws8["up"], ws8["down"])
     y = combine(eo, dest, w, sh)
     return dict(y=y, topk_idx=idx, topk_w=w, counts=counts, exempt=ex, stats=st)
+
+
+def ep_recv_layout(topk_idx_per_rank, E: int, world: int):
+    """Rows each owner receives when `world` ranks share a layer and rank q owns experts
+    [q E/world, (q+1) E/world) (page "15. DeepSeek: MLA, MoE and MTP", section "V3 MoE": one
+    expert group per node). Order at an owner: its experts ascending; inside an expert the source
+    ranks ascending; inside a source its tokens ascending. Returns, per owner q, (rows, offsets):
+    rows [m, 2] = (source rank, source token) of each received row, offsets [E/world + 1] the row
+    range of each owned expert."""
+    Eq = E // world
+    out = []
+    for q in range(world):
+        rows, offsets = [], [0]
+        for e in range(q * Eq, (q + 1) * Eq):
+            for s, idx in enumerate(topk_idx_per_rank):
+                toks = np.nonzero((np.asarray(idx) == e).any(axis=1))[0]
+                rows.extend((s, int(t)) for t in toks)
+            offsets.append(len(rows))
+        out.append((np.asarray(rows, np.int64).reshape(-1, 2), np.asarray(offsets, np.int64)))
+    return out

@@ -612,3 +612,27 @@ def test_round_to_bf16_matches_torch():
     a = np.concatenate([rng.normal(0, 1, 5000) * rng.lognormal(0, 4, 5000), [0.0, -0.0, 1.0, 3.0 / 7.0]])
     ref = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(O.round_to_bf16(a), ref)
+
+
+# ---------------------------------------------------------------- expert parallelism: receive layout
+
+
+@pytest.mark.parametrize("world,E,k", [(1, 8, 2), (2, 8, 2), (4, 16, 3), (8, 64, 6)])
+def test_ep_recv_layout_is_the_global_stable_permutation_split_by_owner(world, E, k):
+    """Pinned to the oracle's C counting sort of the concatenated batch (a separate formulation):
+    the owners' rows, concatenated in owner order, are its permutation, and each owner's expert
+    ranges are its offsets shifted to start at zero."""
+    rng = np.random.default_rng(world * 100 + E)
+    ns = [int(v) for v in rng.integers(0, 40, world)]
+    ns[0] = 0 if world > 1 else ns[0]  # a rank without tokens
+    idx = [np.array([rng.choice(E, k, replace=False) for _ in range(n)], np.int32).reshape(n, k) for n in ns]
+    if world > 1:  # a dropped slot (-1) is never received
+        idx[-1][:1, -1] = -1
+    lay = O.ep_recv_layout(idx, E, world)
+    _, off, perm, _ = O.dispatch(np.concatenate(idx), E)
+    first = np.cumsum([0] + ns)
+    glob = np.concatenate([first[rows[:, 0]] + rows[:, 1] for rows, _ in lay])
+    np.testing.assert_array_equal(glob, perm)
+    Eq = E // world
+    for q, (_, offs) in enumerate(lay):
+        np.testing.assert_array_equal(offs, off[q * Eq:(q + 1) * Eq + 1] - off[q * Eq])

@@ -28,9 +28,12 @@ MOE_F32, MOE_BF16, MOE_FP8 = 0, 1, 2
 
 # Every symbol declared in include/moe.h.
 EXPORTS = ("moe_workspace_size", "moe_route", "moe_route_hash", "moe_bias_update", "moe_permute", "moe_expert_ffn",
-           "moe_combine", "moe_layer_forward", "moe_route_static_scratch", "moe_quantize_fp8", "moe_sync_status",
-           "moe_status_string")
+           "moe_combine", "moe_layer_forward", "moe_route_static_scratch", "moe_quantize_fp8",
+           "moe_ep_workspace_size", "moe_ep_layer_forward", "moe_ep_export_handle", "moe_ep_open_handle",
+           "moe_ep_close_handle", "moe_sync_status", "moe_status_string")
 MOE_STATIC_SCRATCH_BYTES = 8 << 20  # include/moe.h
+MOE_EP_MAX_RANKS = 8
+MOE_EP_HANDLE_BYTES = 72
 
 
 class moe_config(ctypes.Structure):
@@ -56,6 +59,18 @@ class moe_diag(ctypes.Structure):
                 ("reserved", ctypes.c_int32 * 2)]
 
 
+class moe_ep_group(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("reserved", ctypes.c_int32), ("recv_rows", ctypes.c_int64),
+                ("recv_x", ctypes.c_void_p * MOE_EP_MAX_RANKS), ("recv_out", ctypes.c_void_p * MOE_EP_MAX_RANKS),
+                ("counts", ctypes.c_void_p * MOE_EP_MAX_RANKS), ("flags", ctypes.c_void_p * MOE_EP_MAX_RANKS)]
+
+
+class moe_ep_rank(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int64), ("x", ctypes.c_void_p), ("weights", ctypes.POINTER(moe_weights)),
+                ("y", ctypes.c_void_p), ("topk_idx_opt", ctypes.c_void_p), ("topk_w_opt", ctypes.c_void_p),
+                ("ws", ctypes.c_void_p), ("ws_bytes", ctypes.c_size_t)]
+
+
 DIAG_FIELDS = ("overflowed", "dropped", "refined_tokens", "max_load", "refined_logits", "status")
 
 _P, _I64, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
@@ -69,6 +84,11 @@ _lib.moe_route_hash.argtypes = [_P, _I64, _P, _P, _P, ctypes.c_int32, _P, _P, _P
 _lib.moe_bias_update.argtypes = [_P, _P, _P, ctypes.c_float, _P]
 _lib.moe_route_static_scratch.argtypes = [_P, _I64, _P, _P, _P, _P, _P, _P, _P]
 _lib.moe_quantize_fp8.argtypes = [_P, _I64, ctypes.c_int32, _P, _P, _P]
+_lib.moe_ep_workspace_size.argtypes = [_P, ctypes.c_int32, _I64, _I64, ctypes.POINTER(ctypes.c_size_t)]
+_lib.moe_ep_layer_forward.argtypes = [_P, _P, ctypes.c_int32, ctypes.c_int32, _P, _P]
+_lib.moe_ep_export_handle.argtypes = [_P, _P]
+_lib.moe_ep_open_handle.argtypes = [_P, ctypes.POINTER(ctypes.c_void_p)]
+_lib.moe_ep_close_handle.argtypes = [_P]
 _lib.moe_sync_status.argtypes = [_P, _P]
 _lib.moe_status_string.argtypes = [ctypes.c_int]
 _lib.moe_status_string.restype = ctypes.c_char_p
@@ -186,6 +206,87 @@ def moe_quantize_fp8(x, codes, scale_bytes, stream=None):
     rows, cols = x.shape
     _check(_lib.moe_quantize_fp8(_ptr(x), rows, cols, _ptr(codes), _ptr(scale_bytes), _stream(stream)),
            "moe_quantize_fp8")
+
+
+def moe_ep_recv_rows_bound(cfg, world, token_counts) -> int:
+    """Rows an owner can receive at most: each token holds at most min(k, E / world) of its experts."""
+    return max(1, int(sum(token_counts)) * min(cfg.top_k, cfg.n_routed // world))
+
+
+def moe_ep_workspace_size(cfg, world, n, recv_rows) -> int:
+    out = ctypes.c_size_t()
+    _check(_lib.moe_ep_workspace_size(ctypes.byref(cfg), world, n, recv_rows, ctypes.byref(out)),
+           "moe_ep_workspace_size")
+    return out.value
+
+
+def make_ep_group(recv_rows, recv_x, recv_out, counts, flags=None) -> moe_ep_group:
+    """moe_ep_group from per-rank buffers: lists (one entry per rank) of device tensors or integer
+    device addresses (peer mappings from ep_open_peers)."""
+    world = len(recv_x)
+    if not (1 <= world <= MOE_EP_MAX_RANKS) or not (len(recv_out) == len(counts) == world):
+        raise ValueError("one recv_x, recv_out and counts buffer per rank, at most %d ranks" % MOE_EP_MAX_RANKS)
+
+    def addr(v):
+        return v if isinstance(v, int) or v is None else v.data_ptr()
+
+    g = moe_ep_group()
+    g.world, g.recv_rows = world, int(recv_rows)
+    for q in range(world):
+        g.recv_x[q], g.recv_out[q], g.counts[q] = addr(recv_x[q]), addr(recv_out[q]), addr(counts[q])
+        g.flags[q] = addr(flags[q]) if flags is not None else None
+    return g
+
+
+def moe_ep_layer_forward(cfg, group, first_rank, ranks, stream=None):
+    """One layer step of ranks first_rank .. first_rank + len(ranks) - 1. Each entry of `ranks` is a
+    dict with n, x, weights (a moe_weights), y, ws and optionally topk_idx, topk_w."""
+    arr = (moe_ep_rank * len(ranks))()
+    keep = []
+    for i, r in enumerate(ranks):
+        w = r["weights"]
+        keep.append(w)
+        ws = r["ws"]
+        arr[i] = moe_ep_rank(int(r["n"]), _ptr(r["x"]), ctypes.pointer(w), _ptr(r["y"]), _ptr(r.get("topk_idx")),
+                             _ptr(r.get("topk_w")), _ptr(ws), ws.numel() * ws.element_size())
+    _check(_lib.moe_ep_layer_forward(ctypes.byref(cfg), ctypes.byref(group), first_rank, len(ranks), arr,
+                                     _stream(stream)), "moe_ep_layer_forward")
+
+
+def moe_ep_export_handle(t) -> bytes:
+    """Peer-mapping record (MOE_EP_HANDLE_BYTES bytes) of the device allocation holding tensor t."""
+    buf = ctypes.create_string_buffer(MOE_EP_HANDLE_BYTES)
+    _check(_lib.moe_ep_export_handle(_ptr(t), buf), "moe_ep_export_handle")
+    return buf.raw
+
+
+def moe_ep_open_handle(handle: bytes) -> int:
+    if len(handle) != MOE_EP_HANDLE_BYTES:
+        raise ValueError("a peer-mapping record has %d bytes" % MOE_EP_HANDLE_BYTES)
+    out = ctypes.c_void_p()
+    _check(_lib.moe_ep_open_handle(ctypes.create_string_buffer(handle, MOE_EP_HANDLE_BYTES), ctypes.byref(out)),
+           "moe_ep_open_handle")
+    return out.value
+
+
+def moe_ep_close_handle(addr: int) -> None:
+    _check(_lib.moe_ep_close_handle(addr), "moe_ep_close_handle")
+
+
+def ep_open_peers(local: dict, rank: int, world: int, all_gather_object, export=None, open_=None) -> dict:
+    """Exchange the peer-mapping records of this rank's exchange buffers with every rank of a
+    process group and open the peers' buffers. `local` maps buffer names (recv_x, recv_out, counts,
+    flags) to this rank's tensors; `all_gather_object(obj)` returns the list of every rank's obj
+    (e.g. a wrapper of torch.distributed.all_gather_object). Returns name -> per-rank list with
+    this rank's tensor at `rank` and the peers' mapped addresses elsewhere; release those with
+    moe_ep_close_handle."""
+    export = export or moe_ep_export_handle
+    open_ = open_ or moe_ep_open_handle
+    mine = {k: export(t) for k, t in local.items()}
+    records = all_gather_object(mine)
+    if len(records) != world:
+        raise RuntimeError("expected %d records, got %d" % (world, len(records)))
+    return {k: [t if q == rank else open_(records[q][k]) for q in range(world)] for k, t in local.items()}
 
 
 def moe_sync_status(ws, stream=None) -> int:

@@ -1,8 +1,10 @@
 // api.cu -- the C ABI entry points declared in moe.h: argument checks,
 // workspace carving and the launch sequence of each stage on the caller's
 // stream. No allocation, no host synchronisation (except moe_sync_status).
+#include <cuda.h>
 #include <math.h>
 #include <stddef.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <mutex>
@@ -19,6 +21,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Plan {
   size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
   size_t xq, sfx, hq, sfh, xsq, sfxs, hsq, sfhs;  // FP8 experts: E4M3 activations and their scale blocks
+  size_t ep_off;  // expert parallelism: receive offsets of the rank's own experts
   size_t total;
 };
 
@@ -43,9 +46,16 @@ int router_splits(const moe_config& c, int64_t n) {
   return (int)ceil_div(num_kb, kb_per);
 }
 
-Plan make_plan(const moe_config& c, int64_t n) {
+// ep_world > 0: the layout of one expert-parallel rank. The routed experts run over the
+// ep_recv_rows rows of the group's receive buffer in E / ep_world groups, so h and the FP8
+// activations are sized for those; the permuted rows and expert outputs live in the group's
+// buffers, not here.
+Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_recv_rows = 0) {
   const size_t b = act_dtype(c) == MOE_BF16 ? 2 : 4;
   const int64_t nk = n * c.top_k;
+  const bool ep = ep_world > 0;
+  const int64_t fr = ep ? ep_recv_rows : nk;             // rows through the routed experts
+  const int32_t fg = ep ? c.n_routed / ep_world : c.n_routed;  // their groups
   const int64_t Is = (int64_t)c.n_shared * c.moe_intermediate_size;
   Plan p{};
   size_t off = 0;
@@ -64,23 +74,24 @@ Plan make_plan(const moe_config& c, int64_t n) {
   p.offsets = take((size_t)(c.n_routed + 1) * 4);
   p.perm = take((size_t)nk * 4);
   p.dest = take((size_t)nk * 4);
-  p.xperm = take((size_t)nk * c.d_model * b);
-  p.h = take((size_t)nk * c.moe_intermediate_size * b);
-  p.eo = take((size_t)nk * c.d_model * b);
+  p.xperm = take(ep ? 0 : (size_t)nk * c.d_model * b);
+  p.h = take((size_t)fr * c.moe_intermediate_size * b);
+  p.eo = take(ep ? 0 : (size_t)nk * c.d_model * b);
   p.shh = take((size_t)(Is > 0 ? n * Is : 0) * b);
   p.sh = take((size_t)(Is > 0 ? n * c.d_model : 0) * b);
   p.shoff = take(2 * 4);
   p.sched = take(4 * 4);  // tile counters of the SM-pair GEMM launches (routed GEMM1/2, shared GEMM1/2)
   const bool fp8 = c.dtype == MOE_FP8;
   const int64_t I = c.moe_intermediate_size, d = c.d_model;
-  p.xq = take(fp8 ? (size_t)nk * d : 0);
-  p.sfx = take(fp8 ? (size_t)fp8_sf_tiles_bound(nk, c.n_routed) * (d / 128) * 512 : 0);
-  p.hq = take(fp8 ? (size_t)nk * I : 0);
-  p.sfh = take(fp8 ? (size_t)fp8_sf_tiles_bound(nk, c.n_routed) * (I / 128) * 512 : 0);
+  p.xq = take(fp8 ? (size_t)fr * d : 0);
+  p.sfx = take(fp8 ? (size_t)fp8_sf_tiles_bound(fr, fg) * (d / 128) * 512 : 0);
+  p.hq = take(fp8 ? (size_t)fr * I : 0);
+  p.sfh = take(fp8 ? (size_t)fp8_sf_tiles_bound(fr, fg) * (I / 128) * 512 : 0);
   p.xsq = take(fp8 && Is > 0 ? (size_t)n * d : 0);
   p.sfxs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (d / 128) * 512 : 0);
   p.hsq = take(fp8 && Is > 0 ? (size_t)n * Is : 0);
   p.sfhs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (Is / 128) * 512 : 0);
+  p.ep_off = take(ep ? (size_t)(fg + 1) * 4 : 0);
   p.total = off;
   return p;
 }
@@ -360,6 +371,170 @@ SideStream* side_stream() {
   return &ss;
 }
 
+// ---- expert parallelism ------------------------------------------------------------
+
+// Limit of one barrier wait: MOE_EP_TIMEOUT_MS from the environment, default 5 s.
+uint64_t ep_timeout_ns() {
+  const char* v = getenv("MOE_EP_TIMEOUT_MS");
+  long ms = v ? atol(v) : 0;
+  if (ms <= 0) ms = 5000;
+  return (uint64_t)ms * 1000000ull;
+}
+
+moe_status check_ep(const moe_config* cfg, const moe_ep_group* g, int32_t first, int32_t num,
+                    const moe_ep_rank* ranks) {
+  if (!cfg || !g || !ranks) return MOE_ERR_INVALID_ARG;
+  if (g->world < 1) return MOE_ERR_INVALID_ARG;
+  if (g->world > MOE_EP_MAX_RANKS) return MOE_ERR_UNSUPPORTED;
+  if (cfg->n_routed <= 0 || cfg->n_routed % g->world != 0) return MOE_ERR_INVALID_ARG;
+  if (cfg->cap_policy != MOE_CAP_NONE) return MOE_ERR_UNSUPPORTED;
+  if (g->recv_rows <= 0 || g->recv_rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (!(num == 1 || num == g->world) || first < 0 || first + num > g->world) return MOE_ERR_INVALID_ARG;
+  for (int q = 0; q < g->world; ++q) {
+    if (!ptr_ok(g->recv_x[q]) || !ptr_ok(g->recv_out[q]) || !g->counts[q] || !aligned(g->counts[q], 4))
+      return MOE_ERR_INVALID_ARG;
+    if (num == 1 && g->world > 1 && (!g->flags[q] || !aligned(g->flags[q], 4))) return MOE_ERR_INVALID_ARG;
+  }
+  return MOE_OK;
+}
+
+moe_status begin_ep(const moe_config* cfg, const moe_ep_group* g, const moe_ep_rank& r, cudaStream_t s, Ctx* ctx) {
+  MOE_TRY(check_cfg(cfg, r.n));
+  if (!r.ws || !aligned(r.ws, 256)) return MOE_ERR_INVALID_ARG;
+  ctx->c = *cfg;
+  ctx->n = r.n;
+  ctx->p = make_plan(*cfg, r.n, g->world, g->recv_rows);
+  if (r.ws_bytes < ctx->p.total) return MOE_ERR_WORKSPACE;
+  ctx->ws = static_cast<char*>(r.ws);
+  ctx->s = s;
+  if (!tok_ok(r.x, r.n) || !tok_ok(r.y, r.n) || !r.weights || !ptr_ok(r.weights->w_router))
+    return MOE_ERR_INVALID_ARG;
+  if ((r.topk_idx_opt && !tok_ok(r.topk_idx_opt, r.n)) || (r.topk_w_opt && !tok_ok(r.topk_w_opt, r.n)))
+    return MOE_ERR_INVALID_ARG;
+  return check_weights(ctx->c, r.weights, true, true);
+}
+
+// The routed experts of one rank: its E / world experts over the receive buffer's rows.
+Ctx ep_expert_ctx(const Ctx& c, int32_t world, int64_t recv_rows) {
+  Ctx f = c;
+  f.c.n_routed = c.c.n_routed / world;
+  f.c.top_k = 1;
+  f.c.n_group = 1;
+  f.c.topk_group = 1;
+  f.n = recv_rows;
+  return f;
+}
+
+moe_status ep_forward(const moe_config* cfg, const moe_ep_group* g, int32_t first, int32_t num,
+                      const moe_ep_rank* ranks, cudaStream_t s) {
+  MOE_TRY(check_ep(cfg, g, first, num, ranks));
+  const int R = g->world;
+  const bool barriers = num == 1 && R > 1;
+  EpPeers peers{};
+  for (int q = 0; q < R; ++q) {
+    peers.recv_x[q] = g->recv_x[q];
+    peers.recv_out[q] = g->recv_out[q];
+    peers.counts[q] = g->counts[q];
+    peers.flags[q] = g->flags[q];
+  }
+  Ctx cx[kMaxEpRanks];
+  for (int i = 0; i < num; ++i) MOE_TRY(begin_ep(cfg, g, ranks[i], s, &cx[i]));
+  for (int i = 0; i < num; ++i) MOE_TRY(clear_status(cx[i]));
+  const moe_config& c = *cfg;
+  const uint64_t timeout = ep_timeout_ns();
+  auto barrier = [&]() -> moe_status {
+    if (!barriers) return MOE_OK;
+    return cuda_status(launch_ep_barrier(peers, R, first, timeout, cx[0].status(), s));
+  };
+  int32_t* idx[kMaxEpRanks];
+  float* tw[kMaxEpRanks];
+  void* sh[kMaxEpRanks] = {};
+  bool any_shared = false;
+  for (int i = 0; i < num; ++i) {
+    const moe_ep_rank& r = ranks[i];
+    idx[i] = r.topk_idx_opt && r.n > 0 ? r.topk_idx_opt : cx[i].at<int32_t>(cx[i].p.idx);
+    tw[i] = r.topk_w_opt && r.n > 0 ? r.topk_w_opt : cx[i].at<float>(cx[i].p.w);
+    any_shared |= r.n > 0 && c.n_shared > 0;
+  }
+  // Shared experts of every rank on the side stream, overlapping the exchange.
+  SideStream* side = any_shared ? side_stream() : nullptr;
+  if (side) {
+    MOE_CUDA(cudaEventRecord(side->fork, s));
+    MOE_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
+    for (int i = 0; i < num; ++i) {
+      Ctx cs = cx[i];
+      cs.s = side->s;
+      MOE_TRY(shared_impl(cs, ranks[i].x, ranks[i].weights, &sh[i]));
+    }
+    MOE_CUDA(cudaEventRecord(side->join, side->s));
+  }
+  // 1. route, local stable permutation, counts into every rank's table
+  for (int i = 0; i < num; ++i) {
+    const Ctx& x = cx[i];
+    int32_t* counts = x.at<int32_t>(x.p.counts);
+    MOE_TRY(route_impl(x, ranks[i].x, ranks[i].weights, idx[i], tw[i], counts, nullptr));
+    MOE_TRY(permute_impl(x, ranks[i].x, idx[i], x.at<int32_t>(x.p.offsets), x.at<int32_t>(x.p.perm),
+                         x.at<int32_t>(x.p.dest), nullptr));
+    MOE_CUDA(launch_ep_publish(peers, R, c.n_routed, first + i, counts, s));
+  }
+  MOE_TRY(barrier());
+  // 2. token rows into the owners' receive buffers
+  const int64_t row_bytes = (int64_t)c.d_model * (act_dtype(c) == MOE_BF16 ? 2 : 4);
+  for (int i = 0; i < num; ++i) {
+    const Ctx& x = cx[i];
+    const int rank = first + i;
+    MOE_CUDA(launch_ep_dispatch(peers, R, c.n_routed, rank, g->recv_rows, g->counts[rank],
+                                x.at<int32_t>(x.p.offsets), x.at<int32_t>(x.p.perm), ranks[i].x, x.n * c.top_k,
+                                row_bytes, x.at<int32_t>(x.p.ep_off), x.status(), s));
+  }
+  MOE_TRY(barrier());
+  // 3. each rank's experts over the rows it received
+  for (int i = 0; i < num; ++i) {
+    const int rank = first + i;
+    const Ctx f = ep_expert_ctx(cx[i], R, g->recv_rows);
+    MOE_TRY(ffn_impl(f, g->recv_x[rank], cx[i].at<int32_t>(cx[i].p.ep_off), ranks[i].weights, g->recv_out[rank]));
+  }
+  MOE_TRY(barrier());
+  // 4. gate-weighted sum of the owners' output rows, plus the shared experts
+  if (side) MOE_CUDA(cudaStreamWaitEvent(s, side->join, 0));
+  for (int i = 0; i < num; ++i) {
+    const Ctx& x = cx[i];
+    const int rank = first + i;
+    if (!side && c.n_shared > 0) MOE_TRY(shared_impl(x, ranks[i].x, ranks[i].weights, &sh[i]));
+    MOE_CUDA(launch_ep_combine(peers, R, c.n_routed, rank, g->recv_rows, g->counts[rank],
+                               x.at<int32_t>(x.p.offsets), idx[i], x.at<int32_t>(x.p.dest), tw[i], sh[i], x.n,
+                               c.top_k, c.d_model, act_dtype(c), ranks[i].y, s));
+  }
+  return barrier();
+}
+
+// Driver API entry for the base of the allocation holding a device address.
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(p);
+  });
+  return fn;
+}
+
+moe_status allocation_base(const void* ptr, char** base) {
+  AddressRangeFn fn = address_range_fn();
+  if (!fn) return MOE_ERR_CUDA;
+  CUdeviceptr b = 0;
+  size_t size = 0;
+  if (fn(&b, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS) return MOE_ERR_INVALID_ARG;
+  *base = reinterpret_cast<char*>(b);
+  return MOE_OK;
+}
+
+static_assert(sizeof(cudaIpcMemHandle_t) + sizeof(uint64_t) == MOE_EP_HANDLE_BYTES, "handle record size");
+
 }  // namespace
 }  // namespace moe
 
@@ -551,6 +726,51 @@ moe_status moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, uint8_t* 
   if (!ptr_ok(x) || !ptr_ok(codes) || !scale_bytes) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_quantize_rows(x, nullptr, nullptr, 1, rows, cols, codes, nullptr,
                                           reinterpret_cast<cudaStream_t>(stream), scale_bytes));
+}
+
+moe_status moe_ep_workspace_size(const moe_config* cfg, int32_t world, int64_t n, int64_t recv_rows, size_t* bytes) {
+  MOE_TRY(check_cfg(cfg, n));
+  if (!bytes || world < 1 || recv_rows <= 0 || recv_rows >= ((int64_t)1 << 31)) return MOE_ERR_INVALID_ARG;
+  if (world > MOE_EP_MAX_RANKS) return MOE_ERR_UNSUPPORTED;
+  if (cfg->n_routed % world != 0) return MOE_ERR_INVALID_ARG;
+  *bytes = make_plan(*cfg, n, world, recv_rows).total;
+  return MOE_OK;
+}
+
+moe_status moe_ep_layer_forward(const moe_config* cfg, const moe_ep_group* group, int32_t first_rank,
+                                int32_t num_ranks, const moe_ep_rank* ranks, moe_stream_t stream) {
+  return ep_forward(cfg, group, first_rank, num_ranks, ranks, reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_ep_export_handle(const void* ptr, void* handle) {
+  if (!ptr || !handle) return MOE_ERR_INVALID_ARG;
+  char* base = nullptr;
+  MOE_TRY(allocation_base(ptr, &base));
+  cudaIpcMemHandle_t h;
+  MOE_CUDA(cudaIpcGetMemHandle(&h, base));
+  const uint64_t off = (uint64_t)(static_cast<const char*>(ptr) - base);
+  memcpy(handle, &h, sizeof(h));
+  memcpy(static_cast<char*>(handle) + sizeof(h), &off, sizeof(off));
+  return MOE_OK;
+}
+
+moe_status moe_ep_open_handle(const void* handle, void** ptr) {
+  if (!handle || !ptr) return MOE_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  uint64_t off = 0;
+  memcpy(&h, handle, sizeof(h));
+  memcpy(&off, static_cast<const char*>(handle) + sizeof(h), sizeof(off));
+  void* base = nullptr;
+  MOE_CUDA(cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess));
+  *ptr = static_cast<char*>(base) + off;
+  return MOE_OK;
+}
+
+moe_status moe_ep_close_handle(void* ptr) {
+  if (!ptr) return MOE_ERR_INVALID_ARG;
+  char* base = nullptr;
+  MOE_TRY(allocation_base(ptr, &base));
+  return cuda_status(cudaIpcCloseMemHandle(base));
 }
 
 moe_status moe_sync_status(void* ws, moe_stream_t stream) {

@@ -106,6 +106,27 @@ cudaError_t launch_gather(const void* x, const int32_t* perm_token, const int32_
 cudaError_t launch_combine(const void* eo, const int32_t* slot_dest, const float* topk_w, const void* sh,
                            int64_t n, int32_t k, int32_t d, int dtype, void* y, cudaStream_t s);
 
+// Expert parallelism: every rank's exchange buffers as seen from the calling device.
+constexpr int kMaxEpRanks = MOE_EP_MAX_RANKS;
+struct EpPeers {
+  void* recv_x[kMaxEpRanks];
+  void* recv_out[kMaxEpRanks];
+  int32_t* counts[kMaxEpRanks];
+  uint32_t* flags[kMaxEpRanks];
+};
+cudaError_t launch_ep_publish(const EpPeers& p, int32_t R, int32_t E, int32_t rank, const int32_t* counts,
+                              cudaStream_t s);
+cudaError_t launch_ep_dispatch(const EpPeers& p, int32_t R, int32_t E, int32_t rank, int64_t recv_rows,
+                               const int32_t* table, const int32_t* offsets, const int32_t* perm_token,
+                               const void* x, int64_t max_rows, int64_t row_bytes, int32_t* recv_offsets,
+                               moe_diag* status, cudaStream_t s);
+cudaError_t launch_ep_combine(const EpPeers& p, int32_t R, int32_t E, int32_t rank, int64_t recv_rows,
+                              const int32_t* table, const int32_t* offsets, const int32_t* topk_idx,
+                              const int32_t* slot_dest, const float* topk_w, const void* sh, int64_t n, int32_t k,
+                              int32_t d, int dtype, void* y, cudaStream_t s);
+cudaError_t launch_ep_barrier(const EpPeers& p, int32_t R, int32_t rank, uint64_t timeout_ns, moe_diag* status,
+                              cudaStream_t s);
+
 // Small utilities.
 cudaError_t launch_fill_i32(int32_t* p, int64_t count, int32_t value, cudaStream_t s);
 cudaError_t launch_set_offsets2(int32_t* p, int64_t n, cudaStream_t s);
