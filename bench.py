@@ -11,6 +11,11 @@ is the maximum over ranks of the CUDA-event time of K steps.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on the host
 cores on a bounded token sample of the same workload.
+
+--ep R times the expert-parallel layer (moe_ep_layer_forward) of a group of R
+ranks emulated on one GPU: the workload's tokens split evenly over the ranks,
+rank q owning experts [q E/R, (q+1) E/R), every rank's exchange buffers in this
+GPU's memory and the steps of all ranks in stream order.
 """
 from __future__ import annotations
 
@@ -343,6 +348,183 @@ def run_ours(args):
         print(json.dumps(out), flush=True)
 
 
+NVLINK_GBS = 770.0  # measured peer copy per direction per GPU on this kind of node (NVLink 5)
+
+
+def _split(n, world):
+    return [n // world + (1 if q < n % world else 0) for q in range(world)]
+
+
+def _ep_rank_weights(moe, w, dev, q, world):
+    Eq = w.n_routed // world
+    sl = slice(q * Eq, (q + 1) * Eq)
+    if w.dtype == "fp8":
+        mats = ("gate", "up", "down")
+        scales = {k: dev["w_%s_s" % k][sl] for k in mats}
+        scales.update({"ws_" + k: dev["ws_%s_s" % k] for k in mats if "ws_%s_s" % k in dev})
+        return moe.make_weights(dev["w_r"], dev["w_gate_q"][sl], dev["w_up_q"][sl], dev["w_down_q"][sl],
+                                dev.get("ws_gate_q"), dev.get("ws_up_q"), dev.get("ws_down_q"), dev.get("bias"),
+                                scales=scales)
+    return moe.make_weights(dev["w_r"], dev["w_gate"][sl], dev["w_up"][sl], dev["w_down"][sl], dev.get("ws_gate"),
+                            dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
+
+
+def ep_launches_per_rank(w):
+    """Kernels of this library one rank launches in moe_ep_layer_forward (all ranks on one device)."""
+    n = 4  # router GEMM, route, histogram + scan of the counts
+    n += 3  # local stable permutation: histogram + scan + scatter (no local row gather)
+    n += 2  # count publish, row push
+    n += 4 if w.dtype == "fp8" else 2  # owned experts: (quantise,) GEMM1, (quantise,) GEMM2
+    if w.n_shared:
+        n += 4 if w.dtype == "fp8" else 2
+    n += 1  # combine
+    return n
+
+
+def run_ep(args):
+    import torch
+
+    import top_routing_expert_router_b200 as moe
+    from synth import workloads as W
+
+    world, rank, _ = _dist()
+    if world > 1:
+        raise SystemExit("--ep emulates the whole group on one GPU: run it as a single process")
+    R = args.ep
+    torch.cuda.set_device(0)
+    w = W.get(args.workload)
+    dev = W.device_inputs(w, device="cuda")
+    cfg = moe.make_config(dtype=w.dtype, **w.cfg_fields())
+    n, d, E, k = w.n, w.d_model, w.n_routed, w.top_k
+    Eq = E // R
+    splits = _split(n, R)
+    first = [sum(splits[:q]) for q in range(R + 1)]
+    recv_rows = moe.moe_ep_recv_rows_bound(cfg, R, splits)
+    x = dev["x"]
+    bufs = dict(recv_x=[torch.empty((recv_rows, d), dtype=x.dtype, device="cuda") for _ in range(R)],
+                recv_out=[torch.empty((recv_rows, d), dtype=x.dtype, device="cuda") for _ in range(R)],
+                counts=[torch.zeros((R, E), dtype=torch.int32, device="cuda") for _ in range(R)])
+    group = moe.make_ep_group(recv_rows, **bufs)
+    y = torch.empty_like(x)
+    idx = torch.empty((n, k), dtype=torch.int32, device="cuda")
+    ranks = [dict(n=splits[q], x=x[first[q]:first[q + 1]], y=y[first[q]:first[q + 1]],
+                  topk_idx=idx[first[q]:first[q + 1]], weights=_ep_rank_weights(moe, w, dev, q, R),
+                  ws=torch.empty(moe.moe_ep_workspace_size(cfg, R, splits[q], recv_rows), dtype=torch.uint8,
+                                 device="cuda")) for q in range(R)]
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+
+    def step(xin=None, yout=None):
+        rs = ranks
+        if xin is not None:
+            rs = [dict(r, x=xin[first[q]:first[q + 1]], y=yout[first[q]:first[q + 1]]) for q, r in enumerate(ranks)]
+        moe.moe_ep_layer_forward(cfg, group, 0, rs, stream=s)
+
+    for _ in range(args.warmup):
+        step()
+    for r in ranks:
+        st = moe.moe_sync_status(r["ws"], s)
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"device status after warm-up: {moe.moe_status_string(st)}")
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0] or "0") as clk:
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    ms_step = ev0.elapsed_time(ev1) / args.steps
+    clocks = clk.summary()
+
+    # Exchange volume: slot rows whose expert lives on another rank cross NVLink twice (token row
+    # out, expert output back); the busiest rank bounds the time.
+    owner = (idx.cpu() // Eq).numpy()
+    src = __import__("numpy").repeat(__import__("numpy").arange(R), splits)[:, None]
+    bpe = x.element_size()
+    remote = (owner != src) & (idx.cpu().numpy() >= 0)
+    sent = [int(remote[first[q]:first[q + 1]].sum()) for q in range(R)]
+    recvd = [int((remote & (owner == q)).sum()) for q in range(R)]
+    busiest = max(max(sent), max(recvd)) * d * bpe
+    nvlink_ms = 2 * busiest / (NVLINK_GBS * 1e9) * 1e3  # dispatch + combine, each one direction per rank
+
+    # Owned-expert FFN of every rank over the rows it received (the same kernels as in the layer).
+    tables = bufs["counts"][0].cpu()
+    col = tables.sum(0)
+    ffn_cfg = moe.make_config(dtype=w.dtype, **{**w.cfg_fields(), "n_routed": Eq, "top_k": 1, "n_shared": 0,
+                                                "n_group": 1, "topk_group": 1, "score_fn": "softmax",
+                                                "renormalize": False, "routed_scaling_factor": 1.0})
+    ffn_ws = torch.empty(moe.moe_workspace_size(ffn_cfg, recv_rows), dtype=torch.uint8, device="cuda")
+    offs = []
+    for q in range(R):
+        c = col[q * Eq:(q + 1) * Eq]
+        offs.append(torch.cat([torch.zeros(1, dtype=torch.int64), c.cumsum(0)]).to(torch.int32).cuda())
+    reps = max(3, min(args.steps, 10))
+    for q in range(R):
+        moe.moe_expert_ffn(ffn_cfg, recv_rows, bufs["recv_x"][q], offs[q], ranks[q]["weights"], bufs["recv_out"][q],
+                           ffn_ws, s)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(reps):
+        for q in range(R):
+            moe.moe_expert_ffn(ffn_cfg, recv_rows, bufs["recv_x"][q], offs[q], ranks[q]["weights"],
+                               bufs["recv_out"][q], ffn_ws, s)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ffn_ms = a.elapsed_time(b) / reps
+    if moe.moe_sync_status(ffn_ws, s) != moe.MOE_OK:
+        raise RuntimeError("device status after the expert FFN")
+    kept = int(col.sum())
+    ffn_flops = 6.0 * kept * d * w.moe_intermediate_size
+
+    # End to end: every step copies x in from pinned host memory and y out to pinned host memory.
+    x_host = x.cpu().pin_memory()
+    y_host = torch.empty_like(y, device="cpu").pin_memory()
+    xd, yd = torch.empty_like(x), torch.empty_like(y)
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(e2e_steps):
+        xd.copy_(x_host, non_blocking=True)
+        step(xd, yd)
+        y_host.copy_(yd, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / e2e_steps
+    if not torch.equal(y_host, y.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident run")
+
+    hbm, tf_burst, tf_sust, peak_kind = _peaks()
+    peak_dtype = "bf16"
+    if w.dtype == "fp8":
+        tf_burst, tf_sust, peak_dtype = 2 * tf_burst, 2 * tf_sust if tf_sust else None, "bf16 x 2 (nominal fp8/bf16) for fp8"
+    achieved = ffn_flops / (ffn_ms / 1e3) / 1e12
+    out = {
+        "metric": METRIC, "value": n / (ms_step / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 x e4m3 -> f32 (bf16 activations)" if w.dtype == "fp8" else w.dtype,
+        "data": "synthetic (seeded counter-based generator; Irwin-Hall normals)",
+        "config": {"workload": w.name, "n_tokens": n, "tokens_per_rank": splits,
+                   "parallelism": f"ep{R} emulated on 1 GPU (every rank's buffers local, ranks in stream order)",
+                   "recv_rows": recv_rows,
+                   "l2": "inputs larger than L2: every expert's weights streamed per step"},
+        "roofline": {"bound": "tensor", "kernel": "owned-expert FFN of every rank (grouped SwiGLU GEMM1 + GEMM2)",
+                     "achieved": achieved, "peak": tf_burst, "unit": "TFLOP/s", "frac": achieved / tf_burst,
+                     "peak_kind": f"{peak_kind} {peak_dtype} burst", "flops_per_launch": ffn_flops,
+                     "traffic": None},
+        "exchange": {"remote_slots_sent_per_rank": sent, "remote_slots_received_per_rank": recvd,
+                     "busiest_rank_bytes_each_way": busiest, "nvlink_gbs": NVLINK_GBS,
+                     "projected_nvlink_ms_dispatch_plus_combine": nvlink_ms,
+                     "layer_minus_ffn_ms": ms_step - ffn_ms},
+        "e2e": {"value": n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": n * d * bpe,
+                "d2h_bytes_per_step": n * d * bpe, "ms_per_step": e2e_ms},
+        "gpu_launches": ep_launches_per_rank(w) * R * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(out), flush=True)
+
+
 def _oracle_inputs(w, tokens):
     """Host inputs of the oracle's sample: the first `tokens` rows of x and all weights."""
     from synth import workloads as W
@@ -422,11 +604,14 @@ def main():
     ap.add_argument("--cpu-sample", type=int, default=16, help="tokens in the oracle's timed sample")
     ap.add_argument("--ref-sample", type=int, default=1, help="tokens per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ep", type=int, default=0, help="expert-parallel group of this many ranks, emulated on one GPU")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep > 1:
+        run_ep(args)
     else:
         run_ours(args)
 
