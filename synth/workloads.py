@@ -155,6 +155,13 @@ WORKLOADS = {w.name: w for w in [
     _wl("deepseek_v3_small_fp8", n=333, dtype="fp8", **{**_V3, "d_model": 256, "moe_intermediate_size": 128}),
     _wl("fp8_ragged_small", n=300, d_model=384, n_routed=12, top_k=3, moe_intermediate_size=256, n_shared=1,
         dtype="fp8", renormalize=True),
+    _wl("deepseek_v3_decode_small_fp8", n=40, dtype="fp8", **{**_V3, "d_model": 512, "moe_intermediate_size": 256}),
+    # profiling case: DeepSeek-V3 decode shapes with 32 FP8 experts (1.4 GB of weights)
+    _wl("deepseek_v3_decode_fp8_32e", n=64, dtype="fp8",
+        **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4},
+        description="DeepSeek-V3-shaped decode with 32 FP8 experts (profiling size)"),
+    _wl("fp8_skewed_small", n=200, d_model=256, n_routed=16, top_k=1, moe_intermediate_size=128, zipf_s=1.2,
+        dtype="fp8"),
     _wl("tie_softmax", n=256, d_model=64, n_routed=16, top_k=4, moe_intermediate_size=64,
         ternary=True, renormalize=True),
     _wl("tie_sigmoid", n=256, d_model=64, n_routed=32, top_k=4, moe_intermediate_size=64,

@@ -20,7 +20,10 @@ from tests import moe_harness as H
 
 pytestmark = pytest.mark.gpu
 
-FP8_SMALL = ["fp8_ragged_small", "deepseek_v3_small_fp8"]
+# fp8_ragged_small: 75 rows per expert (128 x 128 tiles); the others average at most 16 rows per
+# expert, where the GEMM takes 32-row tiles (fp8_skewed_small: a Zipf-skewed router sends some
+# experts more than 32 rows, so their groups span several short tiles).
+FP8_SMALL = ["fp8_ragged_small", "deepseek_v3_small_fp8", "deepseek_v3_decode_small_fp8", "fp8_skewed_small"]
 MATS = ("gate", "up", "down")
 
 
@@ -73,12 +76,17 @@ def test_quantize_fp8_rejects_bad_shapes():
         moe.moe_quantize_fp8(x, q, s)
 
 
-@pytest.mark.parametrize("bn", ["128", "256"])
+@pytest.mark.parametrize("bn", ["rule", "128", "256", "s128", "s256"])
 @pytest.mark.parametrize("unit_scales", [False, True])
 @pytest.mark.parametrize("name", FP8_SMALL)
 def test_fp8_expert_ffn_parity(name, unit_scales, bn, monkeypatch):
-    """Both tile widths (128 x 128 with two accumulators, 128 x 256 with one) match the oracle."""
-    monkeypatch.setenv("MOE_FP8_BN", bn)
+    """Every tile shape matches the oracle: the one the rows per expert choose, 128-row tiles forced
+    at both widths (128 x 128 with two accumulators, 128 x 256 with one), and short 32-row tiles at
+    both widths where the rows per expert allow them."""
+    if bn == "rule":
+        monkeypatch.delenv("MOE_FP8_BN", raising=False)
+    else:
+        monkeypatch.setenv("MOE_FP8_BN", bn)
     w = W.get(name)
     host, dev = W.host_inputs(w), W.device_inputs(w)
     if unit_scales:  # every weight block scale 2^0: isolates the activation-side scales

@@ -283,13 +283,14 @@ moe_status ffn_fp8(const Ctx& x, const void* A, const int32_t* a_rows, const int
   uint8_t* hq = x.at<uint8_t>(x.p.hq);
   uint32_t* sfh = x.at<uint32_t>(x.p.sfh);
   void* h = x.ws + x.p.h;
-  MOE_CUDA(launch_quantize_rows(A, a_rows, offsets, c.n_routed, nk, (int32_t)d, xq, sfx, x.s));
+  const int32_t tr = fp8_tile_rows(nk, c.n_routed);
+  MOE_CUDA(launch_quantize_rows(A, a_rows, offsets, c.n_routed, nk, (int32_t)d, tr, xq, sfx, x.s));
   GemmFp8Args g1{xq, w->w_gate, w->w_up, sfx, w->w_gate_scale, w->w_up_scale, h, I, offsets, c.n_routed, nk,
-                 (int32_t)I, (int32_t)d};
+                 (int32_t)I, (int32_t)d, tr};
   MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
-  MOE_CUDA(launch_quantize_rows(h, nullptr, offsets, c.n_routed, nk, (int32_t)I, hq, sfh, x.s));
+  MOE_CUDA(launch_quantize_rows(h, nullptr, offsets, c.n_routed, nk, (int32_t)I, tr, hq, sfh, x.s));
   GemmFp8Args g2{hq, w->w_down, nullptr, sfh, w->w_down_scale, nullptr, eo, d, offsets, c.n_routed, nk,
-                 (int32_t)d, (int32_t)I};
+                 (int32_t)d, (int32_t)I, tr};
   MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
   return MOE_OK;
 }
@@ -322,13 +323,14 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
     uint32_t* sfx = x.at<uint32_t>(x.p.sfxs);
     uint8_t* hq = x.at<uint8_t>(x.p.hsq);
     uint32_t* sfh = x.at<uint32_t>(x.p.sfhs);
-    MOE_CUDA(launch_quantize_rows(X, nullptr, nullptr, 1, x.n, (int32_t)d, xq, sfx, x.s));
+    const int32_t tr = fp8_tile_rows(x.n, 1);
+    MOE_CUDA(launch_quantize_rows(X, nullptr, nullptr, 1, x.n, (int32_t)d, tr, xq, sfx, x.s));
     GemmFp8Args g1{xq, w->ws_gate, w->ws_up, sfx, w->ws_gate_scale, w->ws_up_scale, shh, Is, nullptr, 1, x.n,
-                   (int32_t)Is, (int32_t)d};
+                   (int32_t)Is, (int32_t)d, tr};
     MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
-    MOE_CUDA(launch_quantize_rows(shh, nullptr, nullptr, 1, x.n, (int32_t)Is, hq, sfh, x.s));
+    MOE_CUDA(launch_quantize_rows(shh, nullptr, nullptr, 1, x.n, (int32_t)Is, tr, hq, sfh, x.s));
     GemmFp8Args g2{hq, w->ws_down, nullptr, sfh, w->ws_down_scale, nullptr, sh, d, nullptr, 1, x.n, (int32_t)d,
-                   (int32_t)Is};
+                   (int32_t)Is, tr};
     MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
     *sh_out = sh;
     return MOE_OK;
@@ -724,7 +726,7 @@ moe_status moe_quantize_fp8(const void* x, int64_t rows, int32_t cols, uint8_t* 
   if (rows < 0 || cols <= 0 || cols % 128 != 0 || rows * (int64_t)cols >= (int64_t)1 << 40) return MOE_ERR_INVALID_ARG;
   if (rows == 0) return MOE_OK;
   if (!ptr_ok(x) || !ptr_ok(codes) || !scale_bytes) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_quantize_rows(x, nullptr, nullptr, 1, rows, cols, codes, nullptr,
+  return cuda_status(launch_quantize_rows(x, nullptr, nullptr, 1, rows, cols, 128, codes, nullptr,
                                           reinterpret_cast<cudaStream_t>(stream), scale_bytes));
 }
 

@@ -20,6 +20,11 @@
 //               scale byte of their sub-block; tcgen05.commit frees the stage.
 //   warps 2..5  epilogue: tcgen05.ld, SwiGLU in fp32, bf16 stores.
 // Every mbarrier wait is bounded like the bf16 kernels'.
+// Short tiles (groups of a few rows, decode): an m-tile covers 32 rows and a
+// stage holds only those 32 A rows next to the B tile, so 160 KB of weights
+// stay in flight per SM (5 stages of 256-wide tiles, 10 of 128-wide). The MMA
+// still reads a 128-row A operand; its rows 32..127 fall on the stage's B bytes
+// and produce accumulator rows that are never stored.
 #include <cuda.h>
 #include <stdlib.h>
 #include <string.h>
@@ -40,17 +45,21 @@ constexpr uint64_t kDrainNs = 200000000ull;
 
 // Tile shapes: BN = 128 keeps two TMEM accumulators (the epilogue of one tile
 // overlaps the next); BN = 256 halves the copies of A per MMA but leaves TMEM
-// room for one accumulator next to the scale factors.
-template <int BN>
+// room for one accumulator next to the scale factors. BMR = rows of an m-tile
+// (128, or 32 for short tiles).
+template <int BN, int BMR>
 struct Shape {
   static constexpr int ACC_BUFS = BN == 256 ? 1 : 2;
+  static constexpr int A_STAGE = BMR * BK;  // A bytes copied per stage
   static constexpr int B_BYTES = BN * BK;
   static constexpr int SFB_BYTES = (BN / 128) * SF_BYTES;
-  static constexpr int STAGE_BYTES = (A_BYTES + B_BYTES + SF_BYTES + SFB_BYTES + 1023) / 1024 * 1024;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGE_BYTES = (A_STAGE + B_BYTES + SF_BYTES + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGES = BMR == 32 ? (BN == 256 ? 5 : 10) : (BN == 256 ? 4 : 6);
   static constexpr uint32_t SF_COL0 = ACC_BUFS * BN;   // scale factors after the accumulators
   static constexpr uint32_t SF_COLS = 4 + BN / 32;     // per stage: A (128 rows) and B (BN rows)
   static_assert(SF_COL0 + SF_COLS * STAGES <= TMEM_COLS, "TMEM budget");
+  static_assert(A_STAGE + B_BYTES >= A_BYTES, "the MMA's 128-row A operand stays inside its stage");
+  static_assert(BMR == 128 || BMR == 32, "m-tile heights");
 };
 
 struct Fp8Params {
@@ -70,7 +79,7 @@ struct Fp8Params {
   moe_diag* status;
 };
 
-constexpr int kMaxStages = 6;
+constexpr int kMaxStages = 10;
 
 struct __align__(8) Ctl {
   uint64_t full[kMaxStages];
@@ -84,7 +93,7 @@ struct __align__(8) Ctl {
   int32_t n_tiles;
   int32_t row_off[kMaxGroupsFp8 + 1];
   int32_t tile_off[kMaxGroupsFp8 + 1];
-  int32_t sf_off[kMaxGroupsFp8 + 1];  // first 128-row scale tile of each group
+  int32_t sf_off[kMaxGroupsFp8 + 1];  // first scale tile (one per m-tile) of each group
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
@@ -227,12 +236,13 @@ struct Tile {
   int g, m, nt;
 };
 
+template <int BMR>
 __device__ __forceinline__ Tile decode(const Ctl* ctl, int G, int t, int& g_hint) {
   int g = g_hint;
   while (g + 1 <= G && ctl->tile_off[g + 1] <= t) ++g;
   g_hint = g;
   const int local = t - ctl->tile_off[g];
-  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BM - 1) / BM;
+  const int mt = (ctl->row_off[g + 1] - ctl->row_off[g] + BMR - 1) / BMR;
   return Tile{g, local % mt, local / mt};
 }
 
@@ -250,12 +260,12 @@ __device__ __forceinline__ void store16(bf16* C, int64_t ldc, int64_t row, int c
   if (col + 16 <= N) *reinterpret_cast<uint4*>(p + 8) = hi;
 }
 
-template <int BN>
+template <int BN, int BMR>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_fp8_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
                     const __grid_constant__ CUtensorMap map_b2, Fp8Params p) {
-  using S = Shape<BN>;
-  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES, B_BYTES = S::B_BYTES;
+  using S = Shape<BN, BMR>;
+  constexpr int STAGES = S::STAGES, STAGE_BYTES = S::STAGE_BYTES, B_BYTES = S::B_BYTES, A_STAGE = S::A_STAGE;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
@@ -267,7 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = 0; g < p.G; ++g) {
       const int lo = p.offsets ? p.offsets[g] : 0;
       const int hi = p.offsets ? p.offsets[g + 1] : p.M;
-      const int mt = (hi - lo + BM - 1) / BM;
+      const int mt = (hi - lo + BMR - 1) / BMR;
       ctl->row_off[g] = lo;
       ctl->row_off[g + 1] = hi;
       ctl->tile_off[g] = acc;
@@ -313,14 +323,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g_hint = 0;
     bool ok = true;
     uint32_t armed[STAGES] = {};
-    const uint32_t tx = A_BYTES + B_BYTES + SF_BYTES;  // TMA tiles and A's scale block
+    const uint32_t tx = A_STAGE + B_BYTES + SF_BYTES;  // TMA tiles and A's scale block
     // B scale bytes of a tile: lane l keeps k-blocks l, l + 32, l + 64, l + 96 of the gate (or
     // plain) block, the up block and, for plain 256-wide tiles, the next 128-row block. They are
     // loaded one tile ahead, so a tile's first stage does not wait for them.
     int pf_hint = 0;
     auto load_scales = [&](int tt, uint32_t (&g)[4], uint32_t (&u)[4], uint32_t (&nx)[4]) {
       if (tt >= total) return;
-      const Tile tl = decode(ctl, p.G, tt, pf_hint);
+      const Tile tl = decode<BMR>(ctl, p.G, tt, pf_hint);
       const int brow_local = tl.nt * p.n_out;
       const uint8_t* sb_g = p.sb + ((int64_t)tl.g * nbr + brow_local / 128) * nkb;
       const uint8_t* sb2_g = p.swiglu ? p.sb2 + ((int64_t)tl.g * nbr + brow_local / 128) * nkb : sb_g;
@@ -336,8 +346,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t nsbg[4], nsbu[4], nsbn[4];
     load_scales(blockIdx.x, nsbg, nsbu, nsbn);
     for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Tile tl = decode(ctl, p.G, t, g_hint);
-      const int row0 = ctl->row_off[tl.g] + tl.m * BM;
+      const Tile tl = decode<BMR>(ctl, p.G, t, g_hint);
+      const int row0 = ctl->row_off[tl.g] + tl.m * BMR;
       const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
       const uint32_t* sfa_tile = p.sfa + (int64_t)(ctl->sf_off[tl.g] + tl.m) * nkb * 128;
       uint32_t sbg[4], sbu[4], sbn[4];
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         uint8_t* sa = smem + stage * STAGE_BYTES;
-        uint8_t* sbm = sa + A_BYTES;
+        uint8_t* sbm = sa + A_STAGE;
         uint8_t* sfa_s = sbm + B_BYTES;
         uint8_t* sfb_s = sfa_s + SF_BYTES;
         if (lane == 0) {
@@ -424,12 +434,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
           const uint32_t sfa_t = tmem_base + S::SF_COL0 + S::SF_COLS * (uint32_t)stage;
           const uint32_t sfb_t = sfa_t + 4u;
-          sf_copy(sfa_t, sf_desc(sa + A_BYTES + B_BYTES));
+          sf_copy(sfa_t, sf_desc(sa + A_STAGE + B_BYTES));
 #pragma unroll
           for (int blk = 0; blk < BN / 128; ++blk)  // B rows 128 blk .. : TMEM columns 4 blk ..
-            sf_copy(sfb_t + 4u * blk, sf_desc(sa + A_BYTES + B_BYTES + SF_BYTES + SF_BYTES * blk));
+            sf_copy(sfb_t + 4u * blk, sf_desc(sa + A_STAGE + B_BYTES + SF_BYTES + SF_BYTES * blk));
           const uint64_t adesc = sw128_desc(sa);
-          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+          const uint64_t bdesc = sw128_desc(sa + A_STAGE);
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 elements = 32 bytes per MMA
             mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(BN, k), sfa_t, sfb_t,
@@ -458,13 +468,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
       const int buf = S::ACC_BUFS == 2 ? (i & 1) : 0;
       const uint32_t acc_phase = (uint32_t)(S::ACC_BUFS == 2 ? (i >> 1) : i) & 1u;
-      const Tile tl = decode(ctl, p.G, t, g_hint);
+      const Tile tl = decode<BMR>(ctl, p.G, t, g_hint);
       const bool got = mbar_wait(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
       __syncwarp();
       if (!got) break;
       fence_after();
-      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BM + row_in_tile;
-      const bool valid = row < ctl->row_off[tl.g + 1];
+      const int64_t row = (int64_t)ctl->row_off[tl.g] + tl.m * BMR + row_in_tile;
+      const bool valid = row_in_tile < BMR && row < ctl->row_off[tl.g + 1];
+      if (BMR < 128 && q * 32 >= BMR) {  // accumulator rows past a short tile: nothing to store
+        fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+        continue;
+      }
       const int col0 = tl.nt * p.n_out;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * BN);
       bf16* C = static_cast<bf16*>(p.C);
@@ -531,14 +547,18 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, i
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN>
+template <int BN, int BMR>
 constexpr size_t smem_bytes() {
-  return 1024 + Shape<BN>::STAGES * Shape<BN>::STAGE_BYTES + sizeof(Ctl);
+  return 1024 + Shape<BN, BMR>::STAGES * Shape<BN, BMR>::STAGE_BYTES + sizeof(Ctl);
 }
-static_assert(smem_bytes<128>() <= 232448 && smem_bytes<256>() <= 232448, "dynamic shared memory above 227 KB");
-static_assert(Shape<128>::STAGES <= kMaxStages && Shape<256>::STAGES <= kMaxStages, "barrier arrays");
+static_assert(smem_bytes<128, 128>() <= 232448 && smem_bytes<256, 128>() <= 232448 &&
+                  smem_bytes<128, 32>() <= 232448 && smem_bytes<256, 32>() <= 232448,
+              "dynamic shared memory above 227 KB");
+static_assert(Shape<128, 128>::STAGES <= kMaxStages && Shape<256, 128>::STAGES <= kMaxStages &&
+                  Shape<128, 32>::STAGES <= kMaxStages && Shape<256, 32>::STAGES <= kMaxStages,
+              "barrier arrays");
 
-template <int BN>
+template <int BN, int BMR>
 cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
   Fp8Params p{};
   p.G = a.G;
@@ -557,7 +577,7 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
   p.status = status;
   CUtensorMap ma, mb, mb2;
   const int b_box = swiglu ? BN / 2 : BN;
-  if (!make_map_u8(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
+  if (!make_map_u8(&ma, a.A, a.M, a.K, BMR)) return cudaErrorInvalidValue;
   if (!make_map_u8(&mb, a.B, (int64_t)a.G * a.N, a.K, b_box)) return cudaErrorInvalidValue;
   if (swiglu) {
     if (!make_map_u8(&mb2, a.B2, (int64_t)a.G * a.N, a.K, b_box)) return cudaErrorInvalidValue;
@@ -567,7 +587,8 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
   static bool attr = false;
   if (!attr) {
     const cudaError_t e =
-        cudaFuncSetAttribute(gemm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes<BN>());
+        cudaFuncSetAttribute(gemm_fp8_kernel<BN, BMR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem_bytes<BN, BMR>());
     if (e != cudaSuccess) return e;
     attr = true;
   }
@@ -576,20 +597,36 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
   const int64_t n_tiles = ceil_div(a.N, p.n_out);
-  const int64_t max_tiles = (ceil_div(a.M, BM) + (a.offsets ? a.G : 0)) * n_tiles;
+  const int64_t max_tiles = (ceil_div(a.M, BMR) + (a.offsets ? a.G : 0)) * n_tiles;
   const int grid = (int)(max_tiles < sms ? max_tiles : sms);
-  gemm_fp8_kernel<BN><<<grid, kThreads, smem_bytes<BN>(), s>>>(ma, mb, mb2, p);
+  gemm_fp8_kernel<BN, BMR><<<grid, kThreads, smem_bytes<BN, BMR>(), s>>>(ma, mb, mb2, p);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// Groups averaging at least 128 rows (prefill) run 128 x 256 tiles: at the FP8 MMA
-// rate the L2 -> SM copies bound the kernel, and 256-wide tiles copy 25 % fewer
-// bytes per MAC, which outweighs the epilogue no longer overlapping the next tile.
-// Smaller groups (decode) stream weights: 128-wide tiles with two accumulators keep
-// twice as many independent tiles in flight. MOE_FP8_BN=128|256 overrides (tuning
-// and tests).
+// Tile choice from the rows per group (M rows in G groups):
+//  - >= 128 rows (prefill): 128 x 256 tiles. At the FP8 MMA rate the L2 -> SM copies bound the
+//    kernel, and 256-wide tiles copy 25 % fewer bytes per MAC, which outweighs the epilogue no
+//    longer overlapping the next tile.
+//  - <= 16 rows (decode): short 32-row tiles, 128 wide with two accumulators and 10 stages:
+//    weight streaming at HBM rate needs bytes in flight (160 KB of weights per SM), and a group of
+//    a few rows needs none of a 128-row A tile. (256-wide short tiles, 5 stages, measured 13 %
+//    slower on the DeepSeek-V3 decode layer.)
+//  - otherwise 128 x 128 tiles with two accumulators.
+// MOE_FP8_BN (tuning and tests): 128 | 256 force 128-row tiles of that width; s128 | s256 force
+// the width of short tiles where the rule allows them. The workspace holds scale blocks for the
+// short tiles whenever the rule could choose them.
+bool fp8_short_rule(int64_t M, int32_t G) { return M <= 16 * (int64_t)G; }
+
+int fp8_tile_rows(int64_t M, int32_t G) {
+  const char* bn = getenv("MOE_FP8_BN");
+  if (bn && bn[0] != 's') return 128;
+  return fp8_short_rule(M, G) ? 32 : 128;
+}
+
+int64_t fp8_sf_tiles_bound(int64_t rows, int32_t G) { return ceil_div(rows, fp8_short_rule(rows, G) ? 32 : 128) + G; }
+
 cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s) {
   if (a.M <= 0) return cudaSuccess;
   if (a.K % BK != 0 || a.K / BK > 128 || a.N % 16 != 0 || a.N <= 0 || a.G < 1 || a.G > kMaxGroupsFp8)
@@ -598,9 +635,13 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
       reinterpret_cast<uintptr_t>(a.sfa) % 16 || reinterpret_cast<uintptr_t>(a.C) % 16 || a.ldc % 8 != 0 ||
       (swiglu && reinterpret_cast<uintptr_t>(a.B2) % 16))
     return cudaErrorInvalidValue;
+  if (a.tile_rows != fp8_tile_rows(a.M, a.offsets ? a.G : 1)) return cudaErrorInvalidValue;
   const char* bn = getenv("MOE_FP8_BN");
-  const bool wide = bn ? strcmp(bn, "256") == 0 : a.M / (a.offsets ? a.G : 1) >= 128;
-  return wide ? launch_bn<256>(a, swiglu, status, s) : launch_bn<128>(a, swiglu, status, s);
+  if (a.tile_rows == 32)
+    return bn && strcmp(bn, "s256") == 0 ? launch_bn<256, 32>(a, swiglu, status, s)
+                                         : launch_bn<128, 32>(a, swiglu, status, s);
+  const bool wide = bn && bn[0] != 's' ? strcmp(bn, "256") == 0 : a.M / (a.offsets ? a.G : 1) >= 128;
+  return wide ? launch_bn<256, 128>(a, swiglu, status, s) : launch_bn<128, 128>(a, swiglu, status, s);
 }
 
 }  // namespace moe

@@ -52,16 +52,21 @@ struct GemmFp8Args {
   int64_t M;
   int32_t N;
   int32_t K;
+  int32_t tile_rows;      // rows per A tile and scale block: fp8_tile_rows(M, G)
 };
 cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s);
+// Rows per A tile of the FP8 GEMM (32 for groups of a few rows, else 128); the quantiser lays the
+// scale blocks out for the same tiles.
+int fp8_tile_rows(int64_t M, int32_t G);
 
 // E4M3 quantisation of bf16 rows in 1 x 128 tiles (row r reads src[src_row[r]] when
-// src_row is given); scale words go to the GEMM's scale-factor blocks of the groups.
+// src_row is given); scale words go to the GEMM's scale-factor blocks of the groups, one per
+// tile_rows-row tile. fp8_sf_tiles_bound: scale blocks per 128-wide k block for any tile choice.
 int64_t fp8_sf_tiles_bound(int64_t rows, int32_t G);
 // sf_plain given: scale bytes [rows, cols/128] instead of the GEMM's blocks.
 cudaError_t launch_quantize_rows(const void* src, const int32_t* src_row, const int32_t* offsets, int32_t G,
-                                 int64_t rows_bound, int32_t cols, uint8_t* q, uint32_t* sf, cudaStream_t s,
-                                 uint8_t* sf_plain = nullptr);
+                                 int64_t rows_bound, int32_t cols, int32_t tile_rows, uint8_t* q, uint32_t* sf,
+                                 cudaStream_t s, uint8_t* sf_plain = nullptr);
 
 // Router: scoring, group limit, top-k, certification / binary64 refinement, gates.
 struct RouteArgs {

@@ -6,11 +6,12 @@
 //   e      = the smallest integer with amax <= 448 * 2^e (0 when amax = 0),
 //   code_c = E4M3 of v_c * 2^-e, round to nearest even (|v_c * 2^-e| <= 448).
 // The scale of row r, tile t is written where the tensor-core GEMM reads it:
-// 128-row GEMM tiles of each group (tile m of group g covers rows
-// offsets[g] + 128m ...), one 512-byte block per (tile, 128-column tile) in the
-// scale-factor layout of tcgen05.mma block scaling: the 32-bit word of tile
-// row p sits at word 4 (p % 32) + p / 32 and holds the UE8M0 byte four times
-// (one per 32-column sub-block, all equal for 1 x 128 tiles).
+// GEMM row tiles of TR = 128 (or 32) rows of each group (tile m of group g
+// covers rows offsets[g] + TR m ...), one 512-byte block per (row tile,
+// 128-column tile) in the scale-factor layout of tcgen05.mma block scaling: the
+// 32-bit word of tile row p sits at word 4 (p % 32) + p / 32 and holds the
+// UE8M0 byte four times (one per 32-column sub-block, all equal for 1 x 128
+// tiles).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -46,8 +47,8 @@ constexpr int kQuantWarps = 8;
 // One warp per row, two 128-column tiles at a time (one per half-warp).
 __global__ void __launch_bounds__(32 * kQuantWarps)
     quantize_rows_kernel(const bf16* src, const int32_t* src_row, const int32_t* offsets, int G, int64_t rows_single,
-                         int cols, uint8_t* q, uint32_t* sf, uint8_t* sf_plain) {
-  __shared__ int32_t tile_off[kMaxExperts + 1];  // first 128-row tile of each group
+                         int cols, int TR, uint8_t* q, uint32_t* sf, uint8_t* sf_plain) {
+  __shared__ int32_t tile_off[kMaxExperts + 1];  // first row tile of each group
   __shared__ int32_t row_off[kMaxExperts + 1];
   if (threadIdx.x == 0) {
     int32_t acc = 0;
@@ -57,7 +58,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
       row_off[g] = lo;
       row_off[g + 1] = hi;
       tile_off[g] = acc;
-      acc += (hi - lo + 127) / 128;
+      acc += (hi - lo + TR - 1) / TR;
     }
     tile_off[G] = acc;
   }
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t r = warp; r < rows; r += nwarps) {
-    // group of row r (offsets ascending), its 128-row GEMM tile and the row inside it
+    // group of row r (offsets ascending), its GEMM row tile and the row inside it
     int lo = 0, hi = G - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
@@ -76,8 +77,8 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
     }
     const int g = lo;
     const int64_t local = r - row_off[g];
-    const int64_t tile = tile_off[g] + local / 128;
-    const int p = (int)(local % 128);
+    const int64_t tile = tile_off[g] + local / TR;
+    const int p = (int)(local % TR);
     const int64_t srow = src_row ? (int64_t)src_row[r] : r;
     // Half-warp h of the warp owns tile 2c + h of chunk c (256 columns); lane l of a
     // half-warp holds columns 8 (l % 16) .. +7 of its tile: one 16-byte load and one
@@ -136,17 +137,16 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
 
 }  // namespace
 
-int64_t fp8_sf_tiles_bound(int64_t rows, int32_t G) { return ceil_div(rows, 128) + G; }
-
 cudaError_t launch_quantize_rows(const void* src, const int32_t* src_row, const int32_t* offsets, int32_t G,
-                                 int64_t rows_bound, int32_t cols, uint8_t* q, uint32_t* sf, cudaStream_t s,
-                                 uint8_t* sf_plain) {
+                                 int64_t rows_bound, int32_t cols, int32_t tile_rows, uint8_t* q, uint32_t* sf,
+                                 cudaStream_t s, uint8_t* sf_plain) {
   if (rows_bound <= 0) return cudaSuccess;
-  if (cols % 128 != 0 || G < 1 || G > kMaxExperts) return cudaErrorInvalidValue;
+  if (cols % 128 != 0 || G < 1 || G > kMaxExperts || (tile_rows != 128 && tile_rows != 32))
+    return cudaErrorInvalidValue;
   int64_t blocks = ceil_div(rows_bound, kQuantWarps);
   if (blocks > 148 * 16) blocks = 148 * 16;
   quantize_rows_kernel<<<(unsigned)blocks, 32 * kQuantWarps, 0, s>>>(static_cast<const bf16*>(src), src_row, offsets,
-                                                                    G, rows_bound, cols, q, sf, sf_plain);
+                                                                    G, rows_bound, cols, tile_rows, q, sf, sf_plain);
   return cudaGetLastError();
 }
 
