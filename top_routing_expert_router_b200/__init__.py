@@ -15,7 +15,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmoe_b200.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m top_routing_expert_router_b200.build` "
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python top_routing_expert_router_b200/build.py` "
                       "(or __graft_entry__.build()); there is no fallback implementation")
 
 _lib = ctypes.CDLL(LIB_PATH)
