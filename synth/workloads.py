@@ -156,6 +156,13 @@ WORKLOADS = {w.name: w for w in [
     _wl("fp8_ragged_small", n=300, d_model=384, n_routed=12, top_k=3, moe_intermediate_size=256, n_shared=1,
         dtype="fp8", renormalize=True),
     _wl("deepseek_v3_decode_small_fp8", n=40, dtype="fp8", **{**_V3, "d_model": 512, "moe_intermediate_size": 256}),
+    # profiling cases of the HBM-bound kernels at DeepSeek-V3 shapes, a few GB on the device:
+    # routing and permutation of 8192 tokens (experts shrunk to I = 128: the router and the
+    # dispatch do not depend on I), and decode with 32 bf16 experts (2.8 GB of weights)
+    _wl("deepseek_v3_route_8k", n=8192, description="DeepSeek-V3 routing and dispatch, small experts (profiling size)",
+        **{**_V3, "moe_intermediate_size": 128}),
+    _wl("deepseek_v3_decode_32e", n=64, description="DeepSeek-V3-shaped decode with 32 experts (profiling size)",
+        **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4}),
     # profiling case: DeepSeek-V3 decode shapes with 32 FP8 experts (1.4 GB of weights)
     _wl("deepseek_v3_decode_fp8_32e", n=64, dtype="fp8",
         **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4},

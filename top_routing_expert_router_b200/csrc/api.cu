@@ -84,13 +84,15 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   const bool fp8 = c.dtype == MOE_FP8;
   const int64_t I = c.moe_intermediate_size, d = c.d_model;
   p.xq = take(fp8 ? (size_t)fr * d : 0);
-  p.sfx = take(fp8 ? (size_t)fp8_sf_tiles_bound(fr, fg) * (d / 128) * 512 : 0);
+  // scale blocks: 512 bytes per row tile and four 128-wide k blocks
+  auto sf_bytes = [](int64_t rows, int32_t G, int64_t k) { return (size_t)fp8_sf_tiles_bound(rows, G) * ceil_div(k / 128, 4) * 512; };
+  p.sfx = take(fp8 ? sf_bytes(fr, fg, d) : 0);
   p.hq = take(fp8 ? (size_t)fr * I : 0);
-  p.sfh = take(fp8 ? (size_t)fp8_sf_tiles_bound(fr, fg) * (I / 128) * 512 : 0);
+  p.sfh = take(fp8 ? sf_bytes(fr, fg, I) : 0);
   p.xsq = take(fp8 && Is > 0 ? (size_t)n * d : 0);
-  p.sfxs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (d / 128) * 512 : 0);
+  p.sfxs = take(fp8 && Is > 0 ? sf_bytes(n, 1, d) : 0);
   p.hsq = take(fp8 && Is > 0 ? (size_t)n * Is : 0);
-  p.sfhs = take(fp8 && Is > 0 ? (size_t)fp8_sf_tiles_bound(n, 1) * (Is / 128) * 512 : 0);
+  p.sfhs = take(fp8 && Is > 0 ? sf_bytes(n, 1, Is) : 0);
   p.ep_off = take(ep ? (size_t)(fg + 1) * 4 : 0);
   p.total = off;
   return p;

@@ -8,16 +8,22 @@
 // computed by tcgen05.mma kind::mxf8f6f4.block_scale (E4M3 x E4M3 -> fp32 in
 // TMEM, the scales applied by the tensor core per 32-wide k sub-block). C is bf16.
 //
+// Scale factors: a 32-bit scale word in TMEM holds four bytes and each MMA
+// selects one of them. One scale covers a whole 128-wide k block, so the word
+// of a row carries the scales of four consecutive k blocks (byte j: block
+// 4q + j), and one copy into TMEM serves the MMAs of four stages.
+//
 // Design (one CTA per SM, persistent, warp-specialised, 192 threads):
-//   warp 0      producer: per 128-k stage TMA copies of the 128 x 128 A tile,
-//               the 128 x 128 B tile (SwiGLU: 64 gate over 64 up rows) and a
-//               512-byte bulk copy of A's scale-factor block (laid out by the
-//               quantiser); the warp writes B's scale words from the block
-//               scale bytes (prefetched per tile) into the stage.
-//   warp 1      TMEM owner and MMA issuer: tcgen05.cp of both scale-factor
-//               blocks into TMEM (32x128b.warpx4: rows p and p+32k of the tile
-//               in lane p, column k), then four MMAs of K = 32 that select the
-//               scale byte of their sub-block; tcgen05.commit frees the stage.
+//   warp 0      producer: per 128-k stage TMA copies of the 128 x 128 A tile and
+//               the 128 x 128 B tile (SwiGLU: 64 gate over 64 up rows); every
+//               fourth stage also a 512-byte bulk copy of A's scale-factor block
+//               (laid out by the quantiser) and B's scale words, which the warp
+//               writes from the block scale bytes (prefetched per tile).
+//   warp 1      TMEM owner and MMA issuer: every fourth stage tcgen05.cp of both
+//               scale-factor blocks into TMEM (32x128b.warpx4: rows p and p+32k
+//               of the tile in lane p, column k), then per stage four MMAs of
+//               K = 32 that select the scale byte of the stage's k block;
+//               tcgen05.commit frees the stage.
 //   warps 2..5  epilogue: tcgen05.ld, SwiGLU in fp32, bf16 stores.
 // Every mbarrier wait is bounded like the bf16 kernels'.
 // Short tiles (groups of a few rows, decode): an m-tile covers 32 rows and a
@@ -56,8 +62,9 @@ struct Shape {
   static constexpr int STAGE_BYTES = (A_STAGE + B_BYTES + SF_BYTES + SFB_BYTES + 1023) / 1024 * 1024;
   static constexpr int STAGES = BMR == 32 ? (BN == 256 ? 5 : 10) : (BN == 256 ? 4 : 6);
   static constexpr uint32_t SF_COL0 = ACC_BUFS * BN;   // scale factors after the accumulators
-  static constexpr uint32_t SF_COLS = 4 + BN / 32;     // per stage: A (128 rows) and B (BN rows)
-  static_assert(SF_COL0 + SF_COLS * STAGES <= TMEM_COLS, "TMEM budget");
+  static constexpr uint32_t SF_COLS = 4 + BN / 32;     // per slot: A (128 rows) and B (BN rows)
+  static constexpr uint32_t SF_SLOTS = 2;              // four k blocks per slot, two slots in turn
+  static_assert(SF_COL0 + SF_COLS * SF_SLOTS <= TMEM_COLS, "TMEM budget");
   static_assert(A_STAGE + B_BYTES >= A_BYTES, "the MMA's 128-row A operand stays inside its stage");
   static_assert(BMR == 128 || BMR == 32, "m-tile heights");
 };
@@ -194,7 +201,7 @@ __device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
 }
 
 // kind::mxf8f6f4 instruction descriptor: E4M3 A and B (format 0), K-major,
-// UE8M0 scales, M = 128, N = BN; scale-factor byte `id` of A and of B.
+// UE8M0 scales, M = 128, N = BN; scale-factor byte `id` of A's and B's words.
 __device__ __forceinline__ uint32_t idesc_fp8(int bn, int id) {
   return ((uint32_t)id << 4) | ((uint32_t)(bn >> 3) << 17) | (1u << 23) | ((uint32_t)(BM >> 4) << 24) |
          ((uint32_t)id << 29);
@@ -332,7 +339,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     int g_hint = 0;
     bool ok = true;
     uint32_t issued = 0;  // stages armed so far (stage s was armed (issued - 1 - s) / STAGES + 1 times)
-    const uint32_t tx = A_STAGE + B_BYTES + SF_BYTES;  // TMA tiles and A's scale block
+    const uint32_t tx_tiles = A_STAGE + B_BYTES;  // TMA tiles; every fourth stage also A's scale block
+    const int nq = (nkb + 3) / 4;                  // scale blocks per row tile (four k blocks each)
     // B scale bytes of a tile: lane l keeps k-blocks l, l + 32, l + 64, l + 96 of the gate (or
     // plain) block, the up block and, for plain 256-wide tiles, the next 128-row block. They are
     // loaded one tile ahead, so a tile's first stage does not wait for them.
@@ -358,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Tile tl = decode<BMR>(ctl, p.G, t, g_hint);
       const int row0 = ctl->row_off[tl.g] + tl.m * BMR;
       const int brow = tl.g * p.b_rows + tl.nt * p.n_out;
-      const uint32_t* sfa_tile = p.sfa + (int64_t)(ctl->sf_off[tl.g] + tl.m) * nkb * 128;
+      const uint32_t* sfa_tile = p.sfa + (int64_t)(ctl->sf_off[tl.g] + tl.m) * nq * 128;
       uint32_t sbg[4], sbu[4], sbn[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
@@ -381,8 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint8_t* sbm = sa + A_STAGE;
         uint8_t* sfa_s = sbm + B_BYTES;
         uint8_t* sfb_s = sfa_s + SF_BYTES;
+        const bool lead = (kb & 3) == 0;  // first stage of four: carries the scale factors
         if (lane == 0) {
-          mbar_expect_tx(&ctl->full[stage], tx);
+          mbar_expect_tx(&ctl->full[stage], tx_tiles + (lead ? SF_BYTES : 0u));
           tma_load_2d(sa, &map_a, &ctl->full[stage], kb * BK, row0);
           if (p.swiglu) {
             tma_load_2d(sbm, &map_b, &ctl->full[stage], kb * BK, brow);
@@ -390,22 +399,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             tma_load_2d(sbm, &map_b, &ctl->full[stage], kb * BK, brow);
           }
-          bulk_load(sfa_s, sfa_tile + (int64_t)kb * 128, SF_BYTES, &ctl->full[stage]);
+          if (lead) bulk_load(sfa_s, sfa_tile + (int64_t)(kb >> 2) * 128, SF_BYTES, &ctl->full[stage]);
         }
-        // B scale words, one 128-row block per 512 bytes: block row p at word 4 (p % 32) + p / 32.
-        // SwiGLU: the first BN/2 tile rows are gate rows, the rest up rows (one scale block each,
-        // as BN/2 <= 128 rows never straddle a 128-row block); plain: one block per 128 rows.
-        const uint32_t bg = __shfl_sync(0xffffffffu, pick4<BMR == 128>(sbg, kb >> 5), kb & 31) * 0x01010101u;
-        const uint32_t bu = __shfl_sync(0xffffffffu, pick4<BMR == 128>(sbu, kb >> 5), kb & 31) * 0x01010101u;
-        if (BN == 128) {
-          const uint32_t w2 = p.swiglu ? bu : bg;
-          *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, w2, w2);
-        } else {  // BN = 256: block 0 holds tile rows 0..127, block 1 rows 128..255
-          const uint32_t w2 = p.swiglu ? bu : __shfl_sync(0xffffffffu, pick4<BMR == 128>(sbn, kb >> 5), kb & 31) * 0x01010101u;
-          *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, bg, bg);
-          *reinterpret_cast<uint4*>(sfb_s + SF_BYTES + 16 * lane) = make_uint4(w2, w2, w2, w2);
+        // B scale words, one 128-row block per 512 bytes: block row p at word 4 (p % 32) + p / 32,
+        // byte j of the word the scale of k block kb + j. SwiGLU: the first BN/2 tile rows are gate
+        // rows, the rest up rows (one scale block each, as BN/2 <= 128 rows never straddle a
+        // 128-row block); plain: one block per 128 rows.
+        if (lead) {
+          auto quad = [&](const uint32_t(&a)[4]) {  // bytes of k blocks kb .. kb + 3 (kb + 3 <= 127)
+            uint32_t w = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const int x = kb + i;
+              w |= (__shfl_sync(0xffffffffu, pick4<BMR == 128>(a, x >> 5), x & 31) & 0xFFu) << (8 * i);
+            }
+            return w;
+          };
+          const uint32_t bg = quad(sbg);
+          const uint32_t bu = quad(sbu);
+          if (BN == 128) {
+            const uint32_t w2 = p.swiglu ? bu : bg;
+            *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, w2, w2);
+          } else {  // BN = 256: block 0 holds tile rows 0..127, block 1 rows 128..255
+            const uint32_t w2 = p.swiglu ? bu : quad(sbn);
+            *reinterpret_cast<uint4*>(sfb_s + 16 * lane) = make_uint4(bg, bg, bg, bg);
+            *reinterpret_cast<uint4*>(sfb_s + SF_BYTES + 16 * lane) = make_uint4(w2, w2, w2, w2);
+          }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         }
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncwarp();
         if (lane == 0) mbar_arrive(&ctl->full[stage]);
         ++issued;
@@ -443,18 +464,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_after();
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint32_t sfa_t = tmem_base + S::SF_COL0 + S::SF_COLS * (uint32_t)stage;
+          const uint32_t sfa_t = tmem_base + S::SF_COL0 + S::SF_COLS * (uint32_t)((kb >> 2) & 1);
           const uint32_t sfb_t = sfa_t + 4u;
-          sf_copy(sfa_t, sf_desc(sa + A_STAGE + B_BYTES));
+          if ((kb & 3) == 0) {  // scale factors of k blocks kb .. kb + 3, copied once
+            sf_copy(sfa_t, sf_desc(sa + A_STAGE + B_BYTES));
 #pragma unroll
-          for (int blk = 0; blk < BN / 128; ++blk)  // B rows 128 blk .. : TMEM columns 4 blk ..
-            sf_copy(sfb_t + 4u * blk, sf_desc(sa + A_STAGE + B_BYTES + SF_BYTES + SF_BYTES * blk));
+            for (int blk = 0; blk < BN / 128; ++blk)  // B rows 128 blk .. : TMEM columns 4 blk ..
+              sf_copy(sfb_t + 4u * blk, sf_desc(sa + A_STAGE + B_BYTES + SF_BYTES + SF_BYTES * blk));
+          }
           const uint64_t adesc = sw128_desc(sa);
           const uint64_t bdesc = sw128_desc(sa + A_STAGE);
 #pragma unroll
           for (int k = 0; k < BK / 32; ++k)  // 32 E4M3 elements = 32 bytes per MMA
-            mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(BN, k), sfa_t, sfb_t,
-                    (kb | k) != 0);
+            mma_fp8(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc_fp8(BN, kb & 3), sfa_t,
+                    sfb_t, (kb | k) != 0);
           issued = true;
           mma_commit(&ctl->empty[stage]);
           if (++stage == STAGES) {

@@ -7,11 +7,11 @@
 //   code_c = E4M3 of v_c * 2^-e, round to nearest even (|v_c * 2^-e| <= 448).
 // The scale of row r, tile t is written where the tensor-core GEMM reads it:
 // GEMM row tiles of TR = 128 (or 32) rows of each group (tile m of group g
-// covers rows offsets[g] + TR m ...), one 512-byte block per (row tile,
-// 128-column tile) in the scale-factor layout of tcgen05.mma block scaling: the
-// 32-bit word of tile row p sits at word 4 (p % 32) + p / 32 and holds the
-// UE8M0 byte four times (one per 32-column sub-block, all equal for 1 x 128
-// tiles).
+// covers rows offsets[g] + TR m ...), one 512-byte block per (row tile, four
+// consecutive 128-column tiles) in the scale-factor layout of tcgen05.mma block
+// scaling: the 32-bit word of tile row p sits at word 4 (p % 32) + p / 32, and
+// its byte j is the UE8M0 byte of column tile 4q + j (the GEMM's MMAs select the
+// byte of their k block).
 #include <cuda_fp8.h>
 
 #include "common.cuh"
@@ -66,6 +66,7 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
   const int64_t rows = row_off[G];
   const int lane = threadIdx.x & 31;
   const int tiles = cols / 128;
+  const int quads = (tiles + 3) / 4;  // scale blocks per row tile
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   for (int64_t r = warp; r < rows; r += nwarps) {
@@ -128,7 +129,8 @@ __global__ void __launch_bounds__(32 * kQuantWarps)
           if (sf_plain)
             sf_plain[r * tiles + t] = (uint8_t)byte;
           else
-            sf[(tile * tiles + t) * 128 + 4 * (p % 32) + p / 32] = byte * 0x01010101u;
+            reinterpret_cast<uint8_t*>(sf)[(((tile * quads + (t >> 2)) * 128) + 4 * (p % 32) + p / 32) * 4 + (t & 3)] =
+                (uint8_t)byte;
         }
       }
     }
