@@ -58,12 +58,6 @@ def _rank_weights(w, dev, q, world):
                             dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
 
 
-def _full_weights(w, dev):
-    if w.dtype == "fp8":
-        return _rank_weights(w, dev, 0, 1)
-    return H.weights_for(dev)
-
-
 def run_ep(w, dev, world, splits, recv_rows=None):
     cfg = H.cfg_for(w)
     x = dev["x"]
@@ -73,7 +67,7 @@ def run_ep(w, dev, world, splits, recv_rows=None):
                 counts=[torch.zeros((world, w.n_routed), dtype=torch.int32, device="cuda") for _ in range(world)])
     group = moe.make_ep_group(recv_rows, **bufs)
     first = np.concatenate([[0], np.cumsum(splits)])
-    ranks, keep = [], []
+    ranks = []
     for q in range(world):
         n = splits[q]
         r = dict(n=n, x=x[first[q]:first[q + 1]], weights=_rank_weights(w, dev, q, world),
@@ -100,7 +94,10 @@ def _oracle(w, host):
 
 CASES = [("mixtral_small", 2), ("mixtral_small", 4), ("mixtral_small", 8), ("deepseek_v2_small", 4),
          ("deepseek_v2_small", 8), ("deepseek_v3_small", 8), ("deepseek_v4_small", 2), ("ragged_small", 1),
-         ("tiny_f32", 2), ("fp8_ragged_small", 2), ("fp8_ragged_small", 4), ("deepseek_v3_small_fp8", 8)]
+         ("tiny_f32", 2), ("fp8_ragged_small", 2), ("fp8_ragged_small", 4), ("deepseek_v3_small_fp8", 8),
+         # FP8 short tiles (received rows average at most 16 per owned expert); the second has
+         # experts with more than 32 rows, so their groups span several short tiles
+         ("deepseek_v3_decode_small_fp8", 8), ("fp8_skewed_small", 1)]
 
 
 @pytest.mark.parametrize("name,world", CASES)
