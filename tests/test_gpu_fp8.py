@@ -76,13 +76,13 @@ def test_quantize_fp8_rejects_bad_shapes():
         moe.moe_quantize_fp8(x, q, s)
 
 
-@pytest.mark.parametrize("bn", ["rule", "128", "256", "s128", "s256"])
+@pytest.mark.parametrize("bn", ["rule", "128", "256", "pair", "s128", "s256"])
 @pytest.mark.parametrize("unit_scales", [False, True])
 @pytest.mark.parametrize("name", FP8_SMALL)
 def test_fp8_expert_ffn_parity(name, unit_scales, bn, monkeypatch):
-    """Every tile shape matches the oracle: the one the rows per expert choose, 128-row tiles forced
-    at both widths (128 x 128 with two accumulators, 128 x 256 with one), and short 32-row tiles at
-    both widths where the rows per expert allow them."""
+    """Every tile shape matches the oracle: the one the rows per expert choose, one-SM 128-row tiles
+    forced at both widths (128 x 128 with two accumulators, 128 x 256 with one), SM-pair 256 x 256
+    tiles, and short 32-row tiles at both widths where the rows per expert allow them."""
     if bn == "rule":
         monkeypatch.delenv("MOE_FP8_BN", raising=False)
     else:

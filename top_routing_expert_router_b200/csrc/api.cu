@@ -21,9 +21,14 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 struct Plan {
   size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
   size_t xq, sfx, hq, sfh, xsq, sfxs, hsq, sfhs;  // FP8 experts: E4M3 activations and their scale blocks
+  size_t sfb, sfbs;  // FP8 SM-pair GEMMs: B scale blocks (routed, shared experts)
   size_t ep_off;  // expert parallelism: receive offsets of the rank's own experts
   size_t total;
 };
+
+// 512-byte scale blocks of the FP8 activations entering a matrix with k columns: one per row tile
+// and four 128-wide k blocks.
+int64_t fp8_sf_blocks(int64_t rows, int32_t G, int64_t k) { return fp8_sf_tiles_bound(rows, G) * ceil_div(k / 128, 4); }
 
 // Element type of the activations (x, y, x_perm, expert_out) and of the router
 // weight: bf16 for the FP8 experts, whose matrices alone are E4M3.
@@ -85,7 +90,7 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   const int64_t I = c.moe_intermediate_size, d = c.d_model;
   p.xq = take(fp8 ? (size_t)fr * d : 0);
   // scale blocks: 512 bytes per row tile and four 128-wide k blocks
-  auto sf_bytes = [](int64_t rows, int32_t G, int64_t k) { return (size_t)fp8_sf_tiles_bound(rows, G) * ceil_div(k / 128, 4) * 512; };
+  auto sf_bytes = [](int64_t rows, int32_t G, int64_t k) { return (size_t)fp8_sf_blocks(rows, G, k) * 512; };
   p.sfx = take(fp8 ? sf_bytes(fr, fg, d) : 0);
   p.hq = take(fp8 ? (size_t)fr * I : 0);
   p.sfh = take(fp8 ? sf_bytes(fr, fg, I) : 0);
@@ -93,6 +98,13 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   p.sfxs = take(fp8 && Is > 0 ? sf_bytes(n, 1, d) : 0);
   p.hsq = take(fp8 && Is > 0 ? (size_t)n * Is : 0);
   p.sfhs = take(fp8 && Is > 0 ? sf_bytes(n, 1, Is) : 0);
+  auto sfb_bytes = [](int32_t G, int64_t I_, int64_t d_) {
+    const int64_t a = fp8_pair_sfb_bytes(G, (int32_t)I_, (int32_t)d_, true);
+    const int64_t b = fp8_pair_sfb_bytes(G, (int32_t)d_, (int32_t)I_, false);
+    return (size_t)(a > b ? a : b);
+  };
+  p.sfb = take(fp8 ? sfb_bytes(fg, I, d) : 0);
+  p.sfbs = take(fp8 && Is > 0 ? sfb_bytes(1, Is, d) : 0);
   p.ep_off = take(ep ? (size_t)(fg + 1) * 4 : 0);
   p.total = off;
   return p;
@@ -286,13 +298,16 @@ moe_status ffn_fp8(const Ctx& x, const void* A, const int32_t* a_rows, const int
   uint32_t* sfh = x.at<uint32_t>(x.p.sfh);
   void* h = x.ws + x.p.h;
   const int32_t tr = fp8_tile_rows(nk, c.n_routed);
+  int32_t* sched = x.at<int32_t>(x.p.sched);
   MOE_CUDA(launch_quantize_rows(A, a_rows, offsets, c.n_routed, nk, (int32_t)d, tr, xq, sfx, x.s));
   GemmFp8Args g1{xq, w->w_gate, w->w_up, sfx, w->w_gate_scale, w->w_up_scale, h, I, offsets, c.n_routed, nk,
-                 (int32_t)I, (int32_t)d, tr};
+                 (int32_t)I, (int32_t)d, tr, sched, fp8_sf_blocks(nk, c.n_routed, d), x.at<uint32_t>(x.p.sfb),
+                 fp8_pair_sfb_bytes(c.n_routed, (int32_t)I, (int32_t)d, true)};
   MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
   MOE_CUDA(launch_quantize_rows(h, nullptr, offsets, c.n_routed, nk, (int32_t)I, tr, hq, sfh, x.s));
   GemmFp8Args g2{hq, w->w_down, nullptr, sfh, w->w_down_scale, nullptr, eo, d, offsets, c.n_routed, nk,
-                 (int32_t)d, (int32_t)I, tr};
+                 (int32_t)d, (int32_t)I, tr, sched + 1, fp8_sf_blocks(nk, c.n_routed, I), x.at<uint32_t>(x.p.sfb),
+                 fp8_pair_sfb_bytes(c.n_routed, (int32_t)d, (int32_t)I, false)};
   MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
   return MOE_OK;
 }
@@ -326,13 +341,16 @@ moe_status shared_impl(const Ctx& x, const void* X, const moe_weights* w, void**
     uint8_t* hq = x.at<uint8_t>(x.p.hsq);
     uint32_t* sfh = x.at<uint32_t>(x.p.sfhs);
     const int32_t tr = fp8_tile_rows(x.n, 1);
+    int32_t* sched = x.at<int32_t>(x.p.sched);
     MOE_CUDA(launch_quantize_rows(X, nullptr, nullptr, 1, x.n, (int32_t)d, tr, xq, sfx, x.s));
     GemmFp8Args g1{xq, w->ws_gate, w->ws_up, sfx, w->ws_gate_scale, w->ws_up_scale, shh, Is, nullptr, 1, x.n,
-                   (int32_t)Is, (int32_t)d, tr};
+                   (int32_t)Is, (int32_t)d, tr, sched + 2, fp8_sf_blocks(x.n, 1, d), x.at<uint32_t>(x.p.sfbs),
+                   fp8_pair_sfb_bytes(1, (int32_t)Is, (int32_t)d, true)};
     MOE_CUDA(launch_gemm_fp8(g1, true, x.status(), x.s));
     MOE_CUDA(launch_quantize_rows(shh, nullptr, nullptr, 1, x.n, (int32_t)Is, tr, hq, sfh, x.s));
     GemmFp8Args g2{hq, w->ws_down, nullptr, sfh, w->ws_down_scale, nullptr, sh, d, nullptr, 1, x.n, (int32_t)d,
-                   (int32_t)Is, tr};
+                   (int32_t)Is, tr, sched + 3, fp8_sf_blocks(x.n, 1, Is), x.at<uint32_t>(x.p.sfbs),
+                   fp8_pair_sfb_bytes(1, (int32_t)d, (int32_t)Is, false)};
     MOE_CUDA(launch_gemm_fp8(g2, false, x.status(), x.s));
     *sh_out = sh;
     return MOE_OK;

@@ -640,16 +640,16 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
 }  // namespace
 
 // Tile choice from the rows per group (M rows in G groups):
-//  - >= 128 rows (prefill): 128 x 256 tiles. At the FP8 MMA rate the L2 -> SM copies bound the
-//    kernel, and 256-wide tiles copy 25 % fewer bytes per MAC, which outweighs the epilogue no
-//    longer overlapping the next tile.
+//  - >= 128 rows (prefill): 256 x 256 tiles on SM pairs (gemm_fp8_pair.cu). At the FP8 MMA rate
+//    the L2 -> SM copies bound the kernel, and a pair copies 32 KB per SM and 128-k stage where a
+//    one-SM 128 x 256 tile copies 48 KB.
 //  - <= 16 rows (decode): short 32-row tiles, 128 wide with two accumulators and 10 stages:
 //    weight streaming at HBM rate needs bytes in flight (160 KB of weights per SM), and a group of
 //    a few rows needs none of a 128-row A tile. (256-wide short tiles, 5 stages, measured 13 %
 //    slower on the DeepSeek-V3 decode layer.)
 //  - otherwise 128 x 128 tiles with two accumulators.
-// MOE_FP8_BN (tuning and tests): 128 | 256 force 128-row tiles of that width; s128 | s256 force
-// the width of short tiles where the rule allows them. The workspace holds scale blocks for the
+// MOE_FP8_BN (tuning and tests): 128 | 256 force one-SM 128-row tiles of that width; pair forces
+// the SM-pair tiles; s128 | s256 force the width of short tiles where the rule allows them. The workspace holds scale blocks for the
 // short tiles whenever the rule could choose them.
 bool fp8_short_rule(int64_t M, int32_t G) { return M <= 16 * (int64_t)G; }
 
@@ -674,7 +674,10 @@ cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status,
   if (a.tile_rows == 32)
     return bn && strcmp(bn, "s256") == 0 ? launch_bn<256, 32>(a, swiglu, status, s)
                                          : launch_bn<128, 32>(a, swiglu, status, s);
-  const bool wide = bn && bn[0] != 's' ? strcmp(bn, "256") == 0 : a.M / (a.offsets ? a.G : 1) >= 128;
+  const bool big = a.M / (a.offsets ? a.G : 1) >= 128;
+  const bool pair_ok = a.tile_counter && a.sfb && a.sfb_bytes >= fp8_pair_sfb_bytes(a.G, a.N, a.K, swiglu);
+  if (bn ? strcmp(bn, "pair") == 0 : big && pair_ok) return launch_gemm_fp8_pair(a, swiglu, status, s);
+  const bool wide = bn && bn[0] != 's' ? strcmp(bn, "256") == 0 : big;
   return wide ? launch_bn<256, 128>(a, swiglu, status, s) : launch_bn<128, 128>(a, swiglu, status, s);
 }
 

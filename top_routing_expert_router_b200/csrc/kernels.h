@@ -53,8 +53,16 @@ struct GemmFp8Args {
   int32_t N;
   int32_t K;
   int32_t tile_rows;      // rows per A tile and scale block: fp8_tile_rows(M, G)
+  int32_t* tile_counter = nullptr;  // SM-pair kernel: device int32 it hands out tiles from
+  int64_t sf_blocks = 0;            // 512-byte scale blocks the sfa buffer holds
+  uint32_t* sfb = nullptr;          // SM-pair kernel: scratch for B's scale blocks
+  int64_t sfb_bytes = 0;            // at least fp8_pair_sfb_bytes(G, N, K, swiglu)
 };
+int64_t fp8_pair_sfb_bytes(int32_t G, int32_t N, int32_t K, bool swiglu);
 cudaError_t launch_gemm_fp8(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s);
+// The SM-pair kernel (cta_group::2, 256 x 256 tiles); launch_gemm_fp8 calls it for groups of at
+// least 128 rows on average.
+cudaError_t launch_gemm_fp8_pair(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaStream_t s);
 // Rows per A tile of the FP8 GEMM (32 for groups of a few rows, else 128); the quantiser lays the
 // scale blocks out for the same tiles.
 int fp8_tile_rows(int64_t M, int32_t G);
