@@ -618,13 +618,10 @@ cudaError_t launch_bn(const GemmFp8Args& a, bool swiglu, moe_diag* status, cudaS
   } else {
     mb2 = mb;
   }
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_fp8_kernel<BN, BMR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem_bytes<BN, BMR>());
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = set_smem_limit(attr, (const void*)gemm_fp8_kernel<BN, BMR>, smem_bytes<BN, BMR>());
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   int sms = 0, dev = 0;
   cudaGetDevice(&dev);

@@ -707,12 +707,10 @@ cudaError_t launch_gemm_fp8_pair(const GemmFp8Args& a, bool swiglu, moe_diag* st
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  static bool attr = false;
-  if (!attr) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_fp8_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = set_smem_limit(attr, (const void*)gemm_fp8_pair_kernel, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(kThreads, 1, 1);

@@ -1046,12 +1046,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   }
   const int64_t n_tiles_all = ceil_div(a.N, p.n_out);
   if (pair) {
-    static bool attr2 = false;
-    if (!attr2) {
-      cudaError_t e =
-          cudaFuncSetAttribute(gemm_tc2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes2);
+    static std::atomic<uint64_t> attr2{0};
+    {
+      const cudaError_t e = set_smem_limit(attr2, (const void*)gemm_tc2_kernel, kSmemBytes2);
       if (e != cudaSuccess) return e;
-      attr2 = true;
     }
     const int64_t max_pair_tiles = (ceil_div(a.M, BM2) + (a.offsets ? a.G : 0)) * n_tiles_all;
     cudaLaunchConfig_t cfg = {};
@@ -1080,11 +1078,10 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
     return cudaLaunchKernelEx(&cfg, gemm_tc2_kernel, ma, ma_half, mb, mb2, p);
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+  static std::atomic<uint64_t> attr1{0};
+  {
+    const cudaError_t e = set_smem_limit(attr1, (const void*)gemm_tc_kernel, kSmemBytes);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   // Upper bound on the tiles: every group may add one partial m-tile.
   const int64_t n_tiles = ceil_div(a.N, p.n_out);

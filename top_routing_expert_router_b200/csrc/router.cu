@@ -934,15 +934,16 @@ cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32
   if (n <= 0) return cudaSuccess;
   const int P = E < kCapPrefix ? E : kCapPrefix;
   const size_t smem = (size_t)kCapThreads * cap_row_words(P) * sizeof(uint32_t);
-  static bool attr = false;
-  if (!attr) {
-    const int bytes = (int)(kCapThreads * cap_row_words(kCapPrefix) * sizeof(uint32_t));
-    for (const void* f : {(const void*)capacity_kernel<1>, (const void*)capacity_kernel<2>, (const void*)capacity_kernel<4>,
-                          (const void*)capacity_kernel<8>, (const void*)capacity_kernel<0>}) {
-      const cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  static std::atomic<uint64_t> attr[5];
+  {
+    const size_t bytes = (size_t)kCapThreads * cap_row_words(kCapPrefix) * sizeof(uint32_t);
+    const void* fs[5] = {(const void*)capacity_kernel<1>, (const void*)capacity_kernel<2>,
+                         (const void*)capacity_kernel<4>, (const void*)capacity_kernel<8>,
+                         (const void*)capacity_kernel<0>};
+    for (int i = 0; i < 5; ++i) {
+      const cudaError_t e = set_smem_limit(attr[i], fs[i], bytes);
       if (e != cudaSuccess) return e;
     }
-    attr = true;
   }
   switch (k) {
     case 1: capacity_kernel<1><<<1, kCapThreads, smem, s>>>(ranking, n, E, k, C, policy, topk_idx, diag); break;
