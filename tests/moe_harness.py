@@ -49,7 +49,7 @@ def rel_err(y: np.ndarray, r: np.ndarray) -> float:
 
     "Max relative error" is undefined where r ~ 0; the floor is the token's own
     output scale (the row rms), so that tokens with small gates (e.g. capacity
-    overflow onto low-probability experts) are judged against their own size.
+    overflow onto low-probability experts) are measured against their own size.
     """
     if not r.size:
         return 0.0
