@@ -36,9 +36,12 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
+
+using namespace ptx;
 
 constexpr int BK = 128;              // k per stage, in E4M3 elements (128 bytes per row)
 constexpr int SF_BYTES = 512;        // one 128-row scale-factor block
@@ -55,7 +58,6 @@ constexpr int kMaxPairGroups = 256;
 constexpr int kTileSlots = 4;
 constexpr int kTileReaders = 10;     // leader MMA + 4 leader epilogue warps + peer producer + 4 peer epilogue warps
 constexpr uint64_t kTimeoutNs = 2000000000ull;
-constexpr uint64_t kDrainNs = 200000000ull;
 static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
 
 struct PairParams {
@@ -92,60 +94,6 @@ struct __align__(8) Ctl {
   int32_t sf_off[kMaxPairGroups + 1];    // first 128-row scale tile of each group
 };
 
-// ---- PTX wrappers -------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
-}
-
-__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
-  return out;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Cluster-scope acquire: for barriers that order data written by the other CTA of the pair.
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait for the phase of `parity`. False on timeout or abort.
 template <bool CLUSTER>
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl, moe_diag* st) {
@@ -162,59 +110,6 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Ctl* ctl,
       }
     }
   }
-}
-
-__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const uint32_t b = smem_u32(bar);
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try(b, parity))
-    if (globaltimer() - t0 > kDrainNs) return;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-
-// Pair copy: lands in this CTA's shared memory, completes bytes on the leader's barrier.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t leader_bar, int32_t c0,
-                                                 int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// K-major operand, 128-byte swizzle (8-row x 128-byte atoms, 1024 B apart).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)1 << 16;
-  d |= (uint64_t)(1024 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Scale-factor block (32 rows x 16 bytes), no swizzle: core matrices 128 bytes apart.
-__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)(128 >> 4) << 16;
-  d |= (uint64_t)(128 >> 4) << 32;
-  d |= (uint64_t)1 << 46;
-  return d;
 }
 
 // kind::mxf8f6f4: E4M3 A and B, K-major, UE8M0 scales, M = 256, N = 256; scale byte `id`.
@@ -246,19 +141,6 @@ __device__ __forceinline__ void commit_pair(uint64_t* bar) {
           smem_u32(bar)),
       "h"(mask)
       : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void store16(bf16* C, int64_t ldc, int64_t row, int col, int N, const float (&v)[16]) {
@@ -312,12 +194,6 @@ __device__ int take_tile(Ctl* ctl, int i, uint32_t rank, const PairParams& p) {
   else
     mbar_arrive_cluster(map_to_rank(&ctl->tile_empty[slot], 0));
   return t;
-}
-
-__device__ __noinline__ void spin_ns(uint64_t ns) {
-  const uint64_t t0 = globaltimer();
-  while (globaltimer() - t0 < ns) {
-  }
 }
 
 // B scale words of every (group, tile, four k blocks) in the layout the GEMM stages: 256 words,
@@ -589,24 +465,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- host side -----------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* q = nullptr;
-    cudaDriverEntryPointQueryResult r;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &q, cudaEnableDefault, &r) == cudaSuccess &&
-        r == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(q);
-  }
-  return fn;
-}
-
 // 2-D byte tensor [rows, cols], box [box_rows, 128], 128-byte swizzle.
 bool make_map_u8(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();

@@ -29,9 +29,12 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
+
+using namespace ptx;
 
 constexpr int BM = 128;
 constexpr int BK = 64;
@@ -45,7 +48,6 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr int kMaxGroupsTc = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;      // 2 s for any single wait
 constexpr uint64_t kTestTimeoutNs = 50000000ull;    // 50 ms under injected stalls
-constexpr uint64_t kDrainNs = 200000000ull;     // 0.2 s per drain wait after an abort
 
 struct TcParams {
   int32_t G;
@@ -84,33 +86,6 @@ struct __align__(8) SmemCtl {
   int32_t tile_off[kMaxGroupsTc + 1];
 };
 
-// ---- PTX wrappers ------------------------------------------------------------------
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait for the phase of `parity` to complete. False on timeout or abort.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SmemCtl* ctl, moe_diag* st) {
   const uint32_t b = smem_u32(bar);
@@ -129,48 +104,8 @@ __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, SmemCtl* 
   }
 }
 
-// Bounded wait used only while draining after an abort.
-__device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
-  const uint32_t b = smem_u32(bar);
-  const uint64_t t0 = globaltimer();
-  while (!mbar_try(b, parity))
-    if (globaltimer() - t0 > kDrainNs) return;
-}
-
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int32_t c0,
-                                            int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::
-          "r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// K-major operand, 128-byte swizzle: 8-row x 128-byte atoms stacked 1024 B apart.
-__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);  // start address
-  d |= (uint64_t)1 << 16;                   // leading byte offset (unused for swizzled K-major)
-  d |= (uint64_t)(1024 >> 4) << 32;         // stride byte offset: next 8-row group
-  d |= (uint64_t)1 << 46;                   // descriptor version (tcgen05)
-  d |= (uint64_t)2 << 61;                   // SWIZZLE_128B
-  return d;
 }
 
 // kind::f16 instruction descriptor: bf16 A and B, fp32 D, both K-major, M = 128.
@@ -190,19 +125,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-      "%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // ---- tile mapping ----------------------------------------------------------------
@@ -383,8 +305,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-          const uint64_t adesc = sw128_kmajor_desc(sa);
-          const uint64_t bdesc = sw128_kmajor_desc(sa + A_BYTES);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)  // advance 16 elements = 32 bytes inside the swizzle atom
             mma_bf16(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, (kb | k) != 0);
@@ -496,37 +418,6 @@ struct __align__(8) SmemCtl2 {
   int32_t tile_off[kMaxGroupsTc + 1];
 };
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
-}
-
-// Shared-cluster address of the same shared-memory offset in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_u32(p)), "r"(rank));
-  return out;
-}
-
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
-
-// Pair copy: lands in this CTA's shared memory, completes bytes on the leader's barrier.
-__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* map, uint32_t leader_bar, int32_t c0,
-                                                 int32_t c1) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-      "[%2];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
-      : "memory");
-}
-
 __device__ __forceinline__ void mma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
@@ -585,19 +476,6 @@ __device__ __noinline__ bool mbar_wait2(uint64_t* bar, uint32_t parity, SmemCtl2
   }
 }
 
-// Cluster-scope acquire: the tile barriers order data written by the other CTA of the pair.
-__device__ __forceinline__ bool mbar_try_cluster(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 __device__ __noinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, SmemCtl2* ctl, moe_diag* st) {
   const uint32_t b = smem_u32(bar);
   if (mbar_try_cluster(b, parity)) return true;
@@ -643,12 +521,6 @@ __device__ int take_tile(SmemCtl2* ctl, int i, uint32_t rank, const TcParams& p)
   else
     mbar_arrive_cluster(map_to_rank(&ctl->tile_empty[slot], 0));
   return t;
-}
-
-__device__ __noinline__ void spin_ns(uint64_t ns) {
-  const uint64_t t0 = globaltimer();
-  while (globaltimer() - t0 < ns) {
-  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -794,8 +666,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t sa = smem_u32(smem + stage * STAGE2_BYTES);
-          const uint64_t adesc = sw128_kmajor_desc(sa);
-          const uint64_t bdesc = sw128_kmajor_desc(sa + A2_BYTES);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + A2_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k)
             mma_bf16_pair(d_tmem, adesc + (uint64_t)(2 * k), bdesc + (uint64_t)(2 * k), idesc, (kb | k) != 0);
@@ -894,24 +766,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---- host side -----------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
 // 2-D bf16 tensor [rows, cols] (cols contiguous), box [box_rows, 64], 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
   EncodeTiledFn fn = encode_fn();
