@@ -88,3 +88,82 @@ def test_status_strings():
     for code in range(7):
         assert moe.moe_status_string(code)
     assert moe.moe_status_string(99) == "unknown status"
+
+
+# ---------------------------------------------------------------- expert parallelism (host checks)
+
+
+def _mixtral_like(**kw):
+    base = dict(d_model=4096, n_routed=8, top_k=2, moe_intermediate_size=14336, renormalize=True)
+    base.update(kw)
+    return moe.make_config(**base)
+
+
+def test_ep_workspace_size_checks_the_group():
+    cfg = _mixtral_like()
+    one = moe.moe_ep_workspace_size(cfg, 1, 64, 128)
+    eight = moe.moe_ep_workspace_size(cfg, 8, 64, 128)
+    assert one > 0 and eight > 0
+    # more receive rows need more h for the owned experts
+    assert moe.moe_ep_workspace_size(cfg, 2, 64, 4096) > moe.moe_ep_workspace_size(cfg, 2, 64, 128)
+    for world, recv, code in [(3, 128, moe.MOE_ERR_INVALID_ARG),     # 8 experts over 3 ranks
+                              (16, 128, moe.MOE_ERR_UNSUPPORTED),    # above MOE_EP_MAX_RANKS
+                              (0, 128, moe.MOE_ERR_INVALID_ARG),
+                              (2, 0, moe.MOE_ERR_INVALID_ARG)]:      # no receive rows
+        with pytest.raises(moe.MoeError) as e:
+            moe.moe_ep_workspace_size(cfg, world, 64, recv)
+        assert e.value.status == code
+
+
+def test_ep_recv_rows_bound():
+    cfg = _mixtral_like()
+    # a token holds at most min(k, E / world) of one owner's experts
+    assert moe.moe_ep_recv_rows_bound(cfg, 2, [100, 50]) == 150 * 2
+    assert moe.moe_ep_recv_rows_bound(cfg, 8, [100, 50]) == 150 * 1
+    assert moe.moe_ep_recv_rows_bound(cfg, 4, [0, 0]) == 1
+
+
+def _group(world, recv_rows=128, flags=True):
+    addr = lambda q, base: base + 4096 * q  # 16-byte aligned stand-in addresses, never dereferenced
+    return moe.make_ep_group(recv_rows, [addr(q, 1 << 20) for q in range(world)],
+                             [addr(q, 2 << 20) for q in range(world)], [addr(q, 3 << 20) for q in range(world)],
+                             [addr(q, 4 << 20) for q in range(world)] if flags else None)
+
+
+def test_ep_layer_forward_rejects_bad_groups_before_any_launch():
+    lib = moe.lib_handle()
+    cfg = _mixtral_like()
+    cap = _mixtral_like(cap_policy="drop", capacity_factor=1.0)
+    rank = (moe.moe_ep_rank * 2)()
+    call = lambda c, g, first, num: lib.moe_ep_layer_forward(ctypes.byref(c), ctypes.byref(g), first, num, rank, None)
+    assert call(cap, _group(2), 0, 2) == moe.MOE_ERR_UNSUPPORTED         # capacity under expert parallelism
+    assert call(cfg, _group(2), 0, 3) == moe.MOE_ERR_INVALID_ARG        # more ranks than the group
+    assert call(cfg, _group(2), 1, 2) == moe.MOE_ERR_INVALID_ARG        # range past the group
+    assert call(cfg, _group(2, flags=False), 0, 1) == moe.MOE_ERR_INVALID_ARG  # one rank needs flag words
+    assert call(cfg, _group(2, recv_rows=0), 0, 2) == moe.MOE_ERR_INVALID_ARG
+    g = _group(2)
+    g.recv_x[1] = (1 << 20) + 4                                          # misaligned receive buffer
+    assert call(cfg, g, 0, 2) == moe.MOE_ERR_INVALID_ARG
+    g = _group(2)
+    g.world = 9
+    assert call(cfg, g, 0, 1) == moe.MOE_ERR_UNSUPPORTED
+    assert lib.moe_ep_layer_forward(ctypes.byref(cfg), None, 0, 1, rank, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_ep_group_marshalling():
+    g = _group(3, recv_rows=77)
+    assert g.world == 3 and g.recv_rows == 77
+    assert [g.recv_x[q] for q in range(3)] == [(1 << 20) + 4096 * q for q in range(3)]
+    assert g.flags[2] == (4 << 20) + 8192 and g.recv_x[3] is None
+    with pytest.raises(ValueError):
+        moe.make_ep_group(1, [1] * 9, [1] * 9, [1] * 9)
+
+
+def test_ep_handles_reject_bad_arguments():
+    lib = moe.lib_handle()
+    out = ctypes.c_void_p()
+    assert lib.moe_ep_export_handle(None, None) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_open_handle(None, ctypes.byref(out)) == moe.MOE_ERR_INVALID_ARG
+    assert lib.moe_ep_close_handle(None) == moe.MOE_ERR_INVALID_ARG
+    with pytest.raises(ValueError):
+        moe.moe_ep_open_handle(b"short")
