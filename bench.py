@@ -101,7 +101,7 @@ def _sources_sha():
     """Hash of the sources of the dominant kernel (the tensor-core grouped GEMM)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "top_routing_expert_router_b200", "csrc")
-    for fn in ("gemm_tc.cu", "common.cuh"):
+    for fn in ("gemm_tc.cu", "ptx.cuh", "common.cuh"):
         with open(os.path.join(csrc, fn), "rb") as f:
             h.update(fn.encode() + f.read())
     return h.hexdigest()[:16]
