@@ -66,6 +66,16 @@
  *     selection score (logit for softmax, score + bias for sigmoid); equal
  *     scores go to the lower expert index, equal group scores to the lower
  *     group index. Dropped slots carry index -1, weight 0 and slot_dest -1.
+ *   - Environment variables, read at each call (none is needed):
+ *     MOE_TC_MODE=1sm|2sm forces the one-SM or SM-pair bf16 expert GEMM;
+ *     MOE_FP8_BN=128|256|pair|s128|s256 forces an FP8 expert GEMM tile shape
+ *     (one-SM 128-row tiles of that width, SM-pair tiles, or 32-row tiles where
+ *     the rows per expert allow them); these exist for tuning and tests, and
+ *     results are identical up to floating-point summation order.
+ *     MOE_EP_TIMEOUT_MS bounds the expert-parallel barrier wait (see below).
+ *     MOE_TEST_STALL=1 withholds one pipeline stage of the bf16 expert GEMM so
+ *     that its bounded wait runs out and MOE_ERR_TIMEOUT is reported (a test of
+ *     the failure path; never set it otherwise).
  */
 #ifndef MOE_H_
 #define MOE_H_
