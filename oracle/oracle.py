@@ -354,19 +354,26 @@ def dequant_blocks(codes: np.ndarray, scale_bytes: np.ndarray) -> np.ndarray:
 
 
 def round_to_bf16(a64: np.ndarray) -> np.ndarray:
-    """binary64 -> binary32 -> bf16 (each round to nearest even), widened back to binary64: the
-    precision in which the kernel holds h when it quantises it."""
-    u = a64.astype(np.float32).view(np.uint32).astype(np.uint64)
-    u = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
-    return u.astype(np.uint32).view(np.float32).astype(np.float64)
+    """binary64 -> bf16, one rounding to nearest with ties to even, widened back to binary64.
+
+    bf16 keeps 8 significant bits with binary32's exponent range, so a value in [2^(e-1), 2^e)
+    lands on the grid 2^(e-8); below the smallest normal (2^-126) the grid stays 2^-133
+    (subnormals). Magnitudes that round past the largest finite bf16 become infinite."""
+    a64 = np.asarray(a64, np.float64)
+    _, e = np.frexp(a64)
+    q = np.ldexp(1.0, np.maximum(e, -125) - 8)
+    r = np.rint(a64 / q) * q  # the division and product are exact (powers of two); rint ties to even
+    big = np.abs(r) >= 2.0 ** 128
+    return np.where(big, np.copysign(np.inf, a64), r)
 
 
 def swiglu_fp8(x64: np.ndarray, wg, wu, wd) -> np.ndarray:
     """One FP8 expert on rows x64 [m, d]: quantise x, gate/up with dequantised weights, SwiGLU,
-    quantise h, down. wg/wu/wd are (codes, scale bytes) pairs. The E4M3 codes of h are decided on
-    h held in bf16, the precision the kernel stores it in between the two expert matrices (an E4M3
-    step is 2^4 bf16 steps, so deciding the codes from binary64 h instead moves about 1 in 64
-    codes by one E4M3 step)."""
+    quantise h, down. wg/wu/wd are (codes, scale bytes) pairs. h is an activation of the layer,
+    held in the layer's activation type (bf16, like x and y) when it enters the down matrix, so
+    its E4M3 codes are decided on h rounded once from binary64 to bf16 (an E4M3 step is 2^4 bf16
+    steps, so deciding the codes from binary64 h instead moves about 1 in 64 codes by one E4M3
+    step)."""
     xq, xs = quantize_rows(x64)
     xd = dequant_rows(xq, xs)
     g = xd @ dequant_blocks(*wg).T

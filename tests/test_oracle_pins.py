@@ -607,11 +607,64 @@ def test_fp8_layer_close_to_unquantised_layer():
     assert 1e-4 < err < 0.05, err
 
 
-def test_round_to_bf16_matches_torch():
+def test_round_to_bf16_matches_torch_on_binary32_values():
+    """On values that binary32 holds exactly, one rounding to bf16 is torch's binary32 -> bf16 cast."""
     rng = np.random.default_rng(5)
-    a = np.concatenate([rng.normal(0, 1, 5000) * rng.lognormal(0, 4, 5000), [0.0, -0.0, 1.0, 3.0 / 7.0]])
+    a = np.concatenate([rng.normal(0, 1, 5000) * rng.lognormal(0, 4, 5000), [0.0, -0.0, 1.0, 3.0 / 7.0,
+                        2.0 ** -130, -3 * 2.0 ** -133, 2.0 ** 127 * 1.5]])
+    a = a.astype(np.float32).astype(np.float64)
     ref = torch.from_numpy(a.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
     np.testing.assert_array_equal(O.round_to_bf16(a), ref)
+
+
+def test_round_to_bf16_rounds_once_from_binary64():
+    """Ties go to the even neighbour; a value a hair above a tie (2^-30 relative, below binary32's
+    resolution) rounds up, which a rounding through binary32 would get wrong; the grid at
+    [64, 128) is 1/2."""
+    v = np.array([68.25, 68.75, 68.25 + 2.0 ** -24, 68.25 - 2.0 ** -24, -68.25 - 2.0 ** -24, 1.0 + 2.0 ** -8,
+                  1.0 + 3 * 2.0 ** -8, 2.0 ** -126 * (1 + 2.0 ** -8)])
+    want = np.array([68.0, 69.0, 68.5, 68.0, -68.5, 1.0, 1.0 + 2.0 ** -6, 2.0 ** -126])
+    np.testing.assert_array_equal(O.round_to_bf16(v), want)
+    via32 = torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16).to(torch.float64).numpy()
+    assert via32[2] == 68.0  # the double rounding that the one-step rounding avoids
+
+
+def test_swiglu_fp8_hidden_step_on_constructed_boundaries():
+    """The h step of the FP8 expert, exactly: x has four unit entries (quantised exactly), gate rows
+    give g = 64 (silu(64) = 64 in binary64), up rows give u as a sum of four E4M3 values in three
+    k-blocks (the last with scale 2^-21), so h = 64 u is known exactly; W_down is the identity on the
+    first 128 outputs, so the layer returns the dequantised E4M3 codes of h. Expected values by hand:
+    448 sets the tile's scale to 2^0; 68.25 + 2^-24 -> bf16 68.5 -> E4M3 72; 68.25 -> bf16 68 (tie to
+    even) -> E4M3 64 (tie to even; the binary64 value would give 72); 69 -> 72; 67.75 -> bf16 68 ->
+    E4M3 64; 76 -> E4M3 80 (tie to even)."""
+    d, I = 384, 128
+    enc = np.vectorize(O.e4m3_encode, otypes=[np.uint8])
+    x = np.zeros((1, d))
+    x[0, [0, 1, 128, 256]] = 1.0
+    wg = np.zeros((I, d))
+    wg[:, 0] = 64.0
+    u_terms = {0: (7.0, 0, 0, 0),
+               1: (1.0, 2.0 ** -4, 2.0 ** -8, 2.0 ** -30),
+               2: (1.0, 2.0 ** -4, 2.0 ** -8, 0),
+               3: (1.0, 2.0 ** -4, 2.0 ** -6, 0),
+               4: (1.0, 2.0 ** -4, -(2.0 ** -8), 0),
+               5: (1.0, 0.1875, 0, 0)}
+    wu = np.zeros((I, d))
+    for i, (a, b, c, e) in u_terms.items():
+        wu[i, 0], wu[i, 1], wu[i, 128], wu[i, 256] = a, b, c, e
+    sc_u = np.array([[127, 127, 127 - 21]], np.uint8)
+    codes_u = np.zeros((I, d), np.uint8)
+    for blk in range(3):
+        cols = slice(128 * blk, 128 * (blk + 1))
+        codes_u[:, cols] = enc(wu[:, cols] * 2.0 ** -(int(sc_u[0, blk]) - 127))
+    np.testing.assert_array_equal(O.dequant_blocks(codes_u, sc_u), wu)  # the constructed u terms are exact
+    wd = np.zeros((d, I))
+    wd[np.arange(I), np.arange(I)] = 1.0
+    ones = lambda r, c: np.full((r, c), 127, np.uint8)
+    out = O.swiglu_fp8(x, (enc(wg), ones(1, 3)), (codes_u, sc_u), (enc(wd), ones(3, 1)))
+    want = np.zeros((1, d))
+    want[0, :6] = [448.0, 72.0, 64.0, 72.0, 64.0, 80.0]
+    np.testing.assert_array_equal(out, want)
 
 
 # ---------------------------------------------------------------- expert parallelism: receive layout
