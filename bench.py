@@ -4,18 +4,25 @@ python bench.py --gpus N --steps K --warmup W [--impl ours|reference] [--workloa
 
 A step is one moe_layer_forward (route + permute + SwiGLU experts + shared
 experts + combine) over one batch of synthetic tokens whose inputs are already
-resident in HBM. The default workload is the Mixtral-8x7B-shaped layer
-(n = 4096 tokens, d = 4096, 8 experts, top-2, I = 14336, bf16). Ranks are
+resident in HBM. The default workload is the DeepSeek-V3-shaped prefill layer
+(n = 16384 tokens, d = 7168, 256 routed experts + 1 shared, sigmoid scores with
+a selection bias, 8 groups of 32 keep 4, top-8, I = 2048, bf16), the largest
+of the layer shapes that fits one GPU. Ranks are
 independent replicas (weak scaling, no collective on the data path); the time
 is the maximum over ranks of the CUDA-event time of K steps.
 
 The reference arm (--impl reference) times the fp64 CPU oracle on the host
 cores on a bounded token sample of the same workload.
 
+--gpus N run as a plain command starts N ranks itself (torch.distributed.run,
+one process per GPU); launched by torch.distributed.run it is one of them.
+
 --ep R times the expert-parallel layer (moe_ep_layer_forward) of a group of R
-ranks emulated on one GPU: the workload's tokens split evenly over the ranks,
-rank q owning experts [q E/R, (q+1) E/R), every rank's exchange buffers in this
-GPU's memory and the steps of all ranks in stream order.
+ranks: the workload's tokens split evenly over the ranks, rank q owning experts
+[q E/R, (q+1) E/R). With --gpus R (one process per GPU) the ranks exchange rows
+over CUDA IPC peer mappings with flag barriers between the steps; as a single
+process the group is emulated on one GPU, every rank's exchange buffers in its
+memory and the steps of all ranks in stream order.
 """
 from __future__ import annotations
 
@@ -340,7 +347,7 @@ def run_ours(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
+        out["cpu_baseline"] = cpu_baseline(w, args.cpu_sample or default_cpu_sample(w))
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -353,6 +360,17 @@ NVLINK_GBS = 770.0  # measured peer copy per direction per GPU on this kind of n
 
 def _split(n, world):
     return [n // world + (1 if q < n % world else 0) for q in range(world)]
+
+
+def ep_group_plan(n, E, k, world, rank):
+    """One rank of an expert-parallel group over a batch of n tokens: its token slice, the experts it
+    owns and the receive-buffer rows every rank allocates (a token holds at most min(k, E / world) of
+    one owner's experts)."""
+    splits = _split(n, world)
+    first = sum(splits[:rank])
+    Eq = E // world
+    return dict(tokens=(first, first + splits[rank]), experts=(rank * Eq, (rank + 1) * Eq),
+                recv_rows=max(1, n * min(k, Eq)), splits=splits)
 
 
 def _ep_rank_weights(moe, w, dev, q, world):
@@ -525,16 +543,172 @@ def run_ep(args):
     print(json.dumps(out), flush=True)
 
 
-def _oracle_inputs(w, tokens):
-    """Host inputs of the oracle's sample: the first `tokens` rows of x and all weights."""
+def _expert_bytes(w):
+    """Bytes of one routed expert's three matrices in the workload's dtype."""
+    per = 1 if w.dtype == "fp8" else (4 if w.dtype == "f32" else 2)
+    return 3 * w.d_model * w.moe_intermediate_size * per
+
+
+def default_cpu_sample(w):
+    """Tokens in the oracle's timed sample: 16, fewer where the experts that many tokens reach would
+    need more than about 4 GB of host weights (the sample's experts are generated on the host)."""
+    if w.n_routed * _expert_bytes(w) <= 4e9:
+        return min(16, w.n)
+    return max(1, min(16, w.n, int(4e9 // (w.top_k * _expert_bytes(w)))))
+
+
+def run_ep_dist(args):
+    """Expert parallelism with one process per GPU (launched by torch.distributed.run, WORLD_SIZE = R):
+    rank q owns experts [q E/R, (q+1) E/R) and routes its slice of the batch; the exchange buffers are
+    mapped between the processes with CUDA IPC records exchanged through the process group, and the
+    library's flag barriers (bounded waits) separate the steps of each layer call."""
+    from datetime import timedelta
+
+    import torch
+    import torch.distributed as dist
+
+    import top_routing_expert_router_b200 as moe
     from synth import workloads as W
 
-    mats = ["w_gate", "w_up", "w_down"] + (["ws_gate", "ws_up", "ws_down"] if w.n_shared else [])
+    world, rank, local = _dist()
+    if world != args.ep:
+        raise SystemExit(f"--ep {args.ep} with {world} processes: launch one process per rank")
+    if torch.cuda.device_count() <= local:
+        raise SystemExit("one GPU per rank: ranks that wait on one another must not share a GPU")
+    torch.cuda.set_device(local)
+    dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    w = W.get(args.workload)
+    dev = W.device_inputs(w, device=f"cuda:{local}")  # seed 0 on every rank: one batch, split below
+    cfg = moe.make_config(dtype=w.dtype, **w.cfg_fields())
+    plan = ep_group_plan(w.n, w.n_routed, w.top_k, world, rank)
+    t0, t1 = plan["tokens"]
+    n_mine, d, R = t1 - t0, w.d_model, world
+    recv_rows = plan["recv_rows"]
+    x = dev["x"][t0:t1]
+    local_bufs = dict(recv_x=torch.empty((recv_rows, d), dtype=x.dtype, device="cuda"),
+                      recv_out=torch.empty((recv_rows, d), dtype=x.dtype, device="cuda"),
+                      counts=torch.zeros((R, w.n_routed), dtype=torch.int32, device="cuda"),
+                      flags=torch.zeros(R + 1, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+
+    def gather(obj):
+        out = [None] * world
+        dist.all_gather_object(out, obj)
+        return out
+
+    peers = moe.ep_open_peers(local_bufs, rank, world, gather)
+    group = moe.make_ep_group(recv_rows, peers["recv_x"], peers["recv_out"], peers["counts"], peers["flags"])
+    y = torch.empty_like(x)
+    mine = dict(n=n_mine, x=x, y=y, weights=_ep_rank_weights(moe, w, dev, rank, R),
+                ws=torch.empty(moe.moe_ep_workspace_size(cfg, R, n_mine, recv_rows), dtype=torch.uint8,
+                               device="cuda"))
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+
+    def step(xin=None, yout=None):
+        r = mine if xin is None else dict(mine, x=xin, y=yout)
+        moe.moe_ep_layer_forward(cfg, group, rank, [r], stream=s)
+
+    try:
+        for _ in range(args.warmup):
+            step()
+        st = moe.moe_sync_status(mine["ws"], s)
+        if st != moe.MOE_OK:
+            raise RuntimeError(f"rank {rank}: device status after warm-up: {moe.moe_status_string(st)}")
+        # the split layer computes what the single-device layer computes on this rank's tokens
+        full_w = _ep_rank_weights(moe, w, dev, 0, 1)
+        ref = torch.empty_like(y)
+        ws1 = torch.empty(moe.moe_workspace_size(cfg, n_mine), dtype=torch.uint8, device="cuda")
+        moe.moe_layer_forward(cfg, n_mine, x, full_w, ref, ws1, stream=s)
+        torch.cuda.synchronize()
+        same = bool(torch.equal(ref.view(torch.int16), y.view(torch.int16)))
+        del ws1, ref
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        with ClockSampler(phys[local] if len(phys) > local and phys[local] != "" else str(local)) as clk:
+            dist.barrier()
+            torch.cuda.synchronize()
+            ev0.record(stream)
+            for _ in range(args.steps):
+                step()
+            ev1.record(stream)
+            torch.cuda.synchronize()
+            dist.barrier()
+        ms_total = reduce_max(ev0.elapsed_time(ev1), world, "cuda")
+        clocks = clk.summary()
+        st = moe.moe_sync_status(mine["ws"], s)
+        # end to end: this rank's token rows in from pinned host memory, its outputs back
+        x_host = x.cpu().pin_memory()
+        y_host = torch.empty_like(y, device="cpu").pin_memory()
+        xd, yd = torch.empty_like(x), torch.empty_like(y)
+        e2e_steps = max(3, min(args.steps, 10))
+        dist.barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(e2e_steps):
+            xd.copy_(x_host, non_blocking=True)
+            step(xd, yd)
+            y_host.copy_(yd, non_blocking=True)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(ev0.elapsed_time(ev1) / e2e_steps, world, "cuda")
+        ok_all = gather(dict(rank=rank, status=int(st), same=same))
+    finally:
+        torch.cuda.synchronize()
+        dist.barrier()
+        for name, addrs in peers.items():
+            for q, a in enumerate(addrs):
+                if q != rank:
+                    moe.moe_ep_close_handle(a)
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        bpe = x.element_size()
+        out = {
+            "metric": METRIC, "value": w.n * args.steps / (ms_total / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+            "higher_is_better": True, "scaling": "strong", "vs_baseline": None,
+            "dtype": "e4m3 x e4m3 -> f32 (bf16 activations)" if w.dtype == "fp8" else w.dtype,
+            "data": "synthetic (seeded counter-based generator; Irwin-Hall normals)",
+            "config": {"workload": w.name, "n_tokens": w.n, "tokens_per_rank": plan["splits"],
+                       "parallelism": f"ep{world}, one process per GPU (CUDA IPC peer buffers, flag barriers)",
+                       "recv_rows": recv_rows, "l2": "inputs larger than L2: every expert's weights streamed per step"},
+            "ranks": ok_all,
+            "e2e": {"value": w.n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": w.n * d * bpe,
+                    "d2h_bytes_per_step": w.n * d * bpe, "ms_per_step": e2e_ms},
+            "gpu_launches": ep_launches_per_rank(w) * world * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(out), flush=True)
+
+
+def _oracle_inputs(w, tokens):
+    """Host inputs of the oracle's sample: the first `tokens` rows of x, the router, the shared
+    experts, and the routed experts those tokens reach. The other routed experts' matrices are
+    zero-filled arrays the oracle never reads (their pages are never touched), so the sample of a
+    256-expert layer does not hold every expert in host memory."""
+    import numpy as np
+
+    from oracle import oracle as O
+    from synth import workloads as W
+
+    specs = w.tensor_specs()
+    small = ["w_r"] + (["bias"] if w.bias_range else [])
+    shared = ["ws_gate", "ws_up", "ws_down"] if w.n_shared else []
+    routed = ["w_gate", "w_up", "w_down"]
     if w.dtype == "fp8":
-        mats = [m + suffix for m in mats for suffix in ("_q", "_s")]
-    names = ["w_r"] + mats + (["bias"] if w.bias_range else [])
-    inp = W.host_inputs(w, names=names)
+        shared = [m + sfx for m in shared for sfx in ("_q", "_s")]
+        routed = [m + sfx for m in routed for sfx in ("_q", "_s")]
+    inp = W.host_inputs(w, names=small + shared)
     inp["x"] = W.host_rows(w, "x", range(tokens))
+    idx, _, _, _ = O.route_capacity(O.Cfg(**w.cfg_fields()), O.router_logits(inp["x"], inp["w_r"]), inp.get("bias"))
+    used = sorted({int(e) for e in idx.ravel() if e >= 0})
+    for nm in routed:
+        shape, dt = specs[nm][0], specs[nm][5]
+        a = np.zeros(shape, {"u8": np.uint8, "f32": np.float32}.get(dt, np.uint16))
+        if used:
+            a[used] = W.host_rows(w, nm, used)
+        inp[nm] = a
     return inp
 
 
@@ -600,20 +774,44 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mixtral_8x7b")
-    ap.add_argument("--cpu-sample", type=int, default=16, help="tokens in the oracle's timed sample")
+    ap.add_argument("--workload", default="deepseek_v3_prefill")
+    ap.add_argument("--cpu-sample", type=int, default=0,
+                    help="tokens in the oracle's timed sample (0: 16, fewer for layers whose sampled experts "
+                         "would need more than about 4 GB of host weights)")
     ap.add_argument("--ref-sample", type=int, default=1, help="tokens per step of the reference (oracle) arm")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--ep", type=int, default=0, help="expert-parallel group of this many ranks, emulated on one GPU")
+    ap.add_argument("--timeout", type=int, default=900, help="limit (s) of a self-launched multi-rank run")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("at least 3 warm-up steps")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args.gpus, args.timeout))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         run_reference(args)
+    elif args.ep > 1 and world > 1:
+        run_ep_dist(args)
     elif args.ep > 1:
         run_ep(args)
     else:
         run_ours(args)
+
+
+def launch_ranks(n, limit_s, script=None, argv=None):
+    """Run `script argv` (default: this command) as n ranks, one process per GPU, under
+    torch.distributed.run on this node (rendezvous on 127.0.0.1); returns its exit status.
+    `timeout -k 60` bounds the whole run."""
+    import socket
+
+    sock = socket.socket()
+    sock.bind(("127.0.0.1", 0))
+    port = sock.getsockname()[1]
+    sock.close()
+    cmd = ["timeout", "-k", "60", str(limit_s), sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+           script or os.path.abspath(__file__), *(sys.argv[1:] if argv is None else argv)]
+    return subprocess.call(cmd)
 
 
 if __name__ == "__main__":

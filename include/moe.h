@@ -76,6 +76,12 @@
  *     MOE_TEST_STALL=1 withholds one pipeline stage of the bf16 expert GEMM so
  *     that its bounded wait runs out and MOE_ERR_TIMEOUT is reported (a test of
  *     the failure path; never set it otherwise).
+ *     MOE_TEST_NO_TENSOR_MAPS=1 makes the bf16 tensor-core GEMMs report every
+ *     shape as unsupported (a test of that path; never set it otherwise).
+ *   - bf16 matrix products run on the tcgen05 tensor cores only: a shape or
+ *     pointer alignment they cannot take (or a missing tensor-map entry point
+ *     in the driver) is MOE_ERR_UNSUPPORTED, never a slower fallback. binary32
+ *     layers run on the CUDA cores (FFMA), the precision their tolerance needs.
  */
 #ifndef MOE_H_
 #define MOE_H_
@@ -267,15 +273,22 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* 
  * serving engine whose memory planner owns every device allocation, or code on
  * a latency-critical path where a cudaMalloc would synchronise the device. They
  * cannot provide a workspace, so this variant keeps the router's scratch (the
- * binary32 logits, the capacity ranking, per-block counts and the status word)
- * in one array of MOE_STATIC_SCRATCH_BYTES in device memory that is part of
- * this library: every GPU that loads the library holds that array until the
- * process exits. It calls no cudaMalloc, cudaFree or allocating routine.
- *   Arguments and outputs are those of moe_route, without ws/ws_bytes.
+ * binary32 logits, the capacity ranking, per-block counts, the count scan and
+ * the status word) in one array of MOE_STATIC_SCRATCH_BYTES in device memory
+ * that is part of this library. It calls no cudaMalloc, cudaFree or
+ * allocating routine. The array lives in the library's device code, which the
+ * CUDA runtime loads on a device when it is first needed there (lazy module
+ * loading): the first call on each device loads it and reserves its 8 MiB on
+ * that device, which then holds it until the process exits; later calls
+ * reserve nothing.
+ *   Arguments and outputs are those of moe_route, without ws/ws_bytes; diag
+ *   is required here (see below). `stream` must belong to the current device.
  *   Returns MOE_ERR_WORKSPACE when this cfg and n need more scratch than the
- *   array holds (E * 4 bytes of logits per token dominate; e.g. E = 256 fits
- *   about 7000 tokens, E = 8 about 200000), MOE_ERR_CUDA if the array's device
- *   address cannot be found, and the errors of moe_route otherwise.
+ *   array holds (E * 4 bytes of logits per token dominate, plus E * 2 bytes of
+ *   ranking under a capacity; e.g. E = 256 fits about 8000 tokens, E = 8 about
+ *   200000), MOE_ERR_INVALID_ARG for a NULL diag or a stream of another device,
+ *   MOE_ERR_CUDA if the array's device address cannot be found, and the errors
+ *   of moe_route otherwise.
  *   The first call on each device performs a one-time set-up that looks up the
  *   array's device address with that device current; make this first call
  *   before any stream capture begins.
@@ -284,8 +297,8 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* 
  *   Calls that overlap on the GPU, e.g. on two streams at once, race on it and
  *   produce undefined results; order them on one stream. The status word that
  *   moe_sync_status reads lives in the array, so that call does not apply here:
- *   when diag is given, the call copies its device status word (a moe_status
- *   value, 0 = MOE_OK) into diag->status on `stream`.
+ *   the call copies its device status word (a moe_status value, 0 = MOE_OK)
+ *   into diag->status on `stream`.
  */
 moe_status moe_route_static_scratch(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
                                     int32_t* topk_idx, float* topk_w, int32_t* expert_counts, moe_diag* diag,

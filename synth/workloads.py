@@ -46,6 +46,7 @@ class Workload:
     bias_range: tuple | None = None
     zipf_s: float = 0.0
     ternary: bool = False
+    router_scale: float = 1.0  # multiplies the router weights' standard deviation (logit stress cases)
     description: str = ""
 
     @property
@@ -69,7 +70,7 @@ class Workload:
         kind_x = synth.TERNARY if self.ternary else synth.NORMAL
         specs = {
             "x": ((self.n, d), synth.STREAM["x"], kind_x, 1.0, 0.0, dt),
-            "w_r": ((E, d), synth.STREAM["w_r"], kind_x, 1.0 / math.sqrt(d), 0.0, dt),
+            "w_r": ((E, d), synth.STREAM["w_r"], kind_x, self.router_scale / math.sqrt(d), 0.0, dt),
             "w_gate": ((E, I, d), synth.STREAM["w_gate"], synth.NORMAL, 1.0 / math.sqrt(d), 0.0, dt),
             "w_up": ((E, I, d), synth.STREAM["w_up"], synth.NORMAL, 1.0 / math.sqrt(d), 0.0, dt),
             "w_down": ((E, d, I), synth.STREAM["w_down"], synth.NORMAL, 1.0 / math.sqrt(I), 0.0, dt),
@@ -174,6 +175,12 @@ WORKLOADS = {w.name: w for w in [
         description="DeepSeek-V3-shaped decode with 32 FP8 experts (profiling size)"),
     _wl("fp8_skewed_small", n=200, d_model=256, n_routed=16, top_k=1, moe_intermediate_size=128, zipf_s=1.2,
         dtype="fp8"),
+    # router stress cases at d = 7168 (routing only): logits 8x (sigmoid, V3 groups) and 4x (softmax,
+    # no groups) the recipe's scale, so the binary32 logit errors are as large as they get here
+    _wl("deepseek_v3_route_x8", n=16384, router_scale=8.0,
+        description="DeepSeek-V3 routing with router weights 8x the recipe's scale", **_V3),
+    _wl("softmax_7168_route_x4", n=16384, d_model=7168, n_routed=256, top_k=8, moe_intermediate_size=128,
+        router_scale=4.0, description="softmax top-8 of 256 experts at d = 7168, router weights 4x the recipe's scale"),
     _wl("tie_softmax", n=256, d_model=64, n_routed=16, top_k=4, moe_intermediate_size=64,
         ternary=True, renormalize=True),
     _wl("tie_sigmoid", n=256, d_model=64, n_routed=32, top_k=4, moe_intermediate_size=64,

@@ -55,3 +55,33 @@ def test_stalled_stage_reports_timeout_and_context_survives(mode, monkeypatch):
         if hi > lo:
             ref[lo:hi] = O.swiglu(x64[lo:hi], host["w_gate"][e], host["w_up"][e], host["w_down"][e])
     assert H.rel_err(got, ref) <= H.TOL[w.dtype]
+
+
+def test_bf16_gemm_the_tensor_cores_cannot_take_is_unsupported(monkeypatch):
+    """A bf16 layer never runs its matrix products on a slower path: when the tensor-core GEMM
+    cannot take a shape (here forced by MOE_TEST_NO_TENSOR_MAPS=1, as if the driver had no tensor-map
+    entry point) the call returns MOE_ERR_UNSUPPORTED. binary32 layers keep their CUDA-core GEMM."""
+    w = W.get("mixtral_small")
+    dev = W.device_inputs(w)
+    monkeypatch.setenv("MOE_TEST_NO_TENSOR_MAPS", "1")
+    with pytest.raises(moe.MoeError) as e:
+        H.run_layer(w, dev)
+    assert e.value.status == moe.MOE_ERR_UNSUPPORTED
+    wf = W.get("tiny_f32")
+    out = H.run_layer(wf, W.device_inputs(wf))  # binary32: unaffected
+    assert torch.isfinite(out["y"]).all()
+    monkeypatch.delenv("MOE_TEST_NO_TENSOR_MAPS")
+    out = H.run_layer(w, dev)
+    assert torch.isfinite(out["y"]).all()
+
+
+def test_router_with_expert_count_not_a_multiple_of_eight_runs_on_tensor_cores():
+    """E = 5 experts in bf16: the binary32 logits rows are padded to a 16-byte stride and the
+    last columns stored one by one, so the router GEMM stays on the tensor cores (and the
+    indices still equal the oracle's)."""
+    w = W.get("ragged_small")
+    host, dev = W.host_inputs(w), W.device_inputs(w)
+    out = H.run_layer(w, dev)
+    oi, _, ex, _ = O.route_capacity(H.oracle_cfg(w), O.router_logits(host["x"], host["w_r"]), host.get("bias"))
+    got = out["topk_idx"].cpu().numpy()
+    assert (got[~ex] == oi[~ex]).all()

@@ -86,6 +86,30 @@ def test_capacity_route_parity_across_top_k(k, policy):
     test_route_parity(w.name, w)
 
 
+# From 2048 tokens the router decides in the tensor-core epilogue (one pass) and re-decides only
+# the uncertain tokens in binary64; the tie workloads send many tokens down that second path.
+ONE_PASS = ["mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "deepseek_v4_small", "ragged_small",
+            "tie_softmax", "tie_sigmoid"]
+
+
+@pytest.mark.parametrize("name", ONE_PASS)
+def test_one_pass_route_parity(name):
+    w = W.get(name, n=2304 if name != "ragged_small" else 4100)
+    test_route_parity(w.name, w)
+
+
+@pytest.mark.parametrize("mode", ["grid", "1cta"])
+@pytest.mark.parametrize("policy", ["overflow_next", "drop"])
+@pytest.mark.parametrize("k", [1, 2, 3, 8])
+def test_capacity_on_many_ctas(k, policy, mode, monkeypatch):
+    """20 000 tokens: the capacity rule on a cooperative grid of 20 CTAs (one fill event per round)
+    and on the one-CTA kernel, both against the oracle's sequential greedy."""
+    if mode == "1cta":
+        monkeypatch.setenv("MOE_CAP_MODE", "1cta")
+    w = W.get("skewed_small", top_k=k, cap_policy=policy, n=20000)
+    test_route_parity(w.name, w)
+
+
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "skewed_small", "drop_small", "tiny_f32"])
 def test_permute_parity(name):
     w = W.get(name)

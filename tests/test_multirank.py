@@ -57,3 +57,27 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.reduce_max(3.5, 1) == 3.5
     assert bench.job_throughput(64, 2, 1, 1000.0) == 128.0
+
+
+def test_launcher_starts_ranks_that_split_an_expert_parallel_group(tmp_path):
+    """bench.launch_ranks (what `bench.py --gpus N` runs as a plain command) starts N ranks under
+    torch.distributed.run on 127.0.0.1; each rank's group plan (token slice, owned experts, receive
+    rows) is exchanged through the process group: the token slices partition the batch, the owned
+    experts partition the experts, and every rank sizes the same receive buffers. The slowest rank's
+    time is the job's."""
+    import json
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import bench
+
+    out = tmp_path / "ranks.json"
+    probe = os.path.join(os.path.dirname(os.path.abspath(__file__)), "rank_probe.py")
+    rc = bench.launch_ranks(2, 180, script=probe, argv=[str(out), "16387", "256", "8"])
+    assert rc == 0
+    res = json.loads(out.read_text())
+    assert res["world"] == 2 and res["master"] == "127.0.0.1" and res["ms"] == 11.0
+    plans = res["plans"]
+    assert [tuple(p["tokens"]) for p in plans] == [(0, 8194), (8194, 16387)]
+    assert [tuple(p["experts"]) for p in plans] == [(0, 128), (128, 256)]
+    assert plans[0]["recv_rows"] == plans[1]["recv_rows"] == 16387 * 8

@@ -19,7 +19,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace layout; every region starts on a 256-byte boundary.
 struct Plan {
-  size_t diag, logits, ranking, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
+  size_t diag, logits, rq, ranking, capg, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
   size_t xq, sfx, hq, sfh, xsq, sfxs, hsq, sfhs;  // FP8 experts: E4M3 activations and their scale blocks
   size_t sfb, sfbs;  // FP8 SM-pair GEMMs: B scale blocks (routed, shared experts)
   size_t ep_off;  // expert parallelism: receive offsets of the rank's own experts
@@ -34,16 +34,20 @@ int64_t fp8_sf_blocks(int64_t rows, int32_t G, int64_t k) { return fp8_sf_tiles_
 // weight: bf16 for the FP8 experts, whose matrices alone are E4M3.
 int act_dtype(const moe_config& c) { return c.dtype == MOE_FP8 ? MOE_BF16 : c.dtype; }
 
+// Row stride of the binary32 logits: E rounded up to four floats, so that every row
+// starts on a 16-byte boundary for the tensor-core GEMM's vector stores.
+int64_t logits_ld(const moe_config& c) { return align_up(c.n_routed, 4); }
+
 // Split-K factor of the router GEMM: small token counts leave most SMs idle
 // (one 128-row tile per 128 tokens), so the k range is split and the route
 // kernel sums the partial logits in a fixed order. Capped at 4 MiB of partials.
 int router_splits(const moe_config& c, int64_t n) {
-  if (act_dtype(c) != MOE_BF16 || c.n_routed % 8 != 0 || n <= 0) return 1;
+  if (act_dtype(c) != MOE_BF16 || n <= 0) return 1;
   const int64_t tiles = ceil_div(n, 128) * ceil_div(c.n_routed, 256);
   if (tiles >= 74) return 1;
   const int64_t num_kb = ceil_div(c.d_model, 64);
   int64_t s = 148 / tiles;
-  const int64_t cap = ((int64_t)4 << 20) / (n * c.n_routed * 4);
+  const int64_t cap = ((int64_t)4 << 20) / (n * logits_ld(c) * 4);
   if (s > cap) s = cap;
   if (s > num_kb) s = num_kb;
   if (s < 1) s = 1;
@@ -70,8 +74,10 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
     return at;
   };
   p.diag = take(sizeof(moe_diag));
-  p.logits = take((size_t)router_splits(c, n) * n * c.n_routed * 4);
+  p.logits = take((size_t)router_splits(c, n) * n * logits_ld(c) * 4);
+  p.rq = take((size_t)n * 4);  // tokens the one-pass router leaves to the binary64 router
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
+  p.capg = take(c.cap_policy != MOE_CAP_NONE ? (size_t)capacity_grid_scratch_bytes(n, c.n_routed) : 0);
   p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
   p.idx = take((size_t)nk * 4);
   p.w = take((size_t)nk * 4);
@@ -199,27 +205,27 @@ moe_status check_weights(const moe_config& c, const moe_weights* w, bool routed,
   return MOE_OK;
 }
 
-// Grouped GEMM dispatch: tcgen05 tensor cores for bf16 where the shape allows,
-// the CUDA-core kernel otherwise (binary32 layers).
+// Grouped GEMM dispatch: bf16 runs on the tcgen05 tensor cores only (a shape or
+// alignment they cannot take is MOE_ERR_UNSUPPORTED, never a slower path);
+// binary32 layers run on the CUDA cores, whose FFMA meets their 1e-4 tolerance.
 moe_status gemm(const Ctx& x, const GemmArgs& a, bool swiglu, bool out_f32) {
-  if (act_dtype(x.c) == MOE_BF16 && gemm_tc_supported(a, swiglu, out_f32))
+  if (act_dtype(x.c) == MOE_BF16) {
+    if (!gemm_tc_supported(a, swiglu, out_f32)) return MOE_ERR_UNSUPPORTED;
     return cuda_status(launch_gemm_tc(a, swiglu, out_f32, x.status(), x.s));
+  }
   return cuda_status(launch_gemm_simt(a, act_dtype(x.c), out_f32, swiglu, x.s));
 }
 
-// Router logits (binary32, split-K partials for small batches) and the route arguments.
-moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, moe_diag* d,
-                         RouteArgs* out) {
+// Arguments of the warp-per-token router over the logits buffer (splits partial sums).
+RouteArgs route_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, moe_diag* d,
+                     int splits) {
   const moe_config& c = x.c;
-  float* logits = x.at<float>(x.p.logits);
-  const int splits = router_splits(c, x.n);
-  GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, logits, c.n_routed, nullptr, 1, x.n, c.n_routed, c.d_model,
-             splits, x.n * c.n_routed};
-  MOE_TRY(gemm(x, g, false, true));
+  const int64_t ld = logits_ld(c);
   RouteArgs r{};
-  r.logits = logits;
+  r.logits = x.at<float>(x.p.logits);
   r.splits = splits;
-  r.split_stride = x.n * c.n_routed;
+  r.split_stride = x.n * ld;
+  r.ldl = ld;
   r.x = X;
   r.w_r = w->w_router;
   r.bias = c.score_fn != MOE_SCORE_SOFTMAX ? w->bias : nullptr;
@@ -237,8 +243,53 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
   r.topk_w = tw;
   r.diag = d;
   r.ranking = nullptr;
-  *out = r;
+  return r;
+}
+
+// Router logits (binary32, split-K partials for small batches) and the route arguments.
+moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, moe_diag* d,
+                         RouteArgs* out) {
+  const moe_config& c = x.c;
+  const int splits = router_splits(c, x.n);
+  const int64_t ld = logits_ld(c);
+  GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, x.at<float>(x.p.logits), ld, nullptr, 1, x.n, c.n_routed,
+             c.d_model, splits, x.n * ld};
+  MOE_TRY(gemm(x, g, false, true));
+  *out = route_args(x, X, w, idx, tw, d, splits);
   return MOE_OK;
+}
+
+// Batches from this many tokens route in one pass (route_tc.cu) when the configuration allows;
+// smaller ones keep the split-K logits GEMM, which spreads a few token tiles over every SM.
+constexpr int64_t kOnePassMinTokens = 2048;
+
+// The one-pass router's arguments; false when this configuration takes the two-kernel path.
+bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, RouteTcArgs* ra) {
+  const moe_config& c = x.c;
+  if (act_dtype(c) != MOE_BF16 || c.cap_policy != MOE_CAP_NONE || x.n < kOnePassMinTokens) return false;
+  RouteTcArgs a{};
+  a.x = X;
+  a.w_r = w->w_router;
+  a.bias = c.score_fn != MOE_SCORE_SOFTMAX ? w->bias : nullptr;
+  a.n = x.n;
+  a.d = c.d_model;
+  a.E = c.n_routed;
+  a.k = c.top_k;
+  a.G = c.n_group;
+  a.topk_group = c.topk_group;
+  a.score_fn = c.score_fn;
+  a.renorm = c.renormalize;
+  a.rsf = c.routed_scaling_factor;
+  a.topk_idx = idx;
+  a.topk_w = tw;
+  a.logits = x.at<float>(x.p.logits);
+  a.ldl = logits_ld(c);
+  a.queue = x.at<int32_t>(x.p.rq);
+  a.queue_len = &x.status()->reserved[1];
+  a.status = x.status();
+  if (!route_tc_supported(a)) return false;
+  *ra = a;
+  return true;
 }
 
 moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, int32_t* counts,
@@ -251,18 +302,40 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     if (counts) MOE_CUDA(launch_fill_i32(counts, c.n_routed, 0, x.s));
     return MOE_OK;
   }
+  // token cursor of the router's warps and the one-pass router's queue length, in the workspace's
+  // own diag block
+  int32_t* cursor = &x.status()->reserved[0];
+  MOE_CUDA(cudaMemsetAsync(cursor, 0, 2 * sizeof(int32_t), x.s));
+  RouteTcArgs ra;
   RouteArgs r;
-  MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
-  // token cursor of the router's warps, in the workspace's own diag block
-  r.cursor = &x.status()->reserved[0];
-  MOE_CUDA(cudaMemsetAsync(r.cursor, 0, sizeof(int32_t), x.s));
-  if (c.cap_policy == MOE_CAP_NONE) {
-    r.ranking = nullptr;
+  if (one_pass_args(x, X, w, idx, tw, &ra)) {
+    // decisions in the tensor-core epilogue; the queued tokens re-decided from their logits rows
+    MOE_CUDA(launch_route_tc(ra, x.s));
+    r = route_args(x, X, w, idx, tw, d, 1);
+    r.cursor = cursor;
+    r.queue = ra.queue;
+    r.queue_len = ra.queue_len;
+    MOE_CUDA(launch_route(r, x.s));
+  } else if (c.cap_policy == MOE_CAP_NONE) {
+    MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
+    r.cursor = cursor;
     MOE_CUDA(launch_route(r, x.s));
   } else {
+    MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
+    r.cursor = cursor;
     r.ranking = x.at<uint16_t>(x.p.ranking);
     MOE_CUDA(launch_route(r, x.s));
-    MOE_CUDA(launch_capacity(r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, x.s));
+    // the capacity rule on many SMs when its grid fits on the device at once (MOE_CAP_MODE=1cta
+    // forces the one-CTA kernel: tuning and tests)
+    const char* cm = getenv("MOE_CAP_MODE");
+    const bool one_cta = cm && strcmp(cm, "1cta") == 0;
+    if (!one_cta && capacity_grid_fits(x.n, c.top_k)) {
+      CapacityArgs ca{r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, nullptr,
+                      x.status()};
+      MOE_CUDA(launch_capacity_grid(ca, x.ws + x.p.capg, x.s));
+    } else {
+      MOE_CUDA(launch_capacity(r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, x.s));
+    }
     MOE_CUDA(launch_gates(r, x.s));
   }
   // per-expert slot counts and the largest load (histogram + scan, no scatter)
@@ -562,11 +635,17 @@ static_assert(sizeof(cudaIpcMemHandle_t) + sizeof(uint64_t) == MOE_EP_HANDLE_BYT
 
 namespace moe {
 
-// Bytes of the routing part of the workspace layout (the regions moe_route uses).
-size_t route_scratch_bytes(const moe_config& c, int64_t n) {
-  const Plan p = make_plan(c, n);
-  return p.offsets + (size_t)align_up((int64_t)(c.n_routed + 1) * 4, 256);
+// Router-only layout inside a fixed scratch region: the status word, the logits, the capacity
+// ranking, the per-block counts and the offsets of the count scan. The caller's own buffers hold
+// the indices, gates and counts, so the full layout's regions for those are left out.
+Plan route_plan(const moe_config& c, int64_t n) {
+  Plan p = make_plan(c, n);
+  p.offsets = p.idx;
+  p.total = p.offsets + (size_t)align_up((int64_t)(c.n_routed + 1) * 4, 256);
+  return p;
 }
+
+size_t route_scratch_bytes(const moe_config& c, int64_t n) { return route_plan(c, n).total; }
 
 // moe_route over a scratch region that only needs route_scratch_bytes() bytes.
 moe_status route_in_scratch(const moe_config* cfg, int64_t n, const void* x, const moe_weights* weights,
@@ -578,18 +657,18 @@ moe_status route_in_scratch(const moe_config* cfg, int64_t n, const void* x, con
   Ctx c;
   c.c = *cfg;
   c.n = n;
-  c.p = make_plan(*cfg, n);
+  c.p = route_plan(*cfg, n);
   c.ws = static_cast<char*>(scratch);
   c.s = reinterpret_cast<cudaStream_t>(stream);
   if (!weights || !ptr_ok(weights->w_router) || !tok_ok(x, n) || !tok_ok(topk_idx, n) || !tok_ok(topk_w, n))
     return MOE_ERR_INVALID_ARG;
-  if ((expert_counts && !aligned(expert_counts, 4)) || (diag && !aligned(diag, 16))) return MOE_ERR_INVALID_ARG;
+  // diag carries the device status word out of the shared scratch, so it is required here
+  if (!diag || !aligned(diag, 16) || (expert_counts && !aligned(expert_counts, 4))) return MOE_ERR_INVALID_ARG;
   MOE_TRY(check_weights(c.c, weights, false, false));
   MOE_TRY(clear_status(c));
   MOE_TRY(route_impl(c, x, weights, topk_idx, topk_w, expert_counts, diag));
   // The scratch is not the caller's, so hand the device status word over in diag.
-  if (diag)
-    MOE_CUDA(cudaMemcpyAsync(&diag->status, &c.status()->status, sizeof(int32_t), cudaMemcpyDeviceToDevice, c.s));
+  MOE_CUDA(cudaMemcpyAsync(&diag->status, &c.status()->status, sizeof(int32_t), cudaMemcpyDeviceToDevice, c.s));
   return MOE_OK;
 }
 

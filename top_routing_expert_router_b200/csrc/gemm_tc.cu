@@ -152,9 +152,15 @@ __device__ __forceinline__ void store16(void* C, int64_t ldc, int64_t row, int c
   if (f32) {
     float* p = static_cast<float*>(C) + row * ldc + col;
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (col + 4 * q + 4 <= N)
+    for (int q = 0; q < 4; ++q) {
+      if (col + 4 * q + 4 <= N) {
         *reinterpret_cast<float4*>(p + 4 * q) = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)  // last columns of a row whose width is not a multiple of 4
+          if (col + 4 * q + e < N) p[4 * q + e] = v[4 * q + e];
+      }
+    }
   } else {
     bf16* p = static_cast<bf16*>(C) + row * ldc + col;
     uint4 lo, hi;
@@ -828,7 +834,11 @@ bool use_pair_tiles(const GemmArgs& a, bool swiglu, bool out_f32) {
 }  // namespace
 
 bool gemm_tc_supported(const GemmArgs& a, bool swiglu, bool out_f32) {
-  if (a.K % 8 != 0 || a.N % 8 != 0 || a.N <= 0 || a.K <= 0) return false;
+  // MOE_TEST_NO_TENSOR_MAPS=1 makes every shape unsupported (test of the error path).
+  const char* inj = getenv("MOE_TEST_NO_TENSOR_MAPS");
+  if (inj && inj[0] == '1') return false;
+  // binary32 outputs store a row's last columns one by one; bf16 outputs need whole 8-column chunks
+  if (a.K % 8 != 0 || (!out_f32 && a.N % 8 != 0) || a.N <= 0 || a.K <= 0) return false;
   if (a.G > kMaxGroupsTc || a.M >= ((int64_t)1 << 31)) return false;
   if (a.lda != a.K) return false;
   if (swiglu && out_f32) return false;

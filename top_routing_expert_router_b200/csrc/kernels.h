@@ -78,9 +78,10 @@ cudaError_t launch_quantize_rows(const void* src, const int32_t* src_row, const 
 
 // Router: scoring, group limit, top-k, certification / binary64 refinement, gates.
 struct RouteArgs {
-  const float* logits;  // [splits][n, E] partial logits, summed in order
+  const float* logits;  // [splits][n, ldl] partial logits (first E columns), summed in order
   int32_t splits;
   int64_t split_stride;
+  int64_t ldl;          // row stride of the logits (>= E)
   const void* x;        // [n, d] for the binary64 refinement
   const void* w_r;      // [E, d]
   const float* bias;    // [E] or nullptr
@@ -94,9 +95,49 @@ struct RouteArgs {
   float* topk_w;        // [n, k]
   moe_diag* diag;       // refined_tokens / refined_logits counters
   int32_t* cursor;      // zeroed before the launch: next token to route (warps fetch tokens from it)
+  const int32_t* queue = nullptr;      // when set: route only the tokens queue[0 .. *queue_len)
+  const int32_t* queue_len = nullptr;
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
+// Router in one pass (route_tc.cu): logits on the tensor cores and the routing decision of each
+// token in the epilogue, in binary32; tokens whose decision is not certain get their logits row
+// written and their index queued for launch_route (RouteArgs::queue) to re-decide.
+struct RouteTcArgs {
+  const void* x;        // [n, d] bf16
+  const void* w_r;      // [E, d] bf16
+  const float* bias;    // [E] or nullptr
+  int64_t n;
+  int32_t d, E, k, G, topk_group, score_fn, renorm;
+  float rsf;
+  int32_t* topk_idx;    // [n, k]
+  float* topk_w;        // [n, k]
+  float* logits;        // [n, ldl]: rows of the queued tokens
+  int64_t ldl;
+  int32_t* queue;       // [n] tokens left to the binary64 router
+  int32_t* queue_len;   // zeroed before the launch
+  moe_diag* status;
+};
+bool route_tc_supported(const RouteTcArgs& a);
+cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
+
+// Capacity rule over the ranking on many SMs (capacity.cu): a cooperative grid, one token per
+// thread, one round per fill event. Needs capacity_grid_scratch_bytes of scratch (16-byte aligned)
+// and every CTA resident at once (capacity_grid_fits); launch_capacity is the one-CTA form.
+struct CapacityArgs {
+  const uint16_t* ranking;  // [n, E] eligible experts in selection order, 0xFFFF after the last
+  int64_t n;
+  int32_t E, k;
+  int64_t C;
+  int32_t policy;
+  int32_t* topk_idx;        // [n, k]
+  moe_diag* diag;           // overflowed / dropped counters (added to)
+  int32_t* hist;            // set by launch_capacity_grid (inside the scratch)
+  moe_diag* status;         // MOE_ERR_TIMEOUT if a grid barrier wait runs out
+};
+int64_t capacity_grid_scratch_bytes(int64_t n, int32_t E);
+bool capacity_grid_fits(int64_t n, int32_t k);
+cudaError_t launch_capacity_grid(const CapacityArgs& a, void* scratch, cudaStream_t s);
 // Capacity rule over the ranking; writes topk_idx and the overflow/drop counts.
 cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32_t k, int64_t C, int policy,
                             int32_t* topk_idx, moe_diag* diag, cudaStream_t s);

@@ -27,14 +27,17 @@ std::mutex g_lock;
 void* g_scratch_addr[kMaxDevices] = {};
 
 // One-time set-up per device, with that device current: the device address of
-// the array. Returns nullptr when the lookup fails.
-void* scratch_for_current_device() {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+// the array. Returns nullptr when the lookup fails (the failed call's error is
+// cleared, so that it is not reported by a later, unrelated launch check).
+void* scratch_for_device(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
   std::lock_guard<std::mutex> guard(g_lock);
   if (!g_scratch_addr[dev]) {
     void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_route_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
     g_scratch_addr[dev] = ptr;
   }
   return g_scratch_addr[dev];
@@ -50,7 +53,15 @@ extern "C" moe_status moe_route_static_scratch(const moe_config* cfg, int64_t n,
   const moe_status st = moe_workspace_size(cfg, n, &need);  // validates cfg
   if (st != MOE_OK) return st;
   if (moe::route_scratch_bytes(*cfg, n) > kStaticScratchBytes) return MOE_ERR_WORKSPACE;
-  void* scratch = scratch_for_current_device();
+  // The array's address belongs to one device: the stream must belong to the current device.
+  int dev = -1, stream_dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaStreamGetDevice(reinterpret_cast<cudaStream_t>(stream), &stream_dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_INVALID_ARG;
+  }
+  if (stream_dev != dev) return MOE_ERR_INVALID_ARG;
+  void* scratch = scratch_for_device(dev);
   if (!scratch) return MOE_ERR_CUDA;
   return moe::route_in_scratch(cfg, n, x, weights, topk_idx, topk_w, expert_counts, diag, scratch,
                                kStaticScratchBytes, stream);

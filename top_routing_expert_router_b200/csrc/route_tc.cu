@@ -1,0 +1,462 @@
+// route_tc.cu -- the router in one pass: logits x W_r^T on the tensor cores, and
+// the whole routing decision of every token in the epilogue that drains them.
+//
+// Definitions (page "15. DeepSeek: MLA, MoE and MTP", section "V3 MoE: how 8 of
+// 256 experts are chosen"; page "MoE architecture revealed", section 3.1; page
+// "1.8T parameters / 2% per token", section 4.1):
+//   softmax : select on the logits l; gates e^{l_j - m} / sum_E e^{l - m}
+//             (renormalised over the kept slots when asked) times rsf;
+//   sigmoid : s = sigmoid(l), selection value c = s + bias; groups of E/G
+//             experts scored by the sum of their two best c, the topk_group
+//             best groups eligible, top-k of c among them; gates s_j / sum s
+//             (when asked) times rsf; sqrtsoftplus likewise with
+//             s = sqrt(softplus(l)) (section "V4").
+// Ties go to the lower expert (group) index; slots are in descending score.
+//
+// Design (one CTA per SM, persistent over 128-token tiles, 192 threads):
+//   warp 0      TMA producer: 128 x 64 tile of x and E x 64 tile of W_r per
+//               stage, 4-stage ring of 128-byte-swizzled shared memory;
+//   warp 1      TMEM owner (two 128 x 256 fp32 accumulators) and MMA issuer,
+//               tcgen05.mma kind::f16, M = 128, N = E rounded up to 16;
+//   warps 2..5  routing epilogue: thread i of lane quarter q owns token row
+//               32q + i, reads its E logits from TMEM 32 columns at a time and
+//               decides in binary32: group scores, group cut, the k best
+//               eligible experts kept sorted by insertion, gates.
+// Exactness: the logits are binary32 sums, so a decision is kept only when
+// every gap it depends on (group cut, adjacent kept experts, the k-th / (k+1)-th
+// cut) exceeds twice the error bound of the selection values; any other token
+// has its logits row written out and its index appended to a queue, and the
+// warp-per-token router (router.cu) re-decides it, recomputing in binary64 the
+// logits near a boundary. Indices therefore equal the binary64 definition.
+#include <cuda.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+using namespace ptx;
+
+constexpr int BM = 128;
+constexpr int BK = 64;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_MAX_BYTES = 256 * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_MAX_BYTES;
+constexpr int kThreads = 192;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr int kMaxK = 8;  // experts per token the epilogue keeps sorted in registers
+constexpr uint64_t kTimeoutNs = 2000000000ull;
+
+struct __align__(8) Ctl {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+  int32_t abort;
+};
+
+__device__ __noinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Ctl* ctl, moe_diag* st) {
+  const uint32_t b = smem_u32(bar);
+  if (mbar_try(b, parity)) return true;
+  const uint64_t t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(b, parity)) return true;
+    if ((it & 255u) == 0) {
+      if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) return false;
+      if (globaltimer() - t0 > kTimeoutNs) {
+        atomicExch(&ctl->abort, 1);
+        set_status(st, MOE_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+// 32 lanes x 32 columns of fp32 from TMEM.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+}
+
+// Raw score of the routers that add a selection bias, in binary32.
+__device__ __forceinline__ float raw_score32(int score_fn, float l) {
+  if (score_fn == MOE_SCORE_SQRTSOFTPLUS) return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
+  return 1.0f / (1.0f + expf(-l));
+}
+
+// Insert (v, l, e) into the list sorted by v descending; an equal v stays below the entries
+// already there, which hold lower expert indices (experts arrive in ascending order).
+__device__ __forceinline__ void insert(float (&lv)[kMaxK + 1], float (&ll)[kMaxK + 1], int (&le)[kMaxK + 1], float v,
+                                       float l, int e) {
+  if (!(v > lv[kMaxK])) return;
+#pragma unroll
+  for (int j = 0; j <= kMaxK; ++j) {
+    if (v > lv[j]) {
+      const float tv = lv[j], tl = ll[j];
+      const int te = le[j];
+      lv[j] = v;
+      ll[j] = l;
+      le[j] = e;
+      v = tv;
+      l = tl;
+      e = te;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    route_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
+                    RouteTcArgs p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_tiles = (int)((p.n + BM - 1) / BM);
+  const int num_kb = (p.d + BK - 1) / BK;
+  const int n_mma = (p.E + 15) & ~15;
+
+  if (threadIdx.x == 0) {
+    ctl->abort = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&ctl->tmem_full[b], 1);
+      mbar_init(&ctl->tmem_empty[b], 4);
+    }
+    mbar_init(&ctl->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+
+  if (warp == 0) {
+    // ================= TMA producer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed[STAGES] = {0, 0, 0, 0};
+      const uint32_t tx = A_BYTES + (uint32_t)n_mma * BK * 2;
+      bool ok = true;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
+              !wait_bar(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_expect_tx(&ctl->full[stage], tx);
+          ++armed[stage];
+          tma_load_2d(sa, &map_x, &ctl->full[stage], kb * BK, t * BM);
+          tma_load_2d(sa + A_BYTES, &map_w, &ctl->full[stage], kb * BK, 0);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok)
+        for (int s = 0; s < STAGES; ++s)
+          if (armed[s]) mbar_drain(&ctl->full[s], (armed[s] - 1) & 1u);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc = idesc_bf16(n_mma);
+      bool ok = true, issued = false;
+      int i = 0;
+      for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
+        const int buf = i & 1;
+        const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+        if (!wait_bar(&ctl->tmem_empty[buf], acc_phase ^ 1u, ctl, p.status)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * 256);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_try(smem_u32(&ctl->full[stage]), phase) && !wait_bar(&ctl->full[stage], phase, ctl, p.status)) {
+            ok = false;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc = sw128_desc(sa + A_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            asm volatile(
+                "{\n\t.reg .pred p;\n\t"
+                "setp.ne.b32 p, %4, 0;\n\t"
+                "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                "l"(adesc + (uint64_t)(2 * k)), "l"(bdesc + (uint64_t)(2 * k)), "r"(idesc), "r"((kb | k) != 0 ? 1 : 0)
+                : "memory");
+          }
+          issued = true;
+          asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                           smem_u32(&ctl->empty[stage]))
+                       : "memory");
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&ctl->tmem_full[buf]))
+                     : "memory");
+      }
+      if (!ok && issued) {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&ctl->drain))
+                     : "memory");
+        mbar_drain(&ctl->drain, 0);
+      }
+    }
+  } else {
+    // ================= routing epilogue (warps 2..5) =================
+    const int q = warp & 3;
+    const int E = p.E, G = p.G, per = p.E / p.G, k = p.k;
+    const bool soft = p.score_fn == MOE_SCORE_SOFTMAX;
+    // derivative bound of the selection value in the logit (sigmoid' <= 1/4, sqrtsoftplus' < 1/2)
+    const float lip = p.score_fn == MOE_SCORE_SIGMOID ? 0.25f : p.score_fn == MOE_SCORE_SQRTSOFTPLUS ? 0.5f : 1.0f;
+    // binary32 evaluation error of a non-softmax selection value (a few ulp of a value near 1)
+    const float eval_err = soft ? 0.0f : 0x1p-20f;
+    int i = 0;
+    for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+      const int buf = i & 1;
+      const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      const bool got = wait_bar(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
+      __syncwarp();
+      if (!got) break;
+      fence_after();
+      const int64_t tok = (int64_t)t * BM + q * 32 + lane;
+      const bool valid = tok < p.n;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256);
+      // pass 1: |l| max, softmax max and normaliser, group scores (top-2 sums of c)
+      float amax = 0.0f, m = -INFINITY, z = 0.0f;
+      float g1 = -INFINITY, g2 = -INFINITY;
+      float gsc[kMaxGroups];
+      for (int c0 = 0; c0 < E; c0 += 32) {
+        float l[32];
+        tmem_ld32(taddr + (uint32_t)c0, l);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c0 + j;
+          if (e < E) {
+            amax = fmaxf(amax, fabsf(l[j]));
+            if (soft) {
+              if (l[j] > m) {
+                z = z * expf(m - l[j]) + 1.0f;
+                m = l[j];
+              } else {
+                z += expf(l[j] - m);
+              }
+            } else if (G > 1) {
+              const float v = raw_score32(p.score_fn, l[j]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
+              if (v > g1) {
+                g2 = g1;
+                g1 = v;
+              } else if (v > g2) {
+                g2 = v;
+              }
+              if ((e + 1) % per == 0) {
+                gsc[e / per] = g1 + g2;
+                g1 = g2 = -INFINITY;
+              }
+            }
+          }
+        }
+      }
+      const float dl = 0x1p-13f * fmaxf(1.0f, amax);  // binary32 error bound of a logit
+      const float dv = lip * dl + eval_err;              // ... of a selection value
+      // group cut: the topk_group best group scores, ties to the lower group index
+      bool ok = true;
+      uint32_t kept = 0xFFFFFFFFu;
+      if (!soft && G > 1) {
+        kept = 0;
+        float min_kept = INFINITY, max_drop = -INFINITY;
+        for (int g = 0; g < G; ++g) {
+          int better = 0;
+          for (int h = 0; h < G; ++h) better += (gsc[h] > gsc[g]) || (gsc[h] == gsc[g] && h < g);
+          if (better < p.topk_group) {
+            kept |= 1u << g;
+            min_kept = fminf(min_kept, gsc[g]);
+          } else {
+            max_drop = fmaxf(max_drop, gsc[g]);
+          }
+        }
+        if (p.topk_group < G && !(min_kept - max_drop > 4.0f * dv + 0x1p-19f)) ok = false;
+      }
+      // pass 2: the k + 1 best eligible experts, sorted
+      float lv[kMaxK + 1], ll[kMaxK + 1];
+      int le[kMaxK + 1];
+#pragma unroll
+      for (int j = 0; j <= kMaxK; ++j) {
+        lv[j] = -INFINITY;
+        ll[j] = 0.0f;
+        le[j] = -1;
+      }
+      int n_elig = 0;
+      for (int c0 = 0; c0 < E; c0 += 32) {
+        // skip a chunk that lies in a dropped group of every token of the warp (TMEM loads are warp-wide)
+        if (per >= 32 && !__any_sync(0xFFFFFFFFu, (kept >> (c0 / per)) & 1u)) continue;
+        float l[32];
+        tmem_ld32(taddr + (uint32_t)c0, l);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c0 + j;
+          if (e < E && ((kept >> (e / per)) & 1u)) {
+            ++n_elig;
+            const float v = soft ? l[j] : raw_score32(p.score_fn, l[j]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
+            insert(lv, ll, le, v, l[j], e);
+          }
+        }
+      }
+      // every order the result depends on must be certain: adjacent kept experts and the k-th / (k+1)-th cut
+#pragma unroll
+      for (int j = 0; j < kMaxK; ++j)
+        if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) ok = false;
+      const bool spill = valid && !ok;
+      if (valid && ok) {
+        // gates of the k kept experts
+        float w[kMaxK];
+        float denom = 1.0f;
+        if (soft) {
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j) w[j] = j < k ? expf(ll[j] - m) / z : 0.0f;
+        } else {
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j) w[j] = j < k ? raw_score32(p.score_fn, ll[j]) : 0.0f;
+        }
+        if (p.renorm) {
+          float s = 0.0f;
+#pragma unroll
+          for (int j = 0; j < kMaxK; ++j) s += j < k ? w[j] : 0.0f;
+          denom = s;
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j)
+          if (j < k) {
+            p.topk_idx[tok * k + j] = le[j];
+            p.topk_w[tok * k + j] = w[j] / denom * p.rsf;
+          }
+      }
+      // not certain: hand the token to the binary64 router with its logits row (the TMEM loads are
+      // warp-wide, so the whole warp reads when any lane spills)
+      if (__any_sync(0xFFFFFFFFu, spill)) {
+        float* row = p.logits + tok * p.ldl;
+        for (int c0 = 0; c0 < E; c0 += 32) {
+          float l[32];
+          tmem_ld32(taddr + (uint32_t)c0, l);
+          if (spill) {
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+              if (c0 + j + 4 <= E) {
+                *reinterpret_cast<float4*>(row + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  if (c0 + j + u < E) row[c0 + j + u] = l[j + u];
+              }
+          }
+        }
+        if (spill) p.queue[atomicAdd(p.queue_len, 1)] = (int32_t)tok;
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)(cols * 2)};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
+
+}  // namespace
+
+bool route_tc_supported(const RouteTcArgs& a) {
+  const char* inj = getenv("MOE_TEST_NO_TENSOR_MAPS");
+  if (inj && inj[0] == '1') return false;
+  if (a.E < 1 || a.E > 256 || a.k < 1 || a.k > kMaxK || a.G < 1 || a.G > kMaxGroups || a.E % a.G != 0) return false;
+  if (a.d % 8 != 0 || a.ldl % 4 != 0 || a.ldl < a.E) return false;
+  if (reinterpret_cast<uintptr_t>(a.x) % 16 || reinterpret_cast<uintptr_t>(a.w_r) % 16 ||
+      reinterpret_cast<uintptr_t>(a.logits) % 16)
+    return false;
+  return encode_fn() != nullptr;
+}
+
+cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
+  if (!route_tc_supported(a)) return cudaErrorNotSupported;
+  if (a.n <= 0) return cudaSuccess;
+  CUtensorMap mx, mw;
+  if (!make_map(&mx, a.x, a.n, a.d, BM)) return cudaErrorInvalidValue;
+  if (!make_map(&mw, a.w_r, a.E, a.d, (a.E + 15) & ~15)) return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> attr{0};
+  {
+    const cudaError_t e = set_smem_limit(attr, (const void*)route_tc_kernel, kSmemBytes);
+    if (e != cudaSuccess) return e;
+  }
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  const int64_t tiles = ceil_div(a.n, BM);
+  const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+  route_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mx, mw, a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -467,12 +467,71 @@ __device__ double dot64(const RouteArgs& a, int64_t t, int e) {
   return warp_sum(acc0 + acc1);
 }
 
+// Binary64 dot products of x[t] with four rows of W_r at once (independent
+// accumulators, the token's row read once per chunk); e < 0 entries are skipped
+// and return 0.
+__device__ void dot64x4(const RouteArgs& a, int64_t t, const int (&e)[4], double (&out)[4]) {
+  const int lane = threadIdx.x & 31;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  if (a.dtype == MOE_BF16) {
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.x) + t * a.d);
+    const uint4* wr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      wr[q] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.w_r) + (int64_t)(e[q] < 0 ? 0 : e[q]) * a.d);
+#pragma unroll 2
+    for (int i = lane; i < a.d / 8; i += 32) {
+      const uint4 xv = __ldg(xr + i);
+      const bf16* xs = reinterpret_cast<const bf16*>(&xv);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (e[q] < 0) continue;
+        const uint4 wv = __ldg(wr[q] + i);
+        const bf16* ws = reinterpret_cast<const bf16*>(&wv);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) acc[q] = fma(to_f64(xs[c]), to_f64(ws[c]), acc[q]);
+      }
+    }
+  } else {
+    const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + t * a.d);
+    for (int i = lane; i < a.d / 4; i += 32) {
+      const float4 xv = __ldg(xr + i);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (e[q] < 0) continue;
+        const float4 wv = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(a.w_r) + (int64_t)e[q] * a.d) + i);
+        acc[q] = fma((double)xv.x, (double)wv.x, acc[q]);
+        acc[q] = fma((double)xv.y, (double)wv.y, acc[q]);
+        acc[q] = fma((double)xv.z, (double)wv.z, acc[q]);
+        acc[q] = fma((double)xv.w, (double)wv.w, acc[q]);
+      }
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) out[q] = warp_sum(acc[q]);
+}
+
 // Replace the logits of the experts in `which` (bits over j, per lane) by
-// binary64 values. Returns how many were recomputed.
+// binary64 values, four experts per pass over the token's row. Returns how many
+// were recomputed.
 template <int EPL>
 __device__ int refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], uint32_t which) {
   const int lane = threadIdx.x & 31;
   int total = 0;
+  int e[4];
+  int n = 0;
+  auto flush = [&]() {
+    double v[4];
+    dot64x4(a, t, e, v);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (e[q] >= 0 && (e[q] & 31) == lane) {
+#pragma unroll
+        for (int j = 0; j < EPL; ++j)
+          if (j == (e[q] >> 5)) l[j] = v[q];
+      }
+    n = 0;
+  };
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     uint32_t m = __ballot_sync(kFull, (which >> j) & 1u);
@@ -480,9 +539,13 @@ __device__ int refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], ui
     while (m) {
       const int src = __ffs(m) - 1;
       m &= m - 1;
-      const double s = dot64(a, t, src + 32 * j);
-      if (lane == src) l[j] = s;
+      e[n++] = src + 32 * j;
+      if (n == 4) flush();
     }
+  }
+  if (n > 0) {
+    for (int q = n; q < 4; ++q) e[q] = -1;
+    flush();
   }
   return total;
 }
@@ -496,7 +559,7 @@ __device__ __forceinline__ void load_logits(const RouteArgs& a, int64_t t, doubl
     const int e = lane + 32 * j;
     double s = 0.0;
     if (e < a.E)
-      for (int p = 0; p < a.splits; ++p) s += (double)a.logits[(int64_t)p * a.split_stride + t * a.E + e];
+      for (int p = 0; p < a.splits; ++p) s += (double)a.logits[(int64_t)p * a.split_stride + t * a.ldl + e];
     l[j] = s;
   }
 }
@@ -516,11 +579,13 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     if (lane + 32 * j < a.E) valid_mask |= 1u << j;
   // Warps take the next token from a shared cursor: a token that needs binary64
   // refinement holds up only its own warp, never a whole block of tokens.
+  const int64_t count = a.queue ? (int64_t)*a.queue_len : a.n;
   for (;;) {
     int tok = 0;
     if (lane == 0) tok = atomicAdd(a.cursor, 1);
-    const int64_t t = __shfl_sync(kFull, tok, 0);
-    if (t >= a.n) break;
+    const int64_t i = __shfl_sync(kFull, tok, 0);
+    if (i >= count) break;
+    const int64_t t = a.queue ? (int64_t)a.queue[i] : i;
     double l[EPL];
     load_logits<EPL>(a, t, l);
     double amax = 0.0;
