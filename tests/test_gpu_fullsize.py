@@ -79,9 +79,12 @@ def _decision_gap(w, logits, bias):
     return gap
 
 
-def _sample(w, keep, gap, hard=32, rand=30):
-    """Hardest non-exempt tokens by decision gap, plus the first, the last and random ones."""
+def _sample(w, keep, gap, hard=32, rand=32):
+    """Hardest non-exempt tokens by decision gap, plus the first, the last and random ones (every
+    compared token when there are at most hard + rand of them)."""
     cand = np.nonzero(keep)[0]
+    if len(cand) <= hard + rand:
+        return cand.astype(np.int64)
     hardest = cand[np.argsort(gap[cand], kind="stable")[:hard]]
     rng = np.random.default_rng(0)
     pool = np.setdiff1d(cand, hardest)

@@ -21,6 +21,18 @@ SMALL = ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small", 
          "skewed_small", "drop_small", "ragged_small", "deepseek_v4_small", "tie_softmax", "tie_sigmoid"]
 
 
+def _tile_mode(mode, monkeypatch):
+    """1sm: one-SM 128-row tiles; 2sm: SM-pair 256 x 256 tiles; 2sm_wide: SM-pair 256 x 512 tiles."""
+    monkeypatch.setenv("MOE_TC_MODE", "1sm" if mode == "1sm" else "2sm")
+    if mode == "2sm_wide":
+        monkeypatch.setenv("MOE_TC_WIDE", "1")
+    else:
+        monkeypatch.delenv("MOE_TC_WIDE", raising=False)
+
+
+TILE_MODES = ["1sm", "2sm", "2sm_wide"]
+
+
 @pytest.fixture(scope="module", autouse=True)
 def _cuda():
     if not torch.cuda.is_available():
@@ -256,16 +268,18 @@ def _staged_layer(w, dev):
     return y
 
 
-@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+@pytest.mark.parametrize("mode", TILE_MODES)
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "deepseek_v3_small", "ragged_small"])
 def test_layer_equals_staged_path(name, mode, monkeypatch):
     """moe_layer_forward (shared experts on the side stream) equals route -> permute ->
     expert FFN -> combine through the staged entry points bit for bit."""
-    monkeypatch.setenv("MOE_TC_MODE", mode)
+    _tile_mode(mode, monkeypatch)
     w = W.get(name)
     dev = W.device_inputs(w)
     fused = H.run_layer(w, dev)["y"]
     assert torch.equal(fused, _staged_layer(w, dev))
+
+
 
 
 # Group sizes around the 128-row and 256-row tile edges: empty groups, one row,
@@ -273,10 +287,10 @@ def test_layer_equals_staged_path(name, mode, monkeypatch):
 EDGE_COUNTS = [0, 1, 64, 127, 128, 129, 255, 256, 257, 300, 384, 385, 513, 640, 0]
 
 
-@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+@pytest.mark.parametrize("mode", TILE_MODES)
 def test_expert_ffn_tile_edges(mode, monkeypatch):
     """Caller-given group offsets at every tile edge; d and I leave ragged n- and k-tiles."""
-    monkeypatch.setenv("MOE_TC_MODE", mode)
+    _tile_mode(mode, monkeypatch)
     counts = np.array(EDGE_COUNTS, np.int32)
     rows = int(counts.sum())
     w = W.get("ragged_small", n=rows, d_model=320, n_routed=len(counts), top_k=1, moe_intermediate_size=200,
@@ -300,11 +314,11 @@ def test_expert_ffn_tile_edges(mode, monkeypatch):
             assert H.rel_err(got[lo:hi], ref) <= H.TOL[w.dtype], (e, int(counts[e]))
 
 
-@pytest.mark.parametrize("mode", ["1sm", "2sm"])
+@pytest.mark.parametrize("mode", TILE_MODES)
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v3_small", "ragged_small", "deepseek_v2_small"])
 def test_expert_ffn_both_tile_modes(name, mode, monkeypatch):
-    """The 128-row single-SM tiles and the 256-row SM-pair tiles both match the oracle."""
-    monkeypatch.setenv("MOE_TC_MODE", mode)
+    """The 128-row single-SM tiles and the 256-row SM-pair tiles (256 and 512 wide) match the oracle."""
+    _tile_mode(mode, monkeypatch)
     test_expert_ffn_parity(name)
     w = W.get(name)
     dev, host = W.device_inputs(w), W.host_inputs(w)

@@ -329,10 +329,17 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     // forces the one-CTA kernel: tuning and tests)
     const char* cm = getenv("MOE_CAP_MODE");
     const bool one_cta = cm && strcmp(cm, "1cta") == 0;
-    if (!one_cta && capacity_grid_fits(x.n, c.top_k)) {
+    if (!one_cta && capacity_grid_fits(x.n, c.n_routed)) {
       CapacityArgs ca{r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, nullptr,
                       x.status()};
-      MOE_CUDA(launch_capacity_grid(ca, x.ws + x.p.capg, x.s));
+      const cudaError_t e = launch_capacity_grid(ca, x.ws + x.p.capg, x.s);
+      if (e == cudaErrorCooperativeLaunchTooLarge) {
+        // the grid did not fit beside other resident work after all: the one-CTA kernel
+        cudaGetLastError();
+        MOE_CUDA(launch_capacity(r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, x.s));
+      } else {
+        MOE_CUDA(e);
+      }
     } else {
       MOE_CUDA(launch_capacity(r.ranking, x.n, c.n_routed, c.top_k, capacity_of(c, x.n), c.cap_policy, idx, d, x.s));
     }

@@ -136,8 +136,11 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   __shared__ int cross[kMaxExperts];  // CTA where expert e reaches C this round (kNone: nowhere)
   __shared__ int need[kMaxExperts];   // choosers of e in that CTA up to and including the filling one
   __shared__ uint32_t ballots[kThreads / 32];
+  __shared__ int cnt_s[kMaxExperts];        // committed counts at the start of the round
+  __shared__ uint32_t nfull_s[kMaxExperts / 32];
   __shared__ int s_bstar, s_tloc;
   __shared__ unsigned long long s_over, s_drop;
+  extern __shared__ int hist_all[];           // [gridDim.x][E]: every CTA's counts of this round
   const int64_t t = (int64_t)blockIdx.x * kThreads + tid;
   const bool valid = t < a.n;
   const uint16_t* row = a.ranking + (valid ? t : 0) * E;
@@ -192,15 +195,20 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
     for (int e = tid; e < E; e += kThreads) a.hist[(int64_t)blockIdx.x * E + e] = hist[e];
     if (!grid_sync(g, nblocks, gen, a.status)) return;
     // 2. in token order over the CTAs: where does each non-full expert reach C?
+    // (every CTA's row, the counts and the full set are read once, in parallel, from L2: other
+    // CTAs wrote them, so never through a possibly stale L1 line)
     if (tid == 0) s_bstar = kNone;
+    for (int i = tid; i < (int)nblocks * E; i += kThreads) hist_all[i] = __ldcg(&a.hist[i]);
+    for (int e = tid; e < E; e += kThreads) cnt_s[e] = __ldcg(&cur.cnt[e]);
+    for (int w = tid; w < kMaxExperts / 32; w += kThreads) nfull_s[w] = __ldcg(&cur.full[w]);
     __syncthreads();
     if (tid < E) {
       const int e = tid;
-      int run = __ldcg(&cur.cnt[e]);
+      int run = cnt_s[e];
       int cb = kNone, nd = 0;
-      if (!((__ldcg(&cur.full[e >> 5]) >> (e & 31)) & 1u)) {
+      if (!((nfull_s[e >> 5] >> (e & 31)) & 1u)) {
         for (uint32_t b = 0; b < nblocks; ++b) {
-          const int h = __ldcg(&a.hist[(int64_t)b * E + e]);
+          const int h = hist_all[b * E + e];
           if (run + h >= a.C) {
             cb = (int)b;
             nd = (int)(a.C - run);
@@ -248,24 +256,17 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
       __syncthreads();
       for (int j = 0; j < k; ++j) warp_count(hist, (!committed && tid <= tloc) ? slot(j) : -1);
       __syncthreads();
+      // counts up to and including the filling token: the committed ones, every earlier CTA's
+      // row, and this CTA's tokens up to it; an expert is full from C on
       if (tid < E) {
         const int e = tid;
-        int pre = __ldcg(&cur.cnt[e]);
-        for (int b = 0; b < bstar; ++b) pre += __ldcg(&a.hist[(int64_t)b * E + e]);
-        nxt.cnt[e] = pre + hist[e];
+        int c = cnt_s[e] + hist[e];
+        for (int b = 0; b < bstar; ++b) c += hist_all[b * E + e];
+        nxt.cnt[e] = c;
+        if (c >= a.C) atomicOr(&nfull_s[e >> 5], 1u << (e & 31));
       }
-      if (tid < kMaxExperts / 32) {
-        uint32_t m = __ldcg(&cur.full[tid]);
-        for (int q = 0; q < 32; ++q) {
-          const int e = tid * 32 + q;
-          if (e < E) {
-            int pre = __ldcg(&cur.cnt[e]);
-            for (int b = 0; b < bstar; ++b) pre += __ldcg(&a.hist[(int64_t)b * E + e]);
-            if (pre + hist[e] >= a.C) m |= 1u << q;
-          }
-        }
-        nxt.full[tid] = m;
-      }
+      __syncthreads();
+      for (int w = tid; w < kMaxExperts / 32; w += kThreads) nxt.full[w] = nfull_s[w];
       if (tid == 0) nxt.fill_tok = (int)((int64_t)blockIdx.x * kThreads + tloc);
     }
     if (bstar == kNone) {
@@ -327,27 +328,34 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   }
 }
 
+// Dynamic shared memory of a grid of `grid` CTAs: every CTA's row of per-expert counts.
+size_t dyn_smem(unsigned grid, int E) { return (size_t)grid * E * sizeof(int); }
+
 template <int KT>
 cudaError_t launch_t(CapacityArgs a, GridCtl* g, unsigned grid, cudaStream_t s) {
+  static std::atomic<uint64_t> attr{0};
+  const size_t smem = dyn_smem(grid, a.E);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = set_smem_limit(attr, (const void*)capacity_grid_kernel<KT>, 227 * 1024 - 4096);
+    if (e != cudaSuccess) return e;
+  }
   void* args[] = {&a, &g};
-  return cudaLaunchCooperativeKernel((const void*)capacity_grid_kernel<KT>, dim3(grid), dim3(kThreads), args, 0, s);
+  return cudaLaunchCooperativeKernel((const void*)capacity_grid_kernel<KT>, dim3(grid), dim3(kThreads), args, smem, s);
 }
 
 // CTAs of the kernel that fit on the current device at once (queried once per device).
-template <int KT>
+// CTAs of the kernel that fit on the current device at once: one per SM (1024 threads at up to 64
+// registers fill an SM's register file), so the SM count, read once per device.
 int resident_blocks() {
   constexpr int kMaxDevices = 64;
   static std::atomic<int> cached[kMaxDevices];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return 0;
   if (dev < kMaxDevices && cached[dev].load() > 0) return cached[dev].load();
-  int per_sm = 0, sms = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, capacity_grid_kernel<KT>, kThreads, 0) != cudaSuccess)
-    return 0;
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int r = per_sm * sms;
-  if (dev < kMaxDevices && r > 0) cached[dev].store(r);
-  return r;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) return 0;
+  if (dev < kMaxDevices) cached[dev].store(sms);
+  return sms;
 }
 
 }  // namespace
@@ -356,17 +364,10 @@ int64_t capacity_grid_scratch_bytes(int64_t n, int32_t E) {
   return (int64_t)sizeof(GridCtl) + ceil_div(n, kThreads) * E * 4;
 }
 
-bool capacity_grid_fits(int64_t n, int32_t k) {
+bool capacity_grid_fits(int64_t n, int32_t E) {
   const int64_t blocks = ceil_div(n, kThreads);
-  int res = 0;
-  switch (k) {
-    case 1: res = resident_blocks<1>(); break;
-    case 2: res = resident_blocks<2>(); break;
-    case 4: res = resident_blocks<4>(); break;
-    case 8: res = resident_blocks<8>(); break;
-    default: res = resident_blocks<0>(); break;
-  }
-  return blocks >= 1 && blocks <= res;
+  // one CTA per SM, and every CTA's count row in shared memory next to the static arrays
+  return blocks >= 1 && blocks <= resident_blocks() && dyn_smem((unsigned)blocks, E) <= 200 * 1024;
 }
 
 cudaError_t launch_capacity_grid(const CapacityArgs& a, void* scratch, cudaStream_t s) {

@@ -771,6 +771,252 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---- wide SM-pair variant: 256 x 512 tiles ------------------------------------------
+// The pair computes a 256-row (or half-height 128-row) by 512-column tile with two
+// tcgen05.mma.cta_group::2 of N = 256 per 16-wide k step, into one 512-column TMEM
+// accumulator per CTA. Per 64-k stage each CTA stages its A rows (16 KB, 8 KB half) and two
+// 128-row B blocks (32 KB): 48 KB for twice the MMA work of a 256 x 256 tile's 32 KB, so a
+// stage of shared memory carries 25 % fewer bytes per FLOP. SwiGLU: block 0 holds gate rows
+// [j0 + 128r, +128) and block 1 the up rows of the same columns (MMA 0 -> TMEM columns
+// [0, 256) = gate, MMA 1 -> [256, 512) = up), 256 outputs per tile; plain: block 0 rows
+// j0 + 128r, block 1 rows j0 + 256 + 128r, 512 outputs. With one accumulator the epilogue
+// of a tile does not overlap the next tile's main loop, so eight epilogue warps (two per TMEM
+// lane quarter, each half of the columns) drain it.
+constexpr int STAGESW = 4;
+constexpr int BW_BLOCK_BYTES = 128 * BK * 2;
+constexpr int STAGEW_BYTES = A2_BYTES + 2 * BW_BLOCK_BYTES;
+constexpr int kThreadsW = 320;  // producer, MMA issuer, 8 epilogue warps
+constexpr int kTileReadersW = 18;  // leader MMA + 8 leader epilogue warps + peer producer + 8 peer epilogue warps
+static_assert(STAGESW <= STAGES2, "the control block's barrier arrays hold STAGES2 stages");
+
+__global__ void __launch_bounds__(kThreadsW, 1)
+    gemm_tc2w_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_a_half,
+                     const __grid_constant__ CUtensorMap map_b, const __grid_constant__ CUtensorMap map_b2,
+                     TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw_w[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw_w) + 1023) & ~uintptr_t(1023));
+  SmemCtl2* ctl = reinterpret_cast<SmemCtl2*>(smem + STAGESW * STAGEW_BYTES);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    const int n_tiles = (p.N + p.n_out - 1) / p.n_out;
+    for (int g = 0; g < p.G; ++g) {
+      const int lo = p.offsets ? p.offsets[g] : 0;
+      const int hi = p.offsets ? p.offsets[g + 1] : p.M;
+      ctl->tile_off[g] = acc;
+      acc += ((hi - lo + BM2 - 1) / BM2) * n_tiles;
+    }
+    ctl->tile_off[p.G] = acc;
+    ctl->total_tiles = acc;
+    ctl->n_tiles = n_tiles;
+    ctl->abort = 0;
+    ctl->timeout_ns = p.timeout_ns;
+    for (int s = 0; s < STAGESW; ++s) {
+      mbar_init(&ctl->full[s], 1);
+      mbar_init(&ctl->empty[s], 1);
+    }
+    mbar_init(&ctl->tmem_full[0], 1);
+    mbar_init(&ctl->tmem_empty[0], 16);
+    for (int q = 0; q < kTileSlots; ++q) {
+      mbar_init(&ctl->tile_full[q], 1);
+      mbar_init(&ctl->tile_empty[q], kTileReadersW);
+    }
+    mbar_init(&ctl->drain, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&map_a);
+    tma_prefetch_desc(&map_a_half);
+    tma_prefetch_desc(&map_b);
+    if (p.swiglu) tma_prefetch_desc(&map_b2);
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&ctl->tmem_base)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  cluster_sync();
+  fence_after();
+  const uint32_t tmem_base = ctl->tmem_base;
+  const int total = ctl->total_tiles;
+  const int num_kb = (p.K + BK - 1) / BK;
+  bool aborted = false;
+
+  if (warp == 0) {
+    // ================= TMA producer (both CTAs) =================
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int g_hint = 0;
+      for (int i = 0; !aborted; ++i) {
+        const int t = rank == 0 ? publish_tile(ctl, i, p) : take_tile(ctl, i, rank, p);
+        if (t < 0) {
+          aborted = true;
+          break;
+        }
+        if (t >= total) break;
+        const Tile tl = decode2(ctl, p, t, g_hint);
+        const bool half = tl.half != 0;
+        const uint32_t tx = 2u * ((half ? A2_HALF_BYTES : A2_BYTES) + 2 * BW_BLOCK_BYTES);
+        const CUtensorMap* amap = half ? &map_a_half : &map_a;
+        const int row0 = tl.lo + tl.m * BM2 + (int)rank * (half ? 64 : 128);
+        const int brow0 = tl.g * p.b_rows + tl.nt * p.n_out + (int)rank * 128;
+        const int brow1 = p.swiglu ? brow0 : brow0 + 256;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_try(smem_u32(&ctl->empty[stage]), phase ^ 1u) &&
+              !mbar_wait2(&ctl->empty[stage], phase ^ 1u, ctl, p.status)) {
+            aborted = true;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGEW_BYTES;
+          const uint32_t leader_full = map_to_rank(&ctl->full[stage], 0);
+          if (rank == 0) mbar_expect_tx(&ctl->full[stage], tx);
+          tma_load_2d_pair(sa, amap, leader_full, kb * BK, row0);
+          tma_load_2d_pair(sa + A2_BYTES, &map_b, leader_full, kb * BK, brow0);
+          tma_load_2d_pair(sa + A2_BYTES + BW_BLOCK_BYTES, p.swiglu ? &map_b2 : &map_b, leader_full, kb * BK, brow1);
+          if (++stage == STAGESW) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer (leader CTA) =================
+    if (lane == 0 && rank == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t idesc_full = idesc_bf16_pair(BM2, BN_MAX);
+      const uint32_t idesc_half = idesc_bf16_pair(BM2 / 2, BN_MAX);
+      bool issued = false;
+      int g_hint = 0;
+      for (int i = 0; !aborted; ++i) {
+        const int t = take_tile(ctl, i, 0, p);
+        if (t < 0) {
+          aborted = true;
+          break;
+        }
+        if (t >= total) break;
+        const uint32_t idesc = decode2(ctl, p, t, g_hint).half ? idesc_half : idesc_full;
+        if (!mbar_wait2(&ctl->tmem_empty[0], (uint32_t)(i & 1) ^ 1u, ctl, p.status)) {
+          aborted = true;
+          break;
+        }
+        fence_after();
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_try(smem_u32(&ctl->full[stage]), phase) && !mbar_wait2(&ctl->full[stage], phase, ctl, p.status)) {
+            aborted = true;
+            break;
+          }
+          const uint32_t sa = smem_u32(smem + stage * STAGEW_BYTES);
+          const uint64_t adesc = sw128_desc(sa);
+          const uint64_t bdesc0 = sw128_desc(sa + A2_BYTES);
+          const uint64_t bdesc1 = sw128_desc(sa + A2_BYTES + BW_BLOCK_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint32_t acc = (kb | k) != 0;
+            mma_bf16_pair(tmem_base, adesc + (uint64_t)(2 * k), bdesc0 + (uint64_t)(2 * k), idesc, acc);
+            mma_bf16_pair(tmem_base + 256u, adesc + (uint64_t)(2 * k), bdesc1 + (uint64_t)(2 * k), idesc, acc);
+          }
+          issued = true;
+          mma_commit_pair(&ctl->empty[stage]);
+          if (++stage == STAGESW) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (aborted) break;
+        mma_commit_pair(&ctl->tmem_full[0]);
+      }
+      if (aborted && issued) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(&ctl->drain))
+                     : "memory");
+        mbar_drain(&ctl->drain, 0);
+      }
+    }
+  } else {
+    // ================= epilogue (warps 2..9, both CTAs) =================
+    // Lane quarter q = warp % 4 (the TMEM lanes this warp may read), column half hh.
+    // Full tile: lane = row 128r + 32q + lane. Half tile: quarters 0-1 hold MMA columns
+    // [0, 128) and quarters 2-3 columns [128, 256) of each MMA, for rows 64r + 32(q & 1) + lane,
+    // at TMEM columns [0, 128) (MMA 0) and [256, 384) (MMA 1).
+    const int q = warp & 3;
+    const int hh = (warp - 2) >> 2;
+    const uint32_t leader_tmem_empty = map_to_rank(&ctl->tmem_empty[0], 0);
+    int g_hint = 0;
+    for (int i = 0;; ++i) {
+      int t = 0;
+      if (lane == 0) t = take_tile(ctl, i, rank, p);
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (t < 0) {
+        aborted = true;
+        break;
+      }
+      if (t >= total) break;
+      const Tile tl = decode2(ctl, p, t, g_hint);
+      const bool half = tl.half != 0;
+      const bool got = mbar_wait2(&ctl->tmem_full[0], (uint32_t)(i & 1), ctl, p.status);
+      __syncwarp();
+      if (!got) {
+        aborted = true;
+        break;
+      }
+      fence_after();
+      const int row_in_tile = half ? (int)rank * 64 + (q & 1) * 32 + lane : (int)rank * 128 + q * 32 + lane;
+      const int64_t row = (int64_t)tl.lo + tl.m * BM2 + row_in_tile;
+      const bool valid = row < tl.hi;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16);
+      const int tile_col = tl.nt * p.n_out;
+      if (p.swiglu) {
+        // output column j of the tile: gate at MMA-0 column j, up at MMA-1 column j
+        const int j0 = half ? (q >> 1) * 128 + hh * 64 : hh * 128;
+        const int nj = half ? 64 : 128;
+        const uint32_t tcol = half ? (uint32_t)(hh * 64) : (uint32_t)(hh * 128);
+        for (int c = 0; c < nj; c += 16) {
+          float gv[16], uv[16];
+          tmem_ld16(taddr + tcol + (uint32_t)c, gv);
+          tmem_ld16(taddr + 256u + tcol + (uint32_t)c, uv);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) gv[e] = silu(gv[e]) * uv[e];
+          if (valid && tile_col + j0 + c < p.N) store16(p.C, p.ldc, row, tile_col + j0 + c, p.N, gv, false);
+        }
+      } else {
+        // output column j < 256 at MMA-0 column j, j >= 256 at MMA-1 column j - 256
+        const int j0 = half ? hh * 256 + (q >> 1) * 128 : hh * 256;
+        const int nj = half ? 128 : 256;
+        const uint32_t tcol = (uint32_t)(hh * 256);
+        for (int c = 0; c < nj; c += 16) {
+          float v[16];
+          tmem_ld16(taddr + tcol + (uint32_t)c, v);
+          if (valid && tile_col + j0 + c < p.N) store16(p.C, p.ldc, row, tile_col + j0 + c, p.N, v, p.out_f32 != 0);
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tmem_empty);
+    }
+  }
+
+  if (*reinterpret_cast<volatile int32_t*>(&ctl->abort)) spin_ns(1000000);  // let copies in flight land
+  fence_before();
+  __syncthreads();
+  __syncwarp();
+  cluster_sync();
+  fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
 // ---- host side -----------------------------------------------------------------
 // 2-D bf16 tensor [rows, cols] (cols contiguous), box [box_rows, 64], 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int box_rows) {
@@ -796,26 +1042,37 @@ int num_sms() {
   return sms;
 }
 
-// Clusters of two gemm_tc2_kernel CTAs that fit on the device at once, per device.
-int max_resident_pairs(const cudaLaunchConfig_t& cfg) {
-  static int cached[64] = {0};
+// Clusters of two CTAs of a pair kernel (gemm_tc2_kernel, or the wide gemm_tc2w_kernel) that fit
+// on the device at once, per device.
+int max_resident_pairs(const cudaLaunchConfig_t& cfg, bool wide) {
+  static int cached[2][64] = {{0}};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return 0;
-  if (!cached[dev]) {
+  if (!cached[wide][dev]) {
     cudaLaunchConfig_t q = cfg;
     q.gridDim = dim3((unsigned)num_sms(), 1, 1);
     int clusters = 0;
-    if (cudaOccupancyMaxActiveClusters(&clusters, (void*)gemm_tc2_kernel, &q) != cudaSuccess || clusters <= 0)
+    if (cudaOccupancyMaxActiveClusters(&clusters, wide ? (void*)gemm_tc2w_kernel : (void*)gemm_tc2_kernel, &q) !=
+            cudaSuccess ||
+        clusters <= 0)
       return 0;
-    cached[dev] = clusters;
+    cached[wide][dev] = clusters;
   }
-  return cached[dev];
+  return cached[wide][dev];
 }
 
 constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(SmemCtl);
 constexpr size_t kSmemBytes2 = 1024 + STAGES2 * STAGE2_BYTES + sizeof(SmemCtl2);
-static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448, "dynamic shared memory above 227 KB");
+constexpr size_t kSmemBytesW = 1024 + STAGESW * STAGEW_BYTES + sizeof(SmemCtl2);
+static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448 && kSmemBytesW <= 232448,
+              "dynamic shared memory above 227 KB");
+
+// Wide pair tiles (256 x 512): MOE_TC_WIDE=1 selects them for the SM-pair GEMMs.
+bool use_wide_tiles() {
+  const char* w = getenv("MOE_TC_WIDE");
+  return w && w[0] == '1';
+}
 
 // SM-pair tiles stage fewer bytes per FLOP and, with half-height last tiles,
 // pad groups to 128 rows like the single-SM tiles; they are used once groups
@@ -902,11 +1159,44 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
   CUtensorMap ma_half;
   if (pair && !make_map(&ma_half, a.A, a.M, a.K, BM / 2)) return cudaErrorInvalidValue;
-  if (!make_map(&mb, a.B, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
+  const bool wide = pair && use_wide_tiles();
+  const int b_box_used = wide ? 128 : b_box;
+  if (!make_map(&mb, a.B, b_total_rows, a.K, b_box_used)) return cudaErrorInvalidValue;
   if (swiglu) {
-    if (!make_map(&mb2, a.B2, b_total_rows, a.K, b_box)) return cudaErrorInvalidValue;
+    if (!make_map(&mb2, a.B2, b_total_rows, a.K, b_box_used)) return cudaErrorInvalidValue;
   } else {
     mb2 = mb;
+  }
+  if (wide) {
+    // 256 outputs per tile for SwiGLU (gate and up of 256 columns), 512 for plain tiles
+    p.n_out = swiglu ? 256 : 512;
+    static std::atomic<uint64_t> attrw{0};
+    {
+      const cudaError_t e = set_smem_limit(attrw, (const void*)gemm_tc2w_kernel, kSmemBytesW);
+      if (e != cudaSuccess) return e;
+    }
+    const int64_t max_tiles_w = (ceil_div(a.M, BM2) + (a.offsets ? a.G : 0)) * ceil_div(a.N, p.n_out);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kThreadsW, 1, 1);
+    cfg.dynamicSmemBytes = kSmemBytesW;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (!a.tile_counter) return cudaErrorInvalidValue;
+    {
+      const cudaError_t e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s);
+      if (e != cudaSuccess) return e;
+    }
+    const int pairs_resident = max_resident_pairs(cfg, true);
+    if (pairs_resident <= 0) return cudaErrorInvalidConfiguration;
+    const int64_t pairs = max_tiles_w < pairs_resident ? max_tiles_w : pairs_resident;
+    cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+    return cudaLaunchKernelEx(&cfg, gemm_tc2w_kernel, ma, ma_half, mb, mb2, p);
   }
   const int64_t n_tiles_all = ceil_div(a.N, p.n_out);
   if (pair) {
@@ -936,7 +1226,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
       const cudaError_t e = cudaMemsetAsync(a.tile_counter, 0, sizeof(int32_t), s);
       if (e != cudaSuccess) return e;
     }
-    const int pairs_resident = max_resident_pairs(cfg);
+    const int pairs_resident = max_resident_pairs(cfg, false);
     if (pairs_resident <= 0) return cudaErrorInvalidConfiguration;
     const int64_t pairs = max_pair_tiles < pairs_resident ? max_pair_tiles : pairs_resident;
     cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);

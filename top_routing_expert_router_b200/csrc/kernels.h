@@ -136,7 +136,7 @@ struct CapacityArgs {
   moe_diag* status;         // MOE_ERR_TIMEOUT if a grid barrier wait runs out
 };
 int64_t capacity_grid_scratch_bytes(int64_t n, int32_t E);
-bool capacity_grid_fits(int64_t n, int32_t k);
+bool capacity_grid_fits(int64_t n, int32_t E);
 cudaError_t launch_capacity_grid(const CapacityArgs& a, void* scratch, cudaStream_t s);
 // Capacity rule over the ranking; writes topk_idx and the overflow/drop counts.
 cudaError_t launch_capacity(const uint16_t* ranking, int64_t n, int32_t E, int32_t k, int64_t C, int policy,

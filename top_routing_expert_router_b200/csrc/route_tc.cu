@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       float amax = 0.0f, m = -INFINITY, z = 0.0f;
       float g1 = -INFINITY, g2 = -INFINITY;
       float gsc[kMaxGroups];
+      int gpos = 0, gidx = 0;  // place inside the current group, and the group (experts arrive in order)
       for (int c0 = 0; c0 < E; c0 += 32) {
         float l[32];
         tmem_ld32(taddr + (uint32_t)c0, l);
@@ -292,9 +293,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               } else if (v > g2) {
                 g2 = v;
               }
-              if ((e + 1) % per == 0) {
-                gsc[e / per] = g1 + g2;
+              if (++gpos == per) {
+                gsc[gidx++] = g1 + g2;
                 g1 = g2 = -INFINITY;
+                gpos = 0;
               }
             }
           }
@@ -331,17 +333,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int n_elig = 0;
       for (int c0 = 0; c0 < E; c0 += 32) {
+        int g = c0 / per, r = c0 - g * per;  // group of expert c0 and its place in the group
         // skip a chunk that lies in a dropped group of every token of the warp (TMEM loads are warp-wide)
-        if (per >= 32 && !__any_sync(0xFFFFFFFFu, (kept >> (c0 / per)) & 1u)) continue;
+        if (per >= 32 && r + 32 <= per && !__any_sync(0xFFFFFFFFu, (kept >> g) & 1u)) continue;
         float l[32];
         tmem_ld32(taddr + (uint32_t)c0, l);
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
           const int e = c0 + j;
-          if (e < E && ((kept >> (e / per)) & 1u)) {
+          if (e < E && ((kept >> g) & 1u)) {
             ++n_elig;
             const float v = soft ? l[j] : raw_score32(p.score_fn, l[j]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
             insert(lv, ll, le, v, l[j], e);
+          }
+          if (++r == per) {
+            r = 0;
+            ++g;
           }
         }
       }
