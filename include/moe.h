@@ -285,7 +285,7 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* 
  *   is required here (see below). `stream` must belong to the current device.
  *   Returns MOE_ERR_WORKSPACE when this cfg and n need more scratch than the
  *   array holds (E * 4 bytes of logits per token dominate, plus E * 2 bytes of
- *   ranking under a capacity; e.g. E = 256 fits about 8000 tokens, E = 8 about
+ *   ranking under a capacity; e.g. E = 256 fits about 7000 tokens, E = 8 about
  *   200000), MOE_ERR_INVALID_ARG for a NULL diag or a stream of another device,
  *   MOE_ERR_CUDA if the array's device address cannot be found, and the errors
  *   of moe_route otherwise.

@@ -19,7 +19,7 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Workspace layout; every region starts on a 256-byte boundary.
 struct Plan {
-  size_t diag, logits, rq, ranking, capg, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
+  size_t diag, logits, rq, rc, ranking, capg, blk, idx, w, counts, offsets, perm, dest, xperm, h, eo, shh, sh, shoff, sched;
   size_t xq, sfx, hq, sfh, xsq, sfxs, hsq, sfhs;  // FP8 experts: E4M3 activations and their scale blocks
   size_t sfb, sfbs;  // FP8 SM-pair GEMMs: B scale blocks (routed, shared experts)
   size_t ep_off;  // expert parallelism: receive offsets of the rank's own experts
@@ -76,6 +76,7 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   p.diag = take(sizeof(moe_diag));
   p.logits = take((size_t)router_splits(c, n) * n * logits_ld(c) * 4);
   p.rq = take((size_t)n * 4);  // tokens the one-pass router leaves to the binary64 router
+  p.rc = take((size_t)n * (kRouteCandMax + 1) * 4);  // and the experts to refine for each
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
   p.capg = take(c.cap_policy != MOE_CAP_NONE ? (size_t)capacity_grid_scratch_bytes(n, c.n_routed) : 0);
   p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
@@ -286,6 +287,7 @@ bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* i
   a.ldl = logits_ld(c);
   a.queue = x.at<int32_t>(x.p.rq);
   a.queue_len = &x.status()->reserved[1];
+  a.cand = x.at<int32_t>(x.p.rc);
   a.status = x.status();
   if (!route_tc_supported(a)) return false;
   *ra = a;
@@ -315,6 +317,7 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     r.cursor = cursor;
     r.queue = ra.queue;
     r.queue_len = ra.queue_len;
+    r.cand = ra.cand;
     MOE_CUDA(launch_route(r, x.s));
   } else if (c.cap_policy == MOE_CAP_NONE) {
     MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));

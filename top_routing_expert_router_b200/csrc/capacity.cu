@@ -33,6 +33,11 @@ constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kThreads = 1024;  // tokens per CTA
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
 constexpr int kNone = 0x7FFFFFFF;
+constexpr int kPrefix = 64;  // ranking entries per token staged in shared memory
+
+// 32-bit words per staged ranking prefix of P entries: enough for P and odd, so that lanes reading
+// the same position of their rows hit 32 different banks.
+__host__ __device__ constexpr int prefix_words(int P) { return ((P + 1) / 2) | 1; }
 
 // Global state of one round, double-buffered by round parity (CTAs still reading round r's
 // copy while CTA b* writes round r + 1's).
@@ -140,10 +145,31 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   __shared__ uint32_t nfull_s[kMaxExperts / 32];
   __shared__ int s_bstar, s_tloc;
   __shared__ unsigned long long s_over, s_drop;
-  extern __shared__ int hist_all[];           // [gridDim.x][E]: every CTA's counts of this round
+  extern __shared__ int hist_all[];           // [gridDim.x][E]: every CTA's counts of this round, then
+                                              // the tokens' ranking prefixes (kPrefix entries, odd word stride)
   const int64_t t = (int64_t)blockIdx.x * kThreads + tid;
   const bool valid = t < a.n;
   const uint16_t* row = a.ranking + (valid ? t : 0) * E;
+  // the first P entries of this token's ranking in shared memory: a token walking past full experts
+  // reads them at shared-memory latency instead of one dependent global load per step
+  const int P = E < kPrefix ? E : kPrefix;
+  uint32_t* srow32 = reinterpret_cast<uint32_t*>(hist_all + gridDim.x * E) + tid * prefix_words(P);
+  const uint16_t* srow = reinterpret_cast<const uint16_t*>(srow32);
+  if (valid) {
+    if (E % 8 == 0) {
+      const uint4* src = reinterpret_cast<const uint4*>(row);
+      for (int v = 0; v < P / 8; ++v) {
+        const uint4 q4 = src[v];
+        srow32[4 * v] = q4.x;
+        srow32[4 * v + 1] = q4.y;
+        srow32[4 * v + 2] = q4.z;
+        srow32[4 * v + 3] = q4.w;
+      }
+    } else {
+      uint16_t* d16 = reinterpret_cast<uint16_t*>(srow32);
+      for (int c = 0; c < P; ++c) d16[c] = row[c];
+    }
+  }
   uint32_t gen = 0;
   Slots<KA, (KT > 0)> ch, pos;
   int taken = 0, cursor = 0;
@@ -156,7 +182,7 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   // walk on from the cursor until k non-full experts are held
   auto refill = [&]() {
     while (taken < k && cursor < E) {
-      const int e = row[cursor];
+      const int e = cursor < P ? srow[cursor] : row[cursor];
       if (e == 0xFFFF) {
         cursor = E;
         break;
@@ -178,7 +204,7 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
       refill();
     } else {
       for (int j = 0; j < k; ++j) {
-        const int e = row[j];
+        const int e = j < P ? srow[j] : row[j];
         ch.set(j, e != 0xFFFF ? e : -1);
       }
     }
@@ -328,8 +354,12 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   }
 }
 
-// Dynamic shared memory of a grid of `grid` CTAs: every CTA's row of per-expert counts.
-size_t dyn_smem(unsigned grid, int E) { return (size_t)grid * E * sizeof(int); }
+// Dynamic shared memory of a grid of `grid` CTAs: every CTA's row of per-expert counts, and the
+// staged ranking prefixes of the CTA's tokens.
+size_t dyn_smem(unsigned grid, int E) {
+  const int P = E < kPrefix ? E : kPrefix;
+  return (size_t)grid * E * sizeof(int) + (size_t)kThreads * prefix_words(P) * sizeof(uint32_t);
+}
 
 template <int KT>
 cudaError_t launch_t(CapacityArgs a, GridCtl* g, unsigned grid, cudaStream_t s) {

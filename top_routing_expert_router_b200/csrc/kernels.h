@@ -97,8 +97,11 @@ struct RouteArgs {
   int32_t* cursor;      // zeroed before the launch: next token to route (warps fetch tokens from it)
   const int32_t* queue = nullptr;      // when set: route only the tokens queue[0 .. *queue_len)
   const int32_t* queue_len = nullptr;
+  const int32_t* cand = nullptr;       // with queue: experts to recompute in binary64 first (RouteTcArgs::cand)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+
+constexpr int kRouteCandMax = 32;
 
 // Router in one pass (route_tc.cu): logits on the tensor cores and the routing decision of each
 // token in the epilogue, in binary32; tokens whose decision is not certain get their logits row
@@ -116,6 +119,8 @@ struct RouteTcArgs {
   int64_t ldl;
   int32_t* queue;       // [n] tokens left to the binary64 router
   int32_t* queue_len;   // zeroed before the launch
+  int32_t* cand;        // [n][kRouteCandMax + 1] per queued token: count (-1: too many), then the experts
+                        // an uncertain comparison can involve
   moe_diag* status;
 };
 bool route_tc_supported(const RouteTcArgs& a);

@@ -18,10 +18,12 @@
 //               stage, 4-stage ring of 128-byte-swizzled shared memory;
 //   warp 1      TMEM owner (two 128 x 256 fp32 accumulators) and MMA issuer,
 //               tcgen05.mma kind::f16, M = 128, N = E rounded up to 16;
-//   warps 2..5  routing epilogue: thread i of lane quarter q owns token row
-//               32q + i, reads its E logits from TMEM 32 columns at a time and
-//               decides in binary32: group scores, group cut, the k best
-//               eligible experts kept sorted by insertion, gates.
+//   warps 2..9  routing epilogue: two warps per TMEM lane quarter q, thread i
+//               of each owning token row 32q + i, each half of its experts; they
+//               read the logits from TMEM 32 columns at a time and decide in
+//               binary32: group scores, group cut, the k best eligible experts
+//               kept sorted by insertion, gates (partials exchanged through
+//               shared memory, half 0 finishing).
 // Exactness: the logits are binary32 sums, so a decision is kept only when
 // every gap it depends on (group cut, adjacent kept experts, the k-th / (k+1)-th
 // cut) exceeds twice the error bound of the selection values; any other token
@@ -46,10 +48,14 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_MAX_BYTES = 256 * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_MAX_BYTES;
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;  // producer, MMA issuer, 8 epilogue warps
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int kMaxK = 8;  // experts per token the epilogue keeps sorted in registers
+constexpr int kCandMax = kRouteCandMax;  // experts listed for the binary64 refinement of a queued token
 constexpr uint64_t kTimeoutNs = 2000000000ull;
+constexpr int kXg = 2 + 16;                 // per token and half: |l| max, logit max, 16 group scores
+constexpr int kXl = 3 * (kMaxK + 1) + 2;     // per token: half 1's list (values, logits, experts), count, softmax sum
+constexpr int XCHG_BYTES = (2 * BM * kXg + BM * kXl + 256) * 4;  // and the selection bias
 
 struct __align__(8) Ctl {
   uint64_t full[STAGES];
@@ -104,6 +110,14 @@ __device__ __forceinline__ float raw_score32(int score_fn, float l) {
   return 1.0f / (1.0f + expf(-l));
 }
 
+// Selection score of the biased routers in the epilogue's fast form: sigmoid from ex2.approx and a
+// correctly rounded reciprocal (absolute error below 2^-18 for any logit, which the certification
+// margin adds); sqrtsoftplus in the accurate form.
+__device__ __forceinline__ float sel_score(int score_fn, float l) {
+  if (score_fn == MOE_SCORE_SIGMOID) return __frcp_rn(1.0f + __expf(-l));
+  return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
+}
+
 // Insert (v, l, e) into the list sorted by v descending; an equal v stays below the entries
 // already there, which hold lower expert indices (experts arrive in ascending order).
 __device__ __forceinline__ void insert(float (&lv)[kMaxK + 1], float (&ll)[kMaxK + 1], int (&le)[kMaxK + 1], float v,
@@ -130,6 +144,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   Ctl* ctl = reinterpret_cast<Ctl*>(smem + STAGES * STAGE_BYTES);
+  float* xg = reinterpret_cast<float*>(smem + STAGES * STAGE_BYTES + 256);  // partials of the two halves
+  float* xl = xg + 2 * BM * kXg;                                            // half 1's candidate lists
+  volatile int32_t* vote = reinterpret_cast<volatile int32_t*>(smem + STAGES * STAGE_BYTES + 128);
+  float* sbias = xl + BM * kXl;                                             // selection bias (0 without)
+  for (int e = threadIdx.x; e < 256; e += kThreads) sbias[e] = (p.bias && e < p.E) ? p.bias[e] : 0.0f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n_tiles = (int)((p.n + BM - 1) / BM);
   const int num_kb = (p.d + BK - 1) / BK;
@@ -143,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&ctl->tmem_full[b], 1);
-      mbar_init(&ctl->tmem_empty[b], 4);
+      mbar_init(&ctl->tmem_empty[b], 8);
     }
     mbar_init(&ctl->drain, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -246,83 +265,138 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ================= routing epilogue (warps 2..5) =================
+    // ================= routing epilogue (warps 2..9) =================
+    // Two warps per TMEM lane quarter q (the lanes a warp may read): both own the token rows
+    // 32q .. 32q + 31, half 0 the experts [0, e_split), half 1 the rest (a whole number of groups
+    // each). They exchange their partial group scores and softmax sums, decide the group cut
+    // redundantly, each keep their k + 1 best eligible experts, and half 0 merges the two lists,
+    // certifies and writes the token's routing.
     const int q = warp & 3;
+    const int h = (warp - 2) >> 2;
     const int E = p.E, G = p.G, per = p.E / p.G, k = p.k;
     const bool soft = p.score_fn == MOE_SCORE_SOFTMAX;
+    const int Gh = G > 1 ? (G + 1) / 2 : 1;  // groups of half 0
+    const int e_split = G > 1 ? Gh * per : min(E, ((E / 2 + 31) / 32) * 32);
+    const int e_lo = h ? e_split : 0, e_hi = h ? E : e_split;
+    const int g_lo = h ? Gh : 0;
     // derivative bound of the selection value in the logit (sigmoid' <= 1/4, sqrtsoftplus' < 1/2)
     const float lip = p.score_fn == MOE_SCORE_SIGMOID ? 0.25f : p.score_fn == MOE_SCORE_SQRTSOFTPLUS ? 0.5f : 1.0f;
     // binary32 evaluation error of a non-softmax selection value (a few ulp of a value near 1)
-    const float eval_err = soft ? 0.0f : 0x1p-20f;
+    const float eval_err = soft ? 0.0f : 0x1p-18f;
+    // whole 32-expert chunks per half and groups of whole chunks: the loops need no per-expert checks
+    const bool fast = E % 32 == 0 && e_split % 32 == 0 && (G == 1 || per % 32 == 0);
+    const int row = q * 32 + lane;
+    float* xg_mine = xg + ((size_t)h * BM + row) * kXg;
+    const float* xg_other = xg + ((size_t)(h ^ 1) * BM + row) * kXg;
+    float* xl_row = xl + (size_t)row * kXl;
+    auto pair_sync = [&]() { asm volatile("bar.sync %0, %1;" ::"r"(1 + q), "r"(64) : "memory"); };
     int i = 0;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
       const int buf = i & 1;
       const uint32_t acc_phase = (uint32_t)(i >> 1) & 1u;
+      // both warps of the pair go on or stop together (a named barrier waits for both)
       const bool got = wait_bar(&ctl->tmem_full[buf], acc_phase, ctl, p.status);
       __syncwarp();
-      if (!got) break;
+      if (lane == 0) vote[h * 4 + q] = got ? 1 : 0;
+      pair_sync();
+      if (!(vote[q] && vote[4 + q])) break;
       fence_after();
-      const int64_t tok = (int64_t)t * BM + q * 32 + lane;
+      const int64_t tok = (int64_t)t * BM + row;
       const bool valid = tok < p.n;
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256);
-      // pass 1: |l| max, softmax max and normaliser, group scores (top-2 sums of c)
-      float amax = 0.0f, m = -INFINITY, z = 0.0f;
-      float g1 = -INFINITY, g2 = -INFINITY;
-      float gsc[kMaxGroups];
-      int gpos = 0, gidx = 0;  // place inside the current group, and the group (experts arrive in order)
-      for (int c0 = 0; c0 < E; c0 += 32) {
-        float l[32];
-        tmem_ld32(taddr + (uint32_t)c0, l);
+      // pass 1 over this half's experts: |l| max, softmax max, group scores (top-2 sums of c)
+      float amax = 0.0f, m = -INFINITY;
+      if (fast) {
+        // whole 32-expert chunks, groups of whole chunks: no per-expert range or group checks
+        float g1 = -INFINITY, g2 = -INFINITY;
+        for (int c0 = e_lo; c0 < e_hi; c0 += 32) {
+          float l[32];
+          tmem_ld32(taddr + (uint32_t)c0, l);
+          if (soft || G == 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c0 + j;
-          if (e < E) {
-            amax = fmaxf(amax, fabsf(l[j]));
-            if (soft) {
-              if (l[j] > m) {
-                z = z * expf(m - l[j]) + 1.0f;
-                m = l[j];
-              } else {
-                z += expf(l[j] - m);
-              }
-            } else if (G > 1) {
-              const float v = raw_score32(p.score_fn, l[j]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
-              if (v > g1) {
-                g2 = g1;
-                g1 = v;
-              } else if (v > g2) {
-                g2 = v;
-              }
-              if (++gpos == per) {
-                gsc[gidx++] = g1 + g2;
-                g1 = g2 = -INFINITY;
-                gpos = 0;
+            for (int j = 0; j < 32; ++j) {
+              amax = fmaxf(amax, fabsf(l[j]));
+              m = fmaxf(m, l[j]);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              amax = fmaxf(amax, fabsf(l[j]));
+              const float v = sel_score(p.score_fn, l[j]) + sbias[c0 + j];
+              g2 = fmaxf(g2, fminf(g1, v));
+              g1 = fmaxf(g1, v);
+            }
+            if ((c0 + 32) % per == 0) {
+              xg_mine[2 + (c0 / per) - g_lo] = g1 + g2;
+              g1 = g2 = -INFINITY;
+            }
+          }
+        }
+      } else {
+        float g1 = -INFINITY, g2 = -INFINITY;
+        int gpos = 0, gidx = 0;  // place inside the current group, and the group (experts arrive in order)
+        for (int c0 = e_lo & ~31; c0 < e_hi; c0 += 32) {
+          float l[32];
+          tmem_ld32(taddr + (uint32_t)c0, l);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c0 + j;
+            if (e >= e_lo && e < e_hi) {
+              amax = fmaxf(amax, fabsf(l[j]));
+              m = fmaxf(m, l[j]);
+              if (!soft && G > 1) {
+                const float v = sel_score(p.score_fn, l[j]) + sbias[e];
+                g2 = fmaxf(g2, fminf(g1, v));
+                g1 = fmaxf(g1, v);
+                if (++gpos == per) {
+                  xg_mine[2 + gidx++] = g1 + g2;
+                  g1 = g2 = -INFINITY;
+                  gpos = 0;
+                }
               }
             }
           }
         }
       }
+      xg_mine[0] = amax;
+      xg_mine[1] = m;
+      pair_sync();
+      amax = fmaxf(amax, xg_other[0]);
+      m = fmaxf(m, xg_other[1]);
       const float dl = 0x1p-13f * fmaxf(1.0f, amax);  // binary32 error bound of a logit
       const float dv = lip * dl + eval_err;              // ... of a selection value
       // group cut: the topk_group best group scores, ties to the lower group index
       bool ok = true;
-      uint32_t kept = 0xFFFFFFFFu;
+      uint32_t kept = 0xFFFFFFFFu, involved = 0;
       if (!soft && G > 1) {
+        auto gs = [&](int g) { return g < Gh ? (h ? xg_other : xg_mine)[2 + g] : (h ? xg_mine : xg_other)[2 + g - Gh]; };
         kept = 0;
         float min_kept = INFINITY, max_drop = -INFINITY;
         for (int g = 0; g < G; ++g) {
+          const float sg = gs(g);
           int better = 0;
-          for (int h = 0; h < G; ++h) better += (gsc[h] > gsc[g]) || (gsc[h] == gsc[g] && h < g);
+          for (int hh = 0; hh < G; ++hh) {
+            const float so = gs(hh);
+            better += (so > sg) || (so == sg && hh < g);
+          }
           if (better < p.topk_group) {
             kept |= 1u << g;
-            min_kept = fminf(min_kept, gsc[g]);
+            min_kept = fminf(min_kept, sg);
           } else {
-            max_drop = fmaxf(max_drop, gsc[g]);
+            max_drop = fmaxf(max_drop, sg);
           }
         }
-        if (p.topk_group < G && !(min_kept - max_drop > 4.0f * dv + 0x1p-19f)) ok = false;
+        if (p.topk_group < G && !(min_kept - max_drop > 4.0f * dv + 0x1p-19f)) {
+          ok = false;
+          // the groups whose place relative to the cut is uncertain: all their experts are refined
+          for (int g = 0; g < G; ++g) {
+            const float sg = gs(g);
+            const bool in = (kept >> g) & 1u;
+            if (in ? sg <= max_drop + 4.0f * dv + 0x1p-19f : sg >= min_kept - 4.0f * dv - 0x1p-19f) involved |= 1u << g;
+          }
+        }
       }
-      // pass 2: the k + 1 best eligible experts, sorted
+      // pass 2: this half's k + 1 best eligible experts, sorted (and the softmax normaliser)
       float lv[kMaxK + 1], ll[kMaxK + 1];
       int le[kMaxK + 1];
 #pragma unroll
@@ -332,30 +406,88 @@ __global__ void __launch_bounds__(kThreads, 1)
         le[j] = -1;
       }
       int n_elig = 0;
-      for (int c0 = 0; c0 < E; c0 += 32) {
+      float z = 0.0f;
+      for (int c0 = e_lo & ~31; c0 < e_hi; c0 += 32) {
         int g = c0 / per, r = c0 - g * per;  // group of expert c0 and its place in the group
         // skip a chunk that lies in a dropped group of every token of the warp (TMEM loads are warp-wide)
-        if (per >= 32 && r + 32 <= per && !__any_sync(0xFFFFFFFFu, (kept >> g) & 1u)) continue;
+        if (!soft && per >= 32 && r + 32 <= per && !__any_sync(0xFFFFFFFFu, (kept >> g) & 1u)) continue;
         float l[32];
         tmem_ld32(taddr + (uint32_t)c0, l);
+        if (fast) {
+          const bool keptg = (kept >> g) & 1u;  // the whole chunk is in group g
+          n_elig += keptg ? 32 : 0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c0 + j;
-          if (e < E && ((kept >> g) & 1u)) {
-            ++n_elig;
-            const float v = soft ? l[j] : raw_score32(p.score_fn, l[j]) + (p.bias ? __ldg(p.bias + e) : 0.0f);
-            insert(lv, ll, le, v, l[j], e);
+          for (int j = 0; j < 32; ++j) {
+            float v;
+            if (soft) {
+              v = l[j];
+              z += __expf(l[j] - m);
+            } else {
+              v = sel_score(p.score_fn, l[j]) + sbias[c0 + j];
+            }
+            if (keptg && v > lv[kMaxK]) insert(lv, ll, le, v, l[j], c0 + j);
           }
-          if (++r == per) {
-            r = 0;
-            ++g;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const int e = c0 + j;
+            if (e >= e_lo && e < e_hi) {
+              if (soft) z += __expf(l[j] - m);
+              if ((kept >> g) & 1u) {
+                ++n_elig;
+                const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[e];
+                insert(lv, ll, le, v, l[j], e);
+              }
+            }
+            if (++r == per) {
+              r = 0;
+              ++g;
+            }
           }
         }
       }
+      (void)g_lo;
+      if (h == 1) {
+        // hand the list to half 0; this warp is done with the accumulator
+#pragma unroll
+        for (int j = 0; j <= kMaxK; ++j) {
+          xl_row[j] = lv[j];
+          xl_row[kMaxK + 1 + j] = ll[j];
+          xl_row[2 * (kMaxK + 1) + j] = __int_as_float(le[j]);
+        }
+        xl_row[3 * (kMaxK + 1)] = __int_as_float(n_elig);
+        xl_row[3 * (kMaxK + 1) + 1] = z;
+        fence_before();
+        pair_sync();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ctl->tmem_empty[buf]);
+        continue;
+      }
+      pair_sync();
+      {
+        // merge the other half's list (higher expert indices: on equal values this half's come first)
+        float ov[kMaxK + 1], ol[kMaxK + 1];
+        int oe[kMaxK + 1];
+#pragma unroll
+        for (int j = 0; j <= kMaxK; ++j) {
+          ov[j] = xl_row[j];
+          ol[j] = xl_row[kMaxK + 1 + j];
+          oe[j] = __float_as_int(xl_row[2 * (kMaxK + 1) + j]);
+        }
+        n_elig += __float_as_int(xl_row[3 * (kMaxK + 1)]);
+        z += xl_row[3 * (kMaxK + 1) + 1];
+#pragma unroll
+        for (int j = 0; j <= kMaxK; ++j) insert(lv, ll, le, ov[j], ol[j], oe[j] < 0 ? 0x7FFFFFFF : oe[j]);
+      }
       // every order the result depends on must be certain: adjacent kept experts and the k-th / (k+1)-th cut
+      // (and the lowest selection value an expert needs to take part in an uncertain one)
+      float thr = INFINITY;
 #pragma unroll
       for (int j = 0; j < kMaxK; ++j)
-        if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) ok = false;
+        if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) {
+          ok = false;
+          thr = fminf(thr, (j + 1 < k ? lv[j + 1] : lv[j]) - 2.0f * dv);
+        }
       const bool spill = valid && !ok;
       if (valid && ok) {
         // gates of the k kept experts
@@ -384,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // not certain: hand the token to the binary64 router with its logits row (the TMEM loads are
       // warp-wide, so the whole warp reads when any lane spills)
       if (__any_sync(0xFFFFFFFFu, spill)) {
-        float* row = p.logits + tok * p.ldl;
+        float* lrow = p.logits + tok * p.ldl;
         for (int c0 = 0; c0 < E; c0 += 32) {
           float l[32];
           tmem_ld32(taddr + (uint32_t)c0, l);
@@ -392,15 +524,51 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
               if (c0 + j + 4 <= E) {
-                *reinterpret_cast<float4*>(row + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
+                *reinterpret_cast<float4*>(lrow + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
               } else {
 #pragma unroll
                 for (int u = 0; u < 4; ++u)
-                  if (c0 + j + u < E) row[c0 + j + u] = l[j + u];
+                  if (c0 + j + u < E) lrow[c0 + j + u] = l[j + u];
               }
           }
         }
-        if (spill) p.queue[atomicAdd(p.queue_len, 1)] = (int32_t)tok;
+        // the experts an uncertain comparison can involve: eligible ones at or above thr, and every
+        // expert of a group near an uncertain group cut; the binary64 router refines them first
+        int32_t* cand = nullptr;
+        if (spill) {
+          const int qpos = atomicAdd(p.queue_len, 1);
+          p.queue[qpos] = (int32_t)tok;
+          cand = p.cand + (int64_t)qpos * (kCandMax + 1);
+        }
+        int nc = 0;
+        for (int c0 = 0; c0 < E; c0 += 32) {
+          float l[32];
+          tmem_ld32(taddr + (uint32_t)c0, l);
+          if (spill) {
+            int g = c0 / per, r = c0 - g * per;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int e = c0 + j;
+              if (e < E) {
+                const bool el = (kept >> g) & 1u;
+                bool want = (involved >> g) & 1u;
+                if (!want && el && thr != INFINITY) {
+                  const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[e];
+                  want = v >= thr;
+                }
+                if (want) {
+                  if (nc < kCandMax) cand[1 + nc] = e;
+                  ++nc;
+                }
+              }
+              if (++r == per) {
+                r = 0;
+                ++g;
+              }
+            }
+          }
+        }
+        if (spill) cand[0] = nc <= kCandMax ? nc : -1;  // -1: too many, the router finds them itself
       }
       fence_before();
       __syncwarp();
@@ -429,7 +597,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + sizeof(Ctl);
+static_assert(sizeof(Ctl) <= 128, "control block");
+constexpr size_t kSmemBytes = 1024 + STAGES * STAGE_BYTES + 256 + XCHG_BYTES;
 static_assert(kSmemBytes <= 232448, "dynamic shared memory above 227 KB");
 
 }  // namespace
@@ -438,6 +607,7 @@ bool route_tc_supported(const RouteTcArgs& a) {
   const char* inj = getenv("MOE_TEST_NO_TENSOR_MAPS");
   if (inj && inj[0] == '1') return false;
   if (a.E < 1 || a.E > 256 || a.k < 1 || a.k > kMaxK || a.G < 1 || a.G > kMaxGroups || a.E % a.G != 0) return false;
+  if ((a.G + 1) / 2 > 16) return false;  // group scores of a half in the exchange block
   if (a.d % 8 != 0 || a.ldl % 4 != 0 || a.ldl < a.E) return false;
   if (reinterpret_cast<uintptr_t>(a.x) % 16 || reinterpret_cast<uintptr_t>(a.w_r) % 16 ||
       reinterpret_cast<uintptr_t>(a.logits) % 16)

@@ -602,6 +602,21 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     uint32_t exact = 0;
     int nr = 0;
     int n_refined = 0;
+    if (a.cand) {
+      // experts the one-pass router found near a decision boundary: binary64 first, all at once
+      const int32_t* c = a.cand + i * (kRouteCandMax + 1);
+      const int nc = c[0];
+      if (nc > 0) {
+        uint32_t which = 0;
+        for (int q = 0; q < nc; ++q) {
+          const int e = c[1 + q];
+          if ((e & 31) == lane) which |= 1u << (e >> 5);
+        }
+        which &= valid_mask;
+        n_refined += refine_logits<EPL>(a, t, l, which);
+        exact |= which;
+      }
+    }
     for (int it = 0;; ++it) {
       uint32_t refine = 0;
       bool ok;
