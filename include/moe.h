@@ -68,6 +68,10 @@
  *     group index. Dropped slots carry index -1, weight 0 and slot_dest -1.
  *   - Environment variables, read at each call (none is needed):
  *     MOE_TC_MODE=1sm|2sm forces the one-SM or SM-pair bf16 expert GEMM;
+ *     MOE_TC_WIDE=1|gate gives the SM-pair bf16 GEMMs (all, or the gate/up one
+ *     only) 256 x 512 tiles instead of 256 x 256;
+ *     MOE_CAP_MODE=1cta runs the capacity rule on one CTA instead of the
+ *     cooperative grid;
  *     MOE_FP8_BN=128|256|pair|s128|s256 forces an FP8 expert GEMM tile shape
  *     (one-SM 128-row tiles of that width, SM-pair tiles, or 32-row tiles where
  *     the rows per expert allow them); these exist for tuning and tests, and
@@ -285,8 +289,10 @@ moe_status moe_bias_update(const moe_config* cfg, const int32_t* counts, float* 
  *   is required here (see below). `stream` must belong to the current device.
  *   Returns MOE_ERR_WORKSPACE when this cfg and n need more scratch than the
  *   array holds (E * 4 bytes of logits per token dominate, plus E * 2 bytes of
- *   ranking under a capacity; e.g. E = 256 fits about 7000 tokens, E = 8 about
- *   200000), MOE_ERR_INVALID_ARG for a NULL diag or a stream of another device,
+ *   ranking under a capacity, or about 0.5 KB for the queue of tokens re-decided
+ *   in binary64 when bf16 batches of n >= 2048 route without a capacity; e.g.
+ *   E = 256 fits about 5400 tokens, E = 8 about 200000),
+ *   MOE_ERR_INVALID_ARG for a NULL diag or a stream of another device,
  *   MOE_ERR_CUDA if the array's device address cannot be found, and the errors
  *   of moe_route otherwise.
  *   The first call on each device performs a one-time set-up that looks up the

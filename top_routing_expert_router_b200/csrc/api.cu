@@ -55,6 +55,15 @@ int router_splits(const moe_config& c, int64_t n) {
   return (int)ceil_div(num_kb, kb_per);
 }
 
+// Batches from this many tokens route in one pass (route_tc.cu) when the configuration allows;
+// smaller ones keep the split-K logits GEMM, which spreads a few token tiles over every SM.
+constexpr int64_t kOnePassMinTokens = 2048;
+
+// Whether the one-pass router may take this configuration (its kernel checks the rest).
+bool one_pass_possible(const moe_config& c, int64_t n) {
+  return act_dtype(c) == MOE_BF16 && c.cap_policy == MOE_CAP_NONE && n >= kOnePassMinTokens && c.top_k <= 8;
+}
+
 // ep_world > 0: the layout of one expert-parallel rank. The routed experts run over the
 // ep_recv_rows rows of the group's receive buffer in E / ep_world groups, so h and the FP8
 // activations are sized for those; the permuted rows and expert outputs live in the group's
@@ -75,8 +84,11 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   };
   p.diag = take(sizeof(moe_diag));
   p.logits = take((size_t)router_splits(c, n) * n * logits_ld(c) * 4);
-  p.rq = take((size_t)n * 4);  // tokens the one-pass router leaves to the binary64 router
-  p.rc = take((size_t)n * (kRouteCandMax + 1) * 4);  // and the experts to refine for each
+  // the one-pass router's queue of tokens left to the binary64 router, and their candidate experts:
+  // two counters, the candidate table, its binary64 logits, the list of pairs to refine
+  const bool one_pass = one_pass_possible(c, n);
+  p.rq = take(one_pass ? (size_t)n * 4 : 0);
+  p.rc = take(one_pass ? 16 + (size_t)n * (kRouteCandMax + 1) * (4 + 8) + (size_t)n * kRouteCandMax * 4 : 0);
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
   p.capg = take(c.cap_policy != MOE_CAP_NONE ? (size_t)capacity_grid_scratch_bytes(n, c.n_routed) : 0);
   p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
@@ -260,14 +272,10 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
   return MOE_OK;
 }
 
-// Batches from this many tokens route in one pass (route_tc.cu) when the configuration allows;
-// smaller ones keep the split-K logits GEMM, which spreads a few token tiles over every SM.
-constexpr int64_t kOnePassMinTokens = 2048;
-
 // The one-pass router's arguments; false when this configuration takes the two-kernel path.
 bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, RouteTcArgs* ra) {
   const moe_config& c = x.c;
-  if (act_dtype(c) != MOE_BF16 || c.cap_policy != MOE_CAP_NONE || x.n < kOnePassMinTokens) return false;
+  if (!one_pass_possible(c, x.n)) return false;
   RouteTcArgs a{};
   a.x = X;
   a.w_r = w->w_router;
@@ -287,7 +295,11 @@ bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* i
   a.ldl = logits_ld(c);
   a.queue = x.at<int32_t>(x.p.rq);
   a.queue_len = &x.status()->reserved[1];
-  a.cand = x.at<int32_t>(x.p.rc);
+  // candidate region: two counters, then the candidate table, their binary64 logits, the pair list
+  a.pair_count = x.at<int32_t>(x.p.rc);
+  a.cand = x.at<int32_t>(x.p.rc + 16);
+  a.cand_val = reinterpret_cast<double*>(x.ws + x.p.rc + 16 + (size_t)x.n * (kRouteCandMax + 1) * 4);
+  a.pairs = reinterpret_cast<int32_t*>(a.cand_val + (size_t)x.n * (kRouteCandMax + 1));
   a.status = x.status();
   if (!route_tc_supported(a)) return false;
   *ra = a;
@@ -312,12 +324,14 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   RouteArgs r;
   if (one_pass_args(x, X, w, idx, tw, &ra)) {
     // decisions in the tensor-core epilogue; the queued tokens re-decided from their logits rows
+    MOE_CUDA(cudaMemsetAsync(ra.pair_count, 0, 2 * sizeof(int32_t), x.s));
     MOE_CUDA(launch_route_tc(ra, x.s));
     r = route_args(x, X, w, idx, tw, d, 1);
     r.cursor = cursor;
     r.queue = ra.queue;
     r.queue_len = ra.queue_len;
     r.cand = ra.cand;
+    r.cand_val = ra.cand_val;
     MOE_CUDA(launch_route(r, x.s));
   } else if (c.cap_policy == MOE_CAP_NONE) {
     MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));

@@ -34,6 +34,7 @@ constexpr int kThreads = 1024;  // tokens per CTA
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
 constexpr int kNone = 0x7FFFFFFF;
 constexpr int kPrefix = 64;  // ranking entries per token staged in shared memory
+constexpr size_t kMaxDynSmem = 200 * 1024;  // dynamic shared memory of the largest grid
 
 // 32-bit words per staged ranking prefix of P entries: enough for P and odd, so that lanes reading
 // the same position of their rows hit 32 different banks.
@@ -366,7 +367,8 @@ cudaError_t launch_t(CapacityArgs a, GridCtl* g, unsigned grid, cudaStream_t s) 
   static std::atomic<uint64_t> attr{0};
   const size_t smem = dyn_smem(grid, a.E);
   if (smem > 48 * 1024) {
-    const cudaError_t e = set_smem_limit(attr, (const void*)capacity_grid_kernel<KT>, 227 * 1024 - 4096);
+    // the largest grid capacity_grid_fits accepts (static shared memory comes on top)
+    const cudaError_t e = set_smem_limit(attr, (const void*)capacity_grid_kernel<KT>, kMaxDynSmem);
     if (e != cudaSuccess) return e;
   }
   void* args[] = {&a, &g};
@@ -397,7 +399,7 @@ int64_t capacity_grid_scratch_bytes(int64_t n, int32_t E) {
 bool capacity_grid_fits(int64_t n, int32_t E) {
   const int64_t blocks = ceil_div(n, kThreads);
   // one CTA per SM, and every CTA's count row in shared memory next to the static arrays
-  return blocks >= 1 && blocks <= resident_blocks() && dyn_smem((unsigned)blocks, E) <= 200 * 1024;
+  return blocks >= 1 && blocks <= resident_blocks() && dyn_smem((unsigned)blocks, E) <= kMaxDynSmem;
 }
 
 cudaError_t launch_capacity_grid(const CapacityArgs& a, void* scratch, cudaStream_t s) {

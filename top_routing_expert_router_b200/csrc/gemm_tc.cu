@@ -1068,10 +1068,13 @@ constexpr size_t kSmemBytesW = 1024 + STAGESW * STAGEW_BYTES + sizeof(SmemCtl2);
 static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448 && kSmemBytesW <= 232448,
               "dynamic shared memory above 227 KB");
 
-// Wide pair tiles (256 x 512): MOE_TC_WIDE=1 selects them for the SM-pair GEMMs.
-bool use_wide_tiles() {
+// Wide pair tiles (256 x 512): MOE_TC_WIDE=1 selects them for every SM-pair GEMM, MOE_TC_WIDE=gate
+// for the gate/up (SwiGLU) GEMM only.
+bool use_wide_tiles(bool swiglu) {
   const char* w = getenv("MOE_TC_WIDE");
-  return w && w[0] == '1';
+  if (!w) return false;
+  if (w[0] == '1') return true;
+  return swiglu && strcmp(w, "gate") == 0;
 }
 
 // SM-pair tiles stage fewer bytes per FLOP and, with half-height last tiles,
@@ -1159,7 +1162,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
   CUtensorMap ma_half;
   if (pair && !make_map(&ma_half, a.A, a.M, a.K, BM / 2)) return cudaErrorInvalidValue;
-  const bool wide = pair && use_wide_tiles();
+  const bool wide = pair && use_wide_tiles(swiglu);
   const int b_box_used = wide ? 128 : b_box;
   if (!make_map(&mb, a.B, b_total_rows, a.K, b_box_used)) return cudaErrorInvalidValue;
   if (swiglu) {

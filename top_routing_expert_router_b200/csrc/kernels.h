@@ -97,7 +97,8 @@ struct RouteArgs {
   int32_t* cursor;      // zeroed before the launch: next token to route (warps fetch tokens from it)
   const int32_t* queue = nullptr;      // when set: route only the tokens queue[0 .. *queue_len)
   const int32_t* queue_len = nullptr;
-  const int32_t* cand = nullptr;       // with queue: experts to recompute in binary64 first (RouteTcArgs::cand)
+  const int32_t* cand = nullptr;       // with queue: candidate experts and their binary64 logits
+  const double* cand_val = nullptr;    // (RouteTcArgs::cand, cand_val)
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
@@ -121,6 +122,9 @@ struct RouteTcArgs {
   int32_t* queue_len;   // zeroed before the launch
   int32_t* cand;        // [n][kRouteCandMax + 1] per queued token: count (-1: too many), then the experts
                         // an uncertain comparison can involve
+  double* cand_val;     // [n][kRouteCandMax + 1] binary64 logits of those experts (same slots as cand)
+  int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine (one warp each)
+  int32_t* pair_count;  // [2] zeroed before the launch: pairs listed, refine cursor
   moe_diag* status;
 };
 bool route_tc_supported(const RouteTcArgs& a);

@@ -480,14 +480,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j <= kMaxK; ++j) insert(lv, ll, le, ov[j], ol[j], oe[j] < 0 ? 0x7FFFFFFF : oe[j]);
       }
       // every order the result depends on must be certain: adjacent kept experts and the k-th / (k+1)-th cut
-      // (and the lowest selection value an expert needs to take part in an uncertain one)
-      float thr = INFINITY;
+      // (band j: the selection values an expert may have to take part in uncertain comparison j)
+      float band_lo[kMaxK], band_hi[kMaxK];
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j)
+      for (int j = 0; j < kMaxK; ++j) {
+        band_lo[j] = INFINITY;
+        band_hi[j] = -INFINITY;
         if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) {
           ok = false;
-          thr = fminf(thr, (j + 1 < k ? lv[j + 1] : lv[j]) - 2.0f * dv);
+          band_lo[j] = (j + 1 < k ? lv[j + 1] : lv[j]) - 2.0f * dv;
+          band_hi[j] = (j + 1 < k ? lv[j] : lv[j + 1]) + 2.0f * dv;
         }
+      }
       const bool spill = valid && !ok;
       if (valid && ok) {
         // gates of the k kept experts
@@ -532,11 +536,14 @@ __global__ void __launch_bounds__(kThreads, 1)
               }
           }
         }
-        // the experts an uncertain comparison can involve: eligible ones at or above thr, and every
-        // expert of a group near an uncertain group cut; the binary64 router refines them first
+        // the experts an uncertain comparison can involve: eligible ones whose value lies in one of
+        // the bands, and every expert of a group near an uncertain group cut. Their logits are
+        // recomputed in binary64 (one warp per expert, refine_kernel) before the binary64 router
+        // decides the token again.
         int32_t* cand = nullptr;
+        int qpos = 0;
         if (spill) {
-          const int qpos = atomicAdd(p.queue_len, 1);
+          qpos = atomicAdd(p.queue_len, 1);
           p.queue[qpos] = (int32_t)tok;
           cand = p.cand + (int64_t)qpos * (kCandMax + 1);
         }
@@ -550,11 +557,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j) {
               const int e = c0 + j;
               if (e < E) {
-                const bool el = (kept >> g) & 1u;
                 bool want = (involved >> g) & 1u;
-                if (!want && el && thr != INFINITY) {
+                if (!want && ((kept >> g) & 1u)) {
                   const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[e];
-                  want = v >= thr;
+#pragma unroll
+                  for (int b = 0; b < kMaxK; ++b) want |= v >= band_lo[b] && v <= band_hi[b];
                 }
                 if (want) {
                   if (nc < kCandMax) cand[1 + nc] = e;
@@ -568,7 +575,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
         }
-        if (spill) cand[0] = nc <= kCandMax ? nc : -1;  // -1: too many, the router finds them itself
+        if (spill) {
+          if (nc <= kCandMax) {
+            cand[0] = nc;
+            const int base = atomicAdd(p.pair_count, nc);
+            for (int c = 0; c < nc; ++c) p.pairs[base + c] = qpos * (kCandMax + 1) + 1 + c;
+          } else {
+            cand[0] = -1;  // too many: the binary64 router finds and refines them itself
+          }
+        }
       }
       fence_before();
       __syncwarp();
@@ -582,6 +597,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(TMEM_COLS) : "memory");
+  }
+}
+
+// One binary64 logit per warp: x[t] . W_r[e] for every (queued token, candidate expert) pair, with
+// exact bf16 products and DFMA; the lanes take 16-byte chunks of the rows in turn, seven chunks'
+// loads issued before their products.
+__global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_t* cursor_base) {
+  int32_t* cursor = const_cast<int32_t*>(cursor_base);
+  const int lane = threadIdx.x & 31;
+  const int count = *p.pair_count;
+  const int nchunk = p.d / 8;
+  for (;;) {
+    int i = 0;
+    if (lane == 0) i = atomicAdd(cursor, 1);
+    i = __shfl_sync(0xFFFFFFFFu, i, 0);
+    if (i >= count) break;
+    const int slot = p.pairs[i];  // index into the candidate table
+    const int qpos = slot / (kCandMax + 1);
+    const int64_t t = p.queue[qpos];
+    const int e = p.cand[slot];
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.x) + t * p.d);
+    const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.w_r) + (int64_t)e * p.d);
+    double acc0 = 0.0, acc1 = 0.0;
+    for (int c = lane; c < nchunk; c += 32 * 7) {
+      uint4 xv[7], wv[7];
+#pragma unroll
+      for (int u = 0; u < 7; ++u) {
+        const int cc = c + 32 * u;
+        xv[u] = cc < nchunk ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
+        wv[u] = cc < nchunk ? __ldg(wr + cc) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < 7; ++u) {
+        const bf16* xs = reinterpret_cast<const bf16*>(&xv[u]);
+        const bf16* ws = reinterpret_cast<const bf16*>(&wv[u]);
+#pragma unroll
+        for (int q = 0; q < 8; q += 2) {
+          acc0 = fma((double)__bfloat162float(xs[q]), (double)__bfloat162float(ws[q]), acc0);
+          acc1 = fma((double)__bfloat162float(xs[q + 1]), (double)__bfloat162float(ws[q + 1]), acc1);
+        }
+      }
+    }
+    double v = acc0 + acc1;
+#pragma unroll
+    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+    if (lane == 0) p.cand_val[slot] = v;
   }
 }
 
@@ -633,6 +694,10 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
   const int64_t tiles = ceil_div(a.n, BM);
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
   route_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mx, mw, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // binary64 logits of the queued tokens' candidate experts, every pair at once
+  refine_kernel<<<(unsigned)(sms * 8), 256, 0, s>>>(a, a.pair_count + 1);
   return cudaGetLastError();
 }
 

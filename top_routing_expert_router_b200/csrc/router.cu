@@ -603,19 +603,22 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     int nr = 0;
     int n_refined = 0;
     if (a.cand) {
-      // experts the one-pass router found near a decision boundary: binary64 first, all at once
+      // experts the one-pass router found near a decision boundary, already recomputed in binary64
       const int32_t* c = a.cand + i * (kRouteCandMax + 1);
+      const double* cv = a.cand_val + i * (kRouteCandMax + 1);
       const int nc = c[0];
-      if (nc > 0) {
-        uint32_t which = 0;
-        for (int q = 0; q < nc; ++q) {
-          const int e = c[1 + q];
-          if ((e & 31) == lane) which |= 1u << (e >> 5);
+      for (int q = 0; q < nc; ++q) {
+        const int e = c[1 + q];
+        if ((e & 31) == lane) {
+#pragma unroll
+          for (int j = 0; j < EPL; ++j)
+            if (j == (e >> 5)) {
+              l[j] = cv[1 + q];
+              exact |= 1u << j;
+            }
         }
-        which &= valid_mask;
-        n_refined += refine_logits<EPL>(a, t, l, which);
-        exact |= which;
       }
+      n_refined += nc > 0 ? nc : 0;
     }
     for (int it = 0;; ++it) {
       uint32_t refine = 0;
