@@ -164,6 +164,10 @@ WORKLOADS = {w.name: w for w in [
         **{**_V3, "moe_intermediate_size": 128}),
     _wl("deepseek_v3_decode_32e", n=64, description="DeepSeek-V3-shaped decode with 32 experts (profiling size)",
         **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4}),
+    # profiling case: DeepSeek-V3 prefill shapes with 32 bf16 experts (2.8 GB of weights, 512 rows per
+    # expert on average like the full layer, so DRAM traffic per routed slot matches it)
+    _wl("deepseek_v3_prefill_32e", n=2048, **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4},
+        description="DeepSeek-V3-shaped prefill with 32 bf16 experts (profiling size)"),
     # profiling case: DeepSeek-V3 prefill shapes with 32 FP8 experts (1.4 GB of weights, 512 rows
     # per expert: the SM-pair FP8 tiles)
     _wl("deepseek_v3_prefill_fp8_32e", n=2048, dtype="fp8",

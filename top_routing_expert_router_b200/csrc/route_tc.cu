@@ -104,12 +104,6 @@ __device__ __forceinline__ uint32_t idesc_bf16(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
 }
 
-// Raw score of the routers that add a selection bias, in binary32.
-__device__ __forceinline__ float raw_score32(int score_fn, float l) {
-  if (score_fn == MOE_SCORE_SQRTSOFTPLUS) return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
-  return 1.0f / (1.0f + expf(-l));
-}
-
 // Selection score of the biased routers in the epilogue's fast form: sigmoid from ex2.approx and a
 // correctly rounded reciprocal (absolute error below 2^-18 for any logit, which the certification
 // margin adds); sqrtsoftplus in the accurate form.
@@ -118,7 +112,8 @@ __device__ __forceinline__ float sel_score(int score_fn, float l) {
   return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
 }
 
-// Insert (v, l, e) into the list sorted by v descending; an equal v stays below the entries
+// Insert (v, l, e) into the list sorted by v descending (l: what the gate needs, the logit for
+// softmax and the unbiased score otherwise); an equal v stays below the entries
 // already there, which hold lower expert indices (experts arrive in ascending order).
 __device__ __forceinline__ void insert(float (&lv)[kMaxK + 1], float (&ll)[kMaxK + 1], int (&le)[kMaxK + 1], float v,
                                        float l, int e) {
@@ -416,6 +411,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (fast) {
           const bool keptg = (kept >> g) & 1u;  // the whole chunk is in group g
           n_elig += keptg ? 32 : 0;
+          // selection values of the chunk, and which of them beat the list's current floor; the
+          // few that do are inserted one by one (a small loop, not 32 inlined insertions)
+          const float floor0 = lv[kMaxK];
+          uint32_t hit = 0;
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             float v;
@@ -425,7 +424,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
               v = sel_score(p.score_fn, l[j]) + sbias[c0 + j];
             }
-            if (keptg && v > lv[kMaxK]) insert(lv, ll, le, v, l[j], c0 + j);
+            l[j] = v;  // the logit itself is needed only for the few inserted experts (read back below)
+            hit |= (keptg && v > floor0) ? 1u << j : 0u;
+          }
+          while (hit) {
+            const int j = __ffs(hit) - 1;
+            hit &= hit - 1;
+            float v = 0.0f;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) v = u == j ? l[u] : v;
+            // the gate needs the logit (softmax) or the unbiased score (the others)
+            if (v > lv[kMaxK]) insert(lv, ll, le, v, soft ? v : v - sbias[c0 + j], c0 + j);
           }
         } else {
 #pragma unroll
@@ -435,8 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (soft) z += __expf(l[j] - m);
               if ((kept >> g) & 1u) {
                 ++n_elig;
-                const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[e];
-                insert(lv, ll, le, v, l[j], e);
+                const float sc = soft ? l[j] : sel_score(p.score_fn, l[j]);
+                const float v = soft ? sc : sc + sbias[e];
+                insert(lv, ll, le, v, sc, e);
               }
             }
             if (++r == per) {
@@ -502,7 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < kMaxK; ++j) w[j] = j < k ? expf(ll[j] - m) / z : 0.0f;
         } else {
 #pragma unroll
-          for (int j = 0; j < kMaxK; ++j) w[j] = j < k ? raw_score32(p.score_fn, ll[j]) : 0.0f;
+          for (int j = 0; j < kMaxK; ++j) w[j] = j < k ? ll[j] : 0.0f;  // the unbiased scores
         }
         if (p.renorm) {
           float s = 0.0f;
@@ -548,30 +558,49 @@ __global__ void __launch_bounds__(kThreads, 1)
           cand = p.cand + (int64_t)qpos * (kCandMax + 1);
         }
         int nc = 0;
+        float hull_lo = INFINITY, hull_hi = -INFINITY;  // the bands' hull: a cheap first test
+#pragma unroll
+        for (int b = 0; b < kMaxK; ++b) {
+          hull_lo = fminf(hull_lo, band_lo[b]);
+          hull_hi = fmaxf(hull_hi, band_hi[b]);
+        }
         for (int c0 = 0; c0 < E; c0 += 32) {
           float l[32];
           tmem_ld32(taddr + (uint32_t)c0, l);
           if (spill) {
+            // candidates of the chunk as a bit mask: whole groups near an uncertain group cut, and
+            // eligible experts inside the bands' hull (tested against each band below)
+            uint32_t hit = 0, grp = 0;
             int g = c0 / per, r = c0 - g * per;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-              const int e = c0 + j;
-              if (e < E) {
-                bool want = (involved >> g) & 1u;
-                if (!want && ((kept >> g) & 1u)) {
-                  const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[e];
-#pragma unroll
-                  for (int b = 0; b < kMaxK; ++b) want |= v >= band_lo[b] && v <= band_hi[b];
-                }
-                if (want) {
-                  if (nc < kCandMax) cand[1 + nc] = e;
-                  ++nc;
-                }
-              }
+              const bool in = c0 + j < E;
+              const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0];
+              l[j] = v;
+              if (in && ((involved >> g) & 1u)) grp |= 1u << j;
+              if (in && ((kept >> g) & 1u) && v >= hull_lo && v <= hull_hi) hit |= 1u << j;
               if (++r == per) {
                 r = 0;
                 ++g;
               }
+            }
+            uint32_t want = grp;
+            while (hit) {
+              const int j = __ffs(hit) - 1;
+              hit &= hit - 1;
+              float v = 0.0f;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) v = u == j ? l[u] : v;
+              bool in_band = false;
+#pragma unroll
+              for (int b = 0; b < kMaxK; ++b) in_band |= v >= band_lo[b] && v <= band_hi[b];
+              if (in_band) want |= 1u << j;
+            }
+            while (want) {
+              const int j = __ffs(want) - 1;
+              want &= want - 1;
+              if (nc < kCandMax) cand[1 + nc] = c0 + j;
+              ++nc;
             }
           }
         }

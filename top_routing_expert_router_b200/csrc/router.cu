@@ -105,10 +105,16 @@ __device__ __forceinline__ void selection_values(const RouteArgs& a, const doubl
 // true top two only if v >= (second largest v) - 2 delta_v; once all of those
 // are exact the group score is exact.
 template <int EPL>
+__device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
+                                 double delta_v, uint32_t* elig, uint32_t* mark);
+
+template <int EPL>
 __device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
                               double delta_v, uint32_t* elig, uint32_t* mark) {
   const int lane = threadIdx.x & 31;
   const int per = a.E / a.G;
+  // groups of 32 experts, one per lane slot: every group's reduction at once (below)
+  if (per == 32 && a.G == EPL) return decide_groups_32<EPL>(a, v, valid, exact, delta_v, elig, mark);
   double gs[kMaxGroups], gu[kMaxGroups], t2s[kMaxGroups];
   for (int g = 0; g < a.G; ++g) {
     double t1 = -INFINITY, t2 = -INFINITY;
@@ -180,6 +186,76 @@ __device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const 
     if (valid[j] && ((keep >> (e / per)) & 1u)) el |= 1u << j;
   }
   *elig = el;
+  *mark = m;
+  return ok;
+}
+
+// decide_groups for groups of exactly 32 experts with G = EPL: lane slot j of every lane holds
+// expert lane + 32 j, which is in group j, so the two best values of all groups are reduced across
+// the warp together (independent shuffle chains), with no per-expert group arithmetic.
+template <int EPL>
+__device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
+                                 double delta_v, uint32_t* elig, uint32_t* mark) {
+  double t1[EPL], t2[EPL];
+#pragma unroll
+  for (int g = 0; g < EPL; ++g) {
+    t1[g] = valid[g] ? v[g] : -INFINITY;
+    t2[g] = -INFINITY;
+  }
+#pragma unroll
+  for (int off = 16; off; off >>= 1) {
+#pragma unroll
+    for (int g = 0; g < EPL; ++g) {
+      const double o1 = __shfl_xor_sync(kFull, t1[g], off);
+      const double o2 = __shfl_xor_sync(kFull, t2[g], off);
+      const double hi = fmax(t1[g], o1);
+      const double lo = fmax(fmin(t1[g], o1), fmax(t2[g], o2));
+      t1[g] = hi;
+      t2[g] = lo;
+    }
+  }
+  double gs[EPL], gu[EPL];
+#pragma unroll
+  for (int g = 0; g < EPL; ++g) {
+    // an inexact expert could be among the group's true top two if v >= second best - 2 delta_v
+    const bool cand = valid[g] && !((exact >> g) & 1u) && v[g] >= t2[g] - 2.0 * delta_v;
+    gs[g] = t1[g] + t2[g];
+    gu[g] = __any_sync(kFull, cand) ? 2.0 * delta_v : 0.0;
+  }
+  uint32_t keep = 0;
+  double min_kept = INFINITY, max_drop = -INFINITY;
+#pragma unroll
+  for (int g = 0; g < EPL; ++g) {
+    int better = 0;
+#pragma unroll
+    for (int h = 0; h < EPL; ++h) better += (gs[h] > gs[g]) || (gs[h] == gs[g] && h < g);
+    if (better < a.topk_group) {
+      keep |= 1u << g;
+      min_kept = fmin(min_kept, gs[g] - gu[g]);
+    } else {
+      max_drop = fmax(max_drop, gs[g] + gu[g]);
+    }
+  }
+  bool ok = true;
+  uint32_t m = 0;
+  if (a.topk_group < a.G && !(min_kept > max_drop)) {
+    uint32_t involved = 0;
+#pragma unroll
+    for (int g = 0; g < EPL; ++g) {
+      const bool kept = (keep >> g) & 1u;
+      if (gu[g] > 0.0 && (kept ? gs[g] - gu[g] <= max_drop : gs[g] + gu[g] >= min_kept)) involved |= 1u << g;
+    }
+    if (involved) {
+      ok = false;
+#pragma unroll
+      for (int g = 0; g < EPL; ++g)
+        if (valid[g] && ((involved >> g) & 1u) && !((exact >> g) & 1u) && v[g] >= t2[g] - 2.0 * delta_v) m |= 1u << g;
+    }
+  }
+  *elig = 0;
+#pragma unroll
+  for (int g = 0; g < EPL; ++g)
+    if (valid[g] && ((keep >> g) & 1u)) *elig |= 1u << g;
   *mark = m;
   return ok;
 }
