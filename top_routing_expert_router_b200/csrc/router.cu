@@ -509,40 +509,6 @@ __device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* id
   return kept ? (float)(mine / denom * (double)a.rsf) : 0.0f;
 }
 
-// Binary64 dot product x[t] . W_r[e], computed by the whole warp: lanes take
-// 16-byte chunks of the row in turn (coalesced), then a butterfly sum.
-__device__ double dot64(const RouteArgs& a, int64_t t, int e) {
-  const int lane = threadIdx.x & 31;
-  double acc0 = 0.0, acc1 = 0.0;
-  if (a.dtype == MOE_BF16) {
-    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.x) + t * a.d);
-    const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(a.w_r) + (int64_t)e * a.d);
-#pragma unroll 4
-    for (int i = lane; i < a.d / 8; i += 32) {
-      const uint4 xv = __ldg(xr + i), wv = __ldg(wr + i);
-      const bf16* xs = reinterpret_cast<const bf16*>(&xv);
-      const bf16* ws = reinterpret_cast<const bf16*>(&wv);
-#pragma unroll
-      for (int q = 0; q < 8; q += 2) {
-        acc0 = fma(to_f64(xs[q]), to_f64(ws[q]), acc0);
-        acc1 = fma(to_f64(xs[q + 1]), to_f64(ws[q + 1]), acc1);
-      }
-    }
-  } else {
-    const float4* xr = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + t * a.d);
-    const float4* wr = reinterpret_cast<const float4*>(static_cast<const float*>(a.w_r) + (int64_t)e * a.d);
-#pragma unroll 4
-    for (int i = lane; i < a.d / 4; i += 32) {
-      const float4 xv = __ldg(xr + i), wv = __ldg(wr + i);
-      acc0 = fma((double)xv.x, (double)wv.x, acc0);
-      acc1 = fma((double)xv.y, (double)wv.y, acc1);
-      acc0 = fma((double)xv.z, (double)wv.z, acc0);
-      acc1 = fma((double)xv.w, (double)wv.w, acc1);
-    }
-  }
-  return warp_sum(acc0 + acc1);
-}
-
 // Binary64 dot products of x[t] with four rows of W_r at once (independent
 // accumulators, the token's row read once per chunk); e < 0 entries are skipped
 // and return 0.
