@@ -133,6 +133,9 @@ __device__ __forceinline__ void insert(float (&lv)[kMaxK + 1], float (&ll)[kMaxK
   }
 }
 
+// SF: the score function (compile time, so each instance holds one); FAST: whole 32-expert chunks
+// per half and groups of whole chunks, so the loops need no per-expert checks.
+template <int SF, bool FAST>
 __global__ void __launch_bounds__(kThreads, 1)
     route_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_w,
                     RouteTcArgs p) {
@@ -269,17 +272,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
     const int E = p.E, G = p.G, per = p.E / p.G, k = p.k;
-    const bool soft = p.score_fn == MOE_SCORE_SOFTMAX;
+    constexpr bool soft = SF == MOE_SCORE_SOFTMAX;
     const int Gh = G > 1 ? (G + 1) / 2 : 1;  // groups of half 0
     const int e_split = G > 1 ? Gh * per : min(E, ((E / 2 + 31) / 32) * 32);
     const int e_lo = h ? e_split : 0, e_hi = h ? E : e_split;
     const int g_lo = h ? Gh : 0;
     // derivative bound of the selection value in the logit (sigmoid' <= 1/4, sqrtsoftplus' < 1/2)
-    const float lip = p.score_fn == MOE_SCORE_SIGMOID ? 0.25f : p.score_fn == MOE_SCORE_SQRTSOFTPLUS ? 0.5f : 1.0f;
+    constexpr float lip = SF == MOE_SCORE_SIGMOID ? 0.25f : SF == MOE_SCORE_SQRTSOFTPLUS ? 0.5f : 1.0f;
     // binary32 evaluation error of a non-softmax selection value (a few ulp of a value near 1)
-    const float eval_err = soft ? 0.0f : 0x1p-18f;
+    constexpr float eval_err = soft ? 0.0f : 0x1p-18f;
     // whole 32-expert chunks per half and groups of whole chunks: the loops need no per-expert checks
-    const bool fast = E % 32 == 0 && e_split % 32 == 0 && (G == 1 || per % 32 == 0);
+    constexpr bool fast = FAST;
     const int row = q * 32 + lane;
     float* xg_mine = xg + ((size_t)h * BM + row) * kXg;
     const float* xg_other = xg + ((size_t)(h ^ 1) * BM + row) * kXg;
@@ -301,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(buf * 256);
       // pass 1 over this half's experts: |l| max, softmax max, group scores (top-2 sums of c)
       float amax = 0.0f, m = -INFINITY;
-      if (fast) {
+      if constexpr (fast) {
         // whole 32-expert chunks, groups of whole chunks: no per-expert range or group checks
         float g1 = -INFINITY, g2 = -INFINITY;
         for (int c0 = e_lo; c0 < e_hi; c0 += 32) {
@@ -317,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               amax = fmaxf(amax, fabsf(l[j]));
-              const float v = sel_score(p.score_fn, l[j]) + sbias[c0 + j];
+              const float v = sel_score(SF, l[j]) + sbias[c0 + j];
               g2 = fmaxf(g2, fminf(g1, v));
               g1 = fmaxf(g1, v);
             }
@@ -340,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               amax = fmaxf(amax, fabsf(l[j]));
               m = fmaxf(m, l[j]);
               if (!soft && G > 1) {
-                const float v = sel_score(p.score_fn, l[j]) + sbias[e];
+                const float v = sel_score(SF, l[j]) + sbias[e];
                 g2 = fmaxf(g2, fminf(g1, v));
                 g1 = fmaxf(g1, v);
                 if (++gpos == per) {
@@ -408,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!soft && per >= 32 && r + 32 <= per && !__any_sync(0xFFFFFFFFu, (kept >> g) & 1u)) continue;
         float l[32];
         tmem_ld32(taddr + (uint32_t)c0, l);
-        if (fast) {
+        if constexpr (fast) {
           const bool keptg = (kept >> g) & 1u;  // the whole chunk is in group g
           n_elig += keptg ? 32 : 0;
           // selection values of the chunk, and which of them beat the list's current floor; the
@@ -422,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               v = l[j];
               z += __expf(l[j] - m);
             } else {
-              v = sel_score(p.score_fn, l[j]) + sbias[c0 + j];
+              v = sel_score(SF, l[j]) + sbias[c0 + j];
             }
             l[j] = v;  // the logit itself is needed only for the few inserted experts (read back below)
             hit |= (keptg && v > floor0) ? 1u << j : 0u;
@@ -444,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (soft) z += __expf(l[j] - m);
               if ((kept >> g) & 1u) {
                 ++n_elig;
-                const float sc = soft ? l[j] : sel_score(p.score_fn, l[j]);
+                const float sc = soft ? l[j] : sel_score(SF, l[j]);
                 const float v = soft ? sc : sc + sbias[e];
                 insert(lv, ll, le, v, sc, e);
               }
@@ -575,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               const bool in = c0 + j < E;
-              const float v = soft ? l[j] : sel_score(p.score_fn, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0];
+              const float v = soft ? l[j] : sel_score(SF, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0];
               l[j] = v;
               if (in && ((involved >> g) & 1u)) grp |= 1u << j;
               if (in && ((kept >> g) & 1u) && v >= hull_lo && v <= hull_hi) hit |= 1u << j;
@@ -711,9 +714,27 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
   CUtensorMap mx, mw;
   if (!make_map(&mx, a.x, a.n, a.d, BM)) return cudaErrorInvalidValue;
   if (!make_map(&mw, a.w_r, a.E, a.d, (a.E + 15) & ~15)) return cudaErrorInvalidValue;
-  static std::atomic<uint64_t> attr{0};
+  // the instance: score function, and whether every half and group is a whole number of 32-expert chunks
+  const int G = a.G, per = a.E / a.G;
+  const int Gh = G > 1 ? (G + 1) / 2 : 1;
+  const int e_split = G > 1 ? Gh * per : (a.E / 2 + 31) / 32 * 32 < a.E ? (a.E / 2 + 31) / 32 * 32 : a.E;
+  const bool fast = a.E % 32 == 0 && e_split % 32 == 0 && (G == 1 || per % 32 == 0);
+  using Kern = void (*)(const CUtensorMap, const CUtensorMap, RouteTcArgs);
+  Kern kern;
+  static std::atomic<uint64_t> attr[6];
+  int which = 0;
+  if (a.score_fn == MOE_SCORE_SOFTMAX) {
+    kern = fast ? route_tc_kernel<MOE_SCORE_SOFTMAX, true> : route_tc_kernel<MOE_SCORE_SOFTMAX, false>;
+    which = fast ? 0 : 1;
+  } else if (a.score_fn == MOE_SCORE_SIGMOID) {
+    kern = fast ? route_tc_kernel<MOE_SCORE_SIGMOID, true> : route_tc_kernel<MOE_SCORE_SIGMOID, false>;
+    which = fast ? 2 : 3;
+  } else {
+    kern = fast ? route_tc_kernel<MOE_SCORE_SQRTSOFTPLUS, true> : route_tc_kernel<MOE_SCORE_SQRTSOFTPLUS, false>;
+    which = fast ? 4 : 5;
+  }
   {
-    const cudaError_t e = set_smem_limit(attr, (const void*)route_tc_kernel, kSmemBytes);
+    const cudaError_t e = set_smem_limit(attr[which], (const void*)kern, kSmemBytes);
     if (e != cudaSuccess) return e;
   }
   int dev = 0, sms = 0;
@@ -722,7 +743,7 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
   if (sms <= 0) sms = 148;
   const int64_t tiles = ceil_div(a.n, BM);
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-  route_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(mx, mw, a);
+  kern<<<grid, kThreads, kSmemBytes, s>>>(mx, mw, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // binary64 logits of the queued tokens' candidate experts, every pair at once

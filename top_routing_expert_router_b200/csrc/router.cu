@@ -671,7 +671,20 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
         ok = decide<EPL>(a, l, exact, delta_v, s_rank[wib], &nr, &refine);
       if (ok) break;
       refine &= ~exact;
-      if (it >= 3 || !__any_sync(kFull, refine != 0)) refine = valid_mask & ~exact;  // refine the rest
+      if (it >= 3 || !__any_sync(kFull, refine != 0)) {
+        // not settled by the marked experts: first the experts near any boundary under four times
+        // the margin (a superset), and only if that marks nothing new, every remaining logit
+        uint32_t wide = 0;
+        if (it < 6) {
+          int nr_w = 0;
+          if constexpr (FULL)
+            decide_full<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], s_flag[wib], &nr_w, &wide);
+          else
+            decide<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], &nr_w, &wide);
+          wide &= ~exact;
+        }
+        refine = __any_sync(kFull, wide != 0) ? wide : (valid_mask & ~exact);
+      }
       n_refined += refine_logits<EPL>(a, t, l, refine);
       exact |= refine;
     }
