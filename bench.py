@@ -219,15 +219,19 @@ def run_ours(args):
     phys = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
     gpu_index = phys[local] if len(phys) > local and phys[local] != "" else str(local)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # one event after each step as well: the per-step times show the power cap taking the clocks down
+    step_ev = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     with ClockSampler(gpu_index) as clk:
         barrier()
         ev0.record(stream)
-        for _ in range(args.steps):
+        for i in range(args.steps):
             step()
+            step_ev[i].record(stream)
         ev1.record(stream)
         barrier()
     ms_total = reduce_max(ev0.elapsed_time(ev1), world, "cuda")
     ms_step = ms_total / args.steps
+    step_ms = [round((ev0 if i == 0 else step_ev[i - 1]).elapsed_time(step_ev[i]), 3) for i in range(args.steps)]
     value = job_throughput(n, args.steps, world, ms_total)
     clocks = clk.summary()
 
@@ -340,6 +344,7 @@ def run_ours(args):
         "layer_roofline": {"flops": flops, "bytes": bytes_, "t_roof_ms": t_roof * 1e3,
                            "frac": t_roof * 1e3 / ms_step, "active_experts": active, "kept_slots": kept},
         "stages_ms": stage_ms,
+        "step_ms": step_ms,
         "diag": dg,
         "e2e": {"value": world * n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": n * w.d_model * bpe,
                 "d2h_bytes_per_step": n * w.d_model * bpe, "ms_per_step": e2e_ms},

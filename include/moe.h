@@ -184,7 +184,8 @@ moe_status moe_route(const moe_config* cfg, int64_t n, const void* x, const moe_
 
 /*
  * Dispatch: per-expert histogram, exclusive scan and stable permutation
- * (token order within an expert), plus the row gather.
+ * (token order within an expert), plus the row copy x_perm[slot_dest[t, j]] = x[t]
+ * (each token row read once and written to its kept slots).
  *   in : x [n, d], topk_idx [n, k] (-1 = dropped).
  *   out: offsets [E + 1] (offsets[E] = kept slots), perm_token [n * k]
  *        (first offsets[E] entries valid: source token of each permuted row),

@@ -379,7 +379,7 @@ moe_status permute_impl(const Ctx& x, const void* X, const int32_t* idx, int32_t
                            true, nullptr, x.s));
   if (!xperm) return MOE_OK;  // the FP8 quantiser gathers the rows itself
   const int64_t row_bytes = (int64_t)c.d_model * (act_dtype(c) == MOE_BF16 ? 2 : 4);
-  MOE_CUDA(launch_gather(X, perm, offsets, c.n_routed, x.n * c.top_k, row_bytes, xperm, x.s));
+  MOE_CUDA(launch_permute_rows(X, dest, x.n, c.top_k, row_bytes, xperm, x.s));
   return MOE_OK;
 }
 
@@ -816,9 +816,13 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
   int32_t* dest = c.at<int32_t>(c.p.dest);
   void* xperm = c.ws + c.p.xperm;
   void* eo = c.ws + c.p.eo;
-  // Shared experts first, on the side stream, overlapping routing and dispatch.
+  // Routing first: the one-pass router needs a whole SM's shared memory per CTA, so it runs before
+  // the shared experts take the SMs. The shared experts' GEMMs then run on the side stream next to
+  // the permutation, whose HBM-bound kernels fit on the SMs beside the GEMM's CTAs.
+  MOE_TRY(route_impl(c, x, weights, idx, tw, counts, diag_opt));
+  if (n == 0) return MOE_OK;
   void* sh = nullptr;
-  SideStream* side = (n > 0 && c.c.n_shared > 0) ? side_stream() : nullptr;
+  SideStream* side = c.c.n_shared > 0 ? side_stream() : nullptr;
   if (side) {
     MOE_CUDA(cudaEventRecord(side->fork, c.s));
     MOE_CUDA(cudaStreamWaitEvent(side->s, side->fork, 0));
@@ -827,8 +831,6 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
     MOE_TRY(shared_impl(cs, x, weights, &sh));
     MOE_CUDA(cudaEventRecord(side->join, side->s));
   }
-  MOE_TRY(route_impl(c, x, weights, idx, tw, counts, diag_opt));
-  if (n == 0) return MOE_OK;
   if (c.c.dtype == MOE_FP8) {
     // the quantiser gathers the token rows itself: no bf16 permuted copy
     MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, nullptr));

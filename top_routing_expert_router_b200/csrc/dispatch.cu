@@ -98,18 +98,32 @@ __global__ void __launch_bounds__(kThreads) scatter_kernel(const int32_t* idx, i
   }
 }
 
-// x_perm[p] = x[perm_token[p]] for p < offsets[E]; one warp per row, 16-byte vectors.
-__global__ void __launch_bounds__(256) gather_kernel(const uint4* x, const int32_t* perm_token,
-                                                   const int32_t* offsets, int E, int64_t vec_per_row,
-                                                   uint4* x_perm) {
-  const int64_t rows = offsets[E];
+// x_perm[slot_dest[t, j]] = x[t] for every kept slot (slot_dest >= 0), token-major: one warp per
+// token reads its row once (16-byte vectors, four per lane in flight) and writes it to each of its
+// k positions, so x crosses HBM once instead of once per slot.
+__global__ void __launch_bounds__(256) permute_rows_kernel(const uint4* x, const int32_t* slot_dest, int64_t n,
+                                                           int k, int64_t vec_per_row, uint4* x_perm) {
+  constexpr int U = 4;
   const int lane = threadIdx.x & 31;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nw = ((int64_t)gridDim.x * blockDim.x) >> 5;
-  for (int64_t p = warp; p < rows; p += nw) {
-    const uint4* src = x + (int64_t)perm_token[p] * vec_per_row;
-    uint4* dst = x_perm + p * vec_per_row;
-    for (int64_t v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+  for (int64_t t = warp; t < n; t += nw) {
+    const int mine = lane < k ? slot_dest[t * k + lane] : -1;
+    const uint4* src = x + t * vec_per_row;
+    for (int64_t v0 = lane; v0 < vec_per_row; v0 += 32 * U) {
+      uint4 val[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+        if (v0 + 32 * u < vec_per_row) val[u] = __ldg(src + v0 + 32 * u);
+      for (int j = 0; j < k; ++j) {
+        const int p = __shfl_sync(0xffffffffu, mine, j);
+        if (p < 0) continue;  // a slot the capacity rule dropped
+        uint4* dst = x_perm + (int64_t)p * vec_per_row;
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (v0 + 32 * u < vec_per_row) dst[v0 + 32 * u] = val[u];
+      }
+    }
   }
 }
 
@@ -184,11 +198,11 @@ cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t n, int32_t k, int32
   return cudaGetLastError();
 }
 
-cudaError_t launch_gather(const void* x, const int32_t* perm_token, const int32_t* offsets, int32_t E,
-                          int64_t max_rows, int64_t row_bytes, void* x_perm, cudaStream_t s) {
-  if (max_rows <= 0) return cudaSuccess;
-  gather_kernel<<<grid_for(max_rows * 32, 256), 256, 0, s>>>(static_cast<const uint4*>(x), perm_token, offsets, E,
-                                                             row_bytes / 16, static_cast<uint4*>(x_perm));
+cudaError_t launch_permute_rows(const void* x, const int32_t* slot_dest, int64_t n, int32_t k, int64_t row_bytes,
+                                void* x_perm, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  permute_rows_kernel<<<grid_for(n * 32, 256), 256, 0, s>>>(static_cast<const uint4*>(x), slot_dest, n, k,
+                                                            row_bytes / 16, static_cast<uint4*>(x_perm));
   return cudaGetLastError();
 }
 

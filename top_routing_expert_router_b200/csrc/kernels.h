@@ -162,8 +162,9 @@ int64_t dispatch_blocks(int64_t n, int32_t k);
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, int32_t* blk_counts,
                             int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* slot_dest,
                             bool scatter, moe_diag* diag, cudaStream_t s);
-cudaError_t launch_gather(const void* x, const int32_t* perm_token, const int32_t* offsets, int32_t E,
-                          int64_t max_rows, int64_t row_bytes, void* x_perm, cudaStream_t s);
+// x_perm[slot_dest[t, j]] = x[t] for the kept slots (slot_dest >= 0), each token row read once.
+cudaError_t launch_permute_rows(const void* x, const int32_t* slot_dest, int64_t n, int32_t k, int64_t row_bytes,
+                                void* x_perm, cudaStream_t s);
 
 // Combine.
 cudaError_t launch_combine(const void* eo, const int32_t* slot_dest, const float* topk_w, const void* sh,
