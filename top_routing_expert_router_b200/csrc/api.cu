@@ -24,6 +24,7 @@ struct Plan {
   size_t sfb, sfbs;  // FP8 SM-pair GEMMs: B scale blocks (routed, shared experts)
   size_t ep_off;  // expert parallelism: receive offsets of the rank's own experts
   size_t total;
+  bool batched;   // the two-kernel router queues its undecided tokens for launch_refine (rq, rc reserved)
 };
 
 // 512-byte scale blocks of the FP8 activations entering a matrix with k columns: one per row tile
@@ -64,11 +65,24 @@ bool one_pass_possible(const moe_config& c, int64_t n) {
   return act_dtype(c) == MOE_BF16 && c.cap_policy == MOE_CAP_NONE && n >= kOnePassMinTokens && c.top_k <= 8;
 }
 
+// Whether undecided tokens are refined in one batch (launch_refine over a queue) rather than one
+// warp at a time: bf16 rows of a whole number of 16-byte chunks.
+bool batched_refine_possible(const moe_config& c) { return act_dtype(c) == MOE_BF16 && c.d_model % 8 == 0; }
+
+// The candidate region of n queued tokens: 16 bytes of counters, the candidate table
+// [n][kRouteCandMax + 1] int32, their binary64 logits (same shape, 16-byte aligned whatever n),
+// then the pair list [n * kRouteCandMax] int32.
+size_t cand_val_offset(int64_t n) { return (size_t)align_up(16 + n * (kRouteCandMax + 1) * 4, 16); }
+size_t pairs_offset(int64_t n) { return cand_val_offset(n) + (size_t)n * (kRouteCandMax + 1) * 8; }
+size_t cand_region_bytes(int64_t n) { return pairs_offset(n) + (size_t)n * kRouteCandMax * 4; }
+
 // ep_world > 0: the layout of one expert-parallel rank. The routed experts run over the
 // ep_recv_rows rows of the group's receive buffer in E / ep_world groups, so h and the FP8
 // activations are sized for those; the permuted rows and expert outputs live in the group's
 // buffers, not here.
-Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_recv_rows = 0) {
+// batched: reserve the token queue for the two-kernel router too (the router-only scratch layout
+// leaves it out and refines those tokens warp by warp).
+Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_recv_rows = 0, bool batched = true) {
   const size_t b = act_dtype(c) == MOE_BF16 ? 2 : 4;
   const int64_t nk = n * c.top_k;
   const bool ep = ep_world > 0;
@@ -84,11 +98,13 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   };
   p.diag = take(sizeof(moe_diag));
   p.logits = take((size_t)router_splits(c, n) * n * logits_ld(c) * 4);
-  // the one-pass router's queue of tokens left to the binary64 router, and their candidate experts:
-  // two counters, the candidate table, its binary64 logits, the list of pairs to refine
-  const bool one_pass = one_pass_possible(c, n);
-  p.rq = take(one_pass ? (size_t)n * 4 : 0);
-  p.rc = take(one_pass ? 16 + (size_t)n * (kRouteCandMax + 1) * (4 + 8) + (size_t)n * kRouteCandMax * 4 : 0);
+  // the queue of tokens left to the binary64 router (one-pass router, or the first pass of the
+  // two-kernel router), and their candidate experts: four counters, the candidate table, its
+  // binary64 logits, the list of pairs to refine
+  p.batched = batched && batched_refine_possible(c);
+  const bool queued = one_pass_possible(c, n) || p.batched;
+  p.rq = take(queued ? (size_t)n * 4 : 0);
+  p.rc = take(queued ? cand_region_bytes(n) : 0);
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
   p.capg = take(c.cap_policy != MOE_CAP_NONE ? (size_t)capacity_grid_scratch_bytes(n, c.n_routed) : 0);
   p.blk = take((size_t)dispatch_blocks(n, c.top_k) * c.n_routed * 4);
@@ -272,6 +288,18 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
   return MOE_OK;
 }
 
+// The token queue and candidate region: queue length in the workspace's diag block; four counters
+// (pairs listed, refine cursor, second-pass cursor, spare), then the candidate table, their
+// binary64 logits, the pair list.
+void queue_args(const Ctx& x, RouteTcArgs* a) {
+  a->queue = x.at<int32_t>(x.p.rq);
+  a->queue_len = &x.status()->reserved[1];
+  a->pair_count = x.at<int32_t>(x.p.rc);
+  a->cand = x.at<int32_t>(x.p.rc + 16);
+  a->cand_val = reinterpret_cast<double*>(x.ws + x.p.rc + cand_val_offset(x.n));
+  a->pairs = reinterpret_cast<int32_t*>(x.ws + x.p.rc + pairs_offset(x.n));
+}
+
 // The one-pass router's arguments; false when this configuration takes the two-kernel path.
 bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, RouteTcArgs* ra) {
   const moe_config& c = x.c;
@@ -293,15 +321,28 @@ bool one_pass_args(const Ctx& x, const void* X, const moe_weights* w, int32_t* i
   a.topk_w = tw;
   a.logits = x.at<float>(x.p.logits);
   a.ldl = logits_ld(c);
-  a.queue = x.at<int32_t>(x.p.rq);
-  a.queue_len = &x.status()->reserved[1];
-  // candidate region: two counters, then the candidate table, their binary64 logits, the pair list
-  a.pair_count = x.at<int32_t>(x.p.rc);
-  a.cand = x.at<int32_t>(x.p.rc + 16);
-  a.cand_val = reinterpret_cast<double*>(x.ws + x.p.rc + 16 + (size_t)x.n * (kRouteCandMax + 1) * 4);
-  a.pairs = reinterpret_cast<int32_t*>(a.cand_val + (size_t)x.n * (kRouteCandMax + 1));
+  queue_args(x, &a);
   a.status = x.status();
   if (!route_tc_supported(a)) return false;
+  *ra = a;
+  return true;
+}
+
+// The batched refinement's arguments for the two-kernel router; false when its tokens are refined
+// one warp at a time.
+bool refine_args(const Ctx& x, const void* X, const moe_weights* w, RouteTcArgs* ra) {
+  const moe_config& c = x.c;
+  if (!x.p.batched || reinterpret_cast<uintptr_t>(X) % 16 ||
+      reinterpret_cast<uintptr_t>(w->w_router) % 16)
+    return false;
+  RouteTcArgs a{};
+  a.x = X;
+  a.w_r = w->w_router;
+  a.n = x.n;
+  a.d = c.d_model;
+  a.E = c.n_routed;
+  queue_args(x, &a);
+  a.status = x.status();
   *ra = a;
   return true;
 }
@@ -333,15 +374,34 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     r.cand = ra.cand;
     r.cand_val = ra.cand_val;
     MOE_CUDA(launch_route(r, x.s));
-  } else if (c.cap_policy == MOE_CAP_NONE) {
-    MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
-    r.cursor = cursor;
-    MOE_CUDA(launch_route(r, x.s));
   } else {
     MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
     r.cursor = cursor;
-    r.ranking = x.at<uint16_t>(x.p.ranking);
-    MOE_CUDA(launch_route(r, x.s));
+    if (c.cap_policy != MOE_CAP_NONE) r.ranking = x.at<uint16_t>(x.p.ranking);
+    if (refine_args(x, X, w, &ra)) {
+      // first pass decides what binary32 certifies and queues the rest with the experts to refine;
+      // those are refined all at once, then the second pass decides the queued tokens
+      MOE_CUDA(cudaMemsetAsync(ra.pair_count, 0, 4 * sizeof(int32_t), x.s));
+      r.defer_queue = ra.queue;
+      r.defer_len = ra.queue_len;
+      r.defer_cand = ra.cand;
+      r.defer_pairs = ra.pairs;
+      r.defer_pair_count = ra.pair_count;
+      MOE_CUDA(launch_route(r, x.s));
+      MOE_CUDA(launch_refine(ra, x.s));
+      RouteArgs r2 = r;
+      r2.defer_queue = r2.defer_len = r2.defer_cand = r2.defer_pairs = r2.defer_pair_count = nullptr;
+      r2.cursor = ra.pair_count + 2;
+      r2.queue = ra.queue;
+      r2.queue_len = ra.queue_len;
+      r2.cand = ra.cand;
+      r2.cand_val = ra.cand_val;
+      MOE_CUDA(launch_route(r2, x.s));
+    } else {
+      MOE_CUDA(launch_route(r, x.s));
+    }
+  }
+  if (c.cap_policy != MOE_CAP_NONE) {
     // the capacity rule on many SMs when its grid fits on the device at once (MOE_CAP_MODE=1cta
     // forces the one-CTA kernel: tuning and tests)
     const char* cm = getenv("MOE_CAP_MODE");
@@ -663,7 +723,7 @@ namespace moe {
 // ranking, the per-block counts and the offsets of the count scan. The caller's own buffers hold
 // the indices, gates and counts, so the full layout's regions for those are left out.
 Plan route_plan(const moe_config& c, int64_t n) {
-  Plan p = make_plan(c, n);
+  Plan p = make_plan(c, n, 0, 0, false);
   p.offsets = p.idx;
   p.total = p.offsets + (size_t)align_up((int64_t)(c.n_routed + 1) * 4, 256);
   return p;

@@ -99,6 +99,15 @@ struct RouteArgs {
   const int32_t* queue_len = nullptr;
   const int32_t* cand = nullptr;       // with queue: candidate experts and their binary64 logits
   const double* cand_val = nullptr;    // (RouteTcArgs::cand, cand_val)
+  // When defer_queue is set, a token whose first decision is not certain is not refined here: it
+  // is appended to defer_queue with the experts the decision marked (defer_cand, same layout as
+  // RouteTcArgs::cand) and their pairs (defer_pairs), for launch_refine and a second launch_route
+  // over that queue.
+  int32_t* defer_queue = nullptr;
+  int32_t* defer_len = nullptr;        // zeroed before the launch
+  int32_t* defer_cand = nullptr;
+  int32_t* defer_pairs = nullptr;
+  int32_t* defer_pair_count = nullptr; // zeroed before the launch
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
 
@@ -123,12 +132,17 @@ struct RouteTcArgs {
   int32_t* cand;        // [n][kRouteCandMax + 1] per queued token: count (-1: too many), then the experts
                         // an uncertain comparison can involve
   double* cand_val;     // [n][kRouteCandMax + 1] binary64 logits of those experts (same slots as cand)
-  int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine (one warp each)
+  int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine: one run per token, padded
+                        // with -1 to a multiple of four (a warp refines four pairs of one token)
   int32_t* pair_count;  // [2] zeroed before the launch: pairs listed, refine cursor
   moe_diag* status;
 };
 bool route_tc_supported(const RouteTcArgs& a);
 cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s);
+// Binary64 logits of every listed (queued token, candidate expert) pair, one warp each: the refine
+// step of launch_route_tc on its own, for the tokens a deferring launch_route queued. Uses x, w_r,
+// d (bf16 rows, d % 8 == 0, 16-byte aligned), queue, cand, cand_val, pairs and pair_count.
+cudaError_t launch_refine(const RouteTcArgs& a, cudaStream_t s);
 
 // Capacity rule over the ranking on many SMs (capacity.cu): a cooperative grid, one token per
 // thread, one round per fill event. Needs capacity_grid_scratch_bytes of scratch (16-byte aligned)

@@ -112,6 +112,18 @@ __device__ __forceinline__ float sel_score(int score_fn, float l) {
   return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
 }
 
+// Insert v into a list sorted descending (values only).
+__device__ __forceinline__ void insert_value(float (&lv)[kMaxK + 1], float v) {
+  if (!(v > lv[kMaxK])) return;
+#pragma unroll
+  for (int j = 0; j <= kMaxK; ++j)
+    if (v > lv[j]) {
+      const float t = lv[j];
+      lv[j] = v;
+      v = t;
+    }
+}
+
 // Insert (v, l, e) into the list sorted by v descending (l: what the gate needs, the logit for
 // softmax and the unbiased score otherwise); an equal v stays below the entries
 // already there, which hold lower expert indices (experts arrive in ascending order).
@@ -534,25 +546,72 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp-wide, so the whole warp reads when any lane spills)
       if (__any_sync(0xFFFFFFFFu, spill)) {
         float* lrow = p.logits + tok * p.ldl;
-        for (int c0 = 0; c0 < E; c0 += 32) {
-          float l[32];
-          tmem_ld32(taddr + (uint32_t)c0, l);
-          if (spill) {
+        // A token whose group cut is uncertain: once the binary64 values decide the cut, the kept
+        // set is the groups it certainly keeps (W) plus some of the uncertain ones. Its top k then
+        // lies at or above kappa, the k-th best value in W, so the experts that can matter are the
+        // eligible ones within a margin of kappa, and in the uncertain groups those that can be
+        // among their group's top two (v within a margin of the group's second best; g2min is the
+        // lowest of those).
+        const bool gunc = !soft && spill && involved != 0;
+        const bool any_gunc = __any_sync(0xFFFFFFFFu, gunc);
+        float kv[kMaxK + 1];
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              if (c0 + j + 4 <= E) {
-                *reinterpret_cast<float4*>(lrow + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
-              } else {
+        for (int j = 0; j <= kMaxK; ++j) kv[j] = -INFINITY;
+        float g2min = INFINITY;
+        {
+          float t1 = -INFINITY, t2 = -INFINITY;
+          int g = 0, r = 0;
+          for (int c0 = 0; c0 < E; c0 += 32) {
+            float l[32];
+            tmem_ld32(taddr + (uint32_t)c0, l);
+            if (spill) {
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  if (c0 + j + u < E) lrow[c0 + j + u] = l[j + u];
+              for (int j = 0; j < 32; j += 4)
+                if (c0 + j + 4 <= E) {
+                  *reinterpret_cast<float4*>(lrow + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
+                } else {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    if (c0 + j + u < E) lrow[c0 + j + u] = l[j + u];
+                }
+            }
+            if (any_gunc) {
+              uint32_t hit = 0;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float v = c0 + j < E ? sel_score(SF, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0] : -INFINITY;
+                l[j] = v;
+                if (c0 + j < E) {
+                  t2 = fmaxf(t2, fminf(t1, v));
+                  t1 = fmaxf(t1, v);
+                  if ((((kept & ~involved) >> g) & 1u) && v > kv[kMaxK]) hit |= 1u << j;
+                  if (++r == per) {
+                    if ((involved >> g) & 1u) g2min = fminf(g2min, t2);
+                    t1 = t2 = -INFINITY;
+                    r = 0;
+                    ++g;
+                  }
+                }
               }
+              if (!gunc) hit = 0;
+              while (hit) {
+                const int j = __ffs(hit) - 1;
+                hit &= hit - 1;
+                float v = 0.0f;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) v = u == j ? l[u] : v;
+                insert_value(kv, v);
+              }
+            }
           }
         }
+        float kappa = -INFINITY;  // stays -inf when W holds fewer than k experts
+#pragma unroll
+        for (int j = 0; j < kMaxK; ++j) kappa = j == k - 1 ? kv[j] : kappa;
         // the experts an uncertain comparison can involve: eligible ones whose value lies in one of
-        // the bands, and every expert of a group near an uncertain group cut. Their logits are
-        // recomputed in binary64 (one warp per expert, refine_kernel) before the binary64 router
-        // decides the token again.
+        // the bands and, for an uncertain group cut, those picked by kappa and g2min above. Their
+        // logits are recomputed in binary64 (one warp per expert, refine_kernel) before the
+        // binary64 router decides the token again.
         int32_t* cand = nullptr;
         int qpos = 0;
         if (spill) {
@@ -571,8 +630,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float l[32];
           tmem_ld32(taddr + (uint32_t)c0, l);
           if (spill) {
-            // candidates of the chunk as a bit mask: whole groups near an uncertain group cut, and
-            // eligible experts inside the bands' hull (tested against each band below)
+            // candidates of the chunk as a bit mask: after an uncertain group cut, the experts of
+            // kept or uncertain groups within 4 dv of kappa and those of uncertain groups within
+            // 4 dv of g2min; and eligible experts inside the bands' hull (tested against each band below)
             uint32_t hit = 0, grp = 0;
             int g = c0 / per, r = c0 - g * per;
 #pragma unroll
@@ -580,7 +640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
               const bool in = c0 + j < E;
               const float v = soft ? l[j] : sel_score(SF, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0];
               l[j] = v;
-              if (in && ((involved >> g) & 1u)) grp |= 1u << j;
+              if (in && gunc) {
+                if ((((kept | involved) >> g) & 1u) && v >= kappa - 4.0f * dv) grp |= 1u << j;
+                if (((involved >> g) & 1u) && v >= g2min - 4.0f * dv) grp |= 1u << j;
+              }
               if (in && ((kept >> g) & 1u) && v >= hull_lo && v <= hull_hi) hit |= 1u << j;
               if (++r == per) {
                 r = 0;
@@ -610,8 +673,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (spill) {
           if (nc <= kCandMax) {
             cand[0] = nc;
-            const int base = atomicAdd(p.pair_count, nc);
-            for (int c = 0; c < nc; ++c) p.pairs[base + c] = qpos * (kCandMax + 1) + 1 + c;
+            // one run per token, padded to a multiple of four (refine_kernel takes four pairs at a time)
+            const int padded = (nc + 3) & ~3;
+            const int base = atomicAdd(p.pair_count, padded);
+            for (int c = 0; c < padded; ++c) p.pairs[base + c] = c < nc ? qpos * (kCandMax + 1) + 1 + c : -1;
           } else {
             cand[0] = -1;  // too many: the binary64 router finds and refines them itself
           }
@@ -632,49 +697,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// One binary64 logit per warp: x[t] . W_r[e] for every (queued token, candidate expert) pair, with
-// exact bf16 products and DFMA; the lanes take 16-byte chunks of the rows in turn, seven chunks'
-// loads issued before their products.
+// Binary64 logits x[t] . W_r[e] of the listed (queued token, candidate expert) pairs. Each token's
+// pairs are listed as one run padded with -1 to a multiple of four, so a warp takes four pairs of
+// one token: the token's row is read and widened once for the four experts. Products of two bf16
+// values are exact in binary64; the sums are DFMA, the lanes taking 16-byte chunks in turn with
+// four chunks of every row in flight.
 __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_t* cursor_base) {
+  constexpr int U = 4;
   int32_t* cursor = const_cast<int32_t*>(cursor_base);
   const int lane = threadIdx.x & 31;
-  const int count = *p.pair_count;
+  const int quads = *p.pair_count / 4;
   const int nchunk = p.d / 8;
   for (;;) {
     int i = 0;
     if (lane == 0) i = atomicAdd(cursor, 1);
     i = __shfl_sync(0xFFFFFFFFu, i, 0);
-    if (i >= count) break;
-    const int slot = p.pairs[i];  // index into the candidate table
-    const int qpos = slot / (kCandMax + 1);
-    const int64_t t = p.queue[qpos];
-    const int e = p.cand[slot];
-    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.x) + t * p.d);
-    const uint4* wr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.w_r) + (int64_t)e * p.d);
-    double acc0 = 0.0, acc1 = 0.0;
-    for (int c = lane; c < nchunk; c += 32 * 7) {
-      uint4 xv[7], wv[7];
+    if (i >= quads) break;
+    int slot[4], e[4];
 #pragma unroll
-      for (int u = 0; u < 7; ++u) {
+    for (int q = 0; q < 4; ++q) {
+      slot[q] = p.pairs[4 * i + q];
+      e[q] = slot[q] >= 0 ? p.cand[slot[q]] : -1;
+    }
+    const int64_t t = p.queue[slot[0] / (kCandMax + 1)];  // a run starts every group of four
+    const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.x) + t * p.d);
+    const uint4* wr[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      wr[q] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.w_r) + (int64_t)(e[q] < 0 ? 0 : e[q]) * p.d);
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int c = lane; c < nchunk; c += 32 * U) {
+      uint4 xv[U], wv[4][U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
         const int cc = c + 32 * u;
         xv[u] = cc < nchunk ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
-        wv[u] = cc < nchunk ? __ldg(wr + cc) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) wv[q][u] = (cc < nchunk && e[q] >= 0) ? __ldg(wr[q] + cc) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int u = 0; u < 7; ++u) {
+      for (int u = 0; u < U; ++u) {
         const bf16* xs = reinterpret_cast<const bf16*>(&xv[u]);
-        const bf16* ws = reinterpret_cast<const bf16*>(&wv[u]);
 #pragma unroll
-        for (int q = 0; q < 8; q += 2) {
-          acc0 = fma((double)__bfloat162float(xs[q]), (double)__bfloat162float(ws[q]), acc0);
-          acc1 = fma((double)__bfloat162float(xs[q + 1]), (double)__bfloat162float(ws[q + 1]), acc1);
+        for (int h = 0; h < 8; ++h) {
+          const double xd = (double)__bfloat162float(xs[h]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            acc[q] = fma(xd, (double)__bfloat162float(reinterpret_cast<const bf16*>(&wv[q][u])[h]), acc[q]);
         }
       }
     }
-    double v = acc0 + acc1;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-    if (lane == 0) p.cand_val[slot] = v;
+    for (int q = 0; q < 4; ++q) {
+      double v = acc[q];
+#pragma unroll
+      for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
+      if (lane == 0 && slot[q] >= 0) p.cand_val[slot[q]] = v;
+    }
   }
 }
 
@@ -748,6 +827,21 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   // binary64 logits of the queued tokens' candidate experts, every pair at once
   refine_kernel<<<(unsigned)(sms * 8), 256, 0, s>>>(a, a.pair_count + 1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_refine(const RouteTcArgs& a, cudaStream_t s) {
+  if (a.n <= 0) return cudaSuccess;
+  if (a.d % 8 != 0 || reinterpret_cast<uintptr_t>(a.x) % 16 || reinterpret_cast<uintptr_t>(a.w_r) % 16)
+    return cudaErrorInvalidValue;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (sms <= 0) sms = 148;
+  // at most one warp per four listed pairs, and n * kRouteCandMax pairs can be listed
+  const int64_t need = ceil_div(a.n * kCandMax / 4, 8);
+  const unsigned grid = (unsigned)(need < sms * 8 ? need : sms * 8);
+  refine_kernel<<<grid, 256, 0, s>>>(a, a.pair_count + 1);
   return cudaGetLastError();
 }
 

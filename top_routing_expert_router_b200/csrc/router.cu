@@ -606,6 +606,46 @@ __device__ __forceinline__ void load_logits(const RouteArgs& a, int64_t t, doubl
   }
 }
 
+// Queue token t for the batched binary64 refinement: its index, the experts in `refine` (bits
+// over j of expert lane + 32 j, ascending) as its candidate row (count -1 past kRouteCandMax), and
+// one pair per candidate (a run padded to a multiple of four).
+template <int EPL>
+__device__ void defer_token(const RouteArgs& a, int64_t t, uint32_t refine) {
+  const int lane = threadIdx.x & 31;
+  int qpos = 0;
+  if (lane == 0) {
+    qpos = atomicAdd(a.defer_len, 1);
+    a.defer_queue[qpos] = (int32_t)t;
+  }
+  qpos = __shfl_sync(kFull, qpos, 0);
+  int32_t* cand = a.defer_cand + (int64_t)qpos * (kRouteCandMax + 1);
+  const uint32_t below = (1u << lane) - 1u;
+  int nc = 0;
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) {
+    const bool mine = (refine >> j) & 1u;
+    const uint32_t m = __ballot_sync(kFull, mine);
+    const int pos = nc + __popc(m & below);
+    if (mine && pos < kRouteCandMax) cand[1 + pos] = lane + 32 * j;
+    nc += __popc(m);
+  }
+  if (nc <= kRouteCandMax) {
+    // one run, padded with -1 to a multiple of four (the refinement takes four pairs of a token at once)
+    const int padded = (nc + 3) & ~3;
+    int base = 0;
+    if (lane == 0) {
+      cand[0] = nc;
+      base = atomicAdd(a.defer_pair_count, padded);
+    }
+    base = __shfl_sync(kFull, base, 0);
+    for (int c = lane; c < padded; c += 32)
+      a.defer_pairs[base + c] = c < nc ? qpos * (kRouteCandMax + 1) + 1 + c : -1;
+  } else if (lane == 0) {
+    cand[0] = -1;  // too many: the second pass finds and refines them itself
+  }
+  __syncwarp();
+}
+
 template <int EPL, bool FULL>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a) {
   __shared__ int16_t s_rank[kWarpsPerBlock][kMaxExperts];
@@ -662,6 +702,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
       }
       n_refined += nc > 0 ? nc : 0;
     }
+    bool deferred = false;
     for (int it = 0;; ++it) {
       uint32_t refine = 0;
       bool ok;
@@ -671,6 +712,13 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
         ok = decide<EPL>(a, l, exact, delta_v, s_rank[wib], &nr, &refine);
       if (ok) break;
       refine &= ~exact;
+      if (it == 0 && a.defer_queue && __any_sync(kFull, refine != 0)) {
+        // the marked experts of every such token are refined together (launch_refine), and the
+        // token decided again by the second pass over the queue
+        defer_token<EPL>(a, t, refine);
+        deferred = true;
+        break;
+      }
       if (it >= 3 || !__any_sync(kFull, refine != 0)) {
         // not settled by the marked experts: first the experts near any boundary under four times
         // the margin (a superset), and only if that marks nothing new, every remaining logit
@@ -688,6 +736,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
       n_refined += refine_logits<EPL>(a, t, l, refine);
       exact |= refine;
     }
+    if (deferred) continue;
     if (n_refined && lane == 0 && a.diag) {
       atomicAdd(&a.diag->refined_tokens, 1);
       atomicAdd(&a.diag->refined_logits, n_refined);
