@@ -162,6 +162,9 @@ WORKLOADS = {w.name: w for w in [
     # dispatch do not depend on I), and decode with 32 bf16 experts (2.8 GB of weights)
     _wl("deepseek_v3_route_8k", n=8192, description="DeepSeek-V3 routing and dispatch, small experts (profiling size)",
         **{**_V3, "moe_intermediate_size": 128}),
+    # the full layer's router input (x: 235 MB, more than L2) with small experts: router profiling
+    _wl("deepseek_v3_route_16k", n=16384, description="DeepSeek-V3 routing and dispatch at 16384 tokens, small experts "
+        "(router profiling size)", **{**_V3, "moe_intermediate_size": 128}),
     _wl("deepseek_v3_decode_32e", n=64, description="DeepSeek-V3-shaped decode with 32 experts (profiling size)",
         **{**_V3, "n_routed": 32, "n_group": 8, "topk_group": 4}),
     # profiling case: DeepSeek-V3 prefill shapes with 32 bf16 experts (2.8 GB of weights, 512 rows per

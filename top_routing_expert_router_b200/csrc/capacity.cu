@@ -111,8 +111,9 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   __shared__ int hist[kMaxExperts];
   __shared__ uint32_t full_s[kMaxExperts / 32];
   __shared__ int cand[kMaxExperts];
+  __shared__ int8_t cidx[kMaxExperts];   // place of an expert in cand (-1: not a candidate)
   __shared__ int n_cand;
-  __shared__ uint32_t ballots[kThreads / 32];
+  __shared__ uint32_t bal[32][kThreads / 32];  // per candidate of a batch: which tokens of each warp hold it
   __shared__ int s_stop;
   __shared__ int s_ok;
   __shared__ unsigned long long s_over, s_drop;
@@ -147,6 +148,7 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   unsigned long long my_over = 0, my_drop = 0;
   if (tid == 0) s_over = s_drop = 0;
   for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = 0;
+  for (int e = tid; e < kMaxExperts; e += kThreads) cidx[e] = -1;
   __syncthreads();
   auto is_full = [&](int e) { return (full_s[e >> 5] >> (e & 31)) & 1u; };
   // walk on from the cursor until k non-full experts are held
@@ -170,7 +172,8 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
     return ch.get(j);
   };
   // drop the experts that are full now; under OVERFLOW_NEXT walk on to replace them
-  auto drop_full = [&]() {
+  auto drop_full = [&]() -> bool {
+    bool changed = false;
     if (a.policy == MOE_CAP_OVERFLOW_NEXT) {
       int kept = 0;
       for (int j = 0; j < k; ++j)
@@ -186,10 +189,22 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
       if (kept < taken) {
         taken = kept;
         refill();
+        changed = true;
       }
     } else {
       for (int j = 0; j < k; ++j)
-        if (ch.get(j) >= 0 && is_full(ch.get(j))) ch.set(j, -1);
+        if (ch.get(j) >= 0 && is_full(ch.get(j))) {
+          ch.set(j, -1);
+          changed = true;
+        }
+    }
+    return changed;
+  };
+  // this token's choices in or out of the histogram
+  auto count_mine = [&](int sign) {
+    for (int j = 0; j < k; ++j) {
+      const int e = slot(j);
+      if (e >= 0) atomicAdd(&hist[e], sign);
     }
   };
   auto commit = [&]() {
@@ -211,12 +226,29 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
       }
     }
   }
+  ChainState* mine = chain + blockIdx.x;
+  // Full sets only grow along the chain, so the experts full after CTA b - 2 are full at this CTA's
+  // turn too: its tokens walk past them while CTA b - 1 still works, and the histogram of the
+  // resulting choices is taken before the last wait.
+  if (blockIdx.x >= 2) {
+    if (tid == 0) s_ok = wait_for(chain + blockIdx.x - 2, a.status) ? 1 : 0;
+    __syncthreads();
+    if (!s_ok) {
+      if (tid == 0) atomicExch(&mine->flag, 2);  // abandon the rest of the chain at once
+      return;
+    }
+    for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = __ldcg(&chain[blockIdx.x - 2].full[w]);
+    __syncthreads();
+    if (valid) drop_full();
+  }
+  for (int e = tid; e < E; e += kThreads) hist[e] = 0;
+  __syncthreads();
+  for (int j = 0; j < k; ++j) warp_count(hist, valid ? slot(j) : -1);
   // the predecessor's counts and full set (other CTAs wrote them: read from L2, not L1)
   if (tid == 0) s_ok = blockIdx.x == 0 ? 1 : (wait_for(chain + blockIdx.x - 1, a.status) ? 1 : 0);
   __syncthreads();
-  ChainState* mine = chain + blockIdx.x;
   if (!s_ok) {
-    if (tid == 0) atomicExch(&mine->flag, 2);  // abandon the rest of the chain at once
+    if (tid == 0) atomicExch(&mine->flag, 2);
     return;
   }
   if (blockIdx.x == 0) {
@@ -227,47 +259,84 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
     for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = __ldcg(&prev->full[w]);
   }
   __syncthreads();
-  if (valid) drop_full();
+  // tokens that held an expert CTA b - 1 filled walk on; the histogram follows them
+  if (valid) {
+    Slots<KA, (KT > 0)> ch0 = ch;
+    const int taken0 = taken;
+    if (blockIdx.x > 0 && drop_full()) {
+      for (int j = 0; j < k; ++j) {
+        const int e = a.policy == MOE_CAP_OVERFLOW_NEXT ? (j < taken0 ? ch0.get(j) : -1) : ch0.get(j);
+        if (e >= 0) atomicSub(&hist[e], 1);
+      }
+      count_mine(1);
+    }
+  }
+  bool counted = true;  // hist holds the choices of every uncommitted token
   int f = 0;  // first token of the range not committed yet (uniform across the CTA)
   for (;;) {
     const bool active = valid && tid >= f;
-    for (int e = tid; e < E; e += kThreads) hist[e] = 0;
+    if (!counted) {
+      for (int e = tid; e < E; e += kThreads) hist[e] = 0;
+      __syncthreads();
+      for (int j = 0; j < k; ++j) warp_count(hist, active ? slot(j) : -1);
+    }
+    counted = false;
     if (tid == 0) {
       n_cand = 0;
       s_stop = kThreads;
     }
     __syncthreads();
-    for (int j = 0; j < k; ++j) warp_count(hist, active ? slot(j) : -1);
-    __syncthreads();
     for (int e = tid; e < E; e += kThreads)
-      if (!is_full(e) && cnt_s[e] + hist[e] >= a.C) cand[atomicAdd(&n_cand, 1)] = e;
+      if (!is_full(e) && cnt_s[e] + hist[e] >= a.C) {
+        const int c = atomicAdd(&n_cand, 1);
+        cand[c] = e;
+        cidx[e] = (int8_t)(c < 127 ? c : 127);
+      }
     __syncthreads();
     const int nc = n_cand;
-    // the token at which each candidate expert reaches C: its (C - count)-th chooser in order
-    for (int c = 0; c < nc; ++c) {
-      const int e = cand[c];
-      bool me = false;
+    // The token at which each candidate expert reaches C: its (C - count)-th chooser in token
+    // order. Candidates go 32 at a time: every warp ballots all of them, then warp q finds
+    // candidate q's chooser with a prefix over the warps' counts.
+    for (int c0 = 0; c0 < nc; c0 += 32) {
+      const int nb = nc - c0 < 32 ? nc - c0 : 32;
+      uint32_t held = 0;  // bit q: this token holds candidate c0 + q
       if (active)
-        for (int j = 0; j < k; ++j) me |= slot(j) == e;
-      const uint32_t b = __ballot_sync(kFull, me);
-      if (lane == 0) ballots[wid] = b;
-      __syncthreads();
-      if (tid == 0) {
-        int nd = (int)(a.C - cnt_s[e]);
-        for (int w = 0; w < kThreads / 32; ++w) {
-          const int pc = __popc(ballots[w]);
-          if (nd <= pc) {
-            uint32_t bb = ballots[w];
-            for (int q = 1; q < nd; ++q) bb &= bb - 1;
-            const int at = w * 32 + __ffs(bb) - 1;
-            if (at < s_stop) s_stop = at;
-            break;
+        for (int j = 0; j < k; ++j) {
+          const int e = slot(j);
+          if (e >= 0) {
+            const int q = nc <= 127 ? (int)cidx[e] - c0 : -1;
+            if (q >= 0 && q < nb && cand[c0 + q] == e) {
+              held |= 1u << q;
+            } else if (nc > 127) {
+              for (int qq = 0; qq < nb; ++qq) held |= cand[c0 + qq] == e ? 1u << qq : 0u;
+            }
           }
-          nd -= pc;
+        }
+      for (int q = 0; q < nb; ++q) {
+        const uint32_t b = __ballot_sync(kFull, (held >> q) & 1u);
+        if (lane == 0) bal[q][wid] = b;
+      }
+      __syncthreads();
+      if (wid < nb) {
+        const int e = cand[c0 + wid];
+        const int need = (int)(a.C - cnt_s[e]);
+        const uint32_t bw = bal[wid][lane];
+        const int pc = __popc(bw);
+        int incl = pc;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+          const int v = __shfl_up_sync(kFull, incl, off);
+          if (lane >= off) incl += v;
+        }
+        if (incl - pc < need && need <= incl) {
+          uint32_t bb = bw;
+          for (int q = 1; q < need - (incl - pc); ++q) bb &= bb - 1;
+          atomicMin(&s_stop, lane * 32 + __ffs(bb) - 1);
         }
       }
       __syncthreads();
     }
+    for (int c = tid; c < nc; c += kThreads) cidx[cand[c]] = -1;
     const int stop = s_stop;  // last token committed in this step (kThreads: the rest of the range)
     const bool take = active && tid <= stop;
     if (stop < kThreads) {
