@@ -41,7 +41,8 @@ int64_t logits_ld(const moe_config& c) { return align_up(c.n_routed, 4); }
 
 // Split-K factor of the router GEMM: small token counts leave most SMs idle
 // (one 128-row tile per 128 tokens), so the k range is split and the route
-// kernel sums the partial logits in a fixed order. Capped at 4 MiB of partials.
+// kernel sums the partial logits in a fixed order. Capped at 4 MiB of partials
+// and at 32 splits: every logit's sum is a chain through all of them.
 int router_splits(const moe_config& c, int64_t n) {
   if (act_dtype(c) != MOE_BF16 || n <= 0) return 1;
   const int64_t tiles = ceil_div(n, 128) * ceil_div(c.n_routed, 256);
@@ -50,6 +51,7 @@ int router_splits(const moe_config& c, int64_t n) {
   int64_t s = 148 / tiles;
   const int64_t cap = ((int64_t)4 << 20) / (n * logits_ld(c) * 4);
   if (s > cap) s = cap;
+  if (s > 32) s = 32;
   if (s > num_kb) s = num_kb;
   if (s < 1) s = 1;
   const int64_t kb_per = ceil_div(num_kb, s);
@@ -275,7 +277,8 @@ RouteArgs route_args(const Ctx& x, const void* X, const moe_weights* w, int32_t*
   return r;
 }
 
-// Router logits (binary32, split-K partials for small batches) and the route arguments.
+// Router logits (binary32; small batches split K and sum the partials into one row per token)
+// and the route arguments.
 moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int32_t* idx, float* tw, moe_diag* d,
                          RouteArgs* out) {
   const moe_config& c = x.c;
@@ -284,7 +287,9 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
   GemmArgs g{X, c.d_model, w->w_router, nullptr, 0, x.at<float>(x.p.logits), ld, nullptr, 1, x.n, c.n_routed,
              c.d_model, splits, x.n * ld};
   MOE_TRY(gemm(x, g, false, true));
-  *out = route_args(x, X, w, idx, tw, d, splits);
+  // the partials summed once, so every later reader takes one row per token
+  MOE_CUDA(launch_sum_splits(x.at<float>(x.p.logits), splits, x.n * ld, x.n, ld, c.n_routed, x.s));
+  *out = route_args(x, X, w, idx, tw, d, 1);
   return MOE_OK;
 }
 
@@ -428,15 +433,20 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   return MOE_OK;
 }
 
+// counted: route_impl's histogram and scan over the same idx already left the per-block bases and
+// offsets in the workspace, so only the permutation runs.
 moe_status permute_impl(const Ctx& x, const void* X, const int32_t* idx, int32_t* offsets, int32_t* perm,
-                        int32_t* dest, void* xperm) {
+                        int32_t* dest, void* xperm, bool counted = false) {
   const moe_config& c = x.c;
   if (x.n == 0) {
     MOE_CUDA(launch_fill_i32(offsets, c.n_routed + 1, 0, x.s));
     return MOE_OK;
   }
-  MOE_CUDA(launch_dispatch(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), nullptr, offsets, perm, dest,
-                           true, nullptr, x.s));
+  if (counted)
+    MOE_CUDA(launch_scatter(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), offsets, perm, dest, x.s));
+  else
+    MOE_CUDA(launch_dispatch(idx, x.n, c.top_k, c.n_routed, x.at<int32_t>(x.p.blk), nullptr, offsets, perm, dest,
+                             true, nullptr, x.s));
   if (!xperm) return MOE_OK;  // the FP8 quantiser gathers the rows itself
   const int64_t row_bytes = (int64_t)c.d_model * (act_dtype(c) == MOE_BF16 ? 2 : 4);
   MOE_CUDA(launch_permute_rows(X, dest, x.n, c.top_k, row_bytes, xperm, x.s));
@@ -891,12 +901,13 @@ moe_status moe_layer_forward(const moe_config* cfg, int64_t n, const void* x, co
     MOE_TRY(shared_impl(cs, x, weights, &sh));
     MOE_CUDA(cudaEventRecord(side->join, side->s));
   }
+  // route_impl left the histogram's per-block bases and the offsets of idx in the workspace
   if (c.c.dtype == MOE_FP8) {
     // the quantiser gathers the token rows itself: no bf16 permuted copy
-    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, nullptr));
+    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, nullptr, true));
     MOE_TRY(ffn_fp8(c, x, perm, offsets, weights, eo));
   } else {
-    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm));
+    MOE_TRY(permute_impl(c, x, idx, offsets, perm, dest, xperm, true));
     MOE_TRY(ffn_impl(c, xperm, offsets, weights, eo));
   }
   if (side)

@@ -33,31 +33,50 @@ __global__ void __launch_bounds__(kThreads) count_kernel(const int32_t* idx, int
   for (int e = threadIdx.x; e < E; e += kThreads) blk_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
 }
 
-// One block: per-expert exclusive scan over blocks (in place), then over experts.
+// One block: per-expert exclusive scan over blocks (in place), then over experts. Thread e reads
+// eight blocks' counts before it writes their bases, so the walk over blocks costs a few memory
+// latencies; the scan over experts is a warp-shuffle scan.
 __global__ void __launch_bounds__(kMaxExperts) scan_kernel(int32_t* blk_counts, int nblk, int E, int32_t* counts,
                                                          int32_t* offsets, moe_diag* diag) {
-  __shared__ int tot[kMaxExperts];
-  const int e = threadIdx.x;
+  constexpr int B = 8;
+  __shared__ int warp_tot[kMaxExperts / 32], warp_max[kMaxExperts / 32];
+  const int e = threadIdx.x, lane = e & 31, wid = e >> 5;
   int run = 0;
   if (e < E) {
-    for (int b = 0; b < nblk; ++b) {
-      const int c = blk_counts[(int64_t)b * E + e];
-      blk_counts[(int64_t)b * E + e] = run;
-      run += c;
+    for (int b0 = 0; b0 < nblk; b0 += B) {
+      int c[B];
+#pragma unroll
+      for (int q = 0; q < B; ++q) c[q] = b0 + q < nblk ? blk_counts[(int64_t)(b0 + q) * E + e] : 0;
+#pragma unroll
+      for (int q = 0; q < B; ++q)
+        if (b0 + q < nblk) {
+          blk_counts[(int64_t)(b0 + q) * E + e] = run;
+          run += c[q];
+        }
     }
     if (counts) counts[e] = run;
   }
-  tot[e] = e < E ? run : 0;
+  // exclusive scan of the per-expert totals in expert order, and their maximum
+  int incl = run, mx = run;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += v;
+    mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, off));
+  }
+  if (lane == 31) warp_tot[wid] = incl;
+  if (lane == 0) warp_max[wid] = mx;
   __syncthreads();
+  int base = 0, total = 0, gmax = 0;
+  for (int w = 0; w < kMaxExperts / 32; ++w) {
+    base += w < wid ? warp_tot[w] : 0;
+    total += warp_tot[w];
+    gmax = max(gmax, warp_max[w]);
+  }
+  if (e < E) offsets[e] = base + incl - run;
   if (e == 0) {
-    int acc = 0, mx = 0;
-    for (int i = 0; i < E; ++i) {
-      offsets[i] = acc;
-      acc += tot[i];
-      mx = tot[i] > mx ? tot[i] : mx;
-    }
-    offsets[E] = acc;
-    if (diag) diag->max_load = mx;
+    offsets[E] = total;
+    if (diag) diag->max_load = gmax;
   }
 }
 
@@ -184,6 +203,14 @@ unsigned grid_for(int64_t work, int per_block) {
 }  // namespace
 
 int64_t dispatch_blocks(int64_t n, int32_t k) { return ceil_div(n * k, kItems); }
+
+cudaError_t launch_scatter(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, const int32_t* blk_base,
+                           const int32_t* offsets, int32_t* perm_token, int32_t* slot_dest, cudaStream_t s) {
+  const int64_t nblk = dispatch_blocks(n, k);
+  if (nblk > 0)
+    scatter_kernel<<<(unsigned)nblk, kThreads, 0, s>>>(topk_idx, n * k, k, E, blk_base, offsets, perm_token, slot_dest);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, int32_t* blk_counts,
                             int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* slot_dest,

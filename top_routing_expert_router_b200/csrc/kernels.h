@@ -110,6 +110,10 @@ struct RouteArgs {
   int32_t* defer_pair_count = nullptr; // zeroed before the launch
 };
 cudaError_t launch_route(const RouteArgs& a, cudaStream_t s);
+// Sums the split-K partial logits [splits][n, ld] into split 0's rows, in split order (binary64
+// sum rounded to binary32), for the first E columns.
+cudaError_t launch_sum_splits(float* logits, int32_t splits, int64_t split_stride, int64_t n, int64_t ld, int32_t E,
+                              cudaStream_t s);
 
 constexpr int kRouteCandMax = 32;
 
@@ -176,6 +180,10 @@ int64_t dispatch_blocks(int64_t n, int32_t k);
 cudaError_t launch_dispatch(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, int32_t* blk_counts,
                             int32_t* counts, int32_t* offsets, int32_t* perm_token, int32_t* slot_dest,
                             bool scatter, moe_diag* diag, cudaStream_t s);
+// The stable permutation alone, from the per-block bases and offsets a launch_dispatch over the
+// same topk_idx left in blk_base and offsets.
+cudaError_t launch_scatter(const int32_t* topk_idx, int64_t n, int32_t k, int32_t E, const int32_t* blk_base,
+                           const int32_t* offsets, int32_t* perm_token, int32_t* slot_dest, cudaStream_t s);
 // x_perm[slot_dest[t, j]] = x[t] for the kept slots (slot_dest >= 0), each token row read once.
 cudaError_t launch_permute_rows(const void* x, const int32_t* slot_dest, int64_t n, int32_t k, int64_t row_bytes,
                                 void* x_perm, cudaStream_t s);

@@ -592,17 +592,54 @@ __device__ int refine_logits(const RouteArgs& a, int64_t t, double (&l)[EPL], ui
   return total;
 }
 
-// Load a token's logits, summing the split-K partial GEMM results in order.
+// logits[t][e] (split 0's slot) = the sum of the split-K partials of (t, e) in split order: binary64
+// sum, rounded once to binary32. One thread per logit with four splits' loads in flight, so the
+// route kernel's warps read one row per token instead of a serial chain through every split.
+__global__ void __launch_bounds__(256) sum_splits_kernel(float* logits, int splits, int64_t split_stride, int64_t n,
+                                                       int64_t ld, int E) {
+  const int64_t total = n * E;
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < total; i += (int64_t)gridDim.x * 256) {
+    const int64_t t = i / E;
+    float* p0 = logits + t * ld + (i - t * E);
+    double s = 0.0;
+    int p = 0;
+    for (; p + 4 <= splits; p += 4) {
+      const float a0 = p0[(int64_t)p * split_stride], a1 = p0[(int64_t)(p + 1) * split_stride];
+      const float a2 = p0[(int64_t)(p + 2) * split_stride], a3 = p0[(int64_t)(p + 3) * split_stride];
+      s += (double)a0;
+      s += (double)a1;
+      s += (double)a2;
+      s += (double)a3;
+    }
+    for (; p < splits; ++p) s += (double)p0[(int64_t)p * split_stride];
+    *p0 = (float)s;
+  }
+}
+
+// Load a token's logits, summing the split-K partial GEMM results in split order. The partials
+// of four splits are loaded at once before they are added, so a many-way split costs a few
+// memory latencies, not one per split.
 template <int EPL>
 __device__ __forceinline__ void load_logits(const RouteArgs& a, int64_t t, double (&l)[EPL]) {
+  constexpr int P = 4;
   const int lane = threadIdx.x & 31;
+  const float* row = a.logits + t * a.ldl + lane;
 #pragma unroll
-  for (int j = 0; j < EPL; ++j) {
-    const int e = lane + 32 * j;
-    double s = 0.0;
-    if (e < a.E)
-      for (int p = 0; p < a.splits; ++p) s += (double)a.logits[(int64_t)p * a.split_stride + t * a.ldl + e];
-    l[j] = s;
+  for (int j = 0; j < EPL; ++j) l[j] = 0.0;
+  for (int p0 = 0; p0 < a.splits; p0 += P) {
+    float part[P][EPL];
+#pragma unroll
+    for (int q = 0; q < P; ++q)
+#pragma unroll
+      for (int j = 0; j < EPL; ++j)
+        part[q][j] = (p0 + q < a.splits && lane + 32 * j < a.E)
+                         ? __ldg(row + (int64_t)(p0 + q) * a.split_stride + 32 * j)
+                         : 0.0f;
+#pragma unroll
+    for (int q = 0; q < P; ++q)
+      if (p0 + q < a.splits)
+#pragma unroll
+        for (int j = 0; j < EPL; ++j) l[j] += (double)part[q][j];
   }
 }
 
@@ -686,16 +723,20 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     int n_refined = 0;
     if (a.cand) {
       // experts the one-pass router found near a decision boundary, already recomputed in binary64
+      // lane q reads candidate q, then each value goes to the lane that owns its expert
       const int32_t* c = a.cand + i * (kRouteCandMax + 1);
       const double* cv = a.cand_val + i * (kRouteCandMax + 1);
       const int nc = c[0];
+      const int my_e = lane < nc ? c[1 + lane] : -1;
+      const double my_v = lane < nc ? cv[1 + lane] : 0.0;
       for (int q = 0; q < nc; ++q) {
-        const int e = c[1 + q];
+        const int e = __shfl_sync(kFull, my_e, q);
+        const double v = __shfl_sync(kFull, my_v, q);
         if ((e & 31) == lane) {
 #pragma unroll
           for (int j = 0; j < EPL; ++j)
             if (j == (e >> 5)) {
-              l[j] = cv[1 + q];
+              l[j] = v;
               exact |= 1u << j;
             }
         }
@@ -1087,6 +1128,15 @@ cudaError_t launch_route(const RouteArgs& a, cudaStream_t s) {
     case 4: return full ? launch_route_t<4, true>(a, s) : launch_route_t<4, false>(a, s);
     default: return full ? launch_route_t<8, true>(a, s) : launch_route_t<8, false>(a, s);
   }
+}
+
+cudaError_t launch_sum_splits(float* logits, int32_t splits, int64_t split_stride, int64_t n, int64_t ld, int32_t E,
+                              cudaStream_t s) {
+  if (n <= 0 || splits <= 1) return cudaSuccess;
+  const int64_t blocks = ceil_div(n * E, 256);
+  sum_splits_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, s>>>(logits, splits, split_stride, n,
+                                                                                     ld, E);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gates(const RouteArgs& a, cudaStream_t s) {
