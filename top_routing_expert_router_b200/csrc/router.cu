@@ -37,24 +37,35 @@ struct VE {
   int e;
 };
 
-// Best of the warp: larger value, then lower index. Every lane gets the result.
-__device__ __forceinline__ VE warp_best(VE x) {
-#pragma unroll
-  for (int off = 16; off; off >>= 1) {
-    const double ov = __shfl_xor_sync(kFull, x.v, off);
-    const int oe = __shfl_xor_sync(kFull, x.e, off);
-    if (ov > x.v || (ov == x.v && oe < x.e)) {
-      x.v = ov;
-      x.e = oe;
-    }
-  }
-  return x;
+// Order-preserving key of a double: a larger value has a larger key. -0 is taken as +0 first, so
+// that the two have one key as they compare equal.
+__device__ __forceinline__ unsigned long long order_key(double v) {
+  const unsigned long long b = (unsigned long long)__double_as_longlong(v + 0.0);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
+// The value of an order key (-0 comes back as +0).
+__device__ __forceinline__ double key_value(unsigned long long key) {
+  return __longlong_as_double((long long)((key >> 63) ? (key & 0x7FFFFFFFFFFFFFFFull) : ~key));
+}
+
+// Lane holding the largest key of the warp (the lowest such lane on equal keys), by two warp
+// reductions over the key's halves and a ballot.
+__device__ __forceinline__ int warp_argmax_key(unsigned long long key) {
+  const unsigned hi = (unsigned)(key >> 32), lo = (unsigned)key;
+  const unsigned best_hi = __reduce_max_sync(kFull, hi);
+  const unsigned best_lo = __reduce_max_sync(kFull, hi == best_hi ? lo : 0u);
+  return __ffs(__ballot_sync(kFull, hi == best_hi && lo == best_lo)) - 1;
+}
+
+// Largest value of the warp (two warp reductions over its order key, then the value itself).
 __device__ __forceinline__ double warp_max(double v) {
-#pragma unroll
-  for (int off = 16; off; off >>= 1) v = fmax(v, __shfl_xor_sync(kFull, v, off));
-  return v;
+  const unsigned long long key = order_key(v);
+  const unsigned hi = (unsigned)(key >> 32), lo = (unsigned)key;
+  const unsigned best_hi = __reduce_max_sync(kFull, hi);
+  const unsigned best_lo = __reduce_max_sync(kFull, hi == best_hi ? lo : 0u);
+  const int src = __ffs(__ballot_sync(kFull, hi == best_hi && lo == best_lo)) - 1;
+  return __shfl_sync(kFull, v, src);
 }
 
 __device__ __forceinline__ double warp_sum(double v) {
@@ -196,23 +207,18 @@ __device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const 
 template <int EPL>
 __device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
                                  double delta_v, uint32_t* elig, uint32_t* mark) {
+  // The two best values of every group on integer order keys (warp reductions; binary64
+  // comparisons and min/max are slow next to integer ones when many warps decide at once): the
+  // best lane, then the best of the other lanes (equal to the first on a tie).
+  const int lane = threadIdx.x & 31;
   double t1[EPL], t2[EPL];
 #pragma unroll
   for (int g = 0; g < EPL; ++g) {
-    t1[g] = valid[g] ? v[g] : -INFINITY;
-    t2[g] = -INFINITY;
-  }
-#pragma unroll
-  for (int off = 16; off; off >>= 1) {
-#pragma unroll
-    for (int g = 0; g < EPL; ++g) {
-      const double o1 = __shfl_xor_sync(kFull, t1[g], off);
-      const double o2 = __shfl_xor_sync(kFull, t2[g], off);
-      const double hi = fmax(t1[g], o1);
-      const double lo = fmax(fmin(t1[g], o1), fmax(t2[g], o2));
-      t1[g] = hi;
-      t2[g] = lo;
-    }
+    const unsigned long long key = order_key(valid[g] ? v[g] : -INFINITY);
+    const int w1 = warp_argmax_key(key);
+    const int w2 = warp_argmax_key(lane == w1 ? 0ull : key);
+    t1[g] = __shfl_sync(kFull, valid[g] ? v[g] : -INFINITY, w1);
+    t2[g] = __shfl_sync(kFull, valid[g] ? v[g] : -INFINITY, w2);
   }
   double gs[EPL], gu[EPL];
 #pragma unroll
@@ -224,11 +230,14 @@ __device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], con
   }
   uint32_t keep = 0;
   double min_kept = INFINITY, max_drop = -INFINITY;
+  unsigned long long gk[EPL];  // group scores as order keys: larger score, larger key
+#pragma unroll
+  for (int g = 0; g < EPL; ++g) gk[g] = order_key(gs[g]);
 #pragma unroll
   for (int g = 0; g < EPL; ++g) {
     int better = 0;
 #pragma unroll
-    for (int h = 0; h < EPL; ++h) better += (gs[h] > gs[g]) || (gs[h] == gs[g] && h < g);
+    for (int h = 0; h < EPL; ++h) better += (gk[h] > gk[g]) || (gk[h] == gk[g] && h < g);
     if (better < a.topk_group) {
       keep |= 1u << g;
       min_kept = fmin(min_kept, gs[g] - gu[g]);
@@ -294,17 +303,28 @@ __device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exac
   int prev_e = -1;
   bool prev_exact = true;
   double top_lo = INFINITY;  // min over the kept experts of v - u
-  for (int r = 0; r < want; ++r) {
-    VE best{-INFINITY, 0x7FFFFFFF};
+  unsigned long long vk[EPL];  // selection values as order keys
 #pragma unroll
-    for (int j = 0; j < EPL; ++j) {
-      const int e = lane + 32 * j;
-      if (((elig_mask & ~taken) >> j) & 1u && (v[j] > best.v || (v[j] == best.v && e < best.e))) {
-        best.v = v[j];
-        best.e = e;
+  for (int j = 0; j < EPL; ++j) vk[j] = order_key(v[j]);
+  for (int r = 0; r < want; ++r) {
+    // this lane's best untaken eligible expert (lower j first on equal keys), then the warp's
+    unsigned long long bk = 0ull;
+    int bj = -1;
+#pragma unroll
+    for (int j = 0; j < EPL; ++j)
+      if (((elig_mask & ~taken) >> j) & 1u && (bj < 0 || vk[j] > bk)) {
+        bk = vk[j];
+        bj = j;
       }
-    }
-    best = warp_best(best);
+    // the lowest expert index among the lanes holding the best key: lane + 32 j, so the lowest j,
+    // then the lowest lane
+    const unsigned bhi = __reduce_max_sync(kFull, bj >= 0 ? (unsigned)(bk >> 32) : 0u);
+    const unsigned blo = __reduce_max_sync(kFull, bj >= 0 && (unsigned)(bk >> 32) == bhi ? (unsigned)bk : 0u);
+    const bool top = bj >= 0 && (unsigned)(bk >> 32) == bhi && (unsigned)bk == blo;
+    const unsigned be = __reduce_min_sync(kFull, top ? (unsigned)(lane + 32 * bj) : 0xFFFFFFFFu);
+    VE best;
+    best.e = (int)be;
+    best.v = __shfl_sync(kFull, pick(v, bj < 0 ? 0 : bj), (int)(be & 31));
     const int owner = best.e & 31, jb = best.e >> 5;
     const bool b_exact = __shfl_sync(kFull, (int)((exact >> jb) & 1u), owner) != 0;
     const double bu = b_exact ? 0.0 : delta_v;
@@ -348,11 +368,6 @@ __device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exac
   return ok;
 }
 
-// Key order of the ranking: larger value first, then lower expert index.
-__device__ __forceinline__ bool better(double va, int ea, double vb, int eb) {
-  return va > vb || (va == vb && ea < eb);
-}
-
 // Full ranking of one token's eligible experts (the capacity rule needs it),
 // by a bitonic sort across the warp: position p = lane * EPL + j. Each element
 // carries its expert index and exactness. After the sort, adjacent pairs are
@@ -376,16 +391,21 @@ __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t
     for (int j = 0; j < EPL; ++j)
       if (valid[j]) elig_mask |= 1u << j;
   }
-  // keys in sort layout: lane holds positions lane*EPL .. lane*EPL+EPL-1
-  double kv[EPL];
+  // keys in sort layout: lane holds positions lane*EPL .. lane*EPL+EPL-1. The sort compares the
+  // values' integer order keys (binary64 comparisons are slow next to integer ones when many
+  // warps sort at once); the values come back from the keys afterwards.
+  unsigned long long kk[EPL];
   int ke[EPL];  // expert | exact << 16, or -1 for empty
 #pragma unroll
   for (int j = 0; j < EPL; ++j) {
     const int e = lane + 32 * j;
     const bool el = (elig_mask >> j) & 1u;
-    kv[j] = el ? v0[j] : -INFINITY;
+    kk[j] = order_key(el ? v0[j] : -INFINITY);
     ke[j] = el ? (e | (int)(((exact >> j) & 1u) << 16)) : (0x7FFF | (1 << 16));
   }
+  auto key_better = [](unsigned long long ka, int ea, unsigned long long kb, int eb) {
+    return ka > kb || (ka == kb && ea < eb);
+  };
   constexpr int S = 32 * EPL;
 #pragma unroll
   for (int k = 2; k <= S; k <<= 1) {
@@ -398,12 +418,12 @@ __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t
           if (jp > j) {
             const int p = lane * EPL + j;
             const bool up = (p & k) == 0;  // block sorted best-first
-            const bool swap = up ? better(kv[jp], ke[jp] & 0xFFFF, kv[j], ke[j] & 0xFFFF)
-                                 : better(kv[j], ke[j] & 0xFFFF, kv[jp], ke[jp] & 0xFFFF);
+            const bool swap = up ? key_better(kk[jp], ke[jp] & 0xFFFF, kk[j], ke[j] & 0xFFFF)
+                                 : key_better(kk[j], ke[j] & 0xFFFF, kk[jp], ke[jp] & 0xFFFF);
             if (swap) {
-              const double tv = kv[j];
-              kv[j] = kv[jp];
-              kv[jp] = tv;
+              const unsigned long long tk = kk[j];
+              kk[j] = kk[jp];
+              kk[jp] = tk;
               const int te = ke[j];
               ke[j] = ke[jp];
               ke[jp] = te;
@@ -414,22 +434,25 @@ __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t
         const int ld = d / EPL;
 #pragma unroll
         for (int j = 0; j < EPL; ++j) {
-          const double ov = __shfl_xor_sync(kFull, kv[j], ld);
+          const unsigned long long ok_ = __shfl_xor_sync(kFull, kk[j], ld);
           const int oe = __shfl_xor_sync(kFull, ke[j], ld);
           const int p = lane * EPL + j;
           const bool up = (p & k) == 0;
           const bool lower = (lane & ld) == 0;  // this element sits at the smaller position
-          const bool other_better = better(ov, oe & 0xFFFF, kv[j], ke[j] & 0xFFFF);
+          const bool other_better = key_better(ok_, oe & 0xFFFF, kk[j], ke[j] & 0xFFFF);
           // the smaller position keeps the better key in an ascending block
           const bool take = (lower == up) ? other_better : !other_better;
           if (take) {
-            kv[j] = ov;
+            kk[j] = ok_;
             ke[j] = oe;
           }
         }
       }
     }
   }
+  double kv[EPL];
+#pragma unroll
+  for (int j = 0; j < EPL; ++j) kv[j] = key_value(kk[j]);
   int n_elig = __popc(elig_mask);
 #pragma unroll
   for (int off = 16; off; off >>= 1) n_elig += __shfl_xor_sync(kFull, n_elig, off);
@@ -476,8 +499,9 @@ __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t
 
 // Gate weights of the slots in idx[0..k) (entries < 0 are dropped slots).
 // Lane j < k returns the weight of slot j.
+// s_val: this warp's kMaxTopK doubles of shared memory.
 template <int EPL>
-__device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* idx_of_slot) {
+__device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* idx_of_slot, double* s_val) {
   const int lane = threadIdx.x & 31;
   double m = -INFINITY;
   if (a.score_fn == MOE_SCORE_SOFTMAX) {
@@ -493,15 +517,20 @@ __device__ float gates(const RouteArgs& a, const double (&l)[EPL], const int* id
       if (lane + 32 * j < a.E) z += exp(l[j] - m);
     z = warp_sum(z);
   }
-  double mine = 0.0;
+  // the logit of each kept expert to its slot's lane (the lane owning the expert writes it), then
+  // every slot's score at once
   for (int r = 0; r < a.k; ++r) {
     const int e = idx_of_slot[r];
-    const int src = e >= 0 ? (e & 31) : 0;
-    const double le = __shfl_sync(kFull, pick(l, e >= 0 ? (e >> 5) : 0), src);
-    double p = 0.0;
-    if (e >= 0) p = a.score_fn == MOE_SCORE_SOFTMAX ? exp(le - m) / z : raw_score(a.score_fn, le);
-    if (lane == r) mine = p;
+    if (e >= 0 && (e & 31) == lane) s_val[r] = pick(l, e >> 5);
   }
+  __syncwarp();
+  double mine = 0.0;
+  const int e_mine = lane < a.k ? idx_of_slot[lane] : -1;
+  if (e_mine >= 0) {
+    const double le = s_val[lane];
+    mine = a.score_fn == MOE_SCORE_SOFTMAX ? exp(le - m) / z : raw_score(a.score_fn, le);
+  }
+  __syncwarp();  // s_val is the next token's
   double denom = 1.0;
   if (a.renorm) denom = warp_sum(lane < a.k ? mine : 0.0);
   // a dropped slot weighs 0, also when every slot of the token was dropped
@@ -688,6 +717,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
   __shared__ int16_t s_rank[kWarpsPerBlock][kMaxExperts];
   __shared__ uint8_t s_flag[kWarpsPerBlock][kMaxExperts];
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
+  __shared__ double s_val[kWarpsPerBlock][kMaxTopK];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   constexpr bool full_ranking = FULL;  // the capacity rule needs every eligible expert ranked
   for (int i = lane; i < kMaxExperts; i += 32) s_flag[wib][i] = 0;
@@ -789,7 +819,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
     }
     if (lane < a.k) s_idx[wib][lane] = lane < nr ? (int)s_rank[wib][lane] : -1;
     __syncwarp();
-    const float w = gates<EPL>(a, l, s_idx[wib]);
+    const float w = gates<EPL>(a, l, s_idx[wib], s_val[wib]);
     if (lane < a.k) {
       a.topk_idx[t * a.k + lane] = s_idx[wib][lane];
       a.topk_w[t * a.k + lane] = w;
@@ -802,6 +832,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
 template <int EPL>
 __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a) {
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
+  __shared__ double s_val[kWarpsPerBlock][kMaxTopK];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -810,7 +841,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) gates_kernel(RouteArgs a)
     load_logits<EPL>(a, t, l);
     if (lane < a.k) s_idx[wib][lane] = a.topk_idx[t * a.k + lane];
     __syncwarp();
-    const float w = gates<EPL>(a, l, s_idx[wib]);
+    const float w = gates<EPL>(a, l, s_idx[wib], s_val[wib]);
     if (lane < a.k) a.topk_w[t * a.k + lane] = w;
     __syncwarp();
   }
