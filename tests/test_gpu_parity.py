@@ -22,12 +22,10 @@ SMALL = ["tiny_f32", "mixtral_small", "deepseek_v2_small", "deepseek_v3_small", 
 
 
 def _tile_mode(mode, monkeypatch):
-    """1sm: one-SM 128-row tiles; 2sm: SM-pair 256 x 256 tiles; 2sm_wide: SM-pair 256 x 512 tiles."""
+    """1sm: one-SM 128-row tiles; 2sm: SM-pair 256 x 256 tiles; 2sm_wide: SM-pair 256 x 512 tiles
+    (the default mix, wide gate/up tiles for small groups, runs in every other test)."""
     monkeypatch.setenv("MOE_TC_MODE", "1sm" if mode == "1sm" else "2sm")
-    if mode == "2sm_wide":
-        monkeypatch.setenv("MOE_TC_WIDE", "1")
-    else:
-        monkeypatch.delenv("MOE_TC_WIDE", raising=False)
+    monkeypatch.setenv("MOE_TC_WIDE", "1" if mode == "2sm_wide" else "0")
 
 
 TILE_MODES = ["1sm", "2sm", "2sm_wide"]

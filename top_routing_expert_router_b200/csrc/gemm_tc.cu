@@ -1068,11 +1068,14 @@ constexpr size_t kSmemBytesW = 1024 + STAGESW * STAGEW_BYTES + sizeof(SmemCtl2);
 static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448 && kSmemBytesW <= 232448,
               "dynamic shared memory above 227 KB");
 
-// Wide pair tiles (256 x 512): MOE_TC_WIDE=1 selects them for every SM-pair GEMM, MOE_TC_WIDE=gate
-// for the gate/up (SwiGLU) GEMM only.
-bool use_wide_tiles(bool swiglu) {
+// Wide pair tiles (256 x 512) for the gate/up (SwiGLU) GEMM of many small groups (at most 768 rows
+// per group on average, the DeepSeek shapes): half as many n-tiles re-read each group's rows, which
+// measured ~2 % faster there both at full clock and under the power cap, and ~1 % slower on
+// groups of ~1024 rows. MOE_TC_WIDE=1 selects them for every SM-pair GEMM, =gate for the gate/up
+// GEMM only, =0 for none.
+bool use_wide_tiles(bool swiglu, int64_t rows, int32_t groups) {
   const char* w = getenv("MOE_TC_WIDE");
-  if (!w) return false;
+  if (!w) return swiglu && groups > 1 && rows <= 768 * (int64_t)groups;
   if (w[0] == '1') return true;
   return swiglu && strcmp(w, "gate") == 0;
 }
@@ -1162,7 +1165,7 @@ cudaError_t launch_gemm_tc(const GemmArgs& a, bool swiglu, bool out_f32, moe_dia
   if (!make_map(&ma, a.A, a.M, a.K, BM)) return cudaErrorInvalidValue;
   CUtensorMap ma_half;
   if (pair && !make_map(&ma_half, a.A, a.M, a.K, BM / 2)) return cudaErrorInvalidValue;
-  const bool wide = pair && use_wide_tiles(swiglu);
+  const bool wide = pair && use_wide_tiles(swiglu, a.M, a.G);
   const int b_box_used = wide ? 128 : b_box;
   if (!make_map(&mb, a.B, b_total_rows, a.K, b_box_used)) return cudaErrorInvalidValue;
   if (swiglu) {
