@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   const int E = a.E;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
   __shared__ int cnt_s[kMaxExperts];   // counts so far (the predecessor's, then this range's commits)
-  __shared__ int hist[kMaxExperts];
+  __shared__ int hist[kMaxExperts];        // choices of the uncommitted tokens, per expert
+  __shared__ int hist_taken[kMaxExperts];  // choices of the tokens a round commits
   __shared__ uint32_t full_s[kMaxExperts / 32];
   __shared__ int cand[kMaxExperts];
   __shared__ int8_t cidx[kMaxExperts];   // place of an expert in cand (-1: not a candidate)
@@ -271,16 +272,10 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
       count_mine(1);
     }
   }
-  bool counted = true;  // hist holds the choices of every uncommitted token
+  // from here on hist holds the choices of every uncommitted token of the range
   int f = 0;  // first token of the range not committed yet (uniform across the CTA)
   for (;;) {
     const bool active = valid && tid >= f;
-    if (!counted) {
-      for (int e = tid; e < E; e += kThreads) hist[e] = 0;
-      __syncthreads();
-      for (int j = 0; j < k; ++j) warp_count(hist, active ? slot(j) : -1);
-    }
-    counted = false;
     if (tid == 0) {
       n_cand = 0;
       s_stop = kThreads;
@@ -340,20 +335,38 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
     const int stop = s_stop;  // last token committed in this step (kThreads: the rest of the range)
     const bool take = active && tid <= stop;
     if (stop < kThreads) {
-      for (int e = tid; e < E; e += kThreads) hist[e] = 0;
+      // the committed tokens' counts; hist keeps those of the tokens after them
+      for (int e = tid; e < E; e += kThreads) hist_taken[e] = 0;
       __syncthreads();
-      for (int j = 0; j < k; ++j) warp_count(hist, take ? slot(j) : -1);
+      for (int j = 0; j < k; ++j) warp_count(hist_taken, take ? slot(j) : -1);
       __syncthreads();
     }
     if (take) commit();
     for (int e = tid; e < E; e += kThreads) {
-      cnt_s[e] += hist[e];
+      if (stop < kThreads) {
+        cnt_s[e] += hist_taken[e];
+        hist[e] -= hist_taken[e];
+      } else {
+        cnt_s[e] += hist[e];
+      }
       if (cnt_s[e] >= a.C) atomicOr(&full_s[e >> 5], 1u << (e & 31));
     }
     __syncthreads();
     if (stop >= cnt_tok - 1) break;
     f = stop + 1;
-    if (valid && tid >= f) drop_full();
+    // the later tokens holding the expert that just filled walk on; the histogram follows them,
+    // so the next round needs no recount
+    if (valid && tid >= f) {
+      Slots<KA, (KT > 0)> ch0 = ch;
+      const int taken0 = taken;
+      if (drop_full()) {
+        for (int j = 0; j < k; ++j) {
+          const int e = a.policy == MOE_CAP_OVERFLOW_NEXT ? (j < taken0 ? ch0.get(j) : -1) : ch0.get(j);
+          if (e >= 0) atomicSub(&hist[e], 1);
+        }
+        count_mine(1);
+      }
+    }
   }
   // hand the counts and full set on
   for (int e = tid; e < kMaxExperts; e += kThreads) mine->cnt[e] = cnt_s[e];
