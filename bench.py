@@ -86,18 +86,48 @@ def layer_work(w, kept_slots, active_experts):
     return flops, bytes_
 
 
+def _ceil(a, b):
+    return -(-a // b)
+
+
+def _router_splits(w):
+    """Split-K factor of the two-kernel router's logits GEMM (router_splits in csrc/api.cu)."""
+    if w.dtype == "f32":
+        return 1
+    tiles = _ceil(w.n, 128) * _ceil(w.n_routed, 256)
+    if tiles >= 74:
+        return 1
+    num_kb = _ceil(w.d_model, 64)
+    ld = _ceil(w.n_routed, 4) * 4
+    s = max(1, min(148 // tiles, (4 << 20) // (w.n * ld * 4), 32, num_kb))
+    return _ceil(num_kb, _ceil(num_kb, s))
+
+
+def _fp8_gemm_launches(rows, groups):
+    """Kernels of one FP8 expert GEMM: SM-pair tiles lay out the B scale words first."""
+    if rows <= 16 * groups:
+        return 1  # 32-row short tiles
+    return 2 if rows // groups >= 128 else 1
+
+
 def launches_per_step(w):
-    """Kernels of this library launched by one moe_layer_forward."""
-    n = 2  # router GEMM + route
-    if w.cap_policy != "none":
-        n += 2  # capacity + gates
-    n += 2  # counts: histogram + scan
-    if w.dtype == "fp8":
-        n += 3  # permute: histogram + scan + scatter (the quantiser gathers the rows)
-        n += 4  # quantise x, GEMM1 (SwiGLU), quantise h, GEMM2
-        n += 4 if w.n_shared else 0
+    """Kernels of this library launched by one moe_layer_forward (the choices of csrc/api.cu)."""
+    bf16_act = w.dtype != "f32"
+    if bf16_act and w.cap_policy == "none" and w.n >= 2048 and w.top_k <= 8:
+        n = 3  # one-pass router, binary64 refinement of the queued tokens' candidates, queued tokens
     else:
-        n += 4  # permute: histogram + scan + scatter + gather
+        n = 2 if _router_splits(w) > 1 else 1  # logits GEMM (+ sum of the split-K partials)
+        n += 3 if bf16_act and w.d_model % 8 == 0 else 1  # first pass, refinement, second pass
+        if w.cap_policy != "none":
+            n += 2  # capacity + gates
+    n += 2  # histogram + scan (the permutation reuses them)
+    if w.dtype == "fp8":
+        n += 1  # scatter (the quantiser gathers the rows)
+        n += 2 + 2 * _fp8_gemm_launches(w.n * w.top_k, w.n_routed)  # quantise x and h, GEMM1, GEMM2
+        if w.n_shared:
+            n += 2 + 2 * _fp8_gemm_launches(w.n, 1)
+    else:
+        n += 2  # scatter + row copy
         n += 2  # GEMM1 (SwiGLU) + GEMM2
         n += 2 if w.n_shared else 0
     n += 1  # combine
