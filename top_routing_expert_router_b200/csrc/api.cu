@@ -105,7 +105,7 @@ Plan make_plan(const moe_config& c, int64_t n, int32_t ep_world = 0, int64_t ep_
   // binary64 logits, the list of pairs to refine
   p.batched = batched && batched_refine_possible(c);
   const bool queued = one_pass_possible(c, n) || p.batched;
-  p.rq = take(queued ? (size_t)n * 4 : 0);
+  p.rq = take(queued ? (size_t)2 * n * 4 : 0);  // the one-pass router's queue, then the refinement queue
   p.rc = take(queued ? cand_region_bytes(n) : 0);
   p.ranking = take(c.cap_policy != MOE_CAP_NONE ? (size_t)n * c.n_routed * 2 : 0);
   p.capg = take(c.cap_policy != MOE_CAP_NONE ? (size_t)capacity_grid_scratch_bytes(n, c.n_routed) : 0);
@@ -294,8 +294,8 @@ moe_status router_logits(const Ctx& x, const void* X, const moe_weights* w, int3
 }
 
 // The token queue and candidate region: queue length in the workspace's diag block; four counters
-// (pairs listed, refine cursor, second-pass cursor, spare), then the candidate table, their
-// binary64 logits, the pair list.
+// (pairs listed, refine cursor, second-pass cursor, length of the one-pass router's refinement
+// queue), then the candidate table, their binary64 logits, the pair list.
 void queue_args(const Ctx& x, RouteTcArgs* a) {
   a->queue = x.at<int32_t>(x.p.rq);
   a->queue_len = &x.status()->reserved[1];
@@ -369,16 +369,35 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
   RouteTcArgs ra;
   RouteArgs r;
   if (one_pass_args(x, X, w, idx, tw, &ra)) {
-    // decisions in the tensor-core epilogue; the queued tokens re-decided from their logits rows
-    MOE_CUDA(cudaMemsetAsync(ra.pair_count, 0, 2 * sizeof(int32_t), x.s));
+    // Decisions in the tensor-core epilogue. The tokens it could not certify (their logits rows
+    // written, their indices queued) go through the batched binary64 refinement: a first pass
+    // decides what binary64 certifies from the rows and queues the rest with the experts to
+    // refine, refine_kernel computes those, and a second pass decides the tokens it queued.
+    MOE_CUDA(cudaMemsetAsync(ra.pair_count, 0, 4 * sizeof(int32_t), x.s));
     MOE_CUDA(launch_route_tc(ra, x.s));
+    int32_t* queue2 = ra.queue + x.n;
+    int32_t* queue2_len = ra.pair_count + 3;
     r = route_args(x, X, w, idx, tw, d, 1);
     r.cursor = cursor;
     r.queue = ra.queue;
     r.queue_len = ra.queue_len;
-    r.cand = ra.cand;
-    r.cand_val = ra.cand_val;
+    r.defer_queue = queue2;
+    r.defer_len = queue2_len;
+    r.defer_cand = ra.cand;
+    r.defer_pairs = ra.pairs;
+    r.defer_pair_count = ra.pair_count;
     MOE_CUDA(launch_route(r, x.s));
+    RouteTcArgs rb = ra;
+    rb.queue = queue2;
+    MOE_CUDA(launch_refine(rb, x.s));
+    RouteArgs r2 = r;
+    r2.defer_queue = r2.defer_len = r2.defer_cand = r2.defer_pairs = r2.defer_pair_count = nullptr;
+    r2.cursor = ra.pair_count + 2;
+    r2.queue = queue2;
+    r2.queue_len = queue2_len;
+    r2.cand = ra.cand;
+    r2.cand_val = ra.cand_val;
+    MOE_CUDA(launch_route(r2, x.s));
   } else {
     MOE_TRY(router_logits(x, X, w, idx, tw, d, &r));
     r.cursor = cursor;

@@ -131,10 +131,11 @@ struct RouteTcArgs {
   float* topk_w;        // [n, k]
   float* logits;        // [n, ldl]: rows of the queued tokens
   int64_t ldl;
-  int32_t* queue;       // [n] tokens left to the binary64 router
+  int32_t* queue;       // [n] tokens left to the binary64 router (launch_refine: the refinement queue)
   int32_t* queue_len;   // zeroed before the launch
+  // launch_refine only (written by a deferring launch_route):
   int32_t* cand;        // [n][kRouteCandMax + 1] per queued token: count (-1: too many), then the experts
-                        // an uncertain comparison can involve
+                        // an uncertain comparison involves
   double* cand_val;     // [n][kRouteCandMax + 1] binary64 logits of those experts (same slots as cand)
   int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine: one run per token, padded
                         // with -1 to a multiple of four (a warp refines four pairs of one token)

@@ -112,18 +112,6 @@ __device__ __forceinline__ float sel_score(int score_fn, float l) {
   return sqrtf(fmaxf(l, 0.0f) + log1pf(expf(-fabsf(l))));
 }
 
-// Insert v into a list sorted descending (values only).
-__device__ __forceinline__ void insert_value(float (&lv)[kMaxK + 1], float v) {
-  if (!(v > lv[kMaxK])) return;
-#pragma unroll
-  for (int j = 0; j <= kMaxK; ++j)
-    if (v > lv[j]) {
-      const float t = lv[j];
-      lv[j] = v;
-      v = t;
-    }
-}
-
 // Insert (v, l, e) into the list sorted by v descending (l: what the gate needs, the logit for
 // softmax and the unbiased score otherwise); an equal v stays below the entries
 // already there, which hold lower expert indices (experts arrive in ascending order).
@@ -377,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float dv = lip * dl + eval_err;              // ... of a selection value
       // group cut: the topk_group best group scores, ties to the lower group index
       bool ok = true;
-      uint32_t kept = 0xFFFFFFFFu, involved = 0;
+      uint32_t kept = 0xFFFFFFFFu;
       if (!soft && G > 1) {
         auto gs = [&](int g) { return g < Gh ? (h ? xg_other : xg_mine)[2 + g] : (h ? xg_mine : xg_other)[2 + g - Gh]; };
         kept = 0;
@@ -396,15 +384,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             max_drop = fmaxf(max_drop, sg);
           }
         }
-        if (p.topk_group < G && !(min_kept - max_drop > 4.0f * dv + 0x1p-19f)) {
-          ok = false;
-          // the groups whose place relative to the cut is uncertain: all their experts are refined
-          for (int g = 0; g < G; ++g) {
-            const float sg = gs(g);
-            const bool in = (kept >> g) & 1u;
-            if (in ? sg <= max_drop + 4.0f * dv + 0x1p-19f : sg >= min_kept - 4.0f * dv - 0x1p-19f) involved |= 1u << g;
-          }
-        }
+        if (p.topk_group < G && !(min_kept - max_drop > 4.0f * dv + 0x1p-19f)) ok = false;
       }
       // pass 2: this half's k + 1 best eligible experts, sorted (and the softmax normaliser)
       float lv[kMaxK + 1], ll[kMaxK + 1];
@@ -505,18 +485,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j <= kMaxK; ++j) insert(lv, ll, le, ov[j], ol[j], oe[j] < 0 ? 0x7FFFFFFF : oe[j]);
       }
       // every order the result depends on must be certain: adjacent kept experts and the k-th / (k+1)-th cut
-      // (band j: the selection values an expert may have to take part in uncertain comparison j)
-      float band_lo[kMaxK], band_hi[kMaxK];
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j) {
-        band_lo[j] = INFINITY;
-        band_hi[j] = -INFINITY;
-        if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) {
-          ok = false;
-          band_lo[j] = (j + 1 < k ? lv[j + 1] : lv[j]) - 2.0f * dv;
-          band_hi[j] = (j + 1 < k ? lv[j] : lv[j + 1]) + 2.0f * dv;
-        }
-      }
+      for (int j = 0; j < kMaxK; ++j)
+        if (j < k && j + 1 < n_elig && !(lv[j] - lv[j + 1] > 2.0f * dv)) ok = false;
       const bool spill = valid && !ok;
       if (valid && ok) {
         // gates of the k kept experts
@@ -543,144 +514,27 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
       }
       // not certain: hand the token to the binary64 router with its logits row (the TMEM loads are
-      // warp-wide, so the whole warp reads when any lane spills)
+      // warp-wide, so the whole warp reads when any lane spills). That router decides it from the
+      // row in binary64, queues the experts an uncertain comparison involves for refine_kernel, and
+      // decides it again with their binary64 logits.
       if (__any_sync(0xFFFFFFFFu, spill)) {
         float* lrow = p.logits + tok * p.ldl;
-        // A token whose group cut is uncertain: once the binary64 values decide the cut, the kept
-        // set is the groups it certainly keeps (W) plus some of the uncertain ones. Its top k then
-        // lies at or above kappa, the k-th best value in W, so the experts that can matter are the
-        // eligible ones within a margin of kappa, and in the uncertain groups those that can be
-        // among their group's top two (v within a margin of the group's second best; g2min is the
-        // lowest of those).
-        const bool gunc = !soft && spill && involved != 0;
-        const bool any_gunc = __any_sync(0xFFFFFFFFu, gunc);
-        float kv[kMaxK + 1];
-#pragma unroll
-        for (int j = 0; j <= kMaxK; ++j) kv[j] = -INFINITY;
-        float g2min = INFINITY;
-        {
-          float t1 = -INFINITY, t2 = -INFINITY;
-          int g = 0, r = 0;
-          for (int c0 = 0; c0 < E; c0 += 32) {
-            float l[32];
-            tmem_ld32(taddr + (uint32_t)c0, l);
-            if (spill) {
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                if (c0 + j + 4 <= E) {
-                  *reinterpret_cast<float4*>(lrow + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
-                } else {
-#pragma unroll
-                  for (int u = 0; u < 4; ++u)
-                    if (c0 + j + u < E) lrow[c0 + j + u] = l[j + u];
-                }
-            }
-            if (any_gunc) {
-              uint32_t hit = 0;
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                const float v = c0 + j < E ? sel_score(SF, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0] : -INFINITY;
-                l[j] = v;
-                if (c0 + j < E) {
-                  t2 = fmaxf(t2, fminf(t1, v));
-                  t1 = fmaxf(t1, v);
-                  if ((((kept & ~involved) >> g) & 1u) && v > kv[kMaxK]) hit |= 1u << j;
-                  if (++r == per) {
-                    if ((involved >> g) & 1u) g2min = fminf(g2min, t2);
-                    t1 = t2 = -INFINITY;
-                    r = 0;
-                    ++g;
-                  }
-                }
-              }
-              if (!gunc) hit = 0;
-              while (hit) {
-                const int j = __ffs(hit) - 1;
-                hit &= hit - 1;
-                float v = 0.0f;
-#pragma unroll
-                for (int u = 0; u < 32; ++u) v = u == j ? l[u] : v;
-                insert_value(kv, v);
-              }
-            }
-          }
-        }
-        float kappa = -INFINITY;  // stays -inf when W holds fewer than k experts
-#pragma unroll
-        for (int j = 0; j < kMaxK; ++j) kappa = j == k - 1 ? kv[j] : kappa;
-        // the experts an uncertain comparison can involve: eligible ones whose value lies in one of
-        // the bands and, for an uncertain group cut, those picked by kappa and g2min above. Their
-        // logits are recomputed in binary64 (one warp per expert, refine_kernel) before the
-        // binary64 router decides the token again.
-        int32_t* cand = nullptr;
-        int qpos = 0;
-        if (spill) {
-          qpos = atomicAdd(p.queue_len, 1);
-          p.queue[qpos] = (int32_t)tok;
-          cand = p.cand + (int64_t)qpos * (kCandMax + 1);
-        }
-        int nc = 0;
-        float hull_lo = INFINITY, hull_hi = -INFINITY;  // the bands' hull: a cheap first test
-#pragma unroll
-        for (int b = 0; b < kMaxK; ++b) {
-          hull_lo = fminf(hull_lo, band_lo[b]);
-          hull_hi = fmaxf(hull_hi, band_hi[b]);
-        }
         for (int c0 = 0; c0 < E; c0 += 32) {
           float l[32];
           tmem_ld32(taddr + (uint32_t)c0, l);
           if (spill) {
-            // candidates of the chunk as a bit mask: after an uncertain group cut, the experts of
-            // kept or uncertain groups within 4 dv of kappa and those of uncertain groups within
-            // 4 dv of g2min; and eligible experts inside the bands' hull (tested against each band below)
-            uint32_t hit = 0, grp = 0;
-            int g = c0 / per, r = c0 - g * per;
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const bool in = c0 + j < E;
-              const float v = soft ? l[j] : sel_score(SF, l[j]) + sbias[c0 + j < 256 ? c0 + j : 0];
-              l[j] = v;
-              if (in && gunc) {
-                if ((((kept | involved) >> g) & 1u) && v >= kappa - 4.0f * dv) grp |= 1u << j;
-                if (((involved >> g) & 1u) && v >= g2min - 4.0f * dv) grp |= 1u << j;
+            for (int j = 0; j < 32; j += 4)
+              if (c0 + j + 4 <= E) {
+                *reinterpret_cast<float4*>(lrow + c0 + j) = make_float4(l[j], l[j + 1], l[j + 2], l[j + 3]);
+              } else {
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  if (c0 + j + u < E) lrow[c0 + j + u] = l[j + u];
               }
-              if (in && ((kept >> g) & 1u) && v >= hull_lo && v <= hull_hi) hit |= 1u << j;
-              if (++r == per) {
-                r = 0;
-                ++g;
-              }
-            }
-            uint32_t want = grp;
-            while (hit) {
-              const int j = __ffs(hit) - 1;
-              hit &= hit - 1;
-              float v = 0.0f;
-#pragma unroll
-              for (int u = 0; u < 32; ++u) v = u == j ? l[u] : v;
-              bool in_band = false;
-#pragma unroll
-              for (int b = 0; b < kMaxK; ++b) in_band |= v >= band_lo[b] && v <= band_hi[b];
-              if (in_band) want |= 1u << j;
-            }
-            while (want) {
-              const int j = __ffs(want) - 1;
-              want &= want - 1;
-              if (nc < kCandMax) cand[1 + nc] = c0 + j;
-              ++nc;
-            }
           }
         }
-        if (spill) {
-          if (nc <= kCandMax) {
-            cand[0] = nc;
-            // one run per token, padded to a multiple of four (refine_kernel takes four pairs at a time)
-            const int padded = (nc + 3) & ~3;
-            const int base = atomicAdd(p.pair_count, padded);
-            for (int c = 0; c < padded; ++c) p.pairs[base + c] = c < nc ? qpos * (kCandMax + 1) + 1 + c : -1;
-          } else {
-            cand[0] = -1;  // too many: the binary64 router finds and refines them itself
-          }
-        }
+        if (spill) p.queue[atomicAdd(p.queue_len, 1)] = (int32_t)tok;
       }
       fence_before();
       __syncwarp();
@@ -823,10 +677,6 @@ cudaError_t launch_route_tc(const RouteTcArgs& a, cudaStream_t s) {
   const int64_t tiles = ceil_div(a.n, BM);
   const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
   kern<<<grid, kThreads, kSmemBytes, s>>>(mx, mw, a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  // binary64 logits of the queued tokens' candidate experts, every pair at once
-  refine_kernel<<<(unsigned)(sms * 8), 256, 0, s>>>(a, a.pair_count + 1);
   return cudaGetLastError();
 }
 
