@@ -384,6 +384,7 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     r.defer_queue = queue2;
     r.defer_len = queue2_len;
     r.defer_cand = ra.cand;
+    r.defer_cand_val = ra.cand_val;
     r.defer_pairs = ra.pairs;
     r.defer_pair_count = ra.pair_count;
     MOE_CUDA(launch_route(r, x.s));
@@ -392,6 +393,7 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
     MOE_CUDA(launch_refine(rb, x.s));
     RouteArgs r2 = r;
     r2.defer_queue = r2.defer_len = r2.defer_cand = r2.defer_pairs = r2.defer_pair_count = nullptr;
+    r2.defer_cand_val = nullptr;
     r2.cursor = ra.pair_count + 2;
     r2.queue = queue2;
     r2.queue_len = queue2_len;
@@ -409,12 +411,14 @@ moe_status route_impl(const Ctx& x, const void* X, const moe_weights* w, int32_t
       r.defer_queue = ra.queue;
       r.defer_len = ra.queue_len;
       r.defer_cand = ra.cand;
+      r.defer_cand_val = ra.cand_val;
       r.defer_pairs = ra.pairs;
       r.defer_pair_count = ra.pair_count;
       MOE_CUDA(launch_route(r, x.s));
       MOE_CUDA(launch_refine(ra, x.s));
       RouteArgs r2 = r;
       r2.defer_queue = r2.defer_len = r2.defer_cand = r2.defer_pairs = r2.defer_pair_count = nullptr;
+      r2.defer_cand_val = nullptr;
       r2.cursor = ra.pair_count + 2;
       r2.queue = ra.queue;
       r2.queue_len = ra.queue_len;

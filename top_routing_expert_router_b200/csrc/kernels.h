@@ -106,6 +106,7 @@ struct RouteArgs {
   int32_t* defer_queue = nullptr;
   int32_t* defer_len = nullptr;        // zeroed before the launch
   int32_t* defer_cand = nullptr;
+  double* defer_cand_val = nullptr;    // zeroed for every listed candidate (launch_refine adds into it)
   int32_t* defer_pairs = nullptr;
   int32_t* defer_pair_count = nullptr; // zeroed before the launch
 };
@@ -136,7 +137,8 @@ struct RouteTcArgs {
   // launch_refine only (written by a deferring launch_route):
   int32_t* cand;        // [n][kRouteCandMax + 1] per queued token: count (-1: too many), then the experts
                         // an uncertain comparison involves
-  double* cand_val;     // [n][kRouteCandMax + 1] binary64 logits of those experts (same slots as cand)
+  double* cand_val;     // [n][kRouteCandMax + 1] binary64 logits of those experts (same slots as cand;
+                        // zero before launch_refine, which adds two partial sums into each)
   int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine: one run per token, padded
                         // with -1 to a multiple of four (a warp refines four pairs of one token)
   int32_t* pair_count;  // [2] zeroed before the launch: pairs listed, refine cursor

@@ -553,9 +553,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Binary64 logits x[t] . W_r[e] of the listed (queued token, candidate expert) pairs. Each token's
 // pairs are listed as one run padded with -1 to a multiple of four, so a warp takes four pairs of
-// one token: the token's row is read and widened once for the four experts. Products of two bf16
-// values are exact in binary64; the sums are DFMA, the lanes taking 16-byte chunks in turn with
-// four chunks of every row in flight.
+// one token and one half of the rows: the token's row is read and widened once for the four
+// experts. Products of two bf16 values are exact in binary64; the sums are DFMA, the lanes taking
+// 16-byte chunks in turn with four chunks of every row in flight. The two halves' sums are added
+// into the zeroed candidate values (two terms: the same result in either order).
 __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_t* cursor_base) {
   constexpr int U = 4;
   int32_t* cursor = const_cast<int32_t*>(cursor_base);
@@ -563,10 +564,12 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_
   const int quads = *p.pair_count / 4;
   const int nchunk = p.d / 8;
   for (;;) {
-    int i = 0;
-    if (lane == 0) i = atomicAdd(cursor, 1);
-    i = __shfl_sync(0xFFFFFFFFu, i, 0);
-    if (i >= quads) break;
+    int item = 0;
+    if (lane == 0) item = atomicAdd(cursor, 1);
+    item = __shfl_sync(0xFFFFFFFFu, item, 0);
+    if (item >= 2 * quads) break;
+    const int i = item >> 1, half = item & 1;
+    const int c_lo = half ? nchunk / 2 : 0, c_hi = half ? nchunk : nchunk / 2;
     int slot[4], e[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -580,14 +583,14 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_
     for (int q = 0; q < 4; ++q)
       wr[q] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.w_r) + (int64_t)(e[q] < 0 ? 0 : e[q]) * p.d);
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int c = lane; c < nchunk; c += 32 * U) {
+    for (int c = c_lo + lane; c < c_hi; c += 32 * U) {
       uint4 xv[U], wv[4][U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int cc = c + 32 * u;
-        xv[u] = cc < nchunk ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
+        xv[u] = cc < c_hi ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) wv[q][u] = (cc < nchunk && e[q] >= 0) ? __ldg(wr[q] + cc) : make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 4; ++q) wv[q][u] = (cc < c_hi && e[q] >= 0) ? __ldg(wr[q] + cc) : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
@@ -606,7 +609,7 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_
       double v = acc[q];
 #pragma unroll
       for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-      if (lane == 0 && slot[q] >= 0) p.cand_val[slot[q]] = v;
+      if (lane == 0 && slot[q] >= 0) atomicAdd(&p.cand_val[slot[q]], v);
     }
   }
 }
@@ -688,8 +691,8 @@ cudaError_t launch_refine(const RouteTcArgs& a, cudaStream_t s) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (sms <= 0) sms = 148;
-  // at most one warp per four listed pairs, and n * kRouteCandMax pairs can be listed
-  const int64_t need = ceil_div(a.n * kCandMax / 4, 8);
+  // at most two warps per four listed pairs, and n * kRouteCandMax pairs can be listed
+  const int64_t need = ceil_div(a.n * kCandMax / 2, 8);
   const unsigned grid = (unsigned)(need < sms * 8 ? need : sms * 8);
   refine_kernel<<<grid, 256, 0, s>>>(a, a.pair_count + 1);
   return cudaGetLastError();

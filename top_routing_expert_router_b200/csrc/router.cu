@@ -685,6 +685,7 @@ __device__ void defer_token(const RouteArgs& a, int64_t t, uint32_t refine) {
   }
   qpos = __shfl_sync(kFull, qpos, 0);
   int32_t* cand = a.defer_cand + (int64_t)qpos * (kRouteCandMax + 1);
+  double* cand_val = a.defer_cand_val + (int64_t)qpos * (kRouteCandMax + 1);
   const uint32_t below = (1u << lane) - 1u;
   int nc = 0;
 #pragma unroll
@@ -692,7 +693,10 @@ __device__ void defer_token(const RouteArgs& a, int64_t t, uint32_t refine) {
     const bool mine = (refine >> j) & 1u;
     const uint32_t m = __ballot_sync(kFull, mine);
     const int pos = nc + __popc(m & below);
-    if (mine && pos < kRouteCandMax) cand[1 + pos] = lane + 32 * j;
+    if (mine && pos < kRouteCandMax) {
+      cand[1 + pos] = lane + 32 * j;
+      cand_val[1 + pos] = 0.0;  // the refinement adds its two halves' sums here
+    }
     nc += __popc(m);
   }
   if (nc <= kRouteCandMax) {
