@@ -70,8 +70,8 @@
  *     MOE_TC_MODE=1sm|2sm forces the one-SM or SM-pair bf16 expert GEMM;
  *     MOE_TC_WIDE=1|gate|0 gives the SM-pair bf16 GEMMs (all, the gate/up one
  *     only, or none) 256 x 512 tiles instead of 256 x 256; unset, the gate/up
- *     GEMM takes them when its groups average at most 768 rows or it has one
- *     group (the shared experts);
+ *     GEMM takes them when its groups average at most 768 rows, and both GEMMs
+ *     of one group (the shared experts) do;
  *     MOE_CAP_MODE=1cta runs the capacity rule on one CTA instead of the
  *     cooperative grid;
  *     MOE_FP8_BN=128|256|pair|s128|s256 forces an FP8 expert GEMM tile shape

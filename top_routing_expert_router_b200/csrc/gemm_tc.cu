@@ -1068,15 +1068,16 @@ constexpr size_t kSmemBytesW = 1024 + STAGESW * STAGEW_BYTES + sizeof(SmemCtl2);
 static_assert(kSmemBytes <= 232448 && kSmemBytes2 <= 232448 && kSmemBytesW <= 232448,
               "dynamic shared memory above 227 KB");
 
-// Wide pair tiles (256 x 512) for the gate/up (SwiGLU) GEMM of many small groups (at most 768 rows
-// per group on average, the DeepSeek shapes) and of one dense group (the shared experts): half as
-// many n-tiles re-read each group's rows. Measured ~2 % faster on the routed DeepSeek shapes and
-// 4-7 % on the V3 shared expert, at full clock and under the power cap, and ~1 % slower on groups
-// of ~1024 rows. MOE_TC_WIDE=1 selects them for every SM-pair GEMM, =gate for the gate/up GEMM
-// only, =0 for none.
+// Wide pair tiles (256 x 512): half as many n-tiles re-read each group's rows. Taken by the gate/up
+// (SwiGLU) GEMM of many small groups (at most 768 rows per group on average, the DeepSeek shapes)
+// and by both GEMMs of one dense group (the shared experts). Measured ~2 % faster on the routed
+// DeepSeek gate/up GEMM and 4-7 % on the V3 shared expert's, and 3-4 % more on the shared down
+// GEMM, at full clock and under the power cap. The grouped down GEMM (K = 2048 or less) and groups
+// of ~1024 rows are slower with them: a wide tile's epilogue cannot overlap the next tile.
+// MOE_TC_WIDE=1 selects them for every SM-pair GEMM, =gate for the gate/up GEMM only, =0 for none.
 bool use_wide_tiles(bool swiglu, int64_t rows, int32_t groups) {
   const char* w = getenv("MOE_TC_WIDE");
-  if (!w) return swiglu && (groups == 1 || rows <= 768 * (int64_t)groups);
+  if (!w) return groups == 1 || (swiglu && rows <= 768 * (int64_t)groups);
   if (w[0] == '1') return true;
   return swiglu && strcmp(w, "gate") == 0;
 }
