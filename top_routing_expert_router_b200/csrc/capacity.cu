@@ -11,16 +11,18 @@
 //
 // Between two fill events every token's choice depends only on the set F of
 // full experts. The tokens are cut into ranges of 1024, one per CTA, one token
-// per thread; a CTA resolves its own range like the one-CTA kernel does a
-// window: it counts its tokens' choices, finds the first token at which some
-// expert reaches C (ballot prefixes in token order), commits up to it, marks
-// the expert full, lets the later tokens walk on, and repeats. The counts and
-// full set it starts from are its predecessor's final ones, handed over
-// through a flag (release/acquire); while it waits, its tokens' rankings are
-// already staged and their choices taken under no full expert, so only the
-// tokens that held an expert filled upstream walk on afterwards. The grid is
-// launched cooperatively (every CTA resident, so a wait always ends), and
-// every wait is bounded.
+// per thread; a CTA resolves its range in rounds: from its tokens' current
+// choices it finds the first token at which some expert reaches C (ballot
+// prefixes in token order), marks that expert full, lets the later tokens that
+// held it walk on, and repeats. The tokens before the filling token keep their
+// choices for good. The counts it starts from are its predecessor's final ones
+// (an expert is full once its count reaches C, and a full expert's count is
+// exactly C), each handed over as its own self-validating word; while it
+// waits, its tokens' rankings are already staged and their choices taken under
+// the full set of the CTA two places up the chain, so only the tokens that
+// held an expert filled just upstream walk on afterwards. The grid is launched
+// cooperatively (every CTA resident, so a wait always ends), and every wait is
+// bounded.
 #include "common.cuh"
 #include "kernels.h"
 #include "ptx.cuh"
@@ -35,37 +37,73 @@ constexpr int kThreads = 1024;  // tokens per CTA
 constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;
 constexpr int kPrefix = 64;  // ranking entries per token staged in shared memory
 constexpr size_t kMaxDynSmem = 200 * 1024;  // dynamic shared memory of the largest grid
+constexpr int kPosWords = 17;  // 32-bit words per token of the inverse ranking (64 bytes + 4: odd stride)
 
 // 32-bit words per staged ranking prefix of P entries: enough for P and odd, so that lanes reading
 // the same position of their rows hit 32 different banks.
 __host__ __device__ constexpr int prefix_words(int P) { return ((P + 1) / 2) | 1; }
+// Up to 64 experts (E a multiple of 8) every token's whole ranking is staged, and its inverse too.
+__host__ __device__ constexpr bool mask_capable(int E) { return E <= 64 && E % 8 == 0; }
 
-// State handed from CTA b to CTA b + 1: the counts and the full set after CTA b's tokens, and a
-// flag (0: not yet, 1: ready, 2: the chain was abandoned upstream).
+// State handed from CTA b to CTA b + 1: the expert counts after CTA b's tokens, word e holding
+// count[e] + 1 (0: not written yet; kAbandoned: the chain was abandoned upstream). Each word is
+// valid on its own, so a reader waits on exactly the words it needs and no fence or flag orders
+// them; the full set is the experts whose count reached C.
 struct ChainState {
-  int32_t flag;
-  uint32_t full[kMaxExperts / 32];
-  int32_t cnt[kMaxExperts];
+  uint32_t cnt[kMaxExperts];
 };
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+constexpr uint32_t kAbandoned = 0xFFFFFFFFu;
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
   uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
-// Bounded wait (thread 0) for the predecessor's state; false if it never came or was abandoned.
-__device__ bool wait_for(const ChainState* prev, moe_diag* status) {
+// Bounded wait for one word of a predecessor's state: count + 1, or 0 if it never came (timeout,
+// status set) or the chain was abandoned.
+__device__ uint32_t wait_word(const uint32_t* w, moe_diag* status) {
+  uint32_t v = ld_relaxed(w);
+  if (v != 0) return v == kAbandoned ? 0u : v;
   const uint64_t t0 = globaltimer();
   for (;;) {
-    const uint32_t f = ld_acquire(reinterpret_cast<const uint32_t*>(&prev->flag));
-    if (f == 1) return true;
-    if (f == 2) return false;
+    __nanosleep(32);
+    v = ld_relaxed(w);
+    if (v != 0) return v == kAbandoned ? 0u : v;
     if (globaltimer() - t0 > kBarrierTimeoutNs) {
       set_status(status, MOE_ERR_TIMEOUT);
-      return false;
+      return 0;
     }
-    __nanosleep(32);
   }
+}
+
+// Every thread of the CTA: the counts (cnt != nullptr) and the full set of a predecessor's state,
+// thread e waiting on word e; false (uniform) if any word never came.
+__device__ bool take_state(const ChainState* src, int E, int64_t C, int* cnt, uint32_t* full, int* s_ok,
+                           moe_diag* status) {
+  const int tid = threadIdx.x;
+  if (tid == 0) *s_ok = 1;
+  __syncthreads();
+  bool is_full = false;
+  if (tid < E) {
+    const uint32_t v = wait_word(&src->cnt[tid], status);
+    if (v == 0) *s_ok = 0;
+    const int c = (int)(v - 1u);
+    if (cnt) cnt[tid] = v ? c : 0;
+    is_full = v != 0 && c >= C;
+  }
+  const unsigned bits = __ballot_sync(0xFFFFFFFFu, is_full);
+  if (tid < kMaxExperts && (tid & 31) == 0) full[tid >> 5] = bits;
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+// Mark this CTA's state abandoned, so that the CTAs after it stop waiting.
+__device__ void abandon(ChainState* mine, int E) {
+  for (int e = threadIdx.x; e < E; e += blockDim.x) st_relaxed(&mine->cnt[e], kAbandoned);
 }
 
 // counts[e] += 1 for every lane whose slot holds e (e < 0: nothing), one shared-memory atomic per
@@ -107,49 +145,87 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   const int k = KT > 0 ? KT : a.k;
   const int E = a.E;
   const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
-  __shared__ int cnt_s[kMaxExperts];   // counts so far (the predecessor's, then this range's commits)
-  __shared__ int hist[kMaxExperts];        // choices of the uncommitted tokens, per expert
-  __shared__ int hist_taken[kMaxExperts];  // choices of the tokens a round commits
+  __shared__ int cnt0[kMaxExperts];     // counts before this range (the predecessor's)
+  __shared__ int hist[kMaxExperts];     // the current choices of the range's tokens, per expert
+                                        // (exact for experts that are not full)
   __shared__ uint32_t full_s[kMaxExperts / 32];
+  __shared__ uint32_t applied_s[2];     // mask mode: the full set the tokens' masks already exclude
   __shared__ int cand[kMaxExperts];
-  __shared__ int8_t cidx[kMaxExperts];   // place of an expert in cand (-1: not a candidate)
-  __shared__ int n_cand;
+  __shared__ int cstop[kMaxExperts];    // per candidate: the token at which it reaches C
   __shared__ uint32_t bal[32][kThreads / 32];  // per candidate of a batch: which tokens of each warp hold it
   __shared__ int s_stop;
   __shared__ int s_ok;
   __shared__ unsigned long long s_over, s_drop;
   extern __shared__ uint32_t srows[];  // the tokens' ranking prefixes (kPrefix entries, odd word stride)
-  const int64_t t = (int64_t)blockIdx.x * kThreads + tid;
+  const int64_t t0 = (int64_t)blockIdx.x * kThreads;
+  const int64_t t = t0 + tid;
   const bool valid = t < a.n;
-  const int cnt_tok = (int)((a.n - (int64_t)blockIdx.x * kThreads) < kThreads ? (a.n - (int64_t)blockIdx.x * kThreads)
-                                                                               : kThreads);
+  const int cnt_tok = (int)((a.n - t0) < kThreads ? (a.n - t0) : kThreads);
   const uint16_t* row = a.ranking + (valid ? t : 0) * E;
-  // the first P entries of this token's ranking in shared memory: a token walking past full experts
-  // reads them at shared-memory latency instead of one dependent global load per step
+  // the first P entries of every token's ranking in shared memory: a token walking past full
+  // experts reads them at shared-memory latency instead of one dependent global load per step
   const int P = E < kPrefix ? E : kPrefix;
-  uint32_t* srow32 = srows + tid * prefix_words(P);
+  const int pw = prefix_words(P);
+  uint32_t* srow32 = srows + tid * pw;
   const uint16_t* srow = reinterpret_cast<const uint16_t*>(srow32);
-  if (valid) {
-    if (E % 8 == 0) {
-      const uint4* src = reinterpret_cast<const uint4*>(row);
-      for (int v = 0; v < P / 8; ++v) {
-        const uint4 q4 = src[v];
-        srow32[4 * v] = q4.x;
-        srow32[4 * v + 1] = q4.y;
-        srow32[4 * v + 2] = q4.z;
-        srow32[4 * v + 3] = q4.w;
-      }
-    } else {
-      uint16_t* d16 = reinterpret_cast<uint16_t*>(srow32);
-      for (int c = 0; c < P; ++c) d16[c] = row[c];
+  // Mask mode (OVERFLOW_NEXT, at most 64 experts): a token's choices are the first k positions of
+  // its ranking whose experts are not full, kept as a 64-bit mask of the available positions; the
+  // inverse ranking turns an expert that fills into the one bit it clears, so a token whose expert
+  // filled finds its next choice at once instead of stepping past every full expert. The first two
+  // CTAs, whose staging is on the chain's critical path and which meet few full experts, walk.
+  const bool mm = a.policy == MOE_CAP_OVERFLOW_NEXT && mask_capable(E) && blockIdx.x >= 2;
+  uint8_t* pos_of = reinterpret_cast<uint8_t*>(srows + kThreads * pw);  // [kThreads][kPosWords words]
+  if (mm)
+    for (int w = 0; w < kPosWords; ++w) reinterpret_cast<uint32_t*>(pos_of)[tid * kPosWords + w] = 0xFFFFFFFFu;
+  if (E % 8 == 0) {
+    // the range's rows are contiguous: consecutive threads load consecutive 16-byte pieces, all of
+    // a thread's loads in flight before the first store
+    const int U = P / 8, R = E / 8;
+    const int total = cnt_tok * U;
+    const uint4* src = reinterpret_cast<const uint4*>(a.ranking + t0 * E);
+    uint4 q4[kPrefix / 8];
+#pragma unroll
+    for (int v = 0; v < kPrefix / 8; ++v) {
+      const int idx = tid + v * kThreads;
+      if (idx < total) q4[v] = __ldg(&src[(int64_t)(idx / U) * R + idx % U]);
     }
+#pragma unroll
+    for (int v = 0; v < kPrefix / 8; ++v) {
+      const int idx = tid + v * kThreads;
+      if (idx < total) {
+        uint32_t* d = srows + (idx / U) * pw + 4 * (idx % U);
+        d[0] = q4[v].x;
+        d[1] = q4[v].y;
+        d[2] = q4[v].z;
+        d[3] = q4[v].w;
+      }
+    }
+    if (mm) {
+      __syncthreads();  // every row's 0xFF (not ranked) fill is down
+#pragma unroll
+      for (int v = 0; v < kPrefix / 8; ++v) {
+        const int idx = tid + v * kThreads;
+        if (idx < total) {
+          uint8_t* inv = pos_of + (idx / U) * (kPosWords * 4);
+          const uint32_t w4[4] = {q4[v].x, q4[v].y, q4[v].z, q4[v].w};
+#pragma unroll
+          for (int h = 0; h < 8; ++h) {
+            const uint32_t e = (w4[h >> 1] >> (16 * (h & 1))) & 0xFFFFu;
+            if (e < 64u) inv[e] = (uint8_t)(8 * (idx % U) + h);
+          }
+        }
+      }
+    }
+  } else if (valid) {
+    uint16_t* d16 = reinterpret_cast<uint16_t*>(srow32);
+    for (int c = 0; c < P; ++c) d16[c] = row[c];
   }
   Slots<KA, (KT > 0)> ch, pos;
   int taken = 0, cursor = 0;
-  unsigned long long my_over = 0, my_drop = 0;
+  uint64_t avail = P == 64 ? ~0ull : (1ull << P) - 1, chosen = 0;  // mask mode: by ranking position
   if (tid == 0) s_over = s_drop = 0;
+  if (tid < 2) applied_s[tid] = 0;
   for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = 0;
-  for (int e = tid; e < kMaxExperts; e += kThreads) cidx[e] = -1;
   __syncthreads();
   auto is_full = [&](int e) { return (full_s[e >> 5] >> (e & 31)) & 1u; };
   // walk on from the cursor until k non-full experts are held
@@ -172,9 +248,10 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
     if (a.policy == MOE_CAP_OVERFLOW_NEXT) return j < taken ? ch.get(j) : -1;
     return ch.get(j);
   };
-  // drop the experts that are full now; under OVERFLOW_NEXT walk on to replace them
-  auto drop_full = [&]() -> bool {
-    bool changed = false;
+  // Drop the experts that are full now; under OVERFLOW_NEXT walk on to replace them. Returns the
+  // first slot that holds a new choice (k: none). A dropped expert's count is not taken back: a
+  // full expert's count is C, whatever its holders.
+  auto drop_full = [&]() -> int {
     if (a.policy == MOE_CAP_OVERFLOW_NEXT) {
       int kept = 0;
       for (int j = 0; j < k; ++j)
@@ -187,38 +264,62 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
             ++kept;
           }
         }
-      if (kept < taken) {
-        taken = kept;
-        refill();
-        changed = true;
+      if (kept == taken) return k;
+      taken = kept;
+      refill();
+      return kept;
+    }
+    for (int j = 0; j < k; ++j)
+      if (ch.get(j) >= 0 && is_full(ch.get(j))) ch.set(j, -1);
+    return k;
+  };
+  auto count_new = [&](int from) {
+    for (int j = 0; j < k; ++j)
+      if (j >= from && j < taken) atomicAdd(&hist[ch.get(j)], 1);
+  };
+  // mask mode: the choices are the first k available positions (0xFFFF ends the ranking)
+  auto choose = [&]() {
+    uint64_t m = avail;
+    taken = 0;
+    chosen = 0;
+    for (int j = 0; j < k; ++j) {
+      if (m == 0) break;
+      const int p = __ffsll((long long)m) - 1;
+      const int e = srow[p];
+      if (e == 0xFFFF) break;
+      ch.set(j, e);
+      pos.set(j, p);
+      chosen |= 1ull << p;
+      ++taken;
+      m &= m - 1;
+    }
+  };
+  // mask mode: clear the positions of the experts filled since the masks were last brought up to
+  // date; the hist of a new choice goes up (a left expert is full: its count is C anyway)
+  auto apply_full = [&](bool counted) {
+    uint64_t cleared = 0;
+    const uint8_t* inv = pos_of + tid * (kPosWords * 4);
+    for (int w = 0; w < 2; ++w) {
+      uint32_t bits = full_s[w] & ~applied_s[w];
+      while (bits) {
+        const int p = inv[32 * w + __ffs(bits) - 1];
+        bits &= bits - 1;
+        if (p != 0xFF) cleared |= 1ull << p;
       }
-    } else {
+    }
+    avail &= ~cleared;
+    if (!(chosen & cleared)) return;
+    const uint64_t old = chosen;
+    choose();
+    if (counted)
       for (int j = 0; j < k; ++j)
-        if (ch.get(j) >= 0 && is_full(ch.get(j))) {
-          ch.set(j, -1);
-          changed = true;
-        }
-    }
-    return changed;
-  };
-  // this token's choices in or out of the histogram
-  auto count_mine = [&](int sign) {
-    for (int j = 0; j < k; ++j) {
-      const int e = slot(j);
-      if (e >= 0) atomicAdd(&hist[e], sign);
-    }
-  };
-  auto commit = [&]() {
-    for (int j = 0; j < k; ++j) {
-      const int e = slot(j);
-      a.topk_idx[t * k + j] = e;
-      my_drop += e < 0;
-      if (a.policy == MOE_CAP_OVERFLOW_NEXT && j < taken) my_over += pos.get(j) >= k;
-    }
+        if (j < taken && !((old >> pos.get(j)) & 1ull)) atomicAdd(&hist[ch.get(j)], 1);
   };
   // choices under no full expert, while the predecessor resolves its range
   if (valid) {
-    if (a.policy == MOE_CAP_OVERFLOW_NEXT) {
+    if (mm) {
+      choose();
+    } else if (a.policy == MOE_CAP_OVERFLOW_NEXT) {
       refill();
     } else {
       for (int j = 0; j < k; ++j) {
@@ -232,148 +333,130 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
   // turn too: its tokens walk past them while CTA b - 1 still works, and the histogram of the
   // resulting choices is taken before the last wait.
   if (blockIdx.x >= 2) {
-    if (tid == 0) s_ok = wait_for(chain + blockIdx.x - 2, a.status) ? 1 : 0;
-    __syncthreads();
-    if (!s_ok) {
-      if (tid == 0) atomicExch(&mine->flag, 2);  // abandon the rest of the chain at once
+    if (!take_state(chain + blockIdx.x - 2, E, a.C, nullptr, full_s, &s_ok, a.status)) {
+      abandon(mine, E);  // abandon the rest of the chain at once
       return;
     }
-    for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = __ldcg(&chain[blockIdx.x - 2].full[w]);
-    __syncthreads();
-    if (valid) drop_full();
+    if (valid) {
+      if (mm)
+        apply_full(false);
+      else
+        drop_full();
+    }
   }
   for (int e = tid; e < E; e += kThreads) hist[e] = 0;
   __syncthreads();
+  if (tid < 2) applied_s[tid] = full_s[tid];  // before take_state below writes full_s
   for (int j = 0; j < k; ++j) warp_count(hist, valid ? slot(j) : -1);
-  // the predecessor's counts and full set (other CTAs wrote them: read from L2, not L1)
-  if (tid == 0) s_ok = blockIdx.x == 0 ? 1 : (wait_for(chain + blockIdx.x - 1, a.status) ? 1 : 0);
-  __syncthreads();
-  if (!s_ok) {
-    if (tid == 0) atomicExch(&mine->flag, 2);
+  // the predecessor's counts and full set (other CTAs wrote them: read at L2, not L1)
+  if (blockIdx.x == 0) {
+    for (int e = tid; e < kMaxExperts; e += kThreads) cnt0[e] = 0;
+    __syncthreads();
+  } else if (!take_state(chain + blockIdx.x - 1, E, a.C, cnt0, full_s, &s_ok, a.status)) {
+    abandon(mine, E);
     return;
   }
-  if (blockIdx.x == 0) {
-    for (int e = tid; e < kMaxExperts; e += kThreads) cnt_s[e] = 0;
-  } else {
-    const ChainState* prev = chain + blockIdx.x - 1;
-    for (int e = tid; e < kMaxExperts; e += kThreads) cnt_s[e] = __ldcg(&prev->cnt[e]);
-    for (int w = tid; w < kMaxExperts / 32; w += kThreads) full_s[w] = __ldcg(&prev->full[w]);
+  // tokens that held an expert CTA b - 1 filled walk on; the histogram follows their new choices
+  if (valid && blockIdx.x > 0) {
+    if (mm)
+      apply_full(true);
+    else
+      count_new(drop_full());
   }
-  __syncthreads();
-  // tokens that held an expert CTA b - 1 filled walk on; the histogram follows them
-  if (valid) {
-    Slots<KA, (KT > 0)> ch0 = ch;
-    const int taken0 = taken;
-    if (blockIdx.x > 0 && drop_full()) {
-      for (int j = 0; j < k; ++j) {
-        const int e = a.policy == MOE_CAP_OVERFLOW_NEXT ? (j < taken0 ? ch0.get(j) : -1) : ch0.get(j);
-        if (e >= 0) atomicSub(&hist[e], 1);
-      }
-      count_mine(1);
-    }
-  }
-  // from here on hist holds the choices of every uncommitted token of the range
+  // Rounds. Committed tokens (those before f) never change their choices, so the token at which
+  // expert e reaches C is its (C - cnt0[e])-th holder among all of the range's tokens, and an
+  // expert is a candidate when cnt0[e] + hist[e] >= C. The first such token ends the round: the
+  // experts that fill at it become full and the later tokens that held them walk on. Every warp
+  // lists the candidates itself (the same list, in expert order) and ballots its tokens' holdings
+  // of them, 32 candidates a batch; warp 0 finds each candidate's filling token from the warps'
+  // counts and marks the experts that fill first. Three barriers a round, one when none fills.
   int f = 0;  // first token of the range not committed yet (uniform across the CTA)
   for (;;) {
-    const bool active = valid && tid >= f;
-    if (tid == 0) {
-      n_cand = 0;
-      s_stop = kThreads;
-    }
-    __syncthreads();
-    for (int e = tid; e < E; e += kThreads)
-      if (!is_full(e) && cnt_s[e] + hist[e] >= a.C) {
-        const int c = atomicAdd(&n_cand, 1);
-        cand[c] = e;
-        cidx[e] = (int8_t)(c < 127 ? c : 127);
-      }
-    __syncthreads();
-    const int nc = n_cand;
-    // The token at which each candidate expert reaches C: its (C - count)-th chooser in token
-    // order. Candidates go 32 at a time: every warp ballots all of them, then warp q finds
-    // candidate q's chooser with a prefix over the warps' counts.
-    for (int c0 = 0; c0 < nc; c0 += 32) {
-      const int nb = nc - c0 < 32 ? nc - c0 : 32;
-      uint32_t held = 0;  // bit q: this token holds candidate c0 + q
-      if (active)
-        for (int j = 0; j < k; ++j) {
-          const int e = slot(j);
-          if (e >= 0) {
-            const int q = nc <= 127 ? (int)cidx[e] - c0 : -1;
-            if (q >= 0 && q < nb && cand[c0 + q] == e) {
-              held |= 1u << q;
-            } else if (nc > 127) {
-              for (int qq = 0; qq < nb; ++qq) held |= cand[c0 + qq] == e ? 1u << qq : 0u;
-            }
+    __syncthreads();  // choices and hist are up to date
+    if (tid < 2) applied_s[tid] = full_s[tid];  // mask mode: every mask excludes these
+    int nc = 0;
+    int stop = kThreads;  // warp 0: the first filling token so far
+    for (int bt = 0;; ++bt) {
+      int idx = 0;
+      for (int e0 = 0; e0 < E; e0 += 32) {
+        const int e = e0 + lane;
+        uint32_t m = __ballot_sync(kFull, e < E && !is_full(e) && cnt0[e] + hist[e] >= a.C);
+        while (m) {
+          const int ec = e0 + __ffs(m) - 1;
+          m &= m - 1;
+          if (idx >= 32 * bt && idx < 32 * bt + 32) {
+            bool h = false;
+            if (valid)
+              for (int j = 0; j < k; ++j) h |= slot(j) == ec;
+            const uint32_t b = __ballot_sync(kFull, h);
+            if (lane == 0) bal[idx - 32 * bt][wid] = b;
           }
+          if (bt == 0 && tid == 0) cand[idx] = ec;
+          ++idx;
         }
-      for (int q = 0; q < nb; ++q) {
-        const uint32_t b = __ballot_sync(kFull, (held >> q) & 1u);
-        if (lane == 0) bal[q][wid] = b;
       }
-      __syncthreads();
-      if (wid < nb) {
-        const int e = cand[c0 + wid];
-        const int need = (int)(a.C - cnt_s[e]);
-        const uint32_t bw = bal[wid][lane];
-        const int pc = __popc(bw);
-        int incl = pc;
+      nc = idx;
+      if (nc == 0) break;
+      __syncthreads();  // the batch's ballots are down
+      if (wid == 0) {
+        const int nb = nc - 32 * bt < 32 ? nc - 32 * bt : 32;
+        for (int q = 0; q < nb; ++q) {
+          const int e = cand[32 * bt + q];
+          const int need = (int)(a.C - cnt0[e]);
+          const uint32_t bw = bal[q][lane];  // lane w: the holders among warp w's tokens
+          const int pc = __popc(bw);
+          int incl = pc;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const int v = __shfl_up_sync(kFull, incl, off);
-          if (lane >= off) incl += v;
-        }
-        if (incl - pc < need && need <= incl) {
-          uint32_t bb = bw;
-          for (int q = 1; q < need - (incl - pc); ++q) bb &= bb - 1;
-          atomicMin(&s_stop, lane * 32 + __ffs(bb) - 1);
+          for (int off = 1; off < 32; off <<= 1) {
+            const int v = __shfl_up_sync(kFull, incl, off);
+            if (lane >= off) incl += v;
+          }
+          int at = kThreads;  // fewer holders than needed: not while hist is exact
+          if (incl - pc < need && need <= incl) {
+            uint32_t bb = bw;
+            for (int r = 1; r < need - (incl - pc); ++r) bb &= bb - 1;
+            at = lane * 32 + __ffs(bb) - 1;
+          }
+          at = __reduce_min_sync(kFull, at);
+          if (lane == 0) cstop[32 * bt + q] = at;
+          stop = at < stop ? at : stop;
         }
       }
-      __syncthreads();
+      if (32 * (bt + 1) >= nc) break;
+      __syncthreads();  // warp 0 is done with bal before the next batch writes it
     }
-    for (int c = tid; c < nc; c += kThreads) cidx[cand[c]] = -1;
-    const int stop = s_stop;  // last token committed in this step (kThreads: the rest of the range)
-    const bool take = active && tid <= stop;
-    if (stop < kThreads) {
-      // the committed tokens' counts; hist keeps those of the tokens after them
-      for (int e = tid; e < E; e += kThreads) hist_taken[e] = 0;
-      __syncthreads();
-      for (int j = 0; j < k; ++j) warp_count(hist_taken, take ? slot(j) : -1);
-      __syncthreads();
+    if (nc == 0) break;  // no expert fills in the rest of the range
+    if (wid == 0) {
+      __syncwarp();
+      if (stop < kThreads)
+        for (int c = lane; c < nc; c += 32)
+          if (cstop[c] == stop) atomicOr(&full_s[cand[c] >> 5], 1u << (cand[c] & 31));
+      if (lane == 0) s_stop = stop;
     }
-    if (take) commit();
-    for (int e = tid; e < E; e += kThreads) {
-      if (stop < kThreads) {
-        cnt_s[e] += hist_taken[e];
-        hist[e] -= hist_taken[e];
-      } else {
-        cnt_s[e] += hist[e];
-      }
-      if (cnt_s[e] >= a.C) atomicOr(&full_s[e >> 5], 1u << (e & 31));
-    }
-    __syncthreads();
-    if (stop >= cnt_tok - 1) break;
-    f = stop + 1;
-    // the later tokens holding the expert that just filled walk on; the histogram follows them,
-    // so the next round needs no recount
+    __syncthreads();  // the filling token and the new full set are out
+    const int st = s_stop;
+    if (st >= cnt_tok - 1) break;
+    f = st + 1;
+    // the later tokens holding an expert that just filled walk on; the histogram follows them
     if (valid && tid >= f) {
-      Slots<KA, (KT > 0)> ch0 = ch;
-      const int taken0 = taken;
-      if (drop_full()) {
-        for (int j = 0; j < k; ++j) {
-          const int e = a.policy == MOE_CAP_OVERFLOW_NEXT ? (j < taken0 ? ch0.get(j) : -1) : ch0.get(j);
-          if (e >= 0) atomicSub(&hist[e], 1);
-        }
-        count_mine(1);
-      }
+      if (mm)
+        apply_full(true);
+      else
+        count_new(drop_full());
     }
   }
-  // hand the counts and full set on
-  for (int e = tid; e < kMaxExperts; e += kThreads) mine->cnt[e] = cnt_s[e];
-  for (int w = tid; w < kMaxExperts / 32; w += kThreads) mine->full[w] = full_s[w];
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) atomicExch(&mine->flag, 1);
+  // hand the counts on: C for a full expert, else the predecessor's count plus this range's
+  for (int e = tid; e < E; e += kThreads)
+    st_relaxed(&mine->cnt[e], (uint32_t)(is_full(e) ? (int)a.C : cnt0[e] + hist[e]) + 1u);
+  // every token's final choices
+  unsigned long long my_over = 0, my_drop = 0;
+  if (valid)
+    for (int j = 0; j < k; ++j) {
+      const int e = slot(j);
+      a.topk_idx[t * k + j] = e;
+      my_drop += e < 0;
+      if (a.policy == MOE_CAP_OVERFLOW_NEXT && j < taken) my_over += pos.get(j) >= k;
+    }
   atomicAdd(&s_over, my_over);
   atomicAdd(&s_drop, my_drop);
   __syncthreads();
@@ -387,7 +470,7 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
 size_t dyn_smem(unsigned grid, int E) {
   (void)grid;
   const int P = E < kPrefix ? E : kPrefix;
-  return (size_t)kThreads * prefix_words(P) * sizeof(uint32_t);
+  return (size_t)kThreads * (prefix_words(P) + (mask_capable(E) ? kPosWords : 0)) * sizeof(uint32_t);
 }
 
 template <int KT>
@@ -437,7 +520,7 @@ cudaError_t launch_capacity_grid(const CapacityArgs& a, void* scratch, cudaStrea
   ChainState* g = static_cast<ChainState*>(scratch);
   CapacityArgs b = a;
   const unsigned grid = (unsigned)ceil_div(a.n, kThreads);
-  cudaError_t e = cudaMemsetAsync(g, 0, (size_t)grid * sizeof(ChainState), s);  // every flag 0
+  cudaError_t e = cudaMemsetAsync(g, 0, (size_t)grid * sizeof(ChainState), s);  // no word written yet
   if (e != cudaSuccess) return e;
   switch (a.k) {
     case 1: return launch_t<1>(b, g, grid, s);
