@@ -106,6 +106,20 @@ __device__ void abandon(ChainState* mine, int E) {
   for (int e = threadIdx.x; e < E; e += blockDim.x) st_relaxed(&mine->cnt[e], kAbandoned);
 }
 
+// Position of the n-th (from 1) set bit of x, n <= popc(x): a binary search on popcounts.
+__device__ __forceinline__ int nth_set_bit(uint32_t x, int n) {
+  int pos = 0;
+  int c = __popc(x & 0xFFFFu);
+  if (n > c) { n -= c; pos += 16; x >>= 16; }
+  c = __popc(x & 0xFFu);
+  if (n > c) { n -= c; pos += 8; x >>= 8; }
+  c = __popc(x & 0xFu);
+  if (n > c) { n -= c; pos += 4; x >>= 4; }
+  c = __popc(x & 0x3u);
+  if (n > c) { n -= c; pos += 2; x >>= 2; }
+  return pos + (n > (int)(x & 1u) ? 1 : 0);
+}
+
 // counts[e] += 1 for every lane whose slot holds e (e < 0: nothing), one shared-memory atomic per
 // distinct expert in the warp.
 __device__ __forceinline__ void warp_count(int* counts, int e) {
@@ -412,11 +426,7 @@ __global__ void __launch_bounds__(kThreads) capacity_grid_kernel(CapacityArgs a,
             if (lane >= off) incl += v;
           }
           int at = kThreads;  // fewer holders than needed: not while hist is exact
-          if (incl - pc < need && need <= incl) {
-            uint32_t bb = bw;
-            for (int r = 1; r < need - (incl - pc); ++r) bb &= bb - 1;
-            at = lane * 32 + __ffs(bb) - 1;
-          }
+          if (incl - pc < need && need <= incl) at = lane * 32 + nth_set_bit(bw, need - (incl - pc));
           at = __reduce_min_sync(kFull, at);
           if (lane == 0) cstop[32 * bt + q] = at;
           stop = at < stop ? at : stop;
