@@ -94,7 +94,7 @@ struct RouteArgs {
   int32_t* topk_idx;    // [n, k] (written when ranking == nullptr)
   float* topk_w;        // [n, k]
   moe_diag* diag;       // refined_tokens / refined_logits counters
-  int32_t* cursor;      // zeroed before the launch: next token to route (warps fetch tokens from it)
+  int32_t* cursor;      // zeroed before the launch: a warp's tokens after its first come from it
   const int32_t* queue = nullptr;      // when set: route only the tokens queue[0 .. *queue_len)
   const int32_t* queue_len = nullptr;
   const int32_t* cand = nullptr;       // with queue: candidate experts and their binary64 logits
@@ -141,7 +141,8 @@ struct RouteTcArgs {
                         // zero before launch_refine, which adds two partial sums into each)
   int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine: one run per token, padded
                         // with -1 to a multiple of four (a warp refines four pairs of one token)
-  int32_t* pair_count;  // [2] zeroed before the launch: pairs listed, refine cursor
+  int32_t* pair_count;  // [4] zeroed before the launch: pairs listed, (unused), the second route
+                        // pass's cursor, the second queue's length
   moe_diag* status;
 };
 bool route_tc_supported(const RouteTcArgs& a);

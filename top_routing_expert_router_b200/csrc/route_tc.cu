@@ -556,18 +556,16 @@ __global__ void __launch_bounds__(kThreads, 1)
 // one token and one half of the rows: the token's row is read and widened once for the four
 // experts. Products of two bf16 values are exact in binary64; the sums are DFMA, the lanes taking
 // 16-byte chunks in turn with four chunks of every row in flight. The two halves' sums are added
-// into the zeroed candidate values (two terms: the same result in either order).
-__global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, const int32_t* cursor_base) {
+// into the zeroed candidate values (two terms: the same result in either order). Every item is the
+// same work, so warp w takes items w, w + W, ... (W warps in the grid): no shared cursor, and a
+// grid sized for the largest possible list costs the warps without work one load each.
+__global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p) {
   constexpr int U = 4;
-  int32_t* cursor = const_cast<int32_t*>(cursor_base);
   const int lane = threadIdx.x & 31;
   const int quads = *p.pair_count / 4;
   const int nchunk = p.d / 8;
-  for (;;) {
-    int item = 0;
-    if (lane == 0) item = atomicAdd(cursor, 1);
-    item = __shfl_sync(0xFFFFFFFFu, item, 0);
-    if (item >= 2 * quads) break;
+  const int W = (int)(gridDim.x * (blockDim.x / 32));
+  for (int item = (int)(blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)); item < 2 * quads; item += W) {
     const int i = item >> 1, half = item & 1;
     const int c_lo = half ? nchunk / 2 : 0, c_hi = half ? nchunk : nchunk / 2;
     int slot[4], e[4];
@@ -694,7 +692,7 @@ cudaError_t launch_refine(const RouteTcArgs& a, cudaStream_t s) {
   // at most two warps per four listed pairs, and n * kRouteCandMax pairs can be listed
   const int64_t need = ceil_div(a.n * kCandMax / 2, 8);
   const unsigned grid = (unsigned)(need < sms * 8 ? need : sms * 8);
-  refine_kernel<<<grid, 256, 0, s>>>(a, a.pair_count + 1);
+  refine_kernel<<<grid, 256, 0, s>>>(a);
   return cudaGetLastError();
 }
 

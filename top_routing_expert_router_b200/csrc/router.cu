@@ -117,15 +117,15 @@ __device__ __forceinline__ void selection_values(const RouteArgs& a, const doubl
 // are exact the group score is exact.
 template <int EPL>
 __device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
-                                 double delta_v, uint32_t* elig, uint32_t* mark);
+                                 double delta_v, uint32_t* elig, uint32_t* mark, unsigned long long* keys);
 
 template <int EPL>
 __device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
-                              double delta_v, uint32_t* elig, uint32_t* mark) {
+                              double delta_v, uint32_t* elig, uint32_t* mark, unsigned long long* keys) {
   const int lane = threadIdx.x & 31;
   const int per = a.E / a.G;
   // groups of 32 experts, one per lane slot: every group's reduction at once (below)
-  if (per == 32 && a.G == EPL) return decide_groups_32<EPL>(a, v, valid, exact, delta_v, elig, mark);
+  if (per == 32 && a.G == EPL) return decide_groups_32<EPL>(a, v, valid, exact, delta_v, elig, mark, keys);
   double gs[kMaxGroups], gu[kMaxGroups], t2s[kMaxGroups];
   for (int g = 0; g < a.G; ++g) {
     double t1 = -INFINITY, t2 = -INFINITY;
@@ -206,19 +206,44 @@ __device__ bool decide_groups(const RouteArgs& a, const double (&v)[EPL], const 
 // the warp together (independent shuffle chains), with no per-expert group arithmetic.
 template <int EPL>
 __device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], const bool (&valid)[EPL], uint32_t exact,
-                                 double delta_v, uint32_t* elig, uint32_t* mark) {
-  // The two best values of every group on integer order keys (warp reductions; binary64
-  // comparisons and min/max are slow next to integer ones when many warps decide at once): the
-  // best lane, then the best of the other lanes (equal to the first on a tie).
+                                 double delta_v, uint32_t* elig, uint32_t* mark, unsigned long long* keys) {
+  // The two best values of every group (the largest and the largest of the rest, equal to the
+  // first on a tie) on integer order keys, which order like the values (binary64 comparisons and
+  // min/max are slow next to integer ones when many warps decide at once). Group g is slot g of
+  // every lane; through the warp's shared scratch each group goes to 32 / EPL lanes of EPL keys
+  // each, which take their two best and merge them by shuffles, instead of one chain of warp
+  // reductions per group and rank.
   const int lane = threadIdx.x & 31;
+  constexpr int LPG = 32 / EPL;  // lanes per group
+  __syncwarp();  // the scratch's previous readers are done
+#pragma unroll
+  for (int g = 0; g < EPL; ++g) keys[g * 32 + lane] = order_key(valid[g] ? v[g] : -INFINITY);
+  __syncwarp();
+  unsigned long long k1 = 0ull, k2 = 0ull;  // 0 is below the key of every value, -inf included
+  const unsigned long long* mine = keys + (lane / LPG) * 32 + (lane % LPG) * EPL;
+#pragma unroll
+  for (int i = 0; i < EPL; ++i) {
+    const unsigned long long kk = mine[(i + lane) % EPL];
+    if (kk > k1) {
+      k2 = k1;
+      k1 = kk;
+    } else if (kk > k2) {
+      k2 = kk;
+    }
+  }
+#pragma unroll
+  for (int off = 1; off < LPG; off <<= 1) {
+    const unsigned long long o1 = __shfl_xor_sync(kFull, k1, off);
+    const unsigned long long o2 = __shfl_xor_sync(kFull, k2, off);
+    const unsigned long long lo1 = k1 < o1 ? k1 : o1, hi2 = k2 > o2 ? k2 : o2;
+    k1 = k1 > o1 ? k1 : o1;
+    k2 = lo1 > hi2 ? lo1 : hi2;
+  }
   double t1[EPL], t2[EPL];
 #pragma unroll
   for (int g = 0; g < EPL; ++g) {
-    const unsigned long long key = order_key(valid[g] ? v[g] : -INFINITY);
-    const int w1 = warp_argmax_key(key);
-    const int w2 = warp_argmax_key(lane == w1 ? 0ull : key);
-    t1[g] = __shfl_sync(kFull, valid[g] ? v[g] : -INFINITY, w1);
-    t2[g] = __shfl_sync(kFull, valid[g] ? v[g] : -INFINITY, w2);
+    t1[g] = key_value(__shfl_sync(kFull, k1, g * LPG));
+    t2[g] = key_value(__shfl_sync(kFull, k2, g * LPG));
   }
   double gs[EPL], gu[EPL];
 #pragma unroll
@@ -278,7 +303,7 @@ __device__ bool decide_groups_32(const RouteArgs& a, const double (&v)[EPL], con
 // Otherwise sets, in *refine, the inexact experts an uncertain comparison involves.
 template <int EPL>
 __device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exact, double delta_v, int16_t* rank,
-                       int* n_ranked, uint32_t* refine) {
+                       int* n_ranked, uint32_t* refine, unsigned long long* keys) {
   const int lane = threadIdx.x & 31;
   double v[EPL];
   bool valid[EPL];
@@ -288,7 +313,7 @@ __device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exac
   uint32_t mark = 0;
   uint32_t elig_mask = 0;
   if (a.G > 1) {
-    if (!decide_groups<EPL>(a, v, valid, exact, delta_v, &elig_mask, &mark)) ok = false;
+    if (!decide_groups<EPL>(a, v, valid, exact, delta_v, &elig_mask, &mark, keys)) ok = false;
   } else {
 #pragma unroll
     for (int j = 0; j < EPL; ++j)
@@ -375,7 +400,8 @@ __device__ bool decide(const RouteArgs& a, const double (&l)[EPL], uint32_t exac
 // `flags` (per-warp shared, one byte per expert) and returned in *refine.
 template <int EPL>
 __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t exact, double delta_v,
-                            int16_t* rank, uint8_t* flags, int* n_ranked, uint32_t* refine) {
+                            int16_t* rank, uint8_t* flags, int* n_ranked, uint32_t* refine,
+                            unsigned long long* keys) {
   const int lane = threadIdx.x & 31;
   const int E = a.E;
   double v0[EPL];
@@ -385,7 +411,7 @@ __device__ bool decide_full(const RouteArgs& a, const double (&l)[EPL], uint32_t
   bool ok = true;
   uint32_t mark = 0;
   if (a.G > 1) {
-    if (!decide_groups<EPL>(a, v0, valid, exact, delta_v, &elig_mask, &mark)) ok = false;
+    if (!decide_groups<EPL>(a, v0, valid, exact, delta_v, &elig_mask, &mark, keys)) ok = false;
   } else {
 #pragma unroll
     for (int j = 0; j < EPL; ++j)
@@ -722,6 +748,7 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
   __shared__ uint8_t s_flag[kWarpsPerBlock][kMaxExperts];
   __shared__ int s_idx[kWarpsPerBlock][kMaxTopK];
   __shared__ double s_val[kWarpsPerBlock][kMaxTopK];
+  __shared__ unsigned long long s_keys[kWarpsPerBlock][kMaxExperts];  // the group cut's scratch
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   constexpr bool full_ranking = FULL;  // the capacity rule needs every eligible expert ranked
   for (int i = lane; i < kMaxExperts; i += 32) s_flag[wib][i] = 0;
@@ -730,13 +757,19 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
 #pragma unroll
   for (int j = 0; j < EPL; ++j)
     if (lane + 32 * j < a.E) valid_mask |= 1u << j;
-  // Warps take the next token from a shared cursor: a token that needs binary64
-  // refinement holds up only its own warp, never a whole block of tokens.
+  // A warp's first token is fixed by its place in the grid; after that it takes the next one from a
+  // shared cursor (past the first W = the grid's warps), so a token that needs binary64 refinement
+  // holds up only its own warp, and a warp without a token leaves after one load, never touching
+  // the cursor (the grid is sized before the queue's length is known).
   const int64_t count = a.queue ? (int64_t)*a.queue_len : a.n;
-  for (;;) {
-    int tok = 0;
-    if (lane == 0) tok = atomicAdd(a.cursor, 1);
-    const int64_t i = __shfl_sync(kFull, tok, 0);
+  const int64_t W = (int64_t)gridDim.x * kWarpsPerBlock;
+  for (bool first = true;; first = false) {
+    int64_t i = (int64_t)blockIdx.x * kWarpsPerBlock + wib;
+    if (!first) {
+      int tok = 0;
+      if (lane == 0) tok = atomicAdd(a.cursor, 1);
+      i = W + __shfl_sync(kFull, tok, 0);
+    }
     if (i >= count) break;
     const int64_t t = a.queue ? (int64_t)a.queue[i] : i;
     double l[EPL];
@@ -782,9 +815,9 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
       uint32_t refine = 0;
       bool ok;
       if constexpr (FULL)
-        ok = decide_full<EPL>(a, l, exact, delta_v, s_rank[wib], s_flag[wib], &nr, &refine);
+        ok = decide_full<EPL>(a, l, exact, delta_v, s_rank[wib], s_flag[wib], &nr, &refine, s_keys[wib]);
       else
-        ok = decide<EPL>(a, l, exact, delta_v, s_rank[wib], &nr, &refine);
+        ok = decide<EPL>(a, l, exact, delta_v, s_rank[wib], &nr, &refine, s_keys[wib]);
       if (ok) break;
       refine &= ~exact;
       if (it == 0 && a.defer_queue && __any_sync(kFull, refine != 0)) {
@@ -801,9 +834,9 @@ __global__ void __launch_bounds__(32 * kWarpsPerBlock) route_kernel(RouteArgs a)
         if (it < 6) {
           int nr_w = 0;
           if constexpr (FULL)
-            decide_full<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], s_flag[wib], &nr_w, &wide);
+            decide_full<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], s_flag[wib], &nr_w, &wide, s_keys[wib]);
           else
-            decide<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], &nr_w, &wide);
+            decide<EPL>(a, l, exact, 4.0 * delta_v, s_rank[wib], &nr_w, &wide, s_keys[wib]);
           wide &= ~exact;
         }
         refine = __any_sync(kFull, wide != 0) ? wide : (valid_mask & ~exact);
