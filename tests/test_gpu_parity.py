@@ -120,6 +120,17 @@ def test_capacity_on_many_ctas(k, policy, mode, monkeypatch):
     test_route_parity(w.name, w)
 
 
+@pytest.mark.parametrize("policy", ["overflow_next", "drop"])
+@pytest.mark.parametrize("E", [8, 24, 40, 100, 128])
+def test_capacity_grid_expert_counts(E, policy):
+    """6000 tokens on 6 CTAs of the chained grid, across the expert counts its staging and walks
+    distinguish: whole rankings of at most 64 experts with the position masks (E a multiple of 8),
+    rankings staged token by token (E = 100), and walks that go on in global memory past the 64
+    staged entries (E = 128)."""
+    w = W.get("skewed_small", n_routed=E, top_k=2, cap_policy=policy, n=6000)
+    test_route_parity(w.name, w)
+
+
 @pytest.mark.parametrize("name", ["mixtral_small", "deepseek_v2_small", "skewed_small", "drop_small", "tiny_f32"])
 def test_permute_parity(name):
     w = W.get(name)
