@@ -141,8 +141,8 @@ struct RouteTcArgs {
                         // zero before launch_refine, which adds two partial sums into each)
   int32_t* pairs;       // [n * kRouteCandMax] candidate slots to refine: one run per token, padded
                         // with -1 to a multiple of four (a warp refines four pairs of one token)
-  int32_t* pair_count;  // [4] zeroed before the launch: pairs listed, (unused), the second route
-                        // pass's cursor, the second queue's length
+  int32_t* pair_count;  // [4] zeroed before the launch: pairs listed, the refinement's cursor, the
+                        // second route pass's cursor, the second queue's length
   moe_diag* status;
 };
 bool route_tc_supported(const RouteTcArgs& a);

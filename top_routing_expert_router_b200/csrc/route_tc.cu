@@ -556,16 +556,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // one token and one half of the rows: the token's row is read and widened once for the four
 // experts. Products of two bf16 values are exact in binary64; the sums are DFMA, the lanes taking
 // 16-byte chunks in turn with four chunks of every row in flight. The two halves' sums are added
-// into the zeroed candidate values (two terms: the same result in either order). Every item is the
-// same work, so warp w takes items w, w + W, ... (W warps in the grid): no shared cursor, and a
-// grid sized for the largest possible list costs the warps without work one load each.
-__global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p) {
+// into the zeroed candidate values (two terms: the same result in either order). A warp's first
+// item is fixed by its place in the grid (W warps); only a warp that finished one takes the next
+// from the shared cursor, past the first W. A grid sized for the largest possible list then costs
+// the warps without work one load each, and long lists still balance across the warps.
+__global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, int32_t* cursor) {
   constexpr int U = 4;
   const int lane = threadIdx.x & 31;
   const int quads = *p.pair_count / 4;
   const int nchunk = p.d / 8;
   const int W = (int)(gridDim.x * (blockDim.x / 32));
-  for (int item = (int)(blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)); item < 2 * quads; item += W) {
+  for (int item = (int)(blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)); item < 2 * quads;) {
     const int i = item >> 1, half = item & 1;
     const int c_lo = half ? nchunk / 2 : 0, c_hi = half ? nchunk : nchunk / 2;
     int slot[4], e[4];
@@ -609,6 +610,9 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p) {
       for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
       if (lane == 0 && slot[q] >= 0) atomicAdd(&p.cand_val[slot[q]], v);
     }
+    int next = 0;
+    if (lane == 0) next = atomicAdd(cursor, 1);
+    item = W + __shfl_sync(0xFFFFFFFFu, next, 0);
   }
 }
 
@@ -692,7 +696,7 @@ cudaError_t launch_refine(const RouteTcArgs& a, cudaStream_t s) {
   // at most two warps per four listed pairs, and n * kRouteCandMax pairs can be listed
   const int64_t need = ceil_div(a.n * kCandMax / 2, 8);
   const unsigned grid = (unsigned)(need < sms * 8 ? need : sms * 8);
-  refine_kernel<<<grid, 256, 0, s>>>(a);
+  refine_kernel<<<grid, 256, 0, s>>>(a, a.pair_count + 1);
   return cudaGetLastError();
 }
 
