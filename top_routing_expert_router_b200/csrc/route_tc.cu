@@ -551,17 +551,47 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// One item of refine_kernel: the binary64 dot products of x[t] with the NQ listed rows of W_r over
+// chunks [c_lo, c_hi) of 8 elements. NQ is the number of live pairs in the item's group of four (the
+// padding of a token's run is at its end), so no conversion or DFMA is spent on padding.
+template <int NQ>
+__device__ __forceinline__ void refine_rows(const uint4* xr, const uint4* const (&wr)[4], int c_lo, int c_hi, int lane,
+                                            double (&acc)[4]) {
+  constexpr int U = 4;
+  for (int c = c_lo + lane; c < c_hi; c += 32 * U) {
+    uint4 xv[U], wv[NQ][U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int cc = c + 32 * u;
+      xv[u] = cc < c_hi ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) wv[q][u] = cc < c_hi ? __ldg(wr[q] + cc) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const bf16* xs = reinterpret_cast<const bf16*>(&xv[u]);
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const double xd = (double)__bfloat162float(xs[h]);
+#pragma unroll
+        for (int q = 0; q < NQ; ++q)
+          acc[q] = fma(xd, (double)__bfloat162float(reinterpret_cast<const bf16*>(&wv[q][u])[h]), acc[q]);
+      }
+    }
+  }
+}
+
 // Binary64 logits x[t] . W_r[e] of the listed (queued token, candidate expert) pairs. Each token's
 // pairs are listed as one run padded with -1 to a multiple of four, so a warp takes four pairs of
 // one token and one half of the rows: the token's row is read and widened once for the four
-// experts. Products of two bf16 values are exact in binary64; the sums are DFMA, the lanes taking
-// 16-byte chunks in turn with four chunks of every row in flight. The two halves' sums are added
-// into the zeroed candidate values (two terms: the same result in either order). A warp's first
-// item is fixed by its place in the grid (W warps); only a warp that finished one takes the next
-// from the shared cursor, past the first W. A grid sized for the largest possible list then costs
-// the warps without work one load each, and long lists still balance across the warps.
+// experts, and only the live pairs of the four are computed. Products of two bf16 values are exact
+// in binary64; the sums are DFMA, the lanes taking 16-byte chunks in turn with four chunks of every
+// row in flight. The two halves' sums are added into the zeroed candidate values (two terms: the
+// same result in either order). A warp's first item is fixed by its place in the grid (W warps);
+// only a warp that finished one takes the next from the shared cursor, past the first W. A grid
+// sized for the largest possible list then costs the warps without work one load each, and long
+// lists still balance across the warps.
 __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, int32_t* cursor) {
-  constexpr int U = 4;
   const int lane = threadIdx.x & 31;
   const int quads = *p.pair_count / 4;
   const int nchunk = p.d / 8;
@@ -570,10 +600,14 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, int32_t* cur
     const int i = item >> 1, half = item & 1;
     const int c_lo = half ? nchunk / 2 : 0, c_hi = half ? nchunk : nchunk / 2;
     int slot[4], e[4];
+    int live = 0;
+    unsigned live_mask = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       slot[q] = p.pairs[4 * i + q];
       e[q] = slot[q] >= 0 ? p.cand[slot[q]] : -1;
+      live += e[q] >= 0;
+      live_mask |= (e[q] >= 0 ? 1u : 0u) << q;
     }
     const int64_t t = p.queue[slot[0] / (kCandMax + 1)];  // a run starts every group of four
     const uint4* xr = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.x) + t * p.d);
@@ -582,33 +616,23 @@ __global__ void __launch_bounds__(256) refine_kernel(RouteTcArgs p, int32_t* cur
     for (int q = 0; q < 4; ++q)
       wr[q] = reinterpret_cast<const uint4*>(static_cast<const bf16*>(p.w_r) + (int64_t)(e[q] < 0 ? 0 : e[q]) * p.d);
     double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int c = c_lo + lane; c < c_hi; c += 32 * U) {
-      uint4 xv[U], wv[4][U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int cc = c + 32 * u;
-        xv[u] = cc < c_hi ? __ldg(xr + cc) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) wv[q][u] = (cc < c_hi && e[q] >= 0) ? __ldg(wr[q] + cc) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const bf16* xs = reinterpret_cast<const bf16*>(&xv[u]);
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          const double xd = (double)__bfloat162float(xs[h]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            acc[q] = fma(xd, (double)__bfloat162float(reinterpret_cast<const bf16*>(&wv[q][u])[h]), acc[q]);
-        }
-      }
+    // The live pairs lead the group (padding ends a run); every lane reads the same four pairs. Any
+    // other pattern computes all four rows, a dead one from row 0, and keeps only the live sums.
+    if (live == 4 || live_mask != (1u << live) - 1u) {
+      refine_rows<4>(xr, wr, c_lo, c_hi, lane, acc);
+    } else if (live == 3) {
+      refine_rows<3>(xr, wr, c_lo, c_hi, lane, acc);
+    } else if (live == 2) {
+      refine_rows<2>(xr, wr, c_lo, c_hi, lane, acc);
+    } else if (live == 1) {
+      refine_rows<1>(xr, wr, c_lo, c_hi, lane, acc);
     }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       double v = acc[q];
 #pragma unroll
       for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, off);
-      if (lane == 0 && slot[q] >= 0) atomicAdd(&p.cand_val[slot[q]], v);
+      if (lane == 0 && slot[q] >= 0 && e[q] >= 0) atomicAdd(&p.cand_val[slot[q]], v);
     }
     int next = 0;
     if (lane == 0) next = atomicAdd(cursor, 1);
