@@ -55,7 +55,12 @@ def test_device_inputs_equal_host_inputs(name):
 @pytest.mark.parametrize("name", SMALL)
 def test_route_parity(name, w=None):
     w = w or W.get(name)
-    dev, host = W.device_inputs(w), W.host_inputs(w)
+    _check_route(w, W.device_inputs(w), W.host_inputs(w))
+
+
+def _check_route(w, dev, host):
+    """moe_route on the device inputs against the oracle's routing of the host inputs; returns the
+    diagnostics."""
     cfg = H.cfg_for(w)
     ws = H.workspace(cfg, w.n)
     idx = torch.empty((w.n, w.top_k), dtype=torch.int32, device="cuda")
@@ -85,6 +90,29 @@ def test_route_parity(name, w=None):
         np.testing.assert_array_equal(counts.cpu().numpy(), np.bincount(oi[oi >= 0], minlength=w.n_routed))
         assert diag["max_load"] == np.bincount(oi[oi >= 0], minlength=w.n_routed).max()
     assert ex.mean() < 0.05
+    return diag
+
+
+@pytest.mark.parametrize("name,n,refines", [("deepseek_v3_small", 333, True), ("deepseek_v3_small", 3000, True),
+                                            ("mixtral_small", 700, False), ("skewed_small", 2000, True)])
+def test_route_parity_with_subnormal_token_values(name, n, refines):
+    """Every token's row holds bf16 subnormals and a zero next to its normal values. The routing
+    must still equal the oracle's, which takes the exact binary64 values of the same inputs,
+    including for the tokens the binary64 refinement re-decides. From 2048 tokens the one-pass
+    router queues the uncertain tokens for that refinement. The Mixtral-shaped case certifies
+    every token in binary32."""
+    w = W.get(name, n=n)
+    dev, host = W.device_inputs(w), W.host_inputs(w)
+    x = host["x"].copy()
+    assert x.dtype == np.uint16
+    x[:, 0] = 0x0001  # smallest positive subnormal, 2^-133
+    x[:, 1] = 0x807F  # largest negative subnormal
+    x[:, 2] = 0x0000
+    dev = dict(dev, x=torch.from_numpy(x.view(np.int16)).to("cuda").view(torch.bfloat16))
+    host = dict(host, x=x)
+    diag = _check_route(w, dev, host)
+    if refines:
+        assert diag["refined_tokens"] > 0  # the refinement ran on rows holding subnormals
 
 
 @pytest.mark.parametrize("policy", ["overflow_next", "drop"])
