@@ -90,16 +90,18 @@ def _ceil(a, b):
     return -(-a // b)
 
 
-def _router_splits(w):
-    """Split-K factor of the two-kernel router's logits GEMM (router_splits in csrc/api.cu)."""
+def _router_splits(w, n=None):
+    """Split-K factor of the two-kernel router's logits GEMM for a batch of n tokens (router_splits in
+    csrc/api.cu)."""
+    n = w.n if n is None else n
     if w.dtype == "f32":
         return 1
-    tiles = _ceil(w.n, 128) * _ceil(w.n_routed, 256)
+    tiles = _ceil(n, 128) * _ceil(w.n_routed, 256)
     if tiles >= 74:
         return 1
     num_kb = _ceil(w.d_model, 64)
     ld = _ceil(w.n_routed, 4) * 4
-    s = max(1, min(148 // tiles, (4 << 20) // (w.n * ld * 4), 32, num_kb))
+    s = max(1, min(148 // tiles, (4 << 20) // (n * ld * 4), 32, num_kb))
     return _ceil(num_kb, _ceil(num_kb, s))
 
 
@@ -110,26 +112,34 @@ def _fp8_gemm_launches(rows, groups):
     return 2 if rows // groups >= 128 else 1
 
 
+def _router_launches(w, n):
+    """Kernels of this library's router (route_impl in csrc/api.cu) on a batch of n tokens, with the
+    histogram and scan of its expert counts."""
+    bf16_act = w.dtype != "f32"
+    if bf16_act and w.cap_policy == "none" and n >= 2048 and w.top_k <= 8:
+        k = 4  # one-pass router, first binary64 pass over its queue, refinement, second pass
+    else:
+        k = 2 if _router_splits(w, n) > 1 else 1  # logits GEMM (+ sum of the split-K partials)
+        k += 3 if bf16_act and w.d_model % 8 == 0 else 1  # first pass, refinement, second pass
+        if w.cap_policy != "none":
+            k += 2  # capacity + gates
+    return k + 2  # histogram + scan
+
+
+def _ffn_launches(w, rows, groups):
+    """Kernels of the expert FFN over `rows` permuted rows in `groups` experts (ffn_impl / ffn_fp8)."""
+    if w.dtype == "fp8":
+        return 2 + 2 * _fp8_gemm_launches(rows, groups)  # quantise x and h, GEMM1, GEMM2
+    return 2  # GEMM1 (SwiGLU) + GEMM2
+
+
 def launches_per_step(w):
     """Kernels of this library launched by one moe_layer_forward (the choices of csrc/api.cu)."""
-    bf16_act = w.dtype != "f32"
-    if bf16_act and w.cap_policy == "none" and w.n >= 2048 and w.top_k <= 8:
-        n = 3  # one-pass router, binary64 refinement of the queued tokens' candidates, queued tokens
-    else:
-        n = 2 if _router_splits(w) > 1 else 1  # logits GEMM (+ sum of the split-K partials)
-        n += 3 if bf16_act and w.d_model % 8 == 0 else 1  # first pass, refinement, second pass
-        if w.cap_policy != "none":
-            n += 2  # capacity + gates
-    n += 2  # histogram + scan (the permutation reuses them)
-    if w.dtype == "fp8":
-        n += 1  # scatter (the quantiser gathers the rows)
-        n += 2 + 2 * _fp8_gemm_launches(w.n * w.top_k, w.n_routed)  # quantise x and h, GEMM1, GEMM2
-        if w.n_shared:
-            n += 2 + 2 * _fp8_gemm_launches(w.n, 1)
-    else:
-        n += 2  # scatter + row copy
-        n += 2  # GEMM1 (SwiGLU) + GEMM2
-        n += 2 if w.n_shared else 0
+    n = _router_launches(w, w.n)  # the permutation reuses the histogram and scan
+    n += 1 if w.dtype == "fp8" else 2  # scatter (+ row copy; the FP8 quantiser gathers the rows)
+    n += _ffn_launches(w, w.n * w.top_k, w.n_routed)
+    if w.n_shared:
+        n += _ffn_launches(w, w.n, 1)
     n += 1  # combine
     return n
 
@@ -422,15 +432,20 @@ def _ep_rank_weights(moe, w, dev, q, world):
                             dev.get("ws_up"), dev.get("ws_down"), dev.get("bias"))
 
 
-def ep_launches_per_rank(w):
-    """Kernels of this library one rank launches in moe_ep_layer_forward (all ranks on one device)."""
-    n = 4  # router GEMM, route, histogram + scan of the counts
+def ep_launches_per_rank(w, n_rank, world, barriers):
+    """Kernels of this library one rank launches in one moe_ep_layer_forward over its n_rank tokens
+    (ep_forward in csrc/api.cu). The owned experts' row count is taken as the group's average,
+    n k / world over E / world experts. With one process per GPU (barriers) the rank also launches
+    the flag barrier after each of the four steps."""
+    n = _router_launches(w, n_rank)  # route, histogram + scan of the counts
     n += 3  # local stable permutation: histogram + scan + scatter (no local row gather)
     n += 2  # count publish, row push
-    n += 4 if w.dtype == "fp8" else 2  # owned experts: (quantise,) GEMM1, (quantise,) GEMM2
+    n += _ffn_launches(w, _ceil(w.n * w.top_k, world), max(1, w.n_routed // world))
     if w.n_shared:
-        n += 4 if w.dtype == "fp8" else 2
+        n += _ffn_launches(w, n_rank, 1)
     n += 1  # combine
+    if barriers:
+        n += 4
     return n
 
 
@@ -572,7 +587,7 @@ def run_ep(args):
                      "layer_minus_ffn_ms": ms_step - ffn_ms},
         "e2e": {"value": n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": n * d * bpe,
                 "d2h_bytes_per_step": n * d * bpe, "ms_per_step": e2e_ms},
-        "gpu_launches": ep_launches_per_rank(w) * R * args.steps,
+        "gpu_launches": sum(ep_launches_per_rank(w, nq, R, False) for nq in splits) * args.steps,
         "clocks": clocks,
     }
     print(json.dumps(out), flush=True)
@@ -711,7 +726,7 @@ def run_ep_dist(args):
             "ranks": ok_all,
             "e2e": {"value": w.n / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": w.n * d * bpe,
                     "d2h_bytes_per_step": w.n * d * bpe, "ms_per_step": e2e_ms},
-            "gpu_launches": ep_launches_per_rank(w) * world * args.steps,
+            "gpu_launches": sum(ep_launches_per_rank(w, nq, world, True) for nq in plan["splits"]) * args.steps,
             "clocks": clocks,
         }
         print(json.dumps(out), flush=True)
