@@ -167,3 +167,18 @@ def test_ep_handles_reject_bad_arguments():
     assert lib.moe_ep_close_handle(None) == moe.MOE_ERR_INVALID_ARG
     with pytest.raises(ValueError):
         moe.moe_ep_open_handle(b"short")
+
+
+def test_plain_c_caller_links_and_calls_the_host_entry_points(tmp_path):
+    """A C99 program that includes only include/moe.h links against the library, resolves every
+    entry point and gets the same workspace size as the binding (no GPU needed)."""
+    import subprocess
+
+    lib_dir = os.path.dirname(moe.LIB_PATH)
+    exe = str(tmp_path / "c_abi_check")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                           os.path.join(ROOT, "include"), os.path.join(ROOT, "tests", "c_abi_check.c"), "-L",
+                           lib_dir, "-lmoe_b200", "-Wl,-rpath," + lib_dir, "-o", exe])
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.strip()
+    want = moe.moe_workspace_size(_v3(), 16384)
+    assert out == "ok %d" % want, out
